@@ -1,0 +1,390 @@
+"""fp64 CPU oracle of one Grouped Query Experts (GQE) prefill layer.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline / reference arm of ``bench.py`` may import or call this package. The
+CUDA library never calls it, and it shares no code with the CUDA library: the
+two meet only in the seeded input generator ``synth`` (which draws numbers and
+computes nothing of the layer).
+
+What it computes is the plain definition of the layer, evaluated in fp64 on the
+exact values of the bf16 / fp32 inputs, with no tiling, no online softmax and no
+rounding to bf16 anywhere. Sources (all pages describe the same paper,
+"Grouped Query Experts: Mixture-of-Experts on GQA Self-Attention",
+arXiv:2606.20945):
+
+* routed query-head experts inside each fixed GQA group, a per-token router
+  choosing k experts per group, K/V projections dense and unchanged
+  (gist.science summary, "Technical Summary / Methodology: Architecture and
+  Routing"; chatpaper / hotpaper abstract);
+* "softmax first, then top-k" inside each group; every group takes part
+  (pptc.cn blog, section 7 Conclusion and section 5 Related Work);
+* output construction: hard concatenation of the selected experts, one
+  renormalised weighted-sum slot, one always-on shared head (gist.science
+  summary, "Output Construction");
+* W_O of size (kG+2) x d (hotpaper.ai summary, "Core idea" and "Technical
+  approach").
+
+Readings where the pages are silent, ambiguous or garbled:
+
+* R1 the shared head attends to KV group 0; R2 it has its own W_qs [d, dh];
+* R3 the weighted slot is sum_g sum_{j in S_g} w_gj * o_gj with
+  w = p / (sum over all kG selected p) (one slot, renormalised over every
+  selected expert of the token);
+* R4 the router output r is renormalised per group: r = p / sum_{S_g} p;
+* R5 ties go to the lower expert index; R6 routed slots are ordered by group,
+  then by ascending expert index inside the group; R7 top-k is taken on the
+  logits (equal to top-k on the in-group softmax, which is monotone);
+* R8 scale 1/sqrt(dh), no positional encoding, no biases besides the router's;
+* R9 W_O is [(kG+2)*dh, d]; R10 expert e = g*M + j; dense head h uses group
+  h // M; R11 key u is visible to query t iff u <= t in the same sequence.
+
+Parity is pinned by ``tests/test_oracle_pins.py`` (closed forms, brute force on
+tiny inputs, library routines on special cases, the pages' invariants).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from synth import LayerInputs, LayerShape, bf16_to_f64
+
+_U64 = 2.0 ** -53  # unit roundoff of fp64
+
+
+# --------------------------------------------------------------------------
+# a1-a4: router
+# --------------------------------------------------------------------------
+
+def router_logits(x: np.ndarray, W_r: np.ndarray, b_r: np.ndarray | None) -> np.ndarray:
+    """z[t, e] = sum_i x[t, i] * W_r[i, e] + b[e], in fp64.
+
+    Each product of a bf16 value and an fp32 value has at most 8 + 24
+    significant bits, so it is exact in fp64; only the summation rounds.
+    (Router scores over all experts: gist.science summary, "Conditional
+    activation".)
+    """
+    z = np.asarray(x, np.float64) @ np.asarray(W_r, np.float64)
+    if b_r is not None:
+        z = z + np.asarray(b_r, np.float64)[None, :]
+    return z
+
+
+def _exact_logit(xrow: np.ndarray, wcol: np.ndarray, b: float) -> float:
+    # Products are exact in fp64; math.fsum returns the correctly rounded sum.
+    return math.fsum(list(xrow * wcol) + [b])
+
+
+def router(x: np.ndarray, W_r: np.ndarray, b_r: np.ndarray | None, G: int, M: int, k: int):
+    """Per-group softmax, top-k per group, renormalised weights.
+
+    Returns a dict with
+      z     [R, N]    fp64 logits,
+      p     [R, G, M] in-group softmax probabilities,
+      idx   [R, G, k] int32 selected expert-local indices j, ascending,
+      r     [R, G, k] p renormalised inside the group (reading R4),
+      omega [R, G, k] p renormalised over all kG selected experts (reading R3).
+
+    The selection is the one exact arithmetic gives: where the fp64 logits of
+    a group are closer at the top-k boundary than a certified bound on their
+    rounding error, that group's logits are recomputed correctly rounded
+    (math.fsum of exact products) before selecting.
+    """
+    if not (1 <= k <= M):
+        raise ValueError("need 1 <= k <= M")
+    x = np.asarray(x, np.float64)
+    W_r = np.asarray(W_r, np.float64)
+    R, d = x.shape
+    N = G * M
+    assert W_r.shape == (d, N)
+    bvec = np.zeros(N) if b_r is None else np.asarray(b_r, np.float64)
+    z = router_logits(x, W_r, b_r)
+
+    # Certified fp64 error bound of each logit: gamma_{d+1} * (sum |x w| + |b|).
+    gam = (d + 1) * _U64 / (1.0 - (d + 1) * _U64)
+    bound = gam * (np.abs(x) @ np.abs(W_r) + np.abs(bvec)[None, :]) * 2.0
+
+    zg = z.reshape(R, G, M)
+    if k < M:
+        srt = -np.sort(-zg, axis=-1)
+        margin = srt[..., k - 1] - srt[..., k]
+        bg = bound.reshape(R, G, M).max(axis=-1)
+        for t, g in zip(*np.nonzero(margin <= 2.0 * bg)):
+            for j in range(M):
+                e = g * M + j
+                zg[t, g, j] = _exact_logit(x[t], W_r[:, e], bvec[e])
+        z = zg.reshape(R, N)
+
+    # a2: softmax over the M logits of each group (softmax before top-k).
+    zmax = zg.max(axis=-1, keepdims=True)
+    ez = np.exp(zg - zmax)
+    p = ez / ez.sum(axis=-1, keepdims=True)
+
+    # a3: top-k on the logits; a stable sort of -z keeps equal logits in index
+    # order, so ties go to the lower j. Selected indices stored ascending.
+    order = np.argsort(-zg, axis=-1, kind="stable")[..., :k]
+    idx = np.sort(order, axis=-1).astype(np.int32)
+
+    # a4: renormalised weights.
+    psel = np.take_along_axis(p, idx.astype(np.int64), axis=-1)
+    r = psel / psel.sum(axis=-1, keepdims=True)
+    omega = psel / psel.sum(axis=(1, 2), keepdims=True)
+    return {"z": z, "p": p, "idx": idx, "r": r, "omega": omega}
+
+
+# --------------------------------------------------------------------------
+# a5: dispatch (token lists per expert)
+# --------------------------------------------------------------------------
+
+def dispatch(idx: np.ndarray, B: int, T: int, G: int, M: int):
+    """Token lists per (expert, batch element).
+
+    counts[e, b]   number of tokens of sequence b that selected expert e;
+    offsets[e*B+b] exclusive prefix sum of counts in (e, b) order, with
+                   offsets[N*B] the total (= k*G*B*T);
+    tok[...]       for each (e, b), the positions t (0..T-1) that selected e,
+                   ascending;
+    slot_pos[row, g, s] the index in ``tok`` of the entry for that selection.
+    """
+    R, G_, k = idx.shape
+    assert G_ == G and R == B * T
+    N = G * M
+    counts = np.zeros((N, B), dtype=np.int64)
+    lists = [[[] for _ in range(B)] for _ in range(N)]
+    for row in range(R):
+        b, t = divmod(row, T)
+        for g in range(G):
+            for s in range(k):
+                e = g * M + int(idx[row, g, s])
+                lists[e][b].append(t)
+                counts[e, b] += 1
+    offsets = np.zeros(N * B + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts.reshape(-1))
+    tok = np.zeros(int(offsets[-1]), dtype=np.int32)
+    slot_pos = np.zeros((R, G, k), dtype=np.int32)
+    where = {}
+    for e in range(N):
+        for b in range(B):
+            base = int(offsets[e * B + b])
+            for i, t in enumerate(lists[e][b]):
+                tok[base + i] = t
+                where[(e, b, t)] = base + i
+    for row in range(R):
+        b, t = divmod(row, T)
+        for g in range(G):
+            for s in range(k):
+                e = g * M + int(idx[row, g, s])
+                slot_pos[row, g, s] = where[(e, b, t)]
+    return {"counts": counts.astype(np.int32), "offsets": offsets.astype(np.int32),
+            "tok": tok, "slot_pos": slot_pos}
+
+
+# --------------------------------------------------------------------------
+# a6-a7: projections
+# --------------------------------------------------------------------------
+
+def kv_proj(x: np.ndarray, W: np.ndarray, B: int, T: int, G: int, dh: int) -> np.ndarray:
+    """Dense K (or V) of every group: out[b, g, t, :] = x[b*T+t] @ W[:, g*dh:(g+1)*dh].
+
+    The K/V path is the GQA one, dense and unchanged (gist.science summary,
+    "Dense KV path"; pptc.cn blog, section 5).
+    """
+    y = np.asarray(x, np.float64) @ np.asarray(W, np.float64)  # [R, G*dh]
+    return y.reshape(B, T, G, dh).transpose(0, 2, 1, 3).copy()
+
+
+def q_routed(x: np.ndarray, W_q: np.ndarray, idx: np.ndarray, B: int, T: int, G: int,
+             M: int, dh: int) -> np.ndarray:
+    """Query of every selected expert only, slot-major: Qv[b, g, s, t, :].
+
+    Expert e = g*M + idx[row, g, s] computes q = x[row] @ W_q[:, e*dh:(e+1)*dh]
+    for the rows that selected it, and no other rows (conditional query
+    computation: chatpaper / hotpaper abstract).
+    """
+    x = np.asarray(x, np.float64)
+    W_q = np.asarray(W_q, np.float64)
+    R, _, k = idx.shape
+    Qv = np.zeros((B, G, k, T, dh))
+    rows = np.arange(R)
+    for g in range(G):
+        for j in range(M):
+            e = g * M + j
+            We = W_q[:, e * dh:(e + 1) * dh]
+            for s in range(k):
+                sel = rows[idx[:, g, s] == j]
+                if sel.size == 0:
+                    continue
+                q = x[sel] @ We
+                Qv[sel // T, g, s, sel % T, :] = q
+    return Qv
+
+
+def q_shared(x: np.ndarray, W_qs: np.ndarray, B: int, T: int, dh: int) -> np.ndarray:
+    """Always-on shared head query for every token: Qs[b, t, :] (readings R1, R2)."""
+    return (np.asarray(x, np.float64) @ np.asarray(W_qs, np.float64)).reshape(B, T, dh)
+
+
+# --------------------------------------------------------------------------
+# a8-a9: causal attention
+# --------------------------------------------------------------------------
+
+def causal_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, rows=None,
+                     block: int = 512) -> np.ndarray:
+    """o[t] = sum_{u <= t} softmax_u(q[t] . K[u] / sqrt(dh)) V[u] for one head.
+
+    ``q`` holds the queries of the rows ``rows`` (positions in the sequence;
+    all positions 0..len(q)-1 when None). Each row is evaluated on its own
+    from the definition; ``block`` only groups rows to bound memory.
+    """
+    q = np.asarray(q, np.float64)
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    n, dh = q.shape
+    pos = np.arange(n) if rows is None else np.asarray(rows, np.int64)
+    scale = 1.0 / math.sqrt(dh)
+    out = np.empty((n, V.shape[1]))
+    for s in range(0, n, block):
+        ps = pos[s:s + block]
+        hi = int(ps.max()) + 1
+        sc = (q[s:s + block] @ K[:hi].T) * scale          # [rows, hi]
+        mask = np.arange(hi)[None, :] > ps[:, None]
+        sc[mask] = -np.inf
+        sc -= sc.max(axis=1, keepdims=True)
+        w = np.exp(sc)
+        w /= w.sum(axis=1, keepdims=True)
+        out[s:s + block] = w @ V[:hi]
+    return out
+
+
+# --------------------------------------------------------------------------
+# a10-a11: slots and W_O
+# --------------------------------------------------------------------------
+
+def assemble_slots(o_routed: np.ndarray, o_shared: np.ndarray, omega: np.ndarray) -> np.ndarray:
+    """(kG+2) slots per token: [o_{g,s} for g, s] + [o_shared] + [sum w*o].
+
+    o_routed [R, G, k, dh], o_shared [R, dh], omega [R, G, k] -> [R, (kG+2)*dh].
+    """
+    R, G, k, dh = o_routed.shape
+    weighted = np.einsum("rgs,rgsd->rd", omega, o_routed)
+    return np.concatenate([o_routed.reshape(R, G * k * dh), o_shared, weighted], axis=1)
+
+
+def output_proj(slots: np.ndarray, W_o: np.ndarray) -> np.ndarray:
+    """y = slots @ W_O with W_O of shape [(kG+2)*dh, d] (reading R9)."""
+    return np.asarray(slots, np.float64) @ np.asarray(W_o, np.float64)
+
+
+# --------------------------------------------------------------------------
+# whole layers
+# --------------------------------------------------------------------------
+
+def _f64_inputs(inp: LayerInputs):
+    return {
+        "x": bf16_to_f64(inp.x),
+        "W_r": inp.W_r.astype(np.float64),
+        "b_r": None if inp.b_r is None else inp.b_r.astype(np.float64),
+        "W_q": bf16_to_f64(inp.W_q),
+        "W_qs": bf16_to_f64(inp.W_qs),
+        "W_k": bf16_to_f64(inp.W_k),
+        "W_v": bf16_to_f64(inp.W_v),
+        "W_o": bf16_to_f64(inp.W_o),
+        "W_o_dense": bf16_to_f64(inp.W_o_dense),
+    }
+
+
+def gqe_layer(inp: LayerInputs, rows=None, with_dispatch: bool = True) -> dict:
+    """GQE prefill forward (a1-a11).
+
+    ``rows`` (optional) is a list of global row indices b*T+t at which the
+    attention, slots and y are evaluated; router, dispatch, K and V are always
+    computed in full. Without ``rows`` every output is computed in full.
+    """
+    s: LayerShape = inp.shape
+    B, T, G, M, k, dh = s.B, s.T, s.G, s.M, s.k, s.d_head
+    f = _f64_inputs(inp)
+    rt = router(f["x"], f["W_r"], f["b_r"], G, M, k)
+    out = dict(rt)
+    if with_dispatch:
+        out.update(dispatch(rt["idx"], B, T, G, M))
+    K = kv_proj(f["x"], f["W_k"], B, T, G, dh)
+    V = kv_proj(f["x"], f["W_v"], B, T, G, dh)
+    out["K"], out["V"] = K, V
+    idx = rt["idx"]
+    R = B * T
+    sel_rows = np.arange(R) if rows is None else np.asarray(rows, np.int64)
+
+    # Queries (only for the evaluated rows when sampling; same definition).
+    x_sel = f["x"][sel_rows]
+    idx_sel = idx[sel_rows]
+    n = sel_rows.size
+    q_r = np.zeros((n, G, k, dh))
+    for g in range(G):
+        for j in range(M):
+            e = g * M + j
+            We = f["W_q"][:, e * dh:(e + 1) * dh]
+            for si in range(k):
+                m = idx_sel[:, g, si] == j
+                if m.any():
+                    q_r[m, g, si] = x_sel[m] @ We
+    q_s = x_sel @ f["W_qs"]
+    if rows is None:
+        out["Qv"] = q_r.reshape(B, T, G, k, dh).transpose(0, 2, 3, 1, 4).copy()
+        out["Qs"] = q_s.reshape(B, T, dh)
+
+    o_r = np.zeros((n, G, k, dh))
+    o_s = np.zeros((n, dh))
+    for b in range(B):
+        m = (sel_rows // T) == b
+        if not m.any():
+            continue
+        pos = sel_rows[m] % T
+        for g in range(G):
+            for si in range(k):
+                o_r[m, g, si] = causal_attention(q_r[m, g, si], K[b, g], V[b, g], rows=pos)
+        o_s[m] = causal_attention(q_s[m], K[b, 0], V[b, 0], rows=pos)
+    slots = assemble_slots(o_r, o_s, rt["omega"][sel_rows])
+    out["slots"] = slots
+    out["y"] = output_proj(slots, f["W_o"])
+    out["rows"] = sel_rows
+    return out
+
+
+def gqa_dense_layer(inp: LayerInputs, rows=None) -> dict:
+    """Dense GQA layer with every one of the N = G*M query heads active.
+
+    Head h uses KV group h // M; its output fills slot h of [R, N*dh], and
+    y = O @ W_O_dense with W_O_dense [N*dh, d]. This is the all-active
+    baseline the speed-up is measured against (gist.science summary,
+    "Experimental Results"; pptc.cn blog Table 1 first row).
+    """
+    s: LayerShape = inp.shape
+    B, T, G, M, dh = s.B, s.T, s.G, s.M, s.d_head
+    N = G * M
+    f = _f64_inputs(inp)
+    K = kv_proj(f["x"], f["W_k"], B, T, G, dh)
+    V = kv_proj(f["x"], f["W_v"], B, T, G, dh)
+    R = B * T
+    sel_rows = np.arange(R) if rows is None else np.asarray(rows, np.int64)
+    x_sel = f["x"][sel_rows]
+    n = sel_rows.size
+    O = np.zeros((n, N, dh))
+    Q = x_sel @ f["W_q"]  # [n, N*dh]
+    for b in range(B):
+        m = (sel_rows // T) == b
+        if not m.any():
+            continue
+        pos = sel_rows[m] % T
+        for h in range(N):
+            O[m, h] = causal_attention(Q[m][:, h * dh:(h + 1) * dh], K[b, h // M], V[b, h // M],
+                                       rows=pos)
+    O = O.reshape(n, N * dh)
+    out = {"K": K, "V": V, "O": O, "y": O @ f["W_o_dense"], "rows": sel_rows}
+    if rows is None:
+        out["Q"] = Q.reshape(B, T, N, dh).transpose(0, 2, 1, 3).copy()
+    return out
+
+
+def active_query_heads(shape: LayerShape) -> int:
+    """Query heads that run attention per token: k per group plus the shared head."""
+    return shape.k * shape.G + 1
