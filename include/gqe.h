@@ -1,0 +1,218 @@
+/*
+ * gqe.h - C ABI of libgqe.so: the prefill forward of one Grouped Query
+ * Experts (GQE) self-attention layer on an NVIDIA B200 (sm_100a), plus the
+ * dense GQA layer it is compared against.
+ *
+ * The method ("Grouped Query Experts: Mixture-of-Experts on GQA
+ * Self-Attention", arXiv:2606.20945, as summarised by the gist.science
+ * "Technical Summary", the pptc.cn blog and the hotpaper.ai summary):
+ * the N = G*M query heads of a GQA layer are split into G fixed groups of M
+ * "experts" (the heads sharing one KV head). Per token, a router takes a
+ * softmax over each group's M logits and keeps the top k experts of every
+ * group; only those experts, plus one always-on shared head, compute a query
+ * and run causal attention against their group's dense, unchanged K/V. The
+ * outputs fill kG+2 slots (kG routed, the shared head, one renormalised
+ * weighted sum of the routed outputs) that feed W_O of size (kG+2) x d.
+ *
+ * Conventions for every call
+ *  - All tensor pointers are DEVICE pointers, allocated and owned by the
+ *    caller, 16-byte aligned, densely packed row-major in the layout given.
+ *    The library never allocates device memory; scratch comes from the
+ *    caller's workspace (size from gqe_workspace_bytes).
+ *  - gqe_bf16 is a bf16 bit pattern; float is IEEE fp32.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream). Host-side validation errors return at once and launch
+ *    nothing. Device-side failures (a bounded wait that ran out) are recorded
+ *    in a per-device status word read by gqe_read_status.
+ *  - Inputs are never written, except `slots` in gqe_output_proj (the
+ *    weighted slot is filled in place).
+ *  - Index conventions: row = b*T + t; expert e = g*M + j (j = 0..M-1 inside
+ *    group g); routed slot (g, s) holds the s-th selected expert of group g
+ *    in ascending j; the shared head attends to KV group 0; ties in the
+ *    top-k go to the lower j. Dense head h uses KV group h / M.
+ */
+#ifndef GQE_H_
+#define GQE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t gqe_bf16;   /* bf16 bit pattern */
+typedef void* gqe_stream_t;  /* cudaStream_t */
+
+typedef struct gqe_config {
+  int32_t B;       /* sequences (batch) */
+  int32_t T;       /* tokens per sequence (prefill length), >= 1 */
+  int32_t d_model; /* model width, a multiple of 64 */
+  int32_t G;       /* KV groups = KV heads */
+  int32_t M;       /* query-head experts per group; N = G*M <= 64 */
+  int32_t k;       /* experts selected per group per token, 1 <= k <= M */
+  int32_t d_head;  /* head dim: 32 or 64 */
+  uint32_t flags;  /* reserved, must be 0 */
+} gqe_config;
+
+typedef enum gqe_status {
+  GQE_OK = 0,
+  GQE_ERR_INVALID = 1,      /* bad shape, k > M, null or misaligned pointer */
+  GQE_ERR_UNSUPPORTED = 2,  /* valid but not built (e.g. d_head not 32/64) */
+  GQE_ERR_WORKSPACE = 3,    /* workspace smaller than gqe_workspace_bytes */
+  GQE_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  GQE_ERR_TIMEOUT = 5,      /* a device-side bounded wait ran out */
+  GQE_ERR_DEVICE_CHECK = 6  /* a device-side consistency check failed */
+} gqe_status;
+
+/* Workspace kinds for gqe_workspace_bytes / gqe_workspace_offset. */
+enum {
+  GQE_WS_DISPATCH = 1, /* scratch of gqe_dispatch */
+  GQE_WS_LAYER = 2,    /* everything gqe_layer_fwd keeps between its steps */
+  GQE_WS_DENSE = 3     /* everything gqa_dense_fwd keeps between its steps */
+};
+
+/* Items inside the GQE_WS_LAYER / GQE_WS_DENSE workspaces (for inspection). */
+enum {
+  GQE_ITEM_IDX = 1, GQE_ITEM_R, GQE_ITEM_OMEGA, GQE_ITEM_COUNTS, GQE_ITEM_OFFSETS,
+  GQE_ITEM_TOK, GQE_ITEM_SLOT_POS, GQE_ITEM_QV, GQE_ITEM_QS, GQE_ITEM_K, GQE_ITEM_V,
+  GQE_ITEM_SLOTS, GQE_ITEM_DISPATCH_WS,
+  GQE_ITEM_DENSE_Q = 32, GQE_ITEM_DENSE_O
+};
+
+/* Bytes of workspace the given call needs for `cfg` (0 if cfg is invalid). */
+size_t gqe_workspace_bytes(const gqe_config* cfg, int which);
+
+/* Byte offset of `item` inside workspace `which`, or (size_t)-1. */
+size_t gqe_workspace_offset(const gqe_config* cfg, int which, int item);
+
+/*
+ * Router: logits, per-group softmax, top-k per group, renormalised weights
+ * (steps a1-a4). Router scores over the query-head experts and selection of
+ * k experts inside every group: gist.science "Technical Summary", Methodology
+ * ("Conditional activation"); softmax before top-k inside each group: pptc.cn
+ * blog section 7; every group takes part: pptc.cn blog section 5.
+ *
+ *   z[row, e]  = sum_i x[row, i] * W_r[i, e] + b_r[e]      (fp32, with a
+ *                certified error bound; a top-k decision whose margin is
+ *                below the bound is re-taken from fp64 logits, so idx is the
+ *                exact-arithmetic selection)
+ *   p          = softmax over the M logits of each group
+ *   idx[row, g, s] = the k largest j of group g, ascending, ties to lower j
+ *   r[row, g, s]     = p / sum of the selected p of group g
+ *   omega[row, g, s] = p / sum of the selected p of all G groups
+ *
+ * x [B*T, d_model] bf16; W_r [d_model, N] fp32; b_r [N] fp32 or NULL;
+ * idx [B*T, G, k] int32; r, omega [B*T, G, k] fp32.
+ */
+gqe_status gqe_router_topk(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
+                           const float* b_r, int32_t* idx, float* r, float* omega,
+                           gqe_stream_t stream);
+
+/*
+ * Dispatch (step a5) and the grouped query projection over the active rows
+ * only (step a7): only the selected experts compute a query ("reduces only
+ * the active query-head computation": chatpaper / hotpaper abstract).
+ *
+ *   counts[e*B + b]  tokens of sequence b that selected expert e
+ *   offsets[e*B + b] exclusive prefix sum of counts in (e, b) order;
+ *                    offsets[N*B] = k*G*B*T
+ *   tok[offsets[e*B+b] + i] = i-th smallest position t of sequence b that
+ *                    selected e (stable, bit-exact)
+ *   slot_pos[row, g, s] = index in tok of the entry of that selection
+ *   Qv[b, g, s, t, :] = x[row] @ W_q[:, e*dh:(e+1)*dh] for e = g*M + idx[row,g,s]
+ *   Qs[b, t, :]       = x[row] @ W_qs   (the always-on shared head)
+ *
+ * idx [B*T, G, k] int32 (from gqe_router_topk); x [B*T, d_model];
+ * W_q [d_model, N*d_head]; W_qs [d_model, d_head]; counts [N*B];
+ * offsets [N*B + 1]; tok [k*G*B*T]; slot_pos [B*T, G, k];
+ * Qv [B, G, k, T, d_head]; Qs [B, T, d_head].
+ * ws: >= gqe_workspace_bytes(cfg, GQE_WS_DISPATCH) bytes.
+ */
+gqe_status gqe_dispatch(const gqe_config* cfg, const int32_t* idx, const gqe_bf16* x,
+                        const gqe_bf16* W_q, const gqe_bf16* W_qs, int32_t* counts,
+                        int32_t* offsets, int32_t* tok, int32_t* slot_pos, gqe_bf16* Qv,
+                        gqe_bf16* Qs, void* ws, size_t ws_bytes, gqe_stream_t stream);
+
+/*
+ * Dense, unchanged K/V projection of every group (step a6; "the Key-Value
+ * projections and the KV cache stay dense and unchanged": gist.science
+ * "Technical Summary", Dense KV path). The dense GQA path uses this same call.
+ *   K[b, g, t, :] = x[row] @ W_k[:, g*dh:(g+1)*dh], V likewise with W_v.
+ * x [B*T, d_model]; W_k, W_v [d_model, G*d_head]; K, V [B, G, T, d_head].
+ */
+gqe_status gqe_kv_proj(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16* W_k,
+                       const gqe_bf16* W_v, gqe_bf16* K, gqe_bf16* V, gqe_stream_t stream);
+
+/*
+ * Routed and shared causal attention (steps a8, a9): every routed slot stream
+ * (g, s) attends causally to K/V of group g; the shared head to K/V of group
+ * 0. o[t] = sum_{u<=t} softmax_u(q[t].K[u] / sqrt(dh)) V[u], fp32 softmax and
+ * accumulation, bf16 output written straight into the slot buffer:
+ *   slots[row, (g*k+s)*dh ...] routed, slots[row, k*G*dh ...] shared.
+ * Slot kG+1 (weighted) is not touched.
+ * Qv [B, G, k, T, d_head]; Qs [B, T, d_head]; K, V [B, G, T, d_head];
+ * slots [B*T, (k*G+2)*d_head].
+ */
+gqe_status gqe_attention_fwd(const gqe_config* cfg, const gqe_bf16* Qv, const gqe_bf16* Qs,
+                             const gqe_bf16* K, const gqe_bf16* V, gqe_bf16* slots,
+                             gqe_stream_t stream);
+
+/*
+ * Weighted slot and output projection (steps a10, a11): the renormalised
+ * weighted sum of the selected experts' outputs ("Output Construction":
+ * gist.science "Technical Summary"), then y = slots @ W_O with W_O of size
+ * (kG+2) x d (hotpaper.ai summary, Technical approach).
+ *   slots[row, (kG+1)*dh ...] = sum_{g,s} omega[row,g,s] * slots[row, (g*k+s)*dh ...]
+ *   y = slots @ W_o
+ * slots [B*T, (k*G+2)*d_head] (updated in place); omega [B*T, G, k] fp32;
+ * W_o [(k*G+2)*d_head, d_model]; y [B*T, d_model].
+ */
+gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* omega,
+                           const gqe_bf16* W_o, gqe_bf16* y, gqe_stream_t stream);
+
+/*
+ * The whole GQE layer (a1-a11) on one stream; every intermediate lives in
+ * `ws` (>= gqe_workspace_bytes(cfg, GQE_WS_LAYER); see gqe_workspace_offset).
+ * Arguments as in the calls above.
+ */
+gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
+                         const float* b_r, const gqe_bf16* W_q, const gqe_bf16* W_qs,
+                         const gqe_bf16* W_k, const gqe_bf16* W_v, const gqe_bf16* W_o,
+                         gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream_t stream);
+
+/*
+ * Dense GQA layer with all N query heads active: the all-active baseline of
+ * the speed-up (gist.science "Technical Summary", Experimental Results;
+ * pptc.cn blog Table 1, first row). Q = x @ W_q [d_model, N*d_head]; K/V via
+ * gqe_kv_proj; head h attends to group h / M; O [B*T, N*d_head];
+ * y = O @ W_o_dense [N*d_head, d_model]. ws >= gqe_workspace_bytes(cfg,
+ * GQE_WS_DENSE). `k` of cfg is ignored.
+ */
+gqe_status gqa_dense_fwd(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16* W_q,
+                         const gqe_bf16* W_k, const gqe_bf16* W_v, const gqe_bf16* W_o_dense,
+                         gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream_t stream);
+
+/*
+ * Synchronises the current device, returns its status word in
+ * *device_status_out (a gqe_status value; 0 = no device-side failure since
+ * the last read) and clears it. Returns GQE_ERR_CUDA if the device cannot
+ * be synchronised.
+ */
+gqe_status gqe_read_status(int32_t* device_status_out);
+
+/* Launches one CTA that waits, with the given bound, on a barrier nothing
+ * completes; exercises the device-side timeout path (status GQE_ERR_TIMEOUT)
+ * without hanging the GPU. limit_ns must be in [1e3, 5e9]. */
+gqe_status gqe_selftest_wait_timeout(uint64_t limit_ns, gqe_stream_t stream);
+
+const char* gqe_status_string(gqe_status s);
+
+/* Library ABI version (major*100 + minor). */
+int gqe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQE_H_ */

@@ -1,0 +1,311 @@
+// C ABI of libgqe.so: argument validation, workspace layout and the order of
+// the kernel launches. Every call is asynchronous on the caller's stream and
+// launches nothing when validation fails.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "gqe_internal.h"
+#include "ptx.cuh"
+
+namespace gqe {
+
+namespace api_impl {
+
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <typename... P>
+bool all_aligned(const P*... ps) {
+  bool ok = true;
+  ((ok = ok && ps != nullptr && aligned16(ps)), ...);
+  return ok;
+}
+
+gqe_status check_cfg(const gqe_config* c) {
+  if (c == nullptr) return GQE_ERR_INVALID;
+  if (c->B < 1 || c->T < 1 || c->G < 1 || c->M < 1 || c->k < 1 || c->k > c->M) return GQE_ERR_INVALID;
+  if (c->d_model < 64 || c->d_model % 64 != 0 || c->flags != 0) return GQE_ERR_INVALID;
+  if (c->G * c->M > kMaxExperts || c->G > 32) return GQE_ERR_UNSUPPORTED;
+  if (c->d_head != 32 && c->d_head != 64) return GQE_ERR_UNSUPPORTED;
+  // Index arithmetic of the kernels stays within int32 for these extents.
+  const long long R = static_cast<long long>(c->B) * c->T;
+  const long long N = static_cast<long long>(c->G) * c->M;
+  if (R * c->d_model >= (1ll << 31) * 4 || R * (N + 2) * c->d_head >= (1ll << 31) ||
+      R * c->G * c->k * 4 >= (1ll << 31))
+    return GQE_ERR_UNSUPPORTED;
+  const int NP = router_np(static_cast<int>(N));
+  const size_t rsm = static_cast<size_t>(c->d_model) * router_row_floats(NP) * 4 + 2 * NP * 4 +
+                     8 * NP * 12;
+  if (rsm > kRouterSmemLimit) return GQE_ERR_UNSUPPORTED;
+  return GQE_OK;
+}
+
+gqe_status cuda_status(int e) { return e == cudaSuccess ? GQE_OK : GQE_ERR_CUDA; }
+
+struct LayerWs {
+  size_t idx, r, omega, counts, offsets, tok, slot_pos, Qv, Qs, K, V, slots, dws, total;
+};
+
+LayerWs layer_ws(const gqe_config& c) {
+  const size_t R = static_cast<size_t>(c.B) * c.T;
+  const size_t N = static_cast<size_t>(c.G) * c.M;
+  const size_t sel = R * c.G * c.k;
+  const size_t dh = c.d_head;
+  LayerWs L{};
+  size_t o = 0;
+  auto put = [&](size_t& field, size_t bytes) {
+    field = o;
+    o = round256(o + bytes);
+  };
+  put(L.idx, sel * 4);
+  put(L.r, sel * 4);
+  put(L.omega, sel * 4);
+  put(L.counts, N * c.B * 4);
+  put(L.offsets, (N * c.B + 1) * 4);
+  put(L.tok, sel * 4);
+  put(L.slot_pos, sel * 4);
+  put(L.Qv, sel * dh * 2);
+  put(L.Qs, R * dh * 2);
+  put(L.K, R * c.G * dh * 2);
+  put(L.V, R * c.G * dh * 2);
+  put(L.slots, R * (c.G * c.k + 2) * dh * 2);
+  put(L.dws, dispatch_ws_layout(c).total);
+  L.total = o;
+  return L;
+}
+
+struct DenseWs {
+  size_t Q, K, V, O, total;
+};
+
+DenseWs dense_ws(const gqe_config& c) {
+  const size_t R = static_cast<size_t>(c.B) * c.T;
+  const size_t N = static_cast<size_t>(c.G) * c.M;
+  const size_t dh = c.d_head;
+  DenseWs L{};
+  size_t o = 0;
+  auto put = [&](size_t& field, size_t bytes) {
+    field = o;
+    o = round256(o + bytes);
+  };
+  put(L.Q, R * N * dh * 2);
+  put(L.K, R * c.G * dh * 2);
+  put(L.V, R * c.G * dh * 2);
+  put(L.O, R * N * dh * 2);
+  L.total = o;
+  return L;
+}
+
+// One warp waits, with a bound, on a barrier that nothing completes: the
+// wait gives up after limit_ns and records GQE_ERR_TIMEOUT.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, limit_ns);
+  __syncwarp();
+}
+
+}  // namespace api_impl
+using namespace api_impl;
+
+}  // namespace gqe
+
+using namespace gqe;
+
+extern "C" {
+
+size_t gqe_workspace_bytes(const gqe_config* cfg, int which) {
+  if (check_cfg(cfg) != GQE_OK) return 0;
+  switch (which) {
+    case GQE_WS_DISPATCH: return dispatch_ws_layout(*cfg).total;
+    case GQE_WS_LAYER: return layer_ws(*cfg).total;
+    case GQE_WS_DENSE: return dense_ws(*cfg).total;
+    default: return 0;
+  }
+}
+
+size_t gqe_workspace_offset(const gqe_config* cfg, int which, int item) {
+  const size_t bad = static_cast<size_t>(-1);
+  if (check_cfg(cfg) != GQE_OK) return bad;
+  if (which == GQE_WS_LAYER) {
+    const LayerWs L = layer_ws(*cfg);
+    switch (item) {
+      case GQE_ITEM_IDX: return L.idx;
+      case GQE_ITEM_R: return L.r;
+      case GQE_ITEM_OMEGA: return L.omega;
+      case GQE_ITEM_COUNTS: return L.counts;
+      case GQE_ITEM_OFFSETS: return L.offsets;
+      case GQE_ITEM_TOK: return L.tok;
+      case GQE_ITEM_SLOT_POS: return L.slot_pos;
+      case GQE_ITEM_QV: return L.Qv;
+      case GQE_ITEM_QS: return L.Qs;
+      case GQE_ITEM_K: return L.K;
+      case GQE_ITEM_V: return L.V;
+      case GQE_ITEM_SLOTS: return L.slots;
+      case GQE_ITEM_DISPATCH_WS: return L.dws;
+      default: return bad;
+    }
+  }
+  if (which == GQE_WS_DENSE) {
+    const DenseWs L = dense_ws(*cfg);
+    switch (item) {
+      case GQE_ITEM_DENSE_Q: return L.Q;
+      case GQE_ITEM_K: return L.K;
+      case GQE_ITEM_V: return L.V;
+      case GQE_ITEM_DENSE_O: return L.O;
+      default: return bad;
+    }
+  }
+  return bad;
+}
+
+gqe_status gqe_router_topk(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
+                           const float* b_r, int32_t* idx, float* r, float* omega,
+                           gqe_stream_t stream) {
+  const gqe_status s = check_cfg(cfg);
+  if (s != GQE_OK) return s;
+  if (!all_aligned(x, W_r, idx, r, omega)) return GQE_ERR_INVALID;
+  if (b_r != nullptr && (reinterpret_cast<uintptr_t>(b_r) & 3u)) return GQE_ERR_INVALID;
+  return cuda_status(launch_router(*cfg, x, W_r, b_r, idx, r, omega, stream));
+}
+
+gqe_status gqe_dispatch(const gqe_config* cfg, const int32_t* idx, const gqe_bf16* x,
+                        const gqe_bf16* W_q, const gqe_bf16* W_qs, int32_t* counts,
+                        int32_t* offsets, int32_t* tok, int32_t* slot_pos, gqe_bf16* Qv,
+                        gqe_bf16* Qs, void* ws, size_t ws_bytes, gqe_stream_t stream) {
+  const gqe_status s = check_cfg(cfg);
+  if (s != GQE_OK) return s;
+  if (!all_aligned(idx, x, W_q, W_qs, counts, offsets, tok, slot_pos, Qv, Qs) || ws == nullptr ||
+      !aligned16(ws))
+    return GQE_ERR_INVALID;
+  const DispatchWs L = dispatch_ws_layout(*cfg);
+  if (ws_bytes < L.total) return GQE_ERR_WORKSPACE;
+  int e = launch_dispatch_lists(*cfg, idx, counts, offsets, tok, slot_pos, ws, L, stream);
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+  char* w = static_cast<char*>(ws);
+  e = gemm_q_routed(*cfg, x, W_q, idx, offsets, tok, w + L.qtiles,
+                    reinterpret_cast<const int32_t*>(w + L.n_qtiles), L.max_qtiles, Qv, stream);
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+  return cuda_status(gemm_q_shared(*cfg, x, W_qs, Qs, stream));
+}
+
+gqe_status gqe_kv_proj(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16* W_k,
+                       const gqe_bf16* W_v, gqe_bf16* K, gqe_bf16* V, gqe_stream_t stream) {
+  const gqe_status s = check_cfg(cfg);
+  if (s != GQE_OK) return s;
+  if (!all_aligned(x, W_k, W_v, K, V)) return GQE_ERR_INVALID;
+  return cuda_status(gemm_kv(*cfg, x, W_k, W_v, K, V, stream));
+}
+
+gqe_status gqe_attention_fwd(const gqe_config* cfg, const gqe_bf16* Qv, const gqe_bf16* Qs,
+                             const gqe_bf16* K, const gqe_bf16* V, gqe_bf16* slots,
+                             gqe_stream_t stream) {
+  const gqe_status s = check_cfg(cfg);
+  if (s != GQE_OK) return s;
+  if (!all_aligned(Qv, Qs, K, V, slots)) return GQE_ERR_INVALID;
+  return cuda_status(attention_gqe(*cfg, Qv, Qs, K, V, slots, stream));
+}
+
+gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* omega,
+                           const gqe_bf16* W_o, gqe_bf16* y, gqe_stream_t stream) {
+  const gqe_status s = check_cfg(cfg);
+  if (s != GQE_OK) return s;
+  if (!all_aligned(slots, omega, W_o, y)) return GQE_ERR_INVALID;
+  int e = launch_weighted_slot(*cfg, slots, omega, stream);
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+  const int R = cfg->B * cfg->T;
+  return cuda_status(gemm_rowmajor(slots, R, (cfg->G * cfg->k + 2) * cfg->d_head, W_o,
+                                   cfg->d_model, y, stream));
+}
+
+gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
+                         const float* b_r, const gqe_bf16* W_q, const gqe_bf16* W_qs,
+                         const gqe_bf16* W_k, const gqe_bf16* W_v, const gqe_bf16* W_o,
+                         gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream_t stream) {
+  const gqe_status s = check_cfg(cfg);
+  if (s != GQE_OK) return s;
+  if (!all_aligned(x, W_r, W_q, W_qs, W_k, W_v, W_o, y) || ws == nullptr || !aligned16(ws))
+    return GQE_ERR_INVALID;
+  const LayerWs L = layer_ws(*cfg);
+  if (ws_bytes < L.total) return GQE_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  auto I = [&](size_t o) { return reinterpret_cast<int32_t*>(w + o); };
+  auto F = [&](size_t o) { return reinterpret_cast<float*>(w + o); };
+  auto H = [&](size_t o) { return reinterpret_cast<gqe_bf16*>(w + o); };
+  gqe_status st = gqe_router_topk(cfg, x, W_r, b_r, I(L.idx), F(L.r), F(L.omega), stream);
+  if (st != GQE_OK) return st;
+  st = gqe_dispatch(cfg, I(L.idx), x, W_q, W_qs, I(L.counts), I(L.offsets), I(L.tok),
+                    I(L.slot_pos), H(L.Qv), H(L.Qs), w + L.dws, L.total - L.dws, stream);
+  if (st != GQE_OK) return st;
+  st = gqe_kv_proj(cfg, x, W_k, W_v, H(L.K), H(L.V), stream);
+  if (st != GQE_OK) return st;
+  st = gqe_attention_fwd(cfg, H(L.Qv), H(L.Qs), H(L.K), H(L.V), H(L.slots), stream);
+  if (st != GQE_OK) return st;
+  return gqe_output_proj(cfg, H(L.slots), F(L.omega), W_o, y, stream);
+}
+
+gqe_status gqa_dense_fwd(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16* W_q,
+                         const gqe_bf16* W_k, const gqe_bf16* W_v, const gqe_bf16* W_o_dense,
+                         gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream_t stream) {
+  if (cfg == nullptr) return GQE_ERR_INVALID;
+  gqe_config c = *cfg;
+  c.k = 1;  // not used by the dense layer
+  const gqe_status s = check_cfg(&c);
+  if (s != GQE_OK) return s;
+  if (!all_aligned(x, W_q, W_k, W_v, W_o_dense, y) || ws == nullptr || !aligned16(ws))
+    return GQE_ERR_INVALID;
+  const DenseWs L = dense_ws(c);
+  if (ws_bytes < L.total) return GQE_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  auto H = [&](size_t o) { return reinterpret_cast<gqe_bf16*>(w + o); };
+  int e = gemm_q_dense(c, x, W_q, H(L.Q), stream);
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+  e = gemm_kv(c, x, W_k, W_v, H(L.K), H(L.V), stream);
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+  e = attention_dense(c, H(L.Q), H(L.K), H(L.V), H(L.O), stream);
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+  const int N = c.G * c.M;
+  return cuda_status(gemm_rowmajor(H(L.O), c.B * c.T, N * c.d_head, W_o_dense, c.d_model, y, stream));
+}
+
+gqe_status gqe_read_status(int32_t* device_status_out) {
+  if (device_status_out == nullptr) return GQE_ERR_INVALID;
+  if (cudaDeviceSynchronize() != cudaSuccess) return GQE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return GQE_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return GQE_ERR_CUDA;
+  *device_status_out = v;
+  return GQE_OK;
+}
+
+gqe_status gqe_selftest_wait_timeout(uint64_t limit_ns, gqe_stream_t stream) {
+  if (limit_ns < 1000ull || limit_ns > 5000000000ull) return GQE_ERR_INVALID;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return cuda_status(cudaGetLastError());
+}
+
+const char* gqe_status_string(gqe_status s) {
+  switch (s) {
+    case GQE_OK: return "ok";
+    case GQE_ERR_INVALID: return "invalid argument";
+    case GQE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case GQE_ERR_WORKSPACE: return "workspace too small";
+    case GQE_ERR_CUDA: return "CUDA error";
+    case GQE_ERR_TIMEOUT: return "device-side wait timed out";
+    case GQE_ERR_DEVICE_CHECK: return "device-side check failed";
+    default: return "unknown status";
+  }
+}
+
+int gqe_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,376 @@
+// Causal flash attention on tcgen05 for the routed and shared heads of the
+// GQE layer (steps a8, a9) and for the dense GQA comparison layer.
+//
+// Every routed slot stream (b, g, s) is a dense, position-ordered stream of T
+// query rows (each token selects exactly k experts of every group), so it is
+// plain causal attention of T queries against the group's K/V; the shared
+// head is one more stream against group 0. Only the selected experts' queries
+// exist, so the work is (kG+1)/N of the dense layer ("GQE keeps the KV cache
+// benefits of GQA and reduces only the active query-head computation":
+// chatpaper / hotpaper abstract; 9 of 16 heads active: gist.science Technical
+// Summary, Experimental Results).
+//
+// One CTA = one 128-row query tile of one stream; KV tiles of 128 keys up to
+// the diagonal (fully masked tiles are never loaded). Warp roles (192
+// threads):
+//   warps 0-3  softmax: thread i owns query row i (TMEM lane i); online
+//              softmax in fp32 (exp2 with the 1/sqrt(dh)*log2(e) scale folded
+//              in), P written to shared memory as bf16 in the UMMA K-major
+//              128B-swizzled layout, O rescaled in TMEM, final O / l stored;
+//   warp 4     TMA loads of Q and of K/V tiles (3-stage ring);
+//   warp 5     one thread issues S = Q K^T into one of two TMEM S buffers
+//              (S_{j+1} overlaps the softmax of S_j) and O += P V.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+dh).
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "gqe_internal.h"
+#include "ptx.cuh"
+#include "tmap.h"
+
+namespace gqe {
+
+namespace attn_impl {
+
+constexpr int BQ = 128;
+constexpr int BKV = 128;
+constexpr int KV_STAGES = 3;
+
+template <int DH>
+struct AttnCfg {
+  static constexpr int SWB = DH * 2;  // bytes per Q/K/V row = swizzle width
+  static constexpr uint32_t LAYOUT = SWB == 128 ? kLayoutSW128 : kLayoutSW64;
+  static constexpr int TILE_BYTES = BQ * DH * 2;
+  static constexpr int P_BYTES = BQ * BKV * 2;
+  static constexpr size_t SMEM =
+      1024 + static_cast<size_t>(TILE_BYTES) * (1 + 2 * KV_STAGES) + 2 * P_BYTES + 256;
+  static constexpr uint32_t TMEM_COLS = 512;
+};
+
+struct AttnParams {
+  int T, B, H;       // tokens per sequence, sequences, query streams per sequence
+  int G, k, M;       // groups, selected per group, experts per group
+  int dense;         // 0: GQE streams (kG routed + shared), 1: dense GQA heads
+  int n_qt;          // query tiles per stream
+  uint16_t* out;     // [B*T, ldo]
+  int ldo;
+  float scale_log2;  // log2(e) / sqrt(dh)
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int DH>
+__global__ void __launch_bounds__(192, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQs,
+                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                const AttnParams p) {
+  using C = AttnCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* sp = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sQ = sp;
+  uint8_t* sK = sQ + C::TILE_BYTES;
+  uint8_t* sV = sK + KV_STAGES * C::TILE_BYTES;
+  uint8_t* sP = sV + KV_STAGES * C::TILE_BYTES;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sP + 2 * C::P_BYTES);
+  uint64_t* q_full = bar;
+  uint64_t* k_full = bar + 1;
+  uint64_t* v_full = k_full + KV_STAGES;
+  uint64_t* kv_empty = v_full + KV_STAGES;
+  uint64_t* s_full = kv_empty + KV_STAGES;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* drain = o_done + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = p.B * p.H;
+  const int qt = p.n_qt - 1 - static_cast<int>(blockIdx.x) / BH;  // longest tiles first
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int b = bh / p.H, h = bh % p.H;
+  int zq, grp, slot;
+  const CUtensorMap* tq = &tmQ;
+  if (p.dense) {
+    zq = b * p.H + h;
+    grp = h / p.M;
+    slot = h;
+  } else if (h < p.G * p.k) {
+    zq = b * p.G * p.k + h;
+    grp = h / p.k;
+    slot = h;
+  } else {
+    zq = b;
+    grp = 0;
+    slot = p.G * p.k;
+    tq = &tmQs;
+  }
+  const int zkv = b * p.G + grp;
+  const int nkv = qt + 1;  // causal: KV tiles 0..qt
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < KV_STAGES; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(tq);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 5) tmem_alloc(tslot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t tO = tmem + 256;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
+      tma_load_3d(sQ, tq, q_full, 0, qt * BQ, zq);
+      for (int j = 0; j < nkv; ++j) {
+        const int st = j % KV_STAGES;
+        const uint32_t ph = (j / KV_STAGES) & 1;
+        if (!mbar_wait(&kv_empty[st], ph ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(&k_full[st], C::TILE_BYTES);
+        tma_load_3d(sK + st * C::TILE_BYTES, &tmK, &k_full[st], 0, j * BKV, zkv);
+        mbar_arrive_expect_tx(&v_full[st], C::TILE_BYTES);
+        tma_load_3d(sV + st * C::TILE_BYTES, &tmV, &v_full[st], 0, j * BKV, zkv);
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------- UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(BQ, BKV, 0, 0);
+      constexpr uint32_t idO = idesc_bf16_f32(BQ, DH, 0, 1);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+          umma_bf16_ss(tmem, smem_desc(aQ + kk * 32, 16, 8 * C::SWB, C::LAYOUT),
+                       smem_desc(aK + kk * 32, 16, 8 * C::SWB, C::LAYOUT), idS, kk > 0 ? 1u : 0u);
+        umma_commit(&s_full[0]);
+      }
+      for (int j = 0; ok && j < nkv; ++j) {
+        if (j + 1 < nkv) {
+          const int st = (j + 1) % KV_STAGES;
+          if (!mbar_wait(&k_full[st], ((j + 1) / KV_STAGES) & 1, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t tS = tmem + ((j + 1) & 1) * 128;
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk)
+            umma_bf16_ss(tS, smem_desc(aQ + kk * 32, 16, 8 * C::SWB, C::LAYOUT),
+                         smem_desc(aK + st * C::TILE_BYTES + kk * 32, 16, 8 * C::SWB, C::LAYOUT),
+                         idS, kk > 0 ? 1u : 0u);
+          umma_commit(&s_full[(j + 1) & 1]);
+        }
+        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag)) break;
+        const int st = j % KV_STAGES;
+        if (!mbar_wait(&v_full[st], (j / KV_STAGES) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t pb = aP + (j & 1) * C::P_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          umma_bf16_ss(tO,
+                       smem_desc(pb + (kk >> 2) * (BQ * 128) + (kk & 3) * 32, 16, 1024,
+                                 kLayoutSW128),
+                       smem_desc(aV + st * C::TILE_BYTES + kk * 16 * C::SWB, C::TILE_BYTES,
+                                 8 * C::SWB, C::LAYOUT),
+                       idO, (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&kv_empty[st]);
+        umma_commit(o_done);
+      }
+      umma_commit(drain);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- softmax
+    const int i = threadIdx.x;  // row in tile, TMEM lane
+    const int qi = qt * BQ + i;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float sc = p.scale_log2;
+    float m = -INFINITY, l = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      // Waits are made warp-uniform: tcgen05.ld/st below are .sync.aligned.
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[BKV];
+      const uint32_t tS = tmem + lane_off + (j & 1) * 128;
+#pragma unroll
+      for (int c = 0; c < BKV / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + c * 32, v);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(v[x]);
+      }
+      if (j == nkv - 1) {  // diagonal tile: key kj visible iff kj <= qi
+        const int lim = qi - j * BKV;
+#pragma unroll
+        for (int x = 0; x < BKV; ++x)
+          if (x > lim) s[x] = -INFINITY;
+      }
+      float mt = s[0];
+#pragma unroll
+      for (int x = 1; x < BKV; ++x) mt = fmaxf(mt, s[x]);
+      const float m_new = fmaxf(m, mt * sc);
+      if (j > 0) {
+        // O holds PV_{j-1}; rescale it before PV_j is issued.
+        if (!__all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float alpha = ex2(m - m_new);
+        l *= alpha;
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+          for (int c = 0; c < DH / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tO + lane_off + c * 32, v);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
+            tmem_st32(tO + lane_off + c * 32, v);
+          }
+          tmem_st_wait();
+        }
+      }
+      m = m_new;
+      const float neg_m = -m_new;
+      uint8_t* prow = sP + (j & 1) * C::P_BYTES + i * 128;
+#pragma unroll
+      for (int c16 = 0; c16 < BKV / 8; ++c16) {
+        float e8[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          e8[x] = ex2(fmaf(s[c16 * 8 + x], sc, neg_m));
+          l += e8[x];
+        }
+        uint4 o;
+        o.x = pack_bf16x2(e8[0], e8[1]);
+        o.y = pack_bf16x2(e8[2], e8[3]);
+        o.z = pack_bf16x2(e8[4], e8[5]);
+        o.w = pack_bf16x2(e8[6], e8[7]);
+        const int kc = c16 >> 3, cw = c16 & 7;
+        *reinterpret_cast<uint4*>(prow + kc * (BQ * 128) + ((cw ^ (i & 7)) << 4)) = o;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[j & 1]);
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, (nkv - 1) & 1, abort_flag))) {
+      tc_fence_after();
+      const float inv = 1.0f / l;
+      uint16_t* dst = p.out + (static_cast<size_t>(b) * p.T + qi) * p.ldo + slot * DH;
+#pragma unroll
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tO + lane_off + c * 32, v);
+        if (qi < p.T) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv);
+            o.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv);
+            o.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv);
+            o.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv);
+            d4[q4] = o;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    volatile int none = 0;
+    mbar_wait(drain, 0, &none, 500000000ull);
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int DH>
+int launch_attn(const CUtensorMap& q, const CUtensorMap& qs, const CUtensorMap& k,
+                const CUtensorMap& v, const AttnParams& p, void* stream) {
+  using C = AttnCfg<DH>;
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::SMEM));
+  if (e != cudaSuccess) return e;
+  const long long grid = static_cast<long long>(p.n_qt) * p.B * p.H;
+  if (grid <= 0) return cudaSuccess;
+  attn_kernel<DH><<<static_cast<unsigned>(grid), 192, C::SMEM, static_cast<cudaStream_t>(stream)>>>(
+      q, qs, k, v, p);
+  return cudaGetLastError();
+}
+
+int run(const gqe_config& c, const uint16_t* Q, uint64_t nq_streams, const uint16_t* Qs,
+        const uint16_t* K, const uint16_t* V, uint16_t* out, int ldo, int H, int dense,
+        void* stream) {
+  const int dh = c.d_head;
+  CUtensorMap tq, tqs, tk, tv;
+  if (!make_tmap_bf16_3d(&tq, Q, dh, c.T, nq_streams, dh, BQ)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_3d(&tqs, Qs ? Qs : Q, dh, c.T, Qs ? c.B : nq_streams, dh, BQ))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_3d(&tk, K, dh, c.T, static_cast<uint64_t>(c.B) * c.G, dh, BKV))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_3d(&tv, V, dh, c.T, static_cast<uint64_t>(c.B) * c.G, dh, BKV))
+    return cudaErrorInvalidValue;
+  AttnParams p;
+  p.T = c.T;
+  p.B = c.B;
+  p.H = H;
+  p.G = c.G;
+  p.k = c.k;
+  p.M = c.M;
+  p.dense = dense;
+  p.n_qt = (c.T + BQ - 1) / BQ;
+  p.out = out;
+  p.ldo = ldo;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(dh)));
+  if (dh == 64) return launch_attn<64>(tq, tqs, tk, tv, p, stream);
+  return launch_attn<32>(tq, tqs, tk, tv, p, stream);
+}
+
+}  // namespace attn_impl
+using namespace attn_impl;
+
+int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
+                  const uint16_t* V, uint16_t* slots, void* stream) {
+  const int H = c.G * c.k + 1;
+  return run(c, Qv, static_cast<uint64_t>(c.B) * c.G * c.k, Qs, K, V, slots,
+             (c.G * c.k + 2) * c.d_head, H, 0, stream);
+}
+
+int attention_dense(const gqe_config& c, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                    uint16_t* O, void* stream) {
+  const int N = c.G * c.M;
+  return run(c, Q, static_cast<uint64_t>(c.B) * N, nullptr, K, V, O, N * c.d_head, N, 1, stream);
+}
+
+}  // namespace gqe

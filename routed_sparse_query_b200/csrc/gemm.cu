@@ -1,0 +1,379 @@
+// tcgen05 GEMM for the projections of the layer: C[128 x BN] tiles of
+// A[rows, K] (bf16, K contiguous) times B[K, N] (bf16, N contiguous), fp32
+// accumulation in tensor memory, bf16 output through a scatter epilogue.
+//
+//  - K/V projection (step a6) and the shared-head / dense query projections:
+//    A tiles come from TMA (128B swizzle), the epilogue writes head-split
+//    layouts [b][h][t][dh].
+//  - Routed query projection (step a7, "only the selected query experts"):
+//    one tile = up to 128 consecutive entries of one (expert, sequence) token
+//    list; the A rows are gathered by four warps with cp.async into the same
+//    swizzled layout TMA would produce, and the epilogue writes each row to its
+//    slot-major stream Qv[b][g][s][t][:].
+//  - W_O projection (step a11): plain row-major output.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 issues the UMMAs
+// (one thread) and owns the TMEM allocation, warps 2-5 gather A rows (routed
+// mode) and run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// B is read MN-major: 64-column (or 32-column) boxes, LBO = distance between
+// column boxes, SBO = 8 rows.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "gqe_internal.h"
+#include "ptx.cuh"
+#include "tmap.h"
+
+namespace gqe {
+
+namespace gemm_impl {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int B_ATOM = BN >= 64 ? 64 : BN;  // B columns per swizzle row
+  static constexpr int B_SWB = B_ATOM * 2;           // bytes per B swizzle row
+  static constexpr uint32_t B_LAYOUT = B_SWB == 128 ? kLayoutSW128 : kLayoutSW64;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BK * BN * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024 / STAGE_BYTES) > 8 ? 8 : (200 * 1024 / STAGE_BYTES);
+  static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;
+  static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 256;
+};
+
+struct Epi {
+  uint16_t* out;
+  long long sb, sh, st;  // element strides of sequence, head, token
+  int T;                 // rows per sequence
+  int hd;                // columns per head
+  int rows, cols;        // valid extent of C
+};
+
+struct Gather {
+  const uint16_t* x;
+  const int32_t* tok;
+  const int32_t* offsets;
+  const int4* qtiles;
+  const int32_t* n_qtiles;
+  const int32_t* idx;
+  uint16_t* Qv;
+  int d, T, G, M, k, B, dh;
+};
+
+__device__ __forceinline__ void store32_bf16(uint16_t* dst, const uint32_t (&v)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 o;
+    o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+    o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+    o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+    o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+    d4[q] = o;
+  }
+}
+
+template <int BN, bool GATHER>
+__global__ void __launch_bounds__(192, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                const __grid_constant__ CUtensorMap tmB1, const Epi epi0, const Epi epi1,
+                const Gather ga, const int K) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* sp = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sA = sp;
+  uint8_t* sB = sp + C::STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* accb = empty + C::STAGES;
+  uint64_t* drain = accb + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool z1 = blockIdx.z == 1;
+  const CUtensorMap* tmB = z1 ? &tmB1 : &tmB0;
+  const Epi& epi = z1 ? epi1 : epi0;
+
+  int m0 = 0, n0 = 0, e = 0, b = 0, list0 = 0, rows = 0;
+  if (GATHER) {
+    const int q = blockIdx.x;
+    if (q >= *ga.n_qtiles) return;  // uniform: this tile slot is unused
+    const int4 qt = ga.qtiles[q];
+    e = qt.x;
+    b = qt.y;
+    list0 = ga.offsets[e * ga.B + b] + qt.z;
+    rows = qt.w;
+    n0 = e * ga.dh;
+  } else {
+    m0 = blockIdx.x * BM;
+    n0 = blockIdx.y * BN;
+  }
+  const int nk = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], GATHER ? 129u : 1u);
+      mbar_init(&empty[s], 1u);
+    }
+    mbar_init(accb, 1u);
+    mbar_init(drain, 1u);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    if (!GATHER) prefetch_tmap(&tmA);
+    prefetch_tmap(tmB);
+  }
+  if (warp == 1) tmem_alloc(tslot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % C::STAGES;
+        const uint32_t ph = (kb / C::STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[s], (GATHER ? 0 : C::A_BYTES) + C::B_BYTES);
+        if (!GATHER) tma_load_2d(sA + s * C::A_BYTES, &tmA, &full[s], kb * BK, m0);
+#pragma unroll
+        for (int c = 0; c < BN / C::B_ATOM; ++c)
+          tma_load_2d(sB + s * C::B_BYTES + c * (BK * C::B_SWB), tmB, &full[s],
+                      n0 + c * C::B_ATOM, kb * BK);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 1);
+      const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % C::STAGES;
+        const uint32_t ph = (kb / C::STAGES) & 1;
+        if (!mbar_wait(&full[s], ph, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = smem_desc(a0 + s * C::A_BYTES + kk * 32, 16, 1024, kLayoutSW128);
+          const uint64_t bd = smem_desc(b0 + s * C::B_BYTES + kk * 16 * C::B_SWB, BK * C::B_SWB,
+                                        8 * C::B_SWB, C::B_LAYOUT);
+          umma_bf16_ss(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accb);
+      umma_commit(drain);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    if (GATHER) {
+      // Thread i gathers row i of the A tile (zeros past the list's end).
+      const int i = threadIdx.x - 64;
+      const bool valid = i < rows;
+      const int t = valid ? ga.tok[list0 + i] : 0;
+      const uint16_t* src = ga.x + (static_cast<size_t>(b) * ga.T + t) * ga.d;
+      const uint32_t a0 = smem_u32(sA);
+      constexpr int LA = C::STAGES - 1;
+      int kb = 0;
+      for (; kb < nk; ++kb) {
+        const int s = kb % C::STAGES;
+        const uint32_t ph = (kb / C::STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) break;
+        const uint32_t dst = a0 + s * C::A_BYTES + i * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          cp_async_16(dst + ((c ^ (i & 7)) << 4), src + kb * BK + c * 8, valid ? 16u : 0u);
+        cp_async_commit();
+        if (kb >= LA) {
+          cp_async_wait<LA>();
+          fence_proxy_async_smem();
+          mbar_arrive(&full[(kb - LA) % C::STAGES]);
+        }
+      }
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      for (int k2 = (kb - LA > 0 ? kb - LA : 0); k2 < kb; ++k2) mbar_arrive(&full[k2 % C::STAGES]);
+    }
+    const bool have = mbar_wait(accb, 0, abort_flag);
+    tc_fence_after();
+    const int r = q * 32 + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    if (GATHER) {
+      const bool valid = have && r < rows;
+      size_t obase = 0;
+      if (valid) {
+        const int t = ga.tok[list0 + r];
+        const int g = e / ga.M, j = e % ga.M;
+        const int32_t* ip = ga.idx + ((static_cast<size_t>(b) * ga.T + t) * ga.G + g) * ga.k;
+        int s = 0;
+        for (int s2 = 0; s2 < ga.k; ++s2)
+          if (ip[s2] == j) s = s2;
+        obase = (((static_cast<size_t>(b) * ga.G + g) * ga.k + s) * ga.T + t) * ga.dh;
+      }
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(trow + cc * 32, v);
+        if (valid) store32_bf16(ga.Qv + obase + cc * 32, v);
+      }
+    } else {
+      const int row = m0 + r;
+      const bool valid = have && row < epi.rows;
+      const int bb = row / epi.T, t = row % epi.T;
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(trow + cc * 32, v);
+        const int col0 = n0 + cc * 32;
+        if (valid && col0 < epi.cols) {
+          const int h = col0 / epi.hd, c = col0 % epi.hd;
+          store32_bf16(epi.out + bb * epi.sb + h * epi.sh + t * epi.st + c, v);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (*abort_flag) {
+      // Let every issued UMMA finish before the columns are released.
+      volatile int none = 0;
+      mbar_wait(drain, 0, &none, 500000000ull);
+    }
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BN, bool GATHER>
+int launch(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const Epi& e0,
+           const Epi& e1, const Gather& g, int K, dim3 grid, void* stream) {
+  using C = GemmCfg<BN>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, GATHER>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(C::SMEM));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  gemm_kernel<BN, GATHER><<<grid, 192, C::SMEM, static_cast<cudaStream_t>(stream)>>>(
+      A, B0, B1, e0, e1, g, K);
+  return cudaGetLastError();
+}
+
+// Dense GEMM with a head-split epilogue; chooses the tile width.
+int dense_gemm(const uint16_t* A, int rows, int K, const uint16_t* W0, const uint16_t* W1, int N,
+               const Epi& e0, const Epi& e1, int nz, void* stream) {
+  int BN = 256;
+  const long long mt = (rows + BM - 1) / BM;
+  if (N % 256 != 0 || mt * (N / 256) * nz < 148) BN = 128;
+  if (N % 128 != 0) BN = 64;
+  if (N % 64 != 0) BN = 32;
+  if (N % 32 != 0) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb0, tb1;
+  const int batom = BN >= 64 ? 64 : BN;
+  if (!make_tmap_bf16_2d(&ta, A, K, rows, K, 64, BM)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tb0, W0, N, K, N, batom, BK)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tb1, W1 ? W1 : W0, N, K, N, batom, BK)) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(mt), static_cast<unsigned>(N / BN), nz);
+  Gather g{};
+  switch (BN) {
+    case 256: return launch<256, false>(ta, tb0, tb1, e0, e1, g, K, grid, stream);
+    case 128: return launch<128, false>(ta, tb0, tb1, e0, e1, g, K, grid, stream);
+    case 64: return launch<64, false>(ta, tb0, tb1, e0, e1, g, K, grid, stream);
+    default: return launch<32, false>(ta, tb0, tb1, e0, e1, g, K, grid, stream);
+  }
+}
+
+Epi head_split(uint16_t* out, int T, int H, int dh, int R) {
+  Epi e;
+  e.out = out;
+  e.T = T;
+  e.hd = dh;
+  e.sb = static_cast<long long>(H) * T * dh;
+  e.sh = static_cast<long long>(T) * dh;
+  e.st = dh;
+  e.rows = R;
+  e.cols = H * dh;
+  return e;
+}
+
+}  // namespace gemm_impl
+using namespace gemm_impl;
+
+int gemm_kv(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
+            uint16_t* K, uint16_t* V, void* stream) {
+  const int R = c.B * c.T;
+  const Epi ek = head_split(K, c.T, c.G, c.d_head, R);
+  const Epi ev = head_split(V, c.T, c.G, c.d_head, R);
+  return dense_gemm(x, R, c.d_model, W_k, W_v, c.G * c.d_head, ek, ev, 2, stream);
+}
+
+int gemm_q_shared(const gqe_config& c, const uint16_t* x, const uint16_t* W_qs, uint16_t* Qs,
+                  void* stream) {
+  const int R = c.B * c.T;
+  const Epi e = head_split(Qs, c.T, 1, c.d_head, R);
+  return dense_gemm(x, R, c.d_model, W_qs, nullptr, c.d_head, e, e, 1, stream);
+}
+
+int gemm_q_dense(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, uint16_t* Q,
+                 void* stream) {
+  const int R = c.B * c.T;
+  const int N = c.G * c.M;
+  const Epi e = head_split(Q, c.T, N, c.d_head, R);
+  return dense_gemm(x, R, c.d_model, W_q, nullptr, N * c.d_head, e, e, 1, stream);
+}
+
+int gemm_rowmajor(const uint16_t* A, int rows, int K, const uint16_t* W, int N, uint16_t* out,
+                  void* stream) {
+  Epi e;
+  e.out = out;
+  e.T = rows;
+  e.hd = N;
+  e.sb = 0;
+  e.sh = 0;
+  e.st = N;
+  e.rows = rows;
+  e.cols = N;
+  return dense_gemm(A, rows, K, W, nullptr, N, e, e, 1, stream);
+}
+
+int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const int32_t* idx,
+                  const int32_t* offsets, const int32_t* tok, const void* qtiles,
+                  const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, void* stream) {
+  const int N = c.G * c.M;
+  const int dh = c.d_head;
+  CUtensorMap tb;
+  if (!make_tmap_bf16_2d(&tb, W_q, static_cast<uint64_t>(N) * dh, c.d_model,
+                         static_cast<uint64_t>(N) * dh, dh, BK))
+    return cudaErrorInvalidValue;
+  Gather g;
+  g.x = x;
+  g.tok = tok;
+  g.offsets = offsets;
+  g.qtiles = static_cast<const int4*>(qtiles);
+  g.n_qtiles = n_qtiles;
+  g.idx = idx;
+  g.Qv = Qv;
+  g.d = c.d_model;
+  g.T = c.T;
+  g.G = c.G;
+  g.M = c.M;
+  g.k = c.k;
+  g.B = c.B;
+  g.dh = dh;
+  Epi e{};
+  const dim3 grid(static_cast<unsigned>(max_qtiles), 1, 1);
+  if (dh == 64) return launch<64, true>(tb, tb, tb, e, e, g, c.d_model, grid, stream);
+  return launch<32, true>(tb, tb, tb, e, e, g, c.d_model, grid, stream);
+}
+
+}  // namespace gqe

@@ -1,0 +1,71 @@
+// Internal declarations shared by the .cu files of libgqe.so.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include "gqe.h"
+
+namespace gqe {
+
+// Wall-time bound of every device-side wait (2 s).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Router limits: N = G*M experts (<= 64, G <= 32). The logits are reduced
+// over NP = max(4, next power of two >= N) columns; W_r is staged in shared
+// memory with a row stride of router_row_floats(NP) floats, == 4 (mod 8), so
+// that the 16-byte reads of 8 consecutive lanes (consecutive rows) land in
+// distinct bank groups.
+constexpr int kMaxExperts = 64;
+__host__ __device__ constexpr int router_np(int N) {
+  return N <= 4 ? 4 : N <= 8 ? 8 : N <= 16 ? 16 : N <= 32 ? 32 : 64;
+}
+__host__ __device__ constexpr int router_row_floats(int NP) { return NP == 4 ? 4 : NP + 4; }
+constexpr size_t kRouterSmemLimit = 200 * 1024;
+
+// Dispatch tiling: tokens of one sequence are cut into tiles of this size.
+constexpr int kDispatchTile = 1024;
+constexpr int kQTileRows = 128;  // rows of one grouped-GEMM tile
+
+struct DispatchWs {
+  // Byte offsets inside the dispatch workspace.
+  size_t tile_counts;  // int32 [N][num_tiles]
+  size_t tile_base;    // int32 [N][num_tiles]
+  size_t qtiles;       // int4  [max_qtiles]: (e, b, start, rows)
+  size_t n_qtiles;     // int32 [1]
+  size_t total;
+  int num_tiles;
+  int tiles_per_seq;
+  int max_qtiles;
+};
+DispatchWs dispatch_ws_layout(const gqe_config& c);
+
+bool config_ok(const gqe_config* c);
+
+// Launchers (return cudaError_t as int).
+int launch_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r,
+                  int32_t* idx, float* r, float* omega, void* stream);
+int launch_dispatch_lists(const gqe_config& c, const int32_t* idx, int32_t* counts,
+                          int32_t* offsets, int32_t* tok, int32_t* slot_pos, void* ws,
+                          const DispatchWs& L, void* stream);
+int launch_weighted_slot(const gqe_config& c, uint16_t* slots, const float* omega, void* stream);
+
+// GEMM front ends (tcgen05). out layouts are described in gemm.cu.
+int gemm_kv(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
+            uint16_t* K, uint16_t* V, void* stream);
+int gemm_q_shared(const gqe_config& c, const uint16_t* x, const uint16_t* W_qs, uint16_t* Qs,
+                  void* stream);
+int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const int32_t* idx,
+                  const int32_t* offsets, const int32_t* tok, const void* qtiles,
+                  const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, void* stream);
+int gemm_q_dense(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, uint16_t* Q,
+                 void* stream);
+int gemm_rowmajor(const uint16_t* A, int rows, int K, const uint16_t* W, int N, uint16_t* out,
+                  void* stream);
+
+// Attention front ends (tcgen05).
+int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
+                  const uint16_t* V, uint16_t* slots, void* stream);
+int attention_dense(const gqe_config& c, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                    uint16_t* O, void* stream);
+
+}  // namespace gqe

@@ -1,0 +1,7 @@
+// Single translation unit of libgqe.so: the device status word and every
+// kernel live in one module, so no relocatable device code is needed.
+#include "router.cu"
+#include "dispatch.cu"
+#include "gemm.cu"
+#include "attention.cu"
+#include "api.cu"

@@ -1,0 +1,106 @@
+"""Helpers shared by the GPU parity tests: upload seeded inputs, run the CUDA
+path step by step through the C ABI, and compare with the fp64 oracle."""
+import numpy as np
+import torch
+
+import synth
+
+MAX_ABS = 2e-2   # bf16 inputs, fp32 accumulation: max-abs error bound
+MEAN_ABS = 2e-3  # ... and mean-abs error bound
+
+
+def bf16_dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def f32_dev(a) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().double().numpy()
+
+
+def assert_close(got: torch.Tensor, want: np.ndarray, what: str, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
+    """Max-abs / mean-abs check against the oracle.
+
+    Every bf16 rounding on the path (Q, K, V, P, slots, y) is relative to the
+    value rounded, so the error scales with the output's magnitude. The bounds
+    hold as stated for outputs of rms <= 1 (every measured workload: attention
+    averages over many positions); for larger outputs (sequences of a few
+    tokens, where o is a single V row) both bounds scale with rms(want).
+    """
+    g = to_f64(got).reshape(want.shape)
+    scale = max(1.0, float(np.sqrt(np.mean(np.square(want)))) if want.size else 1.0)
+    max_abs, mean_abs = max_abs * scale, mean_abs * scale
+    err = np.abs(g - want)
+    assert np.isfinite(g).all(), f"{what}: non-finite values"
+    assert err.max() <= max_abs and err.mean() <= mean_abs, (
+        f"{what}: max abs err {err.max():.3e} (<= {max_abs}), mean abs err {err.mean():.3e} (<= {mean_abs})")
+    return float(err.max()), float(err.mean())
+
+
+def device_inputs(inp: synth.LayerInputs) -> dict:
+    d = {
+        "x": bf16_dev(inp.x), "W_r": f32_dev(inp.W_r),
+        "b_r": None if inp.b_r is None else f32_dev(inp.b_r),
+        "W_q": bf16_dev(inp.W_q), "W_qs": bf16_dev(inp.W_qs), "W_k": bf16_dev(inp.W_k),
+        "W_v": bf16_dev(inp.W_v), "W_o": bf16_dev(inp.W_o),
+    }
+    if inp.W_o_dense.size:
+        d["W_o_dense"] = bf16_dev(inp.W_o_dense)
+    return d
+
+
+def run_steps(rsq, shape: synth.LayerShape, d: dict) -> dict:
+    """GQE layer through the five step entry points; returns every output."""
+    cfg = rsq.GQEConfig.of(shape)
+    B, T, G, M, k, dh = shape.B, shape.T, shape.G, shape.M, shape.k, shape.d_head
+    R, N = B * T, G * M
+    dev = torch.device("cuda")
+    o = {}
+    o["idx"] = torch.empty(R, G, k, dtype=torch.int32, device=dev)
+    o["r"] = torch.empty(R, G, k, dtype=torch.float32, device=dev)
+    o["omega"] = torch.empty(R, G, k, dtype=torch.float32, device=dev)
+    rsq.gqe_router_topk(cfg, d["x"], d["W_r"], d["b_r"], o["idx"], o["r"], o["omega"])
+    o["counts"] = torch.empty(N * B, dtype=torch.int32, device=dev)
+    o["offsets"] = torch.empty(N * B + 1, dtype=torch.int32, device=dev)
+    o["tok"] = torch.empty(k * G * R, dtype=torch.int32, device=dev)
+    o["slot_pos"] = torch.empty(R, G, k, dtype=torch.int32, device=dev)
+    o["Qv"] = torch.empty(B, G, k, T, dh, dtype=torch.bfloat16, device=dev)
+    o["Qs"] = torch.empty(B, T, dh, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_DISPATCH), 16), dtype=torch.uint8,
+                     device=dev)
+    rsq.gqe_dispatch(cfg, o["idx"], d["x"], d["W_q"], d["W_qs"], o["counts"], o["offsets"],
+                     o["tok"], o["slot_pos"], o["Qv"], o["Qs"], ws)
+    o["K"] = torch.empty(B, G, T, dh, dtype=torch.bfloat16, device=dev)
+    o["V"] = torch.empty(B, G, T, dh, dtype=torch.bfloat16, device=dev)
+    rsq.gqe_kv_proj(cfg, d["x"], d["W_k"], d["W_v"], o["K"], o["V"])
+    o["slots"] = torch.zeros(R, (k * G + 2) * dh, dtype=torch.bfloat16, device=dev)
+    rsq.gqe_attention_fwd(cfg, o["Qv"], o["Qs"], o["K"], o["V"], o["slots"])
+    o["y"] = torch.empty(R, shape.d_model, dtype=torch.bfloat16, device=dev)
+    rsq.gqe_output_proj(cfg, o["slots"], o["omega"], d["W_o"], o["y"])
+    torch.cuda.synchronize()
+    assert rsq.gqe_read_status() == 0
+    return o
+
+
+def run_layer(rsq, shape, d: dict):
+    cfg = rsq.GQEConfig.of(shape)
+    ws = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_LAYER), dtype=torch.uint8, device="cuda")
+    y = torch.empty(shape.R, shape.d_model, dtype=torch.bfloat16, device="cuda")
+    rsq.gqe_layer_fwd(cfg, d["x"], d["W_r"], d["b_r"], d["W_q"], d["W_qs"], d["W_k"], d["W_v"],
+                      d["W_o"], y, ws)
+    torch.cuda.synchronize()
+    assert rsq.gqe_read_status() == 0
+    return y, ws
+
+
+def run_dense(rsq, shape, d: dict):
+    cfg = rsq.GQEConfig.of(shape)
+    ws = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_DENSE), dtype=torch.uint8, device="cuda")
+    y = torch.empty(shape.R, shape.d_model, dtype=torch.bfloat16, device="cuda")
+    rsq.gqa_dense_fwd(cfg, d["x"], d["W_q"], d["W_k"], d["W_v"], d["W_o_dense"], y, ws)
+    torch.cuda.synchronize()
+    assert rsq.gqe_read_status() == 0
+    return y, ws

@@ -1,0 +1,149 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on a B200.
+
+Integer outputs (router indices, token lists, counts, offsets, slot positions)
+must be bit-exact; floating-point outputs must be within max-abs 2e-2 and
+mean-abs 2e-3 of the oracle (bf16 inputs, fp32 accumulation).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import LayerShape
+from gpu_common import (assert_close, device_inputs, run_dense, run_layer, run_steps, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rsq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import routed_sparse_query_b200 as m
+    return m
+
+
+def _check_integer_parts(o, ref, shape):
+    assert np.array_equal(o["idx"].cpu().numpy(), ref["idx"]), "router indices differ"
+    assert np.array_equal(o["counts"].cpu().numpy().reshape(shape.N, shape.B), ref["counts"])
+    assert np.array_equal(o["offsets"].cpu().numpy(), ref["offsets"])
+    assert np.array_equal(o["tok"].cpu().numpy(), ref["tok"]), "token lists differ"
+    assert np.array_equal(o["slot_pos"].cpu().numpy(), ref["slot_pos"])
+
+
+def _check_float_parts(o, ref, shape):
+    np.testing.assert_allclose(o["r"].cpu().numpy(), ref["r"], rtol=0, atol=2e-6)
+    np.testing.assert_allclose(o["omega"].cpu().numpy(), ref["omega"], rtol=0, atol=2e-6)
+    assert_close(o["K"], ref["K"], "K")
+    assert_close(o["V"], ref["V"], "V")
+    assert_close(o["Qv"], ref["Qv"], "Qv")
+    assert_close(o["Qs"], ref["Qs"], "Qs")
+    assert_close(o["slots"], ref["slots"], "slots")
+    assert_close(o["y"], ref["y"], "y")
+
+
+CASES = {
+    "tiny": (synth.TINY, {}),
+    "ragged_b2": (LayerShape(B=2, T=333, d_model=256, G=4, M=2, k=1, d_head=64), {}),
+    "pool4_k2_skew": (LayerShape(B=1, T=700, d_model=512, G=8, M=4, k=2, d_head=64), {"skew": True}),
+    "pool4_k1_skew": (LayerShape(B=2, T=300, d_model=512, G=8, M=4, k=1, d_head=64), {"skew": True}),
+    "k_equals_m": (LayerShape(B=1, T=260, d_model=256, G=4, M=2, k=2, d_head=32), {}),
+    "t1": (LayerShape(B=3, T=1, d_model=128, G=2, M=2, k=1, d_head=64), {}),
+    "t5_dh32": (LayerShape(B=2, T=5, d_model=64, G=2, M=3, k=2, d_head=32), {}),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_layer_steps_match_oracle(rsq, name):
+    shape, kw = CASES[name]
+    inp = synth.make_layer_inputs(shape, seed=101, **kw)
+    ref = oracle.gqe_layer(inp)
+    o = run_steps(rsq, shape, device_inputs(inp))
+    _check_integer_parts(o, ref, shape)
+    _check_float_parts(o, ref, shape)
+
+
+def test_seq2k_layer_matches_oracle(rsq):
+    shape = synth.SEQ2K
+    inp = synth.make_layer_inputs(shape)
+    ref = oracle.gqe_layer(inp)
+    d = device_inputs(inp)
+    o = run_steps(rsq, shape, d)
+    _check_integer_parts(o, ref, shape)
+    _check_float_parts(o, ref, shape)
+    y, ws = run_layer(rsq, shape, d)
+    assert torch.equal(y, o["y"]), "gqe_layer_fwd differs from the step calls"
+
+
+def test_dense_gqa_matches_oracle(rsq):
+    for shape in (synth.TINY, synth.SEQ2K, LayerShape(B=2, T=200, d_model=256, G=2, M=3, k=1, d_head=64)):
+        inp = synth.make_layer_inputs(shape, seed=7)
+        ref = oracle.gqa_dense_layer(inp)
+        d = device_inputs(inp)
+        y, ws = run_dense(rsq, shape, d)
+        assert_close(y, ref["y"], f"dense y {shape}")
+        O = rsq.workspace_view(ws, rsq.GQEConfig.of(shape), rsq.GQE_WS_DENSE, "dense_O",
+                               torch.bfloat16, (shape.R, shape.N * shape.d_head))
+        assert_close(O, ref["O"], f"dense O {shape}")
+
+
+def test_kv_is_identical_in_both_layers(rsq):
+    shape = synth.SEQ2K
+    inp = synth.make_layer_inputs(shape, seed=3)
+    d = device_inputs(inp)
+    cfg = rsq.GQEConfig.of(shape)
+    _, ws_g = run_layer(rsq, shape, d)
+    _, ws_d = run_dense(rsq, shape, d)
+    kv_shape = (shape.B, shape.G, shape.T, shape.d_head)
+    for item in ("K", "V"):
+        a = rsq.workspace_view(ws_g, cfg, rsq.GQE_WS_LAYER, item, torch.bfloat16, kv_shape)
+        b = rsq.workspace_view(ws_d, cfg, rsq.GQE_WS_DENSE, item, torch.bfloat16, kv_shape)
+        assert torch.equal(a, b)
+
+
+def test_k_equals_m_routed_slots_are_dense_heads(rsq):
+    # With k = M every expert of every group is selected in ascending order,
+    # so routed slot (g, s) is dense head g*M + s, computed by the same kernels.
+    shape = LayerShape(B=1, T=384, d_model=256, G=4, M=2, k=2, d_head=64)
+    inp = synth.make_layer_inputs(shape, seed=9)
+    d = device_inputs(inp)
+    o = run_steps(rsq, shape, d)
+    _, ws = run_dense(rsq, shape, d)
+    O = rsq.workspace_view(ws, rsq.GQEConfig.of(shape), rsq.GQE_WS_DENSE, "dense_O", torch.bfloat16,
+                           (shape.R, shape.N * shape.d_head))
+    routed = o["slots"][:, :shape.N * shape.d_head]
+    assert torch.equal(routed, O)
+
+
+def test_empty_expert_lists(rsq):
+    shape = LayerShape(B=2, T=150, d_model=128, G=2, M=3, k=1, d_head=64)
+    inp = synth.make_layer_inputs(shape, seed=5)
+    inp.b_r = np.array([40.0, 0, 0, 40.0, 0, 0], dtype=np.float32)  # every token picks j = 0
+    ref = oracle.gqe_layer(inp)
+    o = run_steps(rsq, shape, device_inputs(inp))
+    _check_integer_parts(o, ref, shape)
+    _check_float_parts(o, ref, shape)
+    assert (o["counts"].cpu().numpy().reshape(shape.N, shape.B)[[1, 2, 4, 5]] == 0).all()
+
+
+def test_router_zero_weights_ties_go_low(rsq):
+    shape = LayerShape(B=1, T=128, d_model=256, G=4, M=4, k=2, d_head=64)
+    inp = synth.make_layer_inputs(shape, seed=4)
+    inp.W_r = np.zeros_like(inp.W_r)
+    o = run_steps(rsq, shape, device_inputs(inp))
+    assert (o["idx"].cpu().numpy() == np.array([0, 1])[None, None, :]).all()
+    np.testing.assert_allclose(o["omega"].cpu().numpy(), 1.0 / 8, rtol=1e-6)
+
+
+def test_device_wait_timeout_is_reported_and_recoverable(rsq):
+    rsq.gqe_selftest_wait_timeout(2_000_000)  # 2 ms bound on a barrier nothing completes
+    assert rsq.gqe_read_status() == rsq.GQE_ERR_TIMEOUT
+    assert rsq.gqe_read_status() == 0  # reading clears it
+    shape = synth.TINY
+    inp = synth.make_layer_inputs(shape, seed=1)
+    ref = oracle.gqe_layer(inp)
+    y, _ = run_layer(rsq, shape, device_inputs(inp))
+    assert_close(y, ref["y"], "y after timeout self-test")
