@@ -1,0 +1,516 @@
+#!/usr/bin/env python
+"""Benchmark of the GQE prefill layer on B200; rank 0 prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole GQE prefill layer (router, dispatch and
+grouped query projection, K/V projection, routed + shared attention, weighted
+slot and W_O) over one batch of the workload, issued through the library's C
+ABI. Timing: CUDA events on the launching stream around every step, L2
+flushed (256 MiB write) before each timed step, max over ranks. Under torchrun
+every rank runs an independent replica of the workload (weak scaling, no
+data-path collective).
+
+--impl reference times the fp64 CPU oracle (the reference of this build) on
+the same workload, on the host cores of rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "GQE prefill layer tokens/s and attn tensor-pipe % of bf16 peak vs seq len"
+WORKLOADS = {
+    "seq2k": synth.SEQ2K,
+    "b4x8k": synth.BATCH4_8K,
+    "seq32k": synth.SEQ32K,
+    "seq256k": synth.SEQ256K,
+    "seq1m": synth.SEQ1M,
+    "pool4_k1": synth.POOL4_K1,
+    "pool4_k2": synth.POOL4_K2,
+}
+HEADLINE = "seq2k"
+SWEEP = ["b4x8k", "seq32k", "seq256k", "seq1m"]
+LAUNCHES = {"router": 1, "dispatch": 5, "kv": 1, "attention": 1, "output": 2}
+FLUSH_BYTES = 256 << 20
+PAGES_SPEEDUP = {"2k": 1.15, "4k..1024k": "1.67-1.80", "1024k": 1.80,
+                 "hardware": "not stated"}
+
+
+def describe(s: synth.LayerShape) -> str:
+    return (f"GQE prefill layer B={s.B} T={s.T} d_model={s.d_model} G={s.G} M={s.M} k={s.k} "
+            f"d_head={s.d_head} (+1 shared head)")
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"bf16": p["bf16_tflops"], "bf16_sustained": p["bf16_tflops_sustained"],
+                "hbm": p["hbm_gbs"], "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
+
+
+def flops(s: synth.LayerShape, dense: bool = False):
+    """Algorithmic FLOPs per layer pass (active work only)."""
+    heads = s.N if dense else s.k * s.G + 1
+    slots = s.N if dense else s.n_slots
+    R, d, dh = s.R, s.d_model, s.d_head
+    attn = 4.0 * dh * heads * s.B * s.T * (s.T + 1) / 2
+    return {"attention": attn, "q": 2.0 * R * d * dh * heads, "kv": 4.0 * R * d * dh * s.G,
+            "wo": 2.0 * R * slots * dh * d, "router": 0.0 if dense else 2.0 * R * d * s.N}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read only)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting"}
+
+    def __init__(self, torch_dev: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_dev).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self.max_mhz = None
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            if not self.samples:
+                self._sample()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
+
+
+# ---------------------------------------------------------------- GPU arm
+class Layer:
+    """Device buffers of one layer instance and the C-ABI calls of one step."""
+
+    def __init__(self, rsq, shape: synth.LayerShape, d: dict):
+        import torch
+        self.rsq, self.s, self.d = rsq, shape, d
+        s = shape
+        B, T, G, M, k, dh, R, N = s.B, s.T, s.G, s.M, s.k, s.d_head, s.R, s.N
+        dev = torch.device("cuda")
+        self.cfg = rsq.GQEConfig.of(s)
+        e = torch.empty
+        self.idx = e(R, G, k, dtype=torch.int32, device=dev)
+        self.r = e(R, G, k, dtype=torch.float32, device=dev)
+        self.omega = e(R, G, k, dtype=torch.float32, device=dev)
+        self.counts = e(N * B, dtype=torch.int32, device=dev)
+        self.offsets = e(N * B + 1, dtype=torch.int32, device=dev)
+        self.tok = e(k * G * R, dtype=torch.int32, device=dev)
+        self.slot_pos = e(R, G, k, dtype=torch.int32, device=dev)
+        self.Qv = e(B, G, k, T, dh, dtype=torch.bfloat16, device=dev)
+        self.Qs = e(B, T, dh, dtype=torch.bfloat16, device=dev)
+        self.K = e(B, G, T, dh, dtype=torch.bfloat16, device=dev)
+        self.V = e(B, G, T, dh, dtype=torch.bfloat16, device=dev)
+        self.slots = e(R, s.n_slots * dh, dtype=torch.bfloat16, device=dev)
+        self.y = e(R, s.d_model, dtype=torch.bfloat16, device=dev)
+        self.wsd = e(rsq.gqe_workspace_bytes(self.cfg, rsq.GQE_WS_DISPATCH), dtype=torch.uint8, device=dev)
+
+    def router(self):
+        d = self.d
+        self.rsq.gqe_router_topk(self.cfg, d["x"], d["W_r"], d["b_r"], self.idx, self.r, self.omega)
+
+    def dispatch(self):
+        d = self.d
+        self.rsq.gqe_dispatch(self.cfg, self.idx, d["x"], d["W_q"], d["W_qs"], self.counts,
+                              self.offsets, self.tok, self.slot_pos, self.Qv, self.Qs, self.wsd)
+
+    def kv(self):
+        d = self.d
+        self.rsq.gqe_kv_proj(self.cfg, d["x"], d["W_k"], d["W_v"], self.K, self.V)
+
+    def attention(self):
+        self.rsq.gqe_attention_fwd(self.cfg, self.Qv, self.Qs, self.K, self.V, self.slots)
+
+    def output(self):
+        self.rsq.gqe_output_proj(self.cfg, self.slots, self.omega, self.d["W_o"], self.y)
+
+    CALLS = ("router", "dispatch", "kv", "attention", "output")
+
+
+def device_inputs_from_synth(inp: synth.LayerInputs) -> dict:
+    import torch
+
+    def b16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    d = {"x": b16(inp.x), "W_r": torch.from_numpy(inp.W_r).cuda(),
+         "b_r": None if inp.b_r is None else torch.from_numpy(inp.b_r).cuda(),
+         "W_q": b16(inp.W_q), "W_qs": b16(inp.W_qs), "W_k": b16(inp.W_k), "W_v": b16(inp.W_v),
+         "W_o": b16(inp.W_o), "W_o_dense": b16(inp.W_o_dense)}
+    return d
+
+
+def device_inputs_seeded(shape: synth.LayerShape, seed: int) -> dict:
+    """Same recipe as synth (x ~ N(0,1), weights ~ N(0, 1/d)), drawn on the
+    device with torch's seeded generator (for sizes too large to draw on the
+    host quickly)."""
+    import torch
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    s, sd = shape, shape.d_model ** -0.5
+    d = {"x": torch.randn(s.R, s.d_model, device="cuda", generator=g).to(torch.bfloat16),
+         "W_r": torch.randn(s.d_model, s.N, device="cuda", generator=g) * sd, "b_r": None}
+    for nm, shp in (("W_q", (s.d_model, s.N * s.d_head)), ("W_qs", (s.d_model, s.d_head)),
+                    ("W_k", (s.d_model, s.G * s.d_head)), ("W_v", (s.d_model, s.G * s.d_head)),
+                    ("W_o", (s.n_slots * s.d_head, s.d_model)),
+                    ("W_o_dense", (s.N * s.d_head, s.d_model))):
+        d[nm] = (torch.randn(*shp, device="cuda", generator=g) * sd).to(torch.bfloat16)
+    return d
+
+
+def time_steps(layer: Layer, steps: int, warmup: int, flush, sync_ranks) -> dict:
+    """Times `steps` layer passes; returns total ms and per-call ms sums."""
+    import torch
+    for _ in range(warmup):
+        for c in Layer.CALLS:
+            getattr(layer, c)()
+    torch.cuda.synchronize()
+    n = len(Layer.CALLS)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+    sync_ranks()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        ev[i][0].record()
+        for j, c in enumerate(Layer.CALLS):
+            getattr(layer, c)()
+            ev[i][j + 1].record()
+    torch.cuda.synchronize()
+    sync_ranks()
+    per = {c: 0.0 for c in Layer.CALLS}
+    total = 0.0
+    for i in range(steps):
+        total += ev[i][0].elapsed_time(ev[i][n])
+        for j, c in enumerate(Layer.CALLS):
+            per[c] += ev[i][j].elapsed_time(ev[i][j + 1])
+    return {"total_ms": total, "per_call_ms": per}
+
+
+def time_dense(rsq, shape, d, steps, warmup, flush) -> float:
+    import torch
+    cfg = rsq.GQEConfig.of(shape)
+    ws = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_DENSE), dtype=torch.uint8, device="cuda")
+    y = torch.empty(shape.R, shape.d_model, dtype=torch.bfloat16, device="cuda")
+
+    def f():
+        rsq.gqa_dense_fwd(cfg, d["x"], d["W_q"], d["W_k"], d["W_v"], d["W_o_dense"], y, ws)
+
+    for _ in range(warmup):
+        f()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        if flush is not None:
+            flush()
+        a.record()
+        f()
+        b.record()
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev)
+
+
+def time_e2e(rsq, shape, d, steps, warmup) -> dict:
+    """gqe_layer_fwd with x copied in from pinned host memory and y copied
+    back, every step, inside the timed region."""
+    import torch
+    cfg = rsq.GQEConfig.of(shape)
+    ws = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_LAYER), dtype=torch.uint8, device="cuda")
+    x_h = d["x"].cpu().pin_memory()
+    y_h = torch.empty(shape.R, shape.d_model, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(d["x"])
+    y_d = torch.empty(shape.R, shape.d_model, dtype=torch.bfloat16, device="cuda")
+
+    def f():
+        x_d.copy_(x_h, non_blocking=True)
+        rsq.gqe_layer_fwd(cfg, x_d, d["W_r"], d["b_r"], d["W_q"], d["W_qs"], d["W_k"], d["W_v"],
+                          d["W_o"], y_d, ws)
+        y_h.copy_(y_d, non_blocking=True)
+
+    for _ in range(warmup):
+        f()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        f()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    return {"ms": ms, "h2d": x_h.numel() * 2, "d2h": y_h.numel() * 2}
+
+
+def roofline_of(shape, per_call_ms: dict, steps: int, pk: dict, traffic=None):
+    fl = flops(shape)
+    s = shape
+    units = {
+        "attention": ("tensor", fl["attention"] / 1e12, "TFLOP/s", pk["bf16"]),
+        "kv": ("tensor", fl["kv"] / 1e12, "TFLOP/s", pk["bf16"]),
+        "output": ("tensor", fl["wo"] / 1e12, "TFLOP/s", pk["bf16"]),
+        "dispatch": ("tensor", fl["q"] / 1e12, "TFLOP/s", pk["bf16"]),
+        "router": ("hbm", (s.R * s.d_model * 2 + s.d_model * s.N * 4 + s.R * s.G * s.k * 12) / 1e9,
+                   "GB/s", pk["hbm"]),
+    }
+    top = max(per_call_ms, key=per_call_ms.get)
+    bound, work, unit, peak = units[top]
+    avg_s = per_call_ms[top] / steps / 1e3
+    ach = work / avg_s if avg_s > 0 else 0.0
+    return {"kernel": top, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+            "frac": ach / peak, "peak_source": f"{pk['source']} burst", "traffic": traffic,
+            "avg_launch_ms": avg_s * 1e3}
+
+
+def cpu_baseline(shape: synth.LayerShape, max_tokens: int | None = None) -> dict:
+    """The oracle as it stands, on this host, on one layer pass."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    T = shape.T if max_tokens is None else min(shape.T, max_tokens)
+    s = synth.LayerShape(1, T, shape.d_model, shape.G, shape.M, shape.k, shape.d_head)
+    inp = synth.make_layer_inputs(s, with_dense=False)
+    t0 = time.perf_counter()
+    oracle.gqe_layer(inp)
+    dt = time.perf_counter() - t0
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": T / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"one full oracle layer pass over {T} tokens of one sequence "
+                      f"(fp64 numpy, {dt:.2f} s)", "seconds": dt}
+
+
+def run_ours(args, rank: int, world: int, dist):
+    import torch
+    import routed_sparse_query_b200 as rsq
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+    pk = peaks()
+    shape = WORKLOADS[args.workload]
+    inp = synth.make_layer_inputs(shape, seed=synth.DEFAULT_SEED + rank)
+    d = device_inputs_from_synth(inp)
+    layer = Layer(rsq, shape, d)
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = flush_buf.zero_
+
+    def sync_ranks():
+        if dist is not None:
+            dist.barrier()
+
+    warmup = max(3, args.warmup)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        res = time_steps(layer, args.steps, warmup, flush, sync_ranks)
+    if rsq.gqe_read_status() != 0:
+        raise RuntimeError("device-side status set during the timed steps")
+    total = torch.tensor([res["total_ms"]], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(total, op=dist.ReduceOp.MAX)
+    max_ms = float(total.item())
+    ms_per_step = max_ms / args.steps
+    tokens = shape.R * world * args.steps
+    value = tokens / (max_ms / 1e3)
+
+    e2e = time_e2e(rsq, shape, d, args.steps, warmup)
+    e2e_t = torch.tensor([e2e["ms"]], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_value = tokens / (float(e2e_t.item()) / 1e3)
+
+    dense_ms = time_dense(rsq, shape, d, args.steps, warmup, flush) / args.steps
+    dense_t = torch.tensor([dense_ms], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(dense_t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    if rank != 0:
+        return None
+
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        try:
+            with open(prof) as f:
+                traffic = json.load(f).get(args.workload)
+        except ValueError:
+            traffic = None
+    roof = roofline_of(shape, res["per_call_ms"], args.steps, pk, traffic)
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {describe(shape)}", "global_batch": shape.B * world,
+                   "seq_len": shape.T, "parallelism": f"replicas{world}",
+                   "l2": "flushed (256 MiB write) before every timed step",
+                   "inputs": "seeded synth recipe: x ~ N(0,1) bf16, weights ~ N(0,1/d_model) bf16, "
+                             "router fp32"},
+        "gpu_launches": sum(LAUNCHES.values()) * args.steps,
+        "clocks": clk.summary(),
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
+                "d2h_bytes_per_step": e2e["d2h"], "api": "gqe_layer_fwd"},
+        "roofline": roof,
+        "breakdown_ms_per_step": {c: v / args.steps for c, v in res["per_call_ms"].items()},
+        "dense_gqa": {"ms_per_step": float(dense_t.item()),
+                      "tokens_per_s": shape.R * world / (float(dense_t.item()) / 1e3),
+                      "speedup_gqe_over_dense": float(dense_t.item()) / ms_per_step},
+        "pages_speedup_context": PAGES_SPEEDUP,
+    }
+    if world == 1 and not args.no_sweep:
+        out["sweep"] = sweep(rsq, pk, args)
+    if world == 1 and not args.no_cpu:
+        out["cpu_baseline"] = cpu_baseline(shape)
+    return out
+
+
+def sweep(rsq, pk, args):
+    """GQE vs dense GQA at every sequence length of the measured workloads."""
+    import torch
+    rows = []
+    names = SWEEP if args.sweep_max is None else SWEEP[:SWEEP.index(args.sweep_max) + 1]
+    for name in names:
+        s = WORKLOADS[name]
+        d = device_inputs_seeded(s, 1234)
+        layer = Layer(rsq, s, d)
+        est = flops(s)["attention"] / 0.5e15  # seconds per step at 0.5 PFLOP/s
+        steps = max(2, min(args.steps, int(2.0 / max(est, 1e-6))))
+        res = time_steps(layer, steps, 2, None, lambda: None)
+        dense_ms = time_dense(rsq, s, d, steps, 1, None) / steps
+        gq_ms = res["total_ms"] / steps
+        attn_s = res["per_call_ms"]["attention"] / steps / 1e3
+        ach = flops(s)["attention"] / attn_s / 1e12
+        rows.append({"workload": f"{name}: {describe(s)}", "T": s.T, "B": s.B, "steps": steps,
+                     "gqe_ms": gq_ms, "gqe_tokens_per_s": s.R / (gq_ms / 1e3),
+                     "dense_ms": dense_ms, "dense_tokens_per_s": s.R / (dense_ms / 1e3),
+                     "speedup": dense_ms / gq_ms, "attn_tflops": ach,
+                     "attn_frac_of_bf16_peak": ach / pk["bf16"],
+                     "l2": "inputs larger than L2, not flushed",
+                     "breakdown_ms": {c: v / steps for c, v in res["per_call_ms"].items()}})
+        if rsq.gqe_read_status() != 0:
+            raise RuntimeError(f"device-side status set in sweep {name}")
+        del layer, d
+        torch.cuda.empty_cache()
+    return rows
+
+
+def run_reference(args):
+    """The fp64 oracle on the host cores, on prefixes of the workload sized so
+    that warmup + steps end within about two minutes."""
+    import oracle  # noqa: F401
+    shape = WORKLOADS[args.workload]
+    budget = 120.0 / (args.steps + max(1, args.warmup))
+    T = shape.T
+    probe = cpu_baseline(shape, max_tokens=min(T, 256))
+    per_tok = probe["seconds"] / min(T, 256)
+    while T > 256 and per_tok * T * (1 + T / 4096) > budget:
+        T //= 2
+    for _ in range(max(1, args.warmup) if T <= 256 else 1):
+        cpu_baseline(shape, max_tokens=T)
+    times = []
+    for _ in range(args.steps):
+        times.append(cpu_baseline(shape, max_tokens=T)["seconds"])
+    value = T * args.steps / sum(times)
+    from threadpoolctl import threadpool_info
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(times) / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {describe(shape)}", "global_batch": shape.B,
+                   "seq_len": shape.T, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: the full oracle layer on the first {T} of {shape.T} "
+                                   f"tokens of the sequence (a causal prefix), fp64 numpy"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default=HEADLINE)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--sweep-max", choices=SWEEP, default=None)
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    dist = None
+    if world > 1:
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        out = run_ours(args, rank, world, dist)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -35,10 +35,7 @@ gqe_status check_cfg(const gqe_config* c) {
   if (R * c->d_model >= (1ll << 31) * 4 || R * (N + 2) * c->d_head >= (1ll << 31) ||
       R * c->G * c->k * 4 >= (1ll << 31))
     return GQE_ERR_UNSUPPORTED;
-  const int NP = router_np(static_cast<int>(N));
-  const size_t rsm = static_cast<size_t>(c->d_model) * router_row_floats(NP) * 4 + 2 * NP * 4 +
-                     8 * NP * 12;
-  if (rsm > kRouterSmemLimit) return GQE_ERR_UNSUPPORTED;
+  if (router_smem_bytes(*c) > kRouterSmemLimit) return GQE_ERR_UNSUPPORTED;
   return GQE_OK;
 }
 

@@ -37,6 +37,12 @@ namespace attn_impl {
 constexpr int BQ = 128;
 constexpr int BKV = 128;
 constexpr int KV_STAGES = 3;
+constexpr int kThreads = 320;  // 2 softmax warpgroups + TMA warp + UMMA warp
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+// O is rescaled only when a row's running max grows by more than this many
+// powers of two; until then the stale max is kept and P may reach 2^8.
+constexpr float kRescaleLog2 = 8.0f;
 
 template <int DH>
 struct AttnCfg {
@@ -45,15 +51,16 @@ struct AttnCfg {
   static constexpr int TILE_BYTES = BQ * DH * 2;
   static constexpr int P_BYTES = BQ * BKV * 2;
   static constexpr size_t SMEM =
-      1024 + static_cast<size_t>(TILE_BYTES) * (1 + 2 * KV_STAGES) + 2 * P_BYTES + 256;
-  static constexpr uint32_t TMEM_COLS = 512;
+      1024 + static_cast<size_t>(TILE_BYTES) * (2 + 2 * KV_STAGES) + 2 * P_BYTES + 512;
+  static constexpr uint32_t TMEM_COLS = 512;  // S_a, S_b (128 each), O_a, O_b (DH each)
 };
 
 struct AttnParams {
   int T, B, H;       // tokens per sequence, sequences, query streams per sequence
   int G, k, M;       // groups, selected per group, experts per group
   int dense;         // 0: GQE streams (kG routed + shared), 1: dense GQA heads
-  int n_qt;          // query tiles per stream
+  int n_qt;          // 128-row query tiles per stream
+  int n_pairs;       // CTAs per stream: pairs of consecutive query tiles
   uint16_t* out;     // [B*T, ldo]
   int ldo;
   float scale_log2;  // log2(e) / sqrt(dh)
@@ -65,8 +72,144 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed fp32 pairs (sm_100 f32x2 instructions: one issue slot for two lanes
+// of arithmetic).
+__device__ __forceinline__ uint64_t as_u64(float2 v) { return *reinterpret_cast<uint64_t*>(&v); }
+__device__ __forceinline__ float2 as_f2(uint64_t v) { return *reinterpret_cast<float2*>(&v); }
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(as_u64(a)), "l"(as_u64(b)), "l"(as_u64(c)));
+  return as_f2(r);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(as_u64(a)), "l"(as_u64(b)));
+  return as_f2(r);
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(as_u64(a)), "l"(as_u64(b)));
+  return as_f2(r);
+}
+
+// 2^x on the FMA pipe for a pair of values: x = n + f with n = round(x)
+// (the 1.5*2^23 shift rounds to nearest), 2^f by a degree-3 minimax
+// polynomial on [-1/2, 1/2] (relative error 7.5e-5; coefficients from
+// exp2_poly_fit.py), 2^n added into the exponent field. Inputs below -125 are
+// clamped (result ~1e-38). Additions and the polynomial use f32x2.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 shift = make_float2(12582912.0f, 12582912.0f);
+  const float2 t = fadd2(x, shift);
+  const float2 f = fsub2(x, fsub2(t, shift));
+  float2 q = ffma2(make_float2(5.517166853e-02f, 5.517166853e-02f), f,
+                   make_float2(2.426111251e-01f, 2.426111251e-01f));
+  q = ffma2(q, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
+  q = ffma2(q, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Online softmax of one query row against one 128-key tile held in TMEM
+// (tS): pass 1 takes the row max, pass 2 writes P = 2^(s*scale - m) as bf16
+// into the UMMA K-major 128B-swizzled layout at prow and adds it to l. Only
+// the diagonal tile (MASK) tests keys against the row's position: key x is
+// visible iff x <= lim. O (tO) is rescaled only when the max grows by more
+// than kRescaleLog2.
+template <int DH, bool MASK>
+__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint8_t* prow, int i,
+                                             int lim, float sc, bool first, float& m, float& l) {
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int c = 0; c < BKV / 64; ++c) {
+    uint32_t v[64];
+    tmem_ld64(tS + c * 64, v);
+#pragma unroll
+    for (int x = 0; x < 64; x += 8) {
+      float a[8];
+#pragma unroll
+      for (int y = 0; y < 8; ++y) {
+        a[y] = __uint_as_float(v[x + y]);
+        if (MASK && c * 64 + x + y > lim) a[y] = -INFINITY;
+      }
+      mx[0] = max3(mx[0], a[0], a[4]);
+      mx[1] = max3(mx[1], a[1], a[5]);
+      mx[2] = max3(mx[2], a[2], a[6]);
+      mx[3] = max3(mx[3], a[3], a[7]);
+    }
+  }
+  const float mc = fmaxf(max3(mx[0], mx[1], mx[2]), mx[3]) * sc;
+  const bool need = mc > m + kRescaleLog2;
+  if (__any_sync(0xffffffffu, need)) {
+    const float m_new = need ? mc : m;
+    const float alpha = ex2(m - m_new);
+    if (!first) {
+#pragma unroll
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tO + c * 32, v);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
+        tmem_st32(tO + c * 32, v);
+      }
+      tmem_st_wait();
+    }
+    l *= alpha;
+    m = m_new;
+  }
+  const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m, -m);
+  float2 lsum = make_float2(0.0f, 0.0f);
+#pragma unroll
+  for (int c = 0; c < BKV / 32; ++c) {
+    uint32_t v[32];
+    tmem_ld32(tS + c * 32, v);
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+      const int c16 = c * 4 + c8;  // 8-key chunk index in the row
+      float e8[8];
+#pragma unroll
+      for (int x = 0; x < 8; x += 2) {
+        float2 z = ffma2(make_float2(__uint_as_float(v[c8 * 8 + x]), __uint_as_float(v[c8 * 8 + x + 1])),
+                         sc2, nm2);
+        if (MASK) {
+          if (c16 * 8 + x > lim) z.x = -INFINITY;
+          if (c16 * 8 + x + 1 > lim) z.y = -INFINITY;
+        }
+        float2 e;
+        if ((c8 & 1) && x >= 4) {  // 4 of every 16 on the FMA pipe, the rest on MUFU
+          e = exp2_poly2(z);
+          if (MASK) {
+            if (c16 * 8 + x > lim) e.x = 0.0f;
+            if (c16 * 8 + x + 1 > lim) e.y = 0.0f;
+          }
+        } else {
+          e = make_float2(ex2(z.x), ex2(z.y));
+        }
+        e8[x] = e.x;
+        e8[x + 1] = e.y;
+        lsum = fadd2(lsum, e);
+      }
+      uint4 o;
+      o.x = pack_bf16x2(e8[0], e8[1]);
+      o.y = pack_bf16x2(e8[2], e8[3]);
+      o.z = pack_bf16x2(e8[4], e8[5]);
+      o.w = pack_bf16x2(e8[6], e8[7]);
+      const int kc = c16 >> 3, cw = c16 & 7;
+      *reinterpret_cast<uint4*>(prow + kc * (BQ * 128) + ((cw ^ (i & 7)) << 4)) = o;
+    }
+  }
+  l += lsum.x + lsum.y;
+}
+
 template <int DH>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQs,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const AttnParams p) {
@@ -74,25 +217,25 @@ __global__ void __launch_bounds__(192, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sp = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sQ = sp;
-  uint8_t* sK = sQ + C::TILE_BYTES;
-  uint8_t* sV = sK + KV_STAGES * C::TILE_BYTES;
-  uint8_t* sP = sV + KV_STAGES * C::TILE_BYTES;
+  uint8_t* sQ = sp;                                // [2][TILE]
+  uint8_t* sK = sQ + 2 * C::TILE_BYTES;            // [KV_STAGES][TILE]
+  uint8_t* sV = sK + KV_STAGES * C::TILE_BYTES;    // [KV_STAGES][TILE]
+  uint8_t* sP = sV + KV_STAGES * C::TILE_BYTES;    // [2][P]
   uint64_t* bar = reinterpret_cast<uint64_t*>(sP + 2 * C::P_BYTES);
   uint64_t* q_full = bar;
   uint64_t* k_full = bar + 1;
   uint64_t* v_full = k_full + KV_STAGES;
   uint64_t* kv_empty = v_full + KV_STAGES;
-  uint64_t* s_full = kv_empty + KV_STAGES;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* drain = o_done + 1;
+  uint64_t* s_full = kv_empty + KV_STAGES;  // [2]
+  uint64_t* p_full = s_full + 2;            // [2]
+  uint64_t* o_done = p_full + 2;            // [2]
+  uint64_t* drain = o_done + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
-  const int qt = p.n_qt - 1 - static_cast<int>(blockIdx.x) / BH;  // longest tiles first
+  const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;  // longest first
   const int bh = static_cast<int>(blockIdx.x) % BH;
   const int b = bh / p.H, h = bh % p.H;
   int zq, grp, slot;
@@ -112,7 +255,10 @@ __global__ void __launch_bounds__(192, 1)
     tq = &tmQs;
   }
   const int zkv = b * p.G + grp;
-  const int nkv = qt + 1;  // causal: KV tiles 0..qt
+  const int qt0 = 2 * pair;
+  const bool has_b = qt0 + 1 < p.n_qt;
+  const int nkv_t[2] = {qt0 + 1, has_b ? qt0 + 2 : 0};  // causal: KV tiles 0..qt
+  const int nkv = has_b ? qt0 + 2 : qt0 + 1;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -121,32 +267,32 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_done[t], 1);
     }
-    mbar_init(o_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kTmaWarp && lane == 0) {
     prefetch_tmap(tq);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
   }
-  if (warp == 5) tmem_alloc(tslot, C::TMEM_COLS);
+  if (warp == kMmaWarp) tmem_alloc(tslot, C::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t tO = tmem + 256;
 
-  if (warp == 4) {
+  if (warp == kTmaWarp) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
-      tma_load_3d(sQ, tq, q_full, 0, qt * BQ, zq);
+      mbar_arrive_expect_tx(q_full, C::TILE_BYTES * (has_b ? 2 : 1));
+      tma_load_3d(sQ, tq, q_full, 0, qt0 * BQ, zq);
+      if (has_b) tma_load_3d(sQ + C::TILE_BYTES, tq, q_full, 0, (qt0 + 1) * BQ, zq);
       for (int j = 0; j < nkv; ++j) {
         const int st = j % KV_STAGES;
         const uint32_t ph = (j / KV_STAGES) & 1;
@@ -157,139 +303,97 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_3d(sV + st * C::TILE_BYTES, &tmV, &v_full[st], 0, j * BKV, zkv);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- UMMA issuer
+    // Order per KV tile j: PV_a(j), S_a(j+1), PV_b(j), S_b(j+1): the tensor
+    // core works on one tile while the other tile's softmax runs.
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(BQ, BKV, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(BQ, DH, 0, 1);
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      auto issue_S = [&](int t, int st) {
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+          umma_bf16_ss(tmem + t * 128,
+                       smem_desc(aQ + t * C::TILE_BYTES + kk * 32, 16, 8 * C::SWB, C::LAYOUT),
+                       smem_desc(aK + st * C::TILE_BYTES + kk * 32, 16, 8 * C::SWB, C::LAYOUT),
+                       idS, kk > 0 ? 1u : 0u);
+        umma_commit(&s_full[t]);
+      };
       bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk)
-          umma_bf16_ss(tmem, smem_desc(aQ + kk * 32, 16, 8 * C::SWB, C::LAYOUT),
-                       smem_desc(aK + kk * 32, 16, 8 * C::SWB, C::LAYOUT), idS, kk > 0 ? 1u : 0u);
-        umma_commit(&s_full[0]);
+        issue_S(0, 0);
+        if (has_b) issue_S(1, 0);
       }
       for (int j = 0; ok && j < nkv; ++j) {
-        if (j + 1 < nkv) {
-          const int st = (j + 1) % KV_STAGES;
-          if (!mbar_wait(&k_full[st], ((j + 1) / KV_STAGES) & 1, abort_flag)) break;
-          tc_fence_after();
-          const uint32_t tS = tmem + ((j + 1) & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk)
-            umma_bf16_ss(tS, smem_desc(aQ + kk * 32, 16, 8 * C::SWB, C::LAYOUT),
-                         smem_desc(aK + st * C::TILE_BYTES + kk * 32, 16, 8 * C::SWB, C::LAYOUT),
-                         idS, kk > 0 ? 1u : 0u);
-          umma_commit(&s_full[(j + 1) & 1]);
-        }
-        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag)) break;
         const int st = j % KV_STAGES;
-        if (!mbar_wait(&v_full[st], (j / KV_STAGES) & 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t pb = aP + (j & 1) * C::P_BYTES;
+        bool v_ready = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= nkv_t[t]) continue;
+          if (!mbar_wait(&p_full[t], j & 1, abort_flag)) { ok = false; break; }
+          if (!v_ready) {
+            if (!mbar_wait(&v_full[st], (j / KV_STAGES) & 1, abort_flag)) { ok = false; break; }
+            v_ready = true;
+          }
+          tc_fence_after();
+          const uint32_t pb = aP + t * C::P_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk)
-          umma_bf16_ss(tO,
-                       smem_desc(pb + (kk >> 2) * (BQ * 128) + (kk & 3) * 32, 16, 1024,
-                                 kLayoutSW128),
-                       smem_desc(aV + st * C::TILE_BYTES + kk * 16 * C::SWB, C::TILE_BYTES,
-                                 8 * C::SWB, C::LAYOUT),
-                       idO, (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&kv_empty[st]);
-        umma_commit(o_done);
+          for (int kk = 0; kk < BKV / 16; ++kk)
+            umma_bf16_ss(tmem + 256 + t * DH,
+                         smem_desc(pb + (kk >> 2) * (BQ * 128) + (kk & 3) * 32, 16, 1024,
+                                   kLayoutSW128),
+                         smem_desc(aV + st * C::TILE_BYTES + kk * 16 * C::SWB, C::TILE_BYTES,
+                                   8 * C::SWB, C::LAYOUT),
+                         idO, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&o_done[t]);
+          if (j + 1 < nkv_t[t]) {
+            const int st1 = (j + 1) % KV_STAGES;
+            if (!mbar_wait(&k_full[st1], ((j + 1) / KV_STAGES) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_S(t, st1);
+          }
+        }
+        if (ok) umma_commit(&kv_empty[st]);
       }
       umma_commit(drain);
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------- softmax
-    const int i = threadIdx.x;  // row in tile, TMEM lane
-    const int qi = qt * BQ + i;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int t = warp >> 2;            // 0: tile a, 1: tile b
+    const int i = threadIdx.x & 127;    // row in tile = TMEM lane
+    const int n_t = nkv_t[t];
+    const int qi = (qt0 + t) * BQ + i;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + t * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + t * DH + lane_off;
+    uint8_t* prow = sP + t * C::P_BYTES + i * 128;
     const float sc = p.scale_log2;
     float m = -INFINITY, l = 0.0f;
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
+    bool ok = n_t > 0;
+    for (int j = 0; ok && j < n_t; ++j) {
       // Waits are made warp-uniform: tcgen05.ld/st below are .sync.aligned.
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag))) {
-        ok = false;
-        break;
-      }
+      bool w = mbar_wait(&s_full[t], j & 1, abort_flag);
+      if (j > 0) w = mbar_wait(&o_done[t], (j - 1) & 1, abort_flag) && w;
+      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
-      float s[BKV];
-      const uint32_t tS = tmem + lane_off + (j & 1) * 128;
-#pragma unroll
-      for (int c = 0; c < BKV / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + c * 32, v);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(v[x]);
-      }
-      if (j == nkv - 1) {  // diagonal tile: key kj visible iff kj <= qi
-        const int lim = qi - j * BKV;
-#pragma unroll
-        for (int x = 0; x < BKV; ++x)
-          if (x > lim) s[x] = -INFINITY;
-      }
-      float mt = s[0];
-#pragma unroll
-      for (int x = 1; x < BKV; ++x) mt = fmaxf(mt, s[x]);
-      const float m_new = fmaxf(m, mt * sc);
-      if (j > 0) {
-        // O holds PV_{j-1}; rescale it before PV_j is issued.
-        if (!__all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const float alpha = ex2(m - m_new);
-        l *= alpha;
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll
-          for (int c = 0; c < DH / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tO + lane_off + c * 32, v);
-#pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
-            tmem_st32(tO + lane_off + c * 32, v);
-          }
-          tmem_st_wait();
-        }
-      }
-      m = m_new;
-      const float neg_m = -m_new;
-      uint8_t* prow = sP + (j & 1) * C::P_BYTES + i * 128;
-#pragma unroll
-      for (int c16 = 0; c16 < BKV / 8; ++c16) {
-        float e8[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          e8[x] = ex2(fmaf(s[c16 * 8 + x], sc, neg_m));
-          l += e8[x];
-        }
-        uint4 o;
-        o.x = pack_bf16x2(e8[0], e8[1]);
-        o.y = pack_bf16x2(e8[2], e8[3]);
-        o.z = pack_bf16x2(e8[4], e8[5]);
-        o.w = pack_bf16x2(e8[6], e8[7]);
-        const int kc = c16 >> 3, cw = c16 & 7;
-        *reinterpret_cast<uint4*>(prow + kc * (BQ * 128) + ((cw ^ (i & 7)) << 4)) = o;
-      }
+      if (j == n_t - 1)
+        softmax_tile<DH, true>(tS, tO, prow, i, qi - j * BKV, sc, j == 0, m, l);
+      else
+        softmax_tile<DH, false>(tS, tO, prow, i, BKV, sc, j == 0, m, l);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
+      mbar_arrive(&p_full[t]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, (nkv - 1) & 1, abort_flag))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&o_done[t], (n_t - 1) & 1, abort_flag))) {
       tc_fence_after();
       const float inv = 1.0f / l;
       uint16_t* dst = p.out + (static_cast<size_t>(b) * p.T + qi) * p.ldo + slot * DH;
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(tO + lane_off + c * 32, v);
+        tmem_ld32(tO + c * 32, v);
         if (qi < p.T) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
@@ -307,7 +411,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     volatile int none = 0;
     mbar_wait(drain, 0, &none, 500000000ull);
     tc_fence_after();
@@ -319,12 +423,11 @@ template <int DH>
 int launch_attn(const CUtensorMap& q, const CUtensorMap& qs, const CUtensorMap& k,
                 const CUtensorMap& v, const AttnParams& p, void* stream) {
   using C = AttnCfg<DH>;
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(C::SMEM));
+  const int e = ensure_smem<attn_kernel<DH>>(static_cast<int>(C::SMEM));
   if (e != cudaSuccess) return e;
-  const long long grid = static_cast<long long>(p.n_qt) * p.B * p.H;
+  const long long grid = static_cast<long long>(p.n_pairs) * p.B * p.H;
   if (grid <= 0) return cudaSuccess;
-  attn_kernel<DH><<<static_cast<unsigned>(grid), 192, C::SMEM, static_cast<cudaStream_t>(stream)>>>(
+  attn_kernel<DH><<<static_cast<unsigned>(grid), kThreads, C::SMEM, static_cast<cudaStream_t>(stream)>>>(
       q, qs, k, v, p);
   return cudaGetLastError();
 }
@@ -350,6 +453,7 @@ int run(const gqe_config& c, const uint16_t* Q, uint64_t nq_streams, const uint1
   p.M = c.M;
   p.dense = dense;
   p.n_qt = (c.T + BQ - 1) / BQ;
+  p.n_pairs = (p.n_qt + 1) / 2;
   p.out = out;
   p.ldo = ldo;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(dh)));

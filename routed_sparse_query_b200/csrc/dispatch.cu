@@ -26,6 +26,7 @@ namespace gqe {
 namespace dispatch_impl {
 
 constexpr int kThreads = 256;
+static_assert(kDispatchTile == kThreads, "one token per thread in count/scatter");
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -63,28 +64,28 @@ __device__ __forceinline__ bool token_mask(const ListArgs& a, size_t row, uint64
   return ok;
 }
 
+// One CTA per tile of kDispatchTile (= kThreads) tokens, one token per
+// thread; per-expert counts by warp ballots, summed over the CTA's warps.
 __global__ void __launch_bounds__(kThreads) count_kernel(ListArgs a) {
-  __shared__ int hist[kMaxExperts];
+  __shared__ int wc[kThreads / 32][kMaxExperts];
   const int tile = blockIdx.x;
   const int b = tile / a.tiles_per_seq;
-  const int t0 = (tile % a.tiles_per_seq) * kDispatchTile;
-  const int t1 = min(a.T, t0 + kDispatchTile);
-  for (int e = threadIdx.x; e < a.N; e += blockDim.x) hist[e] = 0;
-  __syncthreads();
-  bool bad = false;
-  for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
-    uint64_t m;
-    bad |= !token_mask(a, static_cast<size_t>(b) * a.T + t, m);
-    while (m) {
-      const int e = __ffsll(static_cast<long long>(m)) - 1;
-      m &= m - 1;
-      atomicAdd(&hist[e], 1);
-    }
+  const int t = (tile % a.tiles_per_seq) * kDispatchTile + threadIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint64_t m = 0;
+  bool ok = true;
+  if (t < a.T) ok = token_mask(a, static_cast<size_t>(b) * a.T + t, m);
+  if (!ok) set_status(GQE_ERR_DEVICE_CHECK);
+  for (int e = 0; e < a.N; ++e) {
+    const unsigned bal = __ballot_sync(0xffffffffu, (m >> e) & 1ull);
+    if (lane == 0) wc[warp][e] = __popc(bal);
   }
-  if (bad) set_status(GQE_ERR_DEVICE_CHECK);
   __syncthreads();
-  for (int e = threadIdx.x; e < a.N; e += blockDim.x)
-    a.tile_counts[static_cast<size_t>(e) * a.num_tiles + tile] = hist[e];
+  for (int e = threadIdx.x; e < a.N; e += blockDim.x) {
+    int c = 0;
+    for (int w = 0; w < kThreads / 32; ++w) c += wc[w][e];
+    a.tile_counts[static_cast<size_t>(e) * a.num_tiles + tile] = c;
+  }
 }
 
 // Block-wide exclusive scan of one int per thread (1024 threads).

@@ -256,14 +256,8 @@ template <int BN, bool GATHER>
 int launch(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const Epi& e0,
            const Epi& e1, const Gather& g, int K, dim3 grid, void* stream) {
   using C = GemmCfg<BN>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, GATHER>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(C::SMEM));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  const int e = ensure_smem<gemm_kernel<BN, GATHER>>(static_cast<int>(C::SMEM));
+  if (e != cudaSuccess) return e;
   gemm_kernel<BN, GATHER><<<grid, 192, C::SMEM, static_cast<cudaStream_t>(stream)>>>(
       A, B0, B1, e0, e1, g, K);
   return cudaGetLastError();

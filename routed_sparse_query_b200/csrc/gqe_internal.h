@@ -3,6 +3,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda_runtime.h>
+
 #include "gqe.h"
 
 namespace gqe {
@@ -23,7 +25,7 @@ __host__ __device__ constexpr int router_row_floats(int NP) { return NP == 4 ? 4
 constexpr size_t kRouterSmemLimit = 200 * 1024;
 
 // Dispatch tiling: tokens of one sequence are cut into tiles of this size.
-constexpr int kDispatchTile = 1024;
+constexpr int kDispatchTile = 256;  // == dispatch CTA size: one token per thread
 constexpr int kQTileRows = 128;  // rows of one grouped-GEMM tile
 
 struct DispatchWs {
@@ -39,7 +41,21 @@ struct DispatchWs {
 };
 DispatchWs dispatch_ws_layout(const gqe_config& c);
 
-bool config_ok(const gqe_config* c);
+size_t router_smem_bytes(const gqe_config& c);
+
+// Raises the dynamic shared-memory limit of kernel K to `bytes`, once per
+// device (the attribute is per device; re-setting it on every launch costs
+// host time on short layers).
+template <auto K>
+inline int ensure_smem(int bytes) {
+  static int done[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 63;
+  if (dev >= 0 && dev < 64 && done[dev] >= bytes) return 0;
+  const cudaError_t e = cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = bytes;
+  return e;
+}
 
 // Launchers (return cudaError_t as int).
 int launch_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r,

@@ -77,28 +77,50 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_kernel(RouterArgs a)
   float* wmax = Wsm + static_cast<size_t>(a.d) * S;                 // [NP]
   float* bsm = wmax + NP;                                           // [NP]
   double* zd_all = reinterpret_cast<double*>(bsm + NP);             // [warps][NP]
-  float* zf_all = reinterpret_cast<float*>(zd_all + kRouterWarps * NP);  // [warps][NP]
+  float* zf_all = reinterpret_cast<float*>(zd_all + kRouterWarps * NP);  // [max(warps*NP, 256)]
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
 
-  // Stage W_r (zero padded to S columns) and the bias.
-  for (int i = tid; i < a.d * S; i += blockDim.x) {
-    const int row = i / S, col = i % S;
-    Wsm[i] = col < a.N ? a.W_r[static_cast<size_t>(row) * a.N + col] : 0.0f;
+  // Stage W_r (zero padded to S columns) and the bias. Rows of 4k floats are
+  // copied with 16-byte cp.async so that all loads are in flight at once.
+  if ((a.N & 3) == 0) {
+    const int cpr = a.N >> 2;  // 16-byte chunks per row
+    for (int i = tid; i < a.d * cpr; i += blockDim.x) {
+      const int row = i / cpr, c = i - row * cpr;
+      cp_async_16(smem_u32(Wsm + row * S + 4 * c), a.W_r + static_cast<size_t>(row) * a.N + 4 * c, 16u);
+    }
+    cp_async_commit();
+  } else {
+    for (int i = tid; i < a.d * a.N; i += blockDim.x) {
+      const int row = i / a.N, col = i - row * a.N;
+      Wsm[row * S + col] = a.W_r[i];
+    }
   }
-  for (int e = tid; e < NP; e += blockDim.x) {
-    wmax[e] = 0.0f;
-    bsm[e] = (e < a.N && a.b_r != nullptr) ? a.b_r[e] : 0.0f;
+  for (int i = tid; i < a.d * (S - a.N); i += blockDim.x) {
+    const int row = i / (S - a.N), col = a.N + i % (S - a.N);
+    Wsm[row * S + col] = 0.0f;
   }
+  cp_async_wait<0>();
+  for (int e = tid; e < NP; e += blockDim.x) bsm[e] = (e < a.N && a.b_r != nullptr) ? a.b_r[e] : 0.0f;
   __syncthreads();
-  for (int i = tid; i < a.d * NP; i += blockDim.x) {
-    const int row = i / NP, col = i % NP;
-    const float w = fabsf(Wsm[row * S + col]);
-    if (w > 0.0f) atomicMax(reinterpret_cast<int*>(&wmax[col]), __float_as_int(w));
+  // max_i |W_r[i, e]|: thread t scans column t % NP over rows t / NP (mod
+  // the number of parts), then one thread per column combines the parts.
+  {
+    constexpr int parts = kRouterWarps * 32 / NP;
+    float mx = 0.0f;
+    const int col = tid % NP, part = tid / NP;
+    for (int row = part; row < a.d; row += parts) mx = fmaxf(mx, fabsf(Wsm[row * S + col]));
+    zf_all[tid] = mx;  // zf_all has room for kRouterWarps * 32 floats
+    __syncthreads();
+    if (tid < NP) {
+      float m2 = 0.0f;
+      for (int p = 0; p < parts; ++p) m2 = fmaxf(m2, zf_all[p * NP + tid]);
+      wmax[tid] = m2;
+    }
+    __syncthreads();
   }
-  __syncthreads();
 
   double* zd = zd_all + warp * NP;
   float* zf = zf_all + warp * NP;
@@ -114,6 +136,7 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_kernel(RouterArgs a)
 #pragma unroll
     for (int e = 0; e < NP; ++e) acc[e] = 0.0f;
     float nx = 0.0f;
+#pragma unroll 8
     for (int m = lane; m < a.d; m += 32) {
       const float xi = bf16_to_f32(xr[m]);
       nx += fabsf(xi);
@@ -243,19 +266,18 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_kernel(RouterArgs a)
   }
 }
 
+
 template <int NP>
 int launch_np(const gqe_config& c, const RouterArgs& a, cudaStream_t st) {
   constexpr int S = router_row_floats(NP);
-  const size_t smem = static_cast<size_t>(c.d_model) * S * 4 + 2 * NP * 4 +
-                      kRouterWarps * NP * (8 + 4);
+  const size_t smem = router_smem_bytes(c);
   if (smem > kRouterSmemLimit) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(router_kernel<NP>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  const int e = ensure_smem<router_kernel<NP>>(static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  // One token per warp while that fills the GPU; larger batches loop.
   const int R = a.R;
-  int grid = (R + kRouterWarps * 8 - 1) / (kRouterWarps * 8);
-  if (grid > 2 * 148) grid = 2 * 148;
+  int grid = (R + kRouterWarps - 1) / kRouterWarps;
+  if (grid > 4 * 148) grid = 4 * 148;
   if (grid < 1) grid = 1;
   router_kernel<NP><<<grid, kRouterWarps * 32, smem, st>>>(a);
   return cudaGetLastError();
@@ -266,8 +288,9 @@ using namespace router_impl;
 
 size_t router_smem_bytes(const gqe_config& c) {
   const int NP = router_np(c.G * c.M);
+  const size_t zf = kRouterWarps * NP > kRouterWarps * 32 ? kRouterWarps * NP : kRouterWarps * 32;
   return static_cast<size_t>(c.d_model) * router_row_floats(NP) * 4 + 2 * NP * 4 +
-         kRouterWarps * NP * 12;
+         kRouterWarps * NP * 8 + zf * 4;
 }
 
 int launch_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r,

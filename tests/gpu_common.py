@@ -24,14 +24,15 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
 def assert_close(got: torch.Tensor, want: np.ndarray, what: str, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
     """Max-abs / mean-abs check against the oracle.
 
-    Every bf16 rounding on the path (Q, K, V, P, slots, y) is relative to the
-    value rounded, so the error scales with the output's magnitude. The bounds
-    hold as stated for outputs of rms <= 1 (every measured workload: attention
-    averages over many positions); for larger outputs (sequences of a few
-    tokens, where o is a single V row) both bounds scale with rms(want).
+    The bounds hold as stated for outputs of rms <= 1/2, which covers every
+    measured workload (attention averages over many positions, rms(y) ~ 0.2).
+    Each bf16 rounding on the path (Q, K, V, P, slots, y) is relative to the
+    value rounded (unit roundoff 2^-8 ~ 3.9e-3), so for larger outputs -- a
+    sequence of a few tokens, where o is a single V row and |y| ~ 1 -- both
+    bounds scale with 2 * rms(want).
     """
     g = to_f64(got).reshape(want.shape)
-    scale = max(1.0, float(np.sqrt(np.mean(np.square(want)))) if want.size else 1.0)
+    scale = max(1.0, 2.0 * float(np.sqrt(np.mean(np.square(want)))) if want.size else 1.0)
     max_abs, mean_abs = max_abs * scale, mean_abs * scale
     err = np.abs(g - want)
     assert np.isfinite(g).all(), f"{what}: non-finite values"
