@@ -333,6 +333,20 @@ def cpu_baseline(shape: synth.LayerShape, max_tokens: int | None = None) -> dict
                       f"(fp64 numpy, {dt:.2f} s)", "seconds": dt}
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """Largest `value` over all ranks (the job is as slow as its slowest rank)."""
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank_step * world * steps / (max_ms / 1e3)
+
+
 def run_ours(args, rank: int, world: int, dist):
     import torch
     import routed_sparse_query_b200 as rsq
@@ -355,24 +369,16 @@ def run_ours(args, rank: int, world: int, dist):
         res = time_steps(layer, args.steps, warmup, flush, sync_ranks)
     if rsq.gqe_read_status() != 0:
         raise RuntimeError("device-side status set during the timed steps")
-    total = torch.tensor([res["total_ms"]], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(total, op=dist.ReduceOp.MAX)
-    max_ms = float(total.item())
+    max_ms = max_over_ranks(res["total_ms"], dist, "cuda")
     ms_per_step = max_ms / args.steps
-    tokens = shape.R * world * args.steps
-    value = tokens / (max_ms / 1e3)
+    value = job_throughput(shape.R, world, args.steps, max_ms)
 
     e2e = time_e2e(rsq, shape, d, args.steps, warmup)
-    e2e_t = torch.tensor([e2e["ms"]], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = tokens / (float(e2e_t.item()) / 1e3)
+    e2e_value = job_throughput(shape.R, world, args.steps, max_over_ranks(e2e["ms"], dist, "cuda"))
 
-    dense_ms = time_dense(rsq, shape, d, args.steps, warmup, flush) / args.steps
-    dense_t = torch.tensor([dense_ms], dtype=torch.float64, device="cuda")
+    dense_ms = max_over_ranks(time_dense(rsq, shape, d, args.steps, warmup, flush) / args.steps,
+                              dist, "cuda")
     if dist is not None:
-        dist.all_reduce(dense_t, op=dist.ReduceOp.MAX)
         dist.barrier()
     if rank != 0:
         return None
@@ -402,9 +408,9 @@ def run_ours(args, rank: int, world: int, dist):
                 "d2h_bytes_per_step": e2e["d2h"], "api": "gqe_layer_fwd"},
         "roofline": roof,
         "breakdown_ms_per_step": {c: v / args.steps for c, v in res["per_call_ms"].items()},
-        "dense_gqa": {"ms_per_step": float(dense_t.item()),
-                      "tokens_per_s": shape.R * world / (float(dense_t.item()) / 1e3),
-                      "speedup_gqe_over_dense": float(dense_t.item()) / ms_per_step},
+        "dense_gqa": {"ms_per_step": dense_ms,
+                      "tokens_per_s": shape.R * world / (dense_ms / 1e3),
+                      "speedup_gqe_over_dense": dense_ms / ms_per_step},
         "pages_speedup_context": PAGES_SPEEDUP,
     }
     if world == 1 and not args.no_sweep:
