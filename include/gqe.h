@@ -135,6 +135,26 @@ gqe_status gqe_dispatch(const gqe_config* cfg, const int32_t* idx, const gqe_bf1
                         gqe_bf16* Qs, void* ws, size_t ws_bytes, gqe_stream_t stream);
 
 /*
+ * gqe_dispatch without a workspace argument (the paper has no counterpart:
+ * this is a calling convention of this library). For callers that cannot
+ * allocate device memory per call -- their memory belongs to another
+ * allocator, e.g. a serving runtime that reserves the GPU at start-up or a
+ * plugin interface that passes only input and output buffers. The scratch
+ * lives in a 4 MiB static device array of the library (held by every GPU that
+ * loads it, until exit); arguments and results are those of gqe_dispatch.
+ *  - The first call on a device looks up the array's address on that device;
+ *    make it before any stream capture.
+ *  - All calls on a device share the array: calls that overlap on the GPU
+ *    race. Each call writes every scratch word before reading it.
+ *  - Configurations needing more than 4 MiB of dispatch scratch
+ *    (gqe_workspace_bytes(cfg, GQE_WS_DISPATCH)) return GQE_ERR_WORKSPACE.
+ */
+gqe_status gqe_dispatch_noalloc(const gqe_config* cfg, const int32_t* idx, const gqe_bf16* x,
+                                const gqe_bf16* W_q, const gqe_bf16* W_qs, int32_t* counts,
+                                int32_t* offsets, int32_t* tok, int32_t* slot_pos,
+                                gqe_bf16* Qv, gqe_bf16* Qs, gqe_stream_t stream);
+
+/*
  * Dense, unchanged K/V projection of every group (step a6; "the Key-Value
  * projections and the KV cache stay dense and unchanged": gist.science
  * "Technical Summary", Dense KV path). The dense GQA path uses this same call.

@@ -32,7 +32,7 @@ ITEMS = {"idx": 1, "r": 2, "omega": 3, "counts": 4, "offsets": 5, "tok": 6, "slo
 EXPORTED = ("gqe_workspace_bytes", "gqe_workspace_offset", "gqe_router_topk", "gqe_dispatch",
             "gqe_kv_proj", "gqe_attention_fwd", "gqe_output_proj", "gqe_layer_fwd",
             "gqa_dense_fwd", "gqe_read_status", "gqe_selftest_wait_timeout",
-            "gqe_status_string", "gqe_version")
+            "gqe_status_string", "gqe_version", "gqe_dispatch_noalloc")
 
 
 class GQEConfig(ctypes.Structure):
@@ -60,6 +60,7 @@ _sig = {
     "gqe_router_topk": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
     "gqe_dispatch": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                     ctypes.c_size_t, _P]),
+    "gqe_dispatch_noalloc": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "gqe_kv_proj": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),
     "gqe_attention_fwd": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),
     "gqe_output_proj": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P]),
@@ -123,6 +124,15 @@ def gqe_dispatch(cfg, idx, x, W_q, W_qs, counts, offsets, tok, slot_pos, Qv, Qs,
                              _ptr(offsets), _ptr(tok), _ptr(slot_pos), _ptr(Qv), _ptr(Qs),
                              _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "gqe_dispatch")
+
+
+def gqe_dispatch_noalloc(cfg, idx, x, W_q, W_qs, counts, offsets, tok, slot_pos, Qv, Qs,
+                         stream=None):
+    """gqe_dispatch for callers that cannot allocate a workspace: the scratch is
+    a fixed device array of the library (see include/gqe.h)."""
+    _check(_lib.gqe_dispatch_noalloc(_cfg(cfg), _ptr(idx), _ptr(x), _ptr(W_q), _ptr(W_qs),
+                                     _ptr(counts), _ptr(offsets), _ptr(tok), _ptr(slot_pos),
+                                     _ptr(Qv), _ptr(Qs), _stream(stream)), "gqe_dispatch_noalloc")
 
 
 def gqe_kv_proj(cfg, x, W_k, W_v, K, V, stream=None):

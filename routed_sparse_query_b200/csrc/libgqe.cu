@@ -5,3 +5,4 @@
 #include "gemm.cu"
 #include "attention.cu"
 #include "api.cu"
+#include "noalloc.cu"
