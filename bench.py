@@ -40,6 +40,7 @@ WORKLOADS = {
     "seq32k": synth.SEQ32K,
     "seq256k": synth.SEQ256K,
     "seq1m": synth.SEQ1M,
+    "seq64k": synth.LayerShape(B=1, T=65536, d_model=1024, G=8, M=2, k=1, d_head=64),
     "pool4_k1": synth.POOL4_K1,
     "pool4_k2": synth.POOL4_K2,
 }

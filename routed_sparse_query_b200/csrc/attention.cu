@@ -52,7 +52,7 @@ struct AttnCfg {
   static constexpr int P_BYTES = BQ * BKV * 2;
   static constexpr size_t SMEM =
       1024 + static_cast<size_t>(TILE_BYTES) * (2 + 2 * KV_STAGES) + 2 * P_BYTES + 512;
-  static constexpr uint32_t TMEM_COLS = 512;  // S_a, S_b (128 each), O_a, O_b (DH each)
+  static constexpr uint32_t TMEM_COLS = 512;  // 3 rotating S buffers (128 each), O_a, O_b (DH each)
 };
 
 struct AttnParams {
@@ -124,28 +124,50 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 // visible iff x <= lim. O (tO) is rescaled only when the max grows by more
 // than kRescaleLog2.
 template <int DH, bool MASK>
-__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint8_t* prow, int i,
-                                             int lim, float sc, bool first, float& m, float& l) {
+__device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, uint8_t* prow, int i,
+                                             int lim, float sc, bool first, float& m, float& l,
+                                             uint64_t* pv_prev, uint32_t pv_parity,
+                                             volatile int* abort_flag) {
+  // TMEM loads are software-pipelined: chunk c+1 (32 columns) is in flight
+  // while chunk c is processed.
   float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  auto row_max = [&](const uint32_t (&v)[32], int c) {
 #pragma unroll
-  for (int c = 0; c < BKV / 64; ++c) {
-    uint32_t v[64];
-    tmem_ld64(tS + c * 64, v);
-#pragma unroll
-    for (int x = 0; x < 64; x += 8) {
+    for (int x = 0; x < 32; x += 8) {
       float a[8];
 #pragma unroll
       for (int y = 0; y < 8; ++y) {
         a[y] = __uint_as_float(v[x + y]);
-        if (MASK && c * 64 + x + y > lim) a[y] = -INFINITY;
+        if (MASK && c * 32 + x + y > lim) a[y] = -INFINITY;
       }
       mx[0] = max3(mx[0], a[0], a[4]);
       mx[1] = max3(mx[1], a[1], a[5]);
       mx[2] = max3(mx[2], a[2], a[6]);
       mx[3] = max3(mx[3], a[3], a[7]);
     }
-  }
+  };
+  uint32_t va[32], vb[32];
+  tmem_ld32_nowait(tS + 0, va);
+  tmem_ld_wait(va);
+  tmem_ld32_nowait(tS + 32, vb);
+  row_max(va, 0);
+  tmem_ld_wait(vb);
+  tmem_ld32_nowait(tS + 64, va);
+  row_max(vb, 1);
+  tmem_ld_wait(va);
+  tmem_ld32_nowait(tS + 96, vb);
+  row_max(va, 2);
+  tmem_ld_wait(vb);
+  tmem_ld32_nowait(tS + 0, va);  // first chunk of pass 2
+  row_max(vb, 3);
+
   const float mc = fmaxf(max3(mx[0], mx[1], mx[2]), mx[3]) * sc;
+  if (pv_prev != nullptr &&
+      !__all_sync(0xffffffffu, mbar_wait(pv_prev, pv_parity, abort_flag))) {
+    tmem_ld_wait(va);
+    return false;
+  }
+  tc_fence_after();
   const bool need = mc > m + kRescaleLog2;
   if (__any_sync(0xffffffffu, need)) {
     const float m_new = need ? mc : m;
@@ -165,11 +187,9 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint8_t* 
     m = m_new;
   }
   const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m, -m);
-  float2 lsum = make_float2(0.0f, 0.0f);
-#pragma unroll
-  for (int c = 0; c < BKV / 32; ++c) {
-    uint32_t v[32];
-    tmem_ld32(tS + c * 32, v);
+  float2 lsum[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                    make_float2(0.0f, 0.0f)};  // independent partial sums (no serial chain)
+  auto exp_chunk = [&](const uint32_t (&v)[32], int c) {
 #pragma unroll
     for (int c8 = 0; c8 < 4; ++c8) {
       const int c16 = c * 4 + c8;  // 8-key chunk index in the row
@@ -194,7 +214,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint8_t* 
         }
         e8[x] = e.x;
         e8[x + 1] = e.y;
-        lsum = fadd2(lsum, e);
+        lsum[x >> 1] = fadd2(lsum[x >> 1], e);
       }
       uint4 o;
       o.x = pack_bf16x2(e8[0], e8[1]);
@@ -204,8 +224,37 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint8_t* 
       const int kc = c16 >> 3, cw = c16 & 7;
       *reinterpret_cast<uint4*>(prow + kc * (BQ * 128) + ((cw ^ (i & 7)) << 4)) = o;
     }
+  };
+  tmem_ld_wait(va);
+  tmem_ld32_nowait(tS + 32, vb);
+  exp_chunk(va, 0);
+  tmem_ld_wait(vb);
+  tmem_ld32_nowait(tS + 64, va);
+  exp_chunk(vb, 1);
+  tmem_ld_wait(va);
+  tmem_ld32_nowait(tS + 96, vb);
+  exp_chunk(va, 2);
+  tmem_ld_wait(vb);
+  exp_chunk(vb, 3);
+  const float2 l01 = fadd2(lsum[0], lsum[1]), l23 = fadd2(lsum[2], lsum[3]);
+  const float2 l4 = fadd2(l01, l23);
+  l += l4.x + l4.y;
+  return true;
+}
+
+// Item n of a CTA's S sequence: (a,0), (b,0), (a,1), (b,1), ..., and tile b's
+// extra diagonal tile last; tile a alone when the CTA has no tile b.
+__device__ __forceinline__ void seq_item(int n, bool has_b, int nkv_a, int& t, int& j) {
+  if (!has_b) {
+    t = 0;
+    j = n;
+  } else if (n < 2 * nkv_a) {
+    t = n & 1;
+    j = n >> 1;
+  } else {
+    t = 1;
+    j = nkv_a;
   }
-  l += lsum.x + lsum.y;
 }
 
 template <int DH>
@@ -226,8 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_full = bar + 1;
   uint64_t* v_full = k_full + KV_STAGES;
   uint64_t* kv_empty = v_full + KV_STAGES;
-  uint64_t* s_full = kv_empty + KV_STAGES;  // [2]
-  uint64_t* p_full = s_full + 2;            // [2]
+  uint64_t* s_full = kv_empty + KV_STAGES;  // [3] one per S buffer
+  uint64_t* p_full = s_full + 3;            // [2] one per query tile
   uint64_t* o_done = p_full + 2;            // [2]
   uint64_t* drain = o_done + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -257,7 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int zkv = b * p.G + grp;
   const int qt0 = 2 * pair;
   const bool has_b = qt0 + 1 < p.n_qt;
-  const int nkv_t[2] = {qt0 + 1, has_b ? qt0 + 2 : 0};  // causal: KV tiles 0..qt
+  // causal: query tile qt needs KV tiles 0..qt; tile a = qt0, tile b = qt0 + 1
+  const int nkv_a = qt0 + 1, nkv_b = has_b ? qt0 + 2 : 0;
   const int nkv = has_b ? qt0 + 2 : qt0 + 1;
 
   if (threadIdx.x == 0) {
@@ -267,8 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
+    for (int b3 = 0; b3 < 3; ++b3) mbar_init(&s_full[b3], 1);
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 128);
       mbar_init(&o_done[t], 1);
     }
@@ -305,83 +355,103 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- UMMA issuer
-    // Order per KV tile j: PV_a(j), S_a(j+1), PV_b(j), S_b(j+1): the tensor
-    // core works on one tile while the other tile's softmax runs.
-    if (lane == 0) {
+    // S tiles are computed in sequence n = 0, 1, 2, ... ((a,0), (b,0),
+    // (a,1), (b,1), ...) into TMEM buffer n % 3. Once the softmax of item m
+    // has published P (so it has finished reading S(m)), the issuer computes
+    // PV of item m and then S(m+3) into that buffer, so every tile's next S
+    // is ready while its current softmax runs. The whole warp runs this
+    // loop; elect.sync picks the lane that issues.
+    {
       constexpr uint32_t idS = idesc_bf16_f32(BQ, BKV, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(BQ, DH, 0, 1);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-      auto issue_S = [&](int t, int st) {
+      // Descriptors are built once; an operand at a byte offset from its base
+      // is the base descriptor plus (offset >> 4) in the start-address field
+      // (shared-memory addresses stay below 2^18, so the field never carries).
+      const uint64_t dQ = smem_desc(smem_u32(sQ), 16, 8 * C::SWB, C::LAYOUT);
+      const uint64_t dK = smem_desc(smem_u32(sK), 16, 8 * C::SWB, C::LAYOUT);
+      const uint64_t dV = smem_desc(smem_u32(sV), C::TILE_BYTES, 8 * C::SWB, C::LAYOUT);
+      const uint64_t dP = smem_desc(smem_u32(sP), 16, 1024, kLayoutSW128);
+      auto wait_all = [&](uint64_t* b, uint32_t par) {
+        return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag));
+      };
+      auto issue_S = [&](int n) -> bool {
+        int t, j;
+        seq_item(n, has_b, nkv_a, t, j);
+        const int st = j % KV_STAGES;
+        if (!wait_all(&k_full[st], (j / KV_STAGES) & 1)) return false;
+        tc_fence_after();
+        const uint64_t q0 = dQ + static_cast<uint64_t>((t * C::TILE_BYTES) >> 4);
+        const uint64_t k0 = dK + static_cast<uint64_t>((st * C::TILE_BYTES) >> 4);
+        const uint32_t d = tmem + (n % 3) * 128;
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk)
-          umma_bf16_ss(tmem + t * 128,
-                       smem_desc(aQ + t * C::TILE_BYTES + kk * 32, 16, 8 * C::SWB, C::LAYOUT),
-                       smem_desc(aK + st * C::TILE_BYTES + kk * 32, 16, 8 * C::SWB, C::LAYOUT),
-                       idS, kk > 0 ? 1u : 0u);
-        umma_commit(&s_full[t]);
+          umma_bf16_ss_elect(d, q0 + 2 * kk, k0 + 2 * kk, idS, kk > 0 ? 1u : 0u);
+        umma_commit_elect(&s_full[n % 3]);
+        return true;
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_S(0, 0);
-        if (has_b) issue_S(1, 0);
-      }
-      for (int j = 0; ok && j < nkv; ++j) {
+      const int n_total = has_b ? 2 * nkv_a + 1 : nkv_a;
+      bool ok = wait_all(q_full, 0);
+      for (int n = 0; ok && n < 3 && n < n_total; ++n) ok = issue_S(n);
+      for (int m = 0; ok && m < n_total; ++m) {
+        int t, j;
+        seq_item(m, has_b, nkv_a, t, j);
         const int st = j % KV_STAGES;
-        bool v_ready = false;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= nkv_t[t]) continue;
-          if (!mbar_wait(&p_full[t], j & 1, abort_flag)) { ok = false; break; }
-          if (!v_ready) {
-            if (!mbar_wait(&v_full[st], (j / KV_STAGES) & 1, abort_flag)) { ok = false; break; }
-            v_ready = true;
-          }
-          tc_fence_after();
-          const uint32_t pb = aP + t * C::P_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk)
-            umma_bf16_ss(tmem + 256 + t * DH,
-                         smem_desc(pb + (kk >> 2) * (BQ * 128) + (kk & 3) * 32, 16, 1024,
-                                   kLayoutSW128),
-                         smem_desc(aV + st * C::TILE_BYTES + kk * 16 * C::SWB, C::TILE_BYTES,
-                                   8 * C::SWB, C::LAYOUT),
-                         idO, (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&o_done[t]);
-          if (j + 1 < nkv_t[t]) {
-            const int st1 = (j + 1) % KV_STAGES;
-            if (!mbar_wait(&k_full[st1], ((j + 1) / KV_STAGES) & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            issue_S(t, st1);
-          }
+        if (!wait_all(&p_full[t], j & 1) || !wait_all(&v_full[st], (j / KV_STAGES) & 1)) {
+          ok = false;
+          break;
         }
-        if (ok) umma_commit(&kv_empty[st]);
+        tc_fence_after();
+        const uint64_t p0 = dP + static_cast<uint64_t>((t * C::P_BYTES) >> 4);
+        const uint64_t v0 = dV + static_cast<uint64_t>((st * C::TILE_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          umma_bf16_ss_elect(tmem + 384 + t * DH, p0 + ((kk >> 2) * (BQ * 128) + (kk & 3) * 32) / 16,
+                             v0 + (kk * 16 * C::SWB) / 16, idO, (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit_elect(&o_done[t]);
+        if (t == 1 || !has_b) umma_commit_elect(&kv_empty[st]);  // last reader of K_j, V_j
+        // S(m+3) follows PV(m): with one tile it needs K_{j+3}, which shares a
+        // stage with V_j (measured: issuing S first is not faster with two).
+        if (m + 3 < n_total) ok = issue_S(m + 3);
       }
-      umma_commit(drain);
+      umma_commit_elect(drain);
     }
-    __syncwarp();
   } else {
     // ---------------------------------------------------------- softmax
     const int t = warp >> 2;            // 0: tile a, 1: tile b
     const int i = threadIdx.x & 127;    // row in tile = TMEM lane
-    const int n_t = nkv_t[t];
+    const int n_t = t == 0 ? nkv_a : nkv_b;
     const int qi = (qt0 + t) * BQ + i;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + t * 128 + lane_off;
-    const uint32_t tO = tmem + 256 + t * DH + lane_off;
+    const uint32_t tO = tmem + 384 + t * DH + lane_off;
     uint8_t* prow = sP + t * C::P_BYTES + i * 128;
     const float sc = p.scale_log2;
     float m = -INFINITY, l = 0.0f;
     bool ok = n_t > 0;
     for (int j = 0; ok && j < n_t; ++j) {
+      // This tile's S for KV tile j is sequence item n, in TMEM buffer n % 3.
+      const int n = has_b ? (j < nkv_a ? 2 * j + t : 2 * nkv_a) : j;
+      const uint32_t tS = tmem + (n % 3) * 128 + lane_off;
       // Waits are made warp-uniform: tcgen05.ld/st below are .sync.aligned.
-      bool w = mbar_wait(&s_full[t], j & 1, abort_flag);
-      if (j > 0) w = mbar_wait(&o_done[t], (j - 1) & 1, abort_flag) && w;
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[n % 3], (n / 3) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
+      // PV of the previous KV tile must be complete before O is rescaled and
+      // before this tile's single P buffer is overwritten; softmax_tile waits
+      // for it after its max pass.
+      uint64_t* pv_prev = j > 0 ? &o_done[t] : nullptr;
+      bool w_ok = true;
       if (j == n_t - 1)
-        softmax_tile<DH, true>(tS, tO, prow, i, qi - j * BKV, sc, j == 0, m, l);
+        w_ok = softmax_tile<DH, true>(tS, tO, prow, i, qi - j * BKV, sc, j == 0, m, l, pv_prev,
+                                      (j - 1) & 1, abort_flag);
       else
-        softmax_tile<DH, false>(tS, tO, prow, i, BKV, sc, j == 0, m, l);
+        w_ok = softmax_tile<DH, false>(tS, tO, prow, i, BKV, sc, j == 0, m, l, pv_prev,
+                                       (j - 1) & 1, abort_flag);
+      if (!w_ok) {
+        ok = false;
+        break;
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[t]);

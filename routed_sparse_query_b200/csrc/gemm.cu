@@ -150,27 +150,27 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 1);
-      const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % C::STAGES;
-        const uint32_t ph = (kb / C::STAGES) & 1;
-        if (!mbar_wait(&full[s], ph, abort_flag)) break;
-        tc_fence_after();
+    // The whole warp runs the issue loop; elect.sync picks the issuing lane.
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 1);
+    // Base descriptors built once; stage / k offsets are added to the
+    // start-address field (units of 16 bytes; addresses stay below 2^18).
+    const uint64_t dA = smem_desc(smem_u32(sA), 16, 1024, kLayoutSW128);
+    const uint64_t dB = smem_desc(smem_u32(sB), BK * C::B_SWB, 8 * C::B_SWB, C::B_LAYOUT);
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % C::STAGES;
+      const uint32_t ph = (kb / C::STAGES) & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag))) break;
+      tc_fence_after();
+      const uint64_t a0 = dA + static_cast<uint64_t>((s * C::A_BYTES) >> 4);
+      const uint64_t b0 = dB + static_cast<uint64_t>((s * C::B_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = smem_desc(a0 + s * C::A_BYTES + kk * 32, 16, 1024, kLayoutSW128);
-          const uint64_t bd = smem_desc(b0 + s * C::B_BYTES + kk * 16 * C::B_SWB, BK * C::B_SWB,
-                                        8 * C::B_SWB, C::B_LAYOUT);
-          umma_bf16_ss(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-        }
-        umma_commit(&empty[s]);
-      }
-      umma_commit(accb);
-      umma_commit(drain);
+      for (int kk = 0; kk < BK / 16; ++kk)
+        umma_bf16_ss_elect(tmem, a0 + 2 * kk, b0 + (kk * 16 * C::B_SWB) / 16, idesc,
+                           (kb | kk) != 0 ? 1u : 0u);
+      umma_commit_elect(&empty[s]);
     }
-    __syncwarp();
+    umma_commit_elect(accb);
+    umma_commit_elect(drain);
   } else {
     const int q = warp & 3;
     if (GATHER) {
