@@ -162,6 +162,7 @@ class Layer:
         self.slots = e(R, s.n_slots * dh, dtype=torch.bfloat16, device=dev)
         self.y = e(R, s.d_model, dtype=torch.bfloat16, device=dev)
         self.wsd = e(rsq.gqe_workspace_bytes(self.cfg, rsq.GQE_WS_DISPATCH), dtype=torch.uint8, device=dev)
+        self.wsa = e(rsq.gqe_workspace_bytes(self.cfg, rsq.GQE_WS_ATTENTION), dtype=torch.uint8, device=dev)
 
     def router(self):
         d = self.d
@@ -177,7 +178,7 @@ class Layer:
         self.rsq.gqe_kv_proj(self.cfg, d["x"], d["W_k"], d["W_v"], self.K, self.V)
 
     def attention(self):
-        self.rsq.gqe_attention_fwd(self.cfg, self.Qv, self.Qs, self.K, self.V, self.slots)
+        self.rsq.gqe_attention_fwd(self.cfg, self.Qv, self.Qs, self.K, self.V, self.slots, self.wsa)
 
     def output(self):
         self.rsq.gqe_output_proj(self.cfg, self.slots, self.omega, self.d["W_o"], self.y)

@@ -69,18 +69,20 @@ typedef enum gqe_status {
 enum {
   GQE_WS_DISPATCH = 1, /* scratch of gqe_dispatch */
   GQE_WS_LAYER = 2,    /* everything gqe_layer_fwd keeps between its steps */
-  GQE_WS_DENSE = 3     /* everything gqa_dense_fwd keeps between its steps */
+  GQE_WS_DENSE = 3,    /* everything gqa_dense_fwd keeps between its steps */
+  GQE_WS_ATTENTION = 4 /* scratch of gqe_attention_fwd (split-KV partials) */
 };
 
 /* Items inside the GQE_WS_LAYER / GQE_WS_DENSE workspaces (for inspection). */
 enum {
   GQE_ITEM_IDX = 1, GQE_ITEM_R, GQE_ITEM_OMEGA, GQE_ITEM_COUNTS, GQE_ITEM_OFFSETS,
   GQE_ITEM_TOK, GQE_ITEM_SLOT_POS, GQE_ITEM_QV, GQE_ITEM_QS, GQE_ITEM_K, GQE_ITEM_V,
-  GQE_ITEM_SLOTS, GQE_ITEM_DISPATCH_WS,
+  GQE_ITEM_SLOTS, GQE_ITEM_DISPATCH_WS, GQE_ITEM_ATTENTION_WS,
   GQE_ITEM_DENSE_Q = 32, GQE_ITEM_DENSE_O
 };
 
-/* Bytes of workspace the given call needs for `cfg` (0 if cfg is invalid). */
+/* Bytes of workspace the given call needs for `cfg` (0 if cfg is invalid;
+ * at least 256 otherwise). */
 size_t gqe_workspace_bytes(const gqe_config* cfg, int which);
 
 /* Byte offset of `item` inside workspace `which`, or (size_t)-1. */
@@ -171,12 +173,16 @@ gqe_status gqe_kv_proj(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16*
  * accumulation, bf16 output written straight into the slot buffer:
  *   slots[row, (g*k+s)*dh ...] routed, slots[row, k*G*dh ...] shared.
  * Slot kG+1 (weighted) is not touched.
+ * Short sequences are split along the keys (each CTA takes a chunk of KV
+ * tiles; the last CTA of a query-tile pair merges the chunks' unnormalised
+ * rows), which needs scratch from ws: >= gqe_workspace_bytes(cfg,
+ * GQE_WS_ATTENTION). Calls sharing one ws must not overlap on the GPU.
  * Qv [B, G, k, T, d_head]; Qs [B, T, d_head]; K, V [B, G, T, d_head];
  * slots [B*T, (k*G+2)*d_head].
  */
 gqe_status gqe_attention_fwd(const gqe_config* cfg, const gqe_bf16* Qv, const gqe_bf16* Qs,
-                             const gqe_bf16* K, const gqe_bf16* V, gqe_bf16* slots,
-                             gqe_stream_t stream);
+                             const gqe_bf16* K, const gqe_bf16* V, gqe_bf16* slots, void* ws,
+                             size_t ws_bytes, gqe_stream_t stream);
 
 /*
  * Weighted slot and output projection (steps a10, a11): the renormalised

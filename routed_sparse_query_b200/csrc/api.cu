@@ -42,7 +42,7 @@ gqe_status check_cfg(const gqe_config* c) {
 gqe_status cuda_status(int e) { return e == cudaSuccess ? GQE_OK : GQE_ERR_CUDA; }
 
 struct LayerWs {
-  size_t idx, r, omega, counts, offsets, tok, slot_pos, Qv, Qs, K, V, slots, dws, total;
+  size_t idx, r, omega, counts, offsets, tok, slot_pos, Qv, Qs, K, V, slots, dws, aws, total;
 };
 
 LayerWs layer_ws(const gqe_config& c) {
@@ -69,12 +69,13 @@ LayerWs layer_ws(const gqe_config& c) {
   put(L.V, R * c.G * dh * 2);
   put(L.slots, R * (c.G * c.k + 2) * dh * 2);
   put(L.dws, dispatch_ws_layout(c).total);
+  put(L.aws, attention_plan(c, c.G * c.k + 1).total);
   L.total = o;
   return L;
 }
 
 struct DenseWs {
-  size_t Q, K, V, O, total;
+  size_t Q, K, V, O, aws, total;
 };
 
 DenseWs dense_ws(const gqe_config& c) {
@@ -91,6 +92,7 @@ DenseWs dense_ws(const gqe_config& c) {
   put(L.K, R * c.G * dh * 2);
   put(L.V, R * c.G * dh * 2);
   put(L.O, R * N * dh * 2);
+  put(L.aws, attention_plan(c, static_cast<int>(N)).total);
   L.total = o;
   return L;
 }
@@ -125,6 +127,10 @@ size_t gqe_workspace_bytes(const gqe_config* cfg, int which) {
     case GQE_WS_DISPATCH: return dispatch_ws_layout(*cfg).total;
     case GQE_WS_LAYER: return layer_ws(*cfg).total;
     case GQE_WS_DENSE: return dense_ws(*cfg).total;
+    case GQE_WS_ATTENTION: {
+      const size_t t = attention_plan(*cfg, cfg->G * cfg->k + 1).total;
+      return t > 256 ? t : 256;
+    }
     default: return 0;
   }
 }
@@ -148,6 +154,7 @@ size_t gqe_workspace_offset(const gqe_config* cfg, int which, int item) {
       case GQE_ITEM_V: return L.V;
       case GQE_ITEM_SLOTS: return L.slots;
       case GQE_ITEM_DISPATCH_WS: return L.dws;
+      case GQE_ITEM_ATTENTION_WS: return L.aws;
       default: return bad;
     }
   }
@@ -203,12 +210,15 @@ gqe_status gqe_kv_proj(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16*
 }
 
 gqe_status gqe_attention_fwd(const gqe_config* cfg, const gqe_bf16* Qv, const gqe_bf16* Qs,
-                             const gqe_bf16* K, const gqe_bf16* V, gqe_bf16* slots,
-                             gqe_stream_t stream) {
+                             const gqe_bf16* K, const gqe_bf16* V, gqe_bf16* slots, void* ws,
+                             size_t ws_bytes, gqe_stream_t stream) {
   const gqe_status s = check_cfg(cfg);
   if (s != GQE_OK) return s;
   if (!all_aligned(Qv, Qs, K, V, slots)) return GQE_ERR_INVALID;
-  return cuda_status(attention_gqe(*cfg, Qv, Qs, K, V, slots, stream));
+  const size_t need = attention_plan(*cfg, cfg->G * cfg->k + 1).total;
+  if (need > 0 && (ws == nullptr || !aligned16(ws))) return GQE_ERR_INVALID;
+  if (ws_bytes < need) return GQE_ERR_WORKSPACE;
+  return cuda_status(attention_gqe(*cfg, Qv, Qs, K, V, slots, ws, ws_bytes, stream));
 }
 
 gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* omega,
@@ -244,7 +254,8 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
   if (st != GQE_OK) return st;
   st = gqe_kv_proj(cfg, x, W_k, W_v, H(L.K), H(L.V), stream);
   if (st != GQE_OK) return st;
-  st = gqe_attention_fwd(cfg, H(L.Qv), H(L.Qs), H(L.K), H(L.V), H(L.slots), stream);
+  st = gqe_attention_fwd(cfg, H(L.Qv), H(L.Qs), H(L.K), H(L.V), H(L.slots), w + L.aws,
+                         L.total - L.aws, stream);
   if (st != GQE_OK) return st;
   return gqe_output_proj(cfg, H(L.slots), F(L.omega), W_o, y, stream);
 }
@@ -267,7 +278,7 @@ gqe_status gqa_dense_fwd(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf1
   if (e != cudaSuccess) return GQE_ERR_CUDA;
   e = gemm_kv(c, x, W_k, W_v, H(L.K), H(L.V), stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
-  e = attention_dense(c, H(L.Q), H(L.K), H(L.V), H(L.O), stream);
+  e = attention_dense(c, H(L.Q), H(L.K), H(L.V), H(L.O), w + L.aws, L.total - L.aws, stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
   const int N = c.G * c.M;
   return cuda_status(gemm_rowmajor(H(L.O), c.B * c.T, N * c.d_head, W_o_dense, c.d_model, y, stream));

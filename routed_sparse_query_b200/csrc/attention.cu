@@ -60,10 +60,15 @@ struct AttnParams {
   int G, k, M;       // groups, selected per group, experts per group
   int dense;         // 0: GQE streams (kG routed + shared), 1: dense GQA heads
   int n_qt;          // 128-row query tiles per stream
-  int n_pairs;       // CTAs per stream: pairs of consecutive query tiles
+  int n_pairs;       // pairs of consecutive query tiles per stream
+  int chunk;         // KV tiles per CTA (split-KV); >= n_qt: no split
+  int items;         // CTAs per stream
   uint16_t* out;     // [B*T, ldo]
   int ldo;
   float scale_log2;  // log2(e) / sqrt(dh)
+  float* part;       // split-KV partial O: [B*H][items][2][128][dh] fp32
+  float2* part_ml;   // split-KV partial (m, l): [B*H][items][2][128]
+  int* counters;     // split-KV arrivals per (stream, pair), zero between calls
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -242,18 +247,37 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, uint8_t* 
   return true;
 }
 
-// Item n of a CTA's S sequence: (a,0), (b,0), (a,1), (b,1), ..., and tile b's
-// extra diagonal tile last; tile a alone when the CTA has no tile b.
-__device__ __forceinline__ void seq_item(int n, bool has_b, int nkv_a, int& t, int& j) {
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Stores 32 fp32 values times `scale` as bf16 (64 contiguous bytes).
+__device__ __forceinline__ void store_row32(uint16_t* dst, const uint32_t (&v)[32], float scale) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint4 o;
+    o.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * scale, __uint_as_float(v[8 * q4 + 1]) * scale);
+    o.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * scale, __uint_as_float(v[8 * q4 + 3]) * scale);
+    o.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * scale, __uint_as_float(v[8 * q4 + 5]) * scale);
+    o.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * scale, __uint_as_float(v[8 * q4 + 7]) * scale);
+    d4[q4] = o;
+  }
+}
+
+// Item n of a CTA's S sequence over its KV tiles j0..: (a,j0), (b,j0),
+// (a,j0+1), (b,j0+1), ..., and tile b's extra diagonal tile last; tile a
+// alone when the CTA has no tile b. na = tile a's KV tiles in the CTA.
+__device__ __forceinline__ void seq_item(int n, bool has_b, int j0, int na, int& t, int& j) {
   if (!has_b) {
     t = 0;
-    j = n;
-  } else if (n < 2 * nkv_a) {
+    j = j0 + n;
+  } else if (n < 2 * na) {
     t = n & 1;
-    j = n >> 1;
+    j = j0 + (n >> 1);
   } else {
     t = 1;
-    j = nkv_a;
+    j = j0 + na;
   }
 }
 
@@ -281,11 +305,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = o_done + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  volatile int* s_last = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
-  const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;  // longest first
   const int bh = static_cast<int>(blockIdx.x) % BH;
+  // Work item: (stream bh, query-tile pair, KV chunk), longest pairs first.
+  int ord = static_cast<int>(blockIdx.x) / BH;
+  int pair, chunk_id = 0, n_chunks = 1, item_base = ord;
+  if (p.chunk >= p.n_qt) {
+    pair = p.n_pairs - 1 - ord;
+  } else {
+    item_base = 0;
+    for (pair = p.n_pairs - 1; pair > 0; --pair) {
+      const int nc = (2 * pair + 1 + p.chunk - 1) / p.chunk;
+      if (ord < nc) break;
+      ord -= nc;
+      item_base += nc;
+    }
+    n_chunks = (2 * pair + 1 + p.chunk - 1) / p.chunk;
+    chunk_id = ord;
+  }
   const int b = bh / p.H, h = bh % p.H;
   int zq, grp, slot;
   const CUtensorMap* tq = &tmQ;
@@ -306,9 +346,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int zkv = b * p.G + grp;
   const int qt0 = 2 * pair;
   const bool has_b = qt0 + 1 < p.n_qt;
-  // causal: query tile qt needs KV tiles 0..qt; tile a = qt0, tile b = qt0 + 1
-  const int nkv_a = qt0 + 1, nkv_b = has_b ? qt0 + 2 : 0;
-  const int nkv = has_b ? qt0 + 2 : qt0 + 1;
+  // Causal: query tile qt needs KV tiles 0..qt (tile a = qt0, tile b = qt0+1).
+  // This CTA takes KV tiles [j0, ja1) for tile a and [j0, jb1) for tile b;
+  // the last chunk also holds tile b's extra diagonal tile.
+  const int j0 = chunk_id * (p.chunk < p.n_qt ? p.chunk : 0);
+  const bool last_chunk = chunk_id == n_chunks - 1;
+  const int ja1 = last_chunk ? qt0 + 1 : j0 + p.chunk;
+  const int jb1 = has_b ? (last_chunk ? qt0 + 2 : ja1) : j0;
+  const int na = ja1 - j0;
+  const int jend = has_b ? jb1 : ja1;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -343,9 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(q_full, C::TILE_BYTES * (has_b ? 2 : 1));
       tma_load_3d(sQ, tq, q_full, 0, qt0 * BQ, zq);
       if (has_b) tma_load_3d(sQ + C::TILE_BYTES, tq, q_full, 0, (qt0 + 1) * BQ, zq);
-      for (int j = 0; j < nkv; ++j) {
-        const int st = j % KV_STAGES;
-        const uint32_t ph = (j / KV_STAGES) & 1;
+      for (int j = j0; j < jend; ++j) {
+        const int st = (j - j0) % KV_STAGES;
+        const uint32_t ph = ((j - j0) / KV_STAGES) & 1;
         if (!mbar_wait(&kv_empty[st], ph ^ 1u, abort_flag)) break;
         mbar_arrive_expect_tx(&k_full[st], C::TILE_BYTES);
         tma_load_3d(sK + st * C::TILE_BYTES, &tmK, &k_full[st], 0, j * BKV, zkv);
@@ -376,9 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_S = [&](int n) -> bool {
         int t, j;
-        seq_item(n, has_b, nkv_a, t, j);
-        const int st = j % KV_STAGES;
-        if (!wait_all(&k_full[st], (j / KV_STAGES) & 1)) return false;
+        seq_item(n, has_b, j0, na, t, j);
+        const int st = (j - j0) % KV_STAGES;
+        if (!wait_all(&k_full[st], ((j - j0) / KV_STAGES) & 1)) return false;
         tc_fence_after();
         const uint64_t q0 = dQ + static_cast<uint64_t>((t * C::TILE_BYTES) >> 4);
         const uint64_t k0 = dK + static_cast<uint64_t>((st * C::TILE_BYTES) >> 4);
@@ -389,14 +435,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit_elect(&s_full[n % 3]);
         return true;
       };
-      const int n_total = has_b ? 2 * nkv_a + 1 : nkv_a;
+      const int n_total = has_b ? 2 * na + (jb1 - ja1) : na;
       bool ok = wait_all(q_full, 0);
       for (int n = 0; ok && n < 3 && n < n_total; ++n) ok = issue_S(n);
       for (int m = 0; ok && m < n_total; ++m) {
         int t, j;
-        seq_item(m, has_b, nkv_a, t, j);
-        const int st = j % KV_STAGES;
-        if (!wait_all(&p_full[t], j & 1) || !wait_all(&v_full[st], (j / KV_STAGES) & 1)) {
+        seq_item(m, has_b, j0, na, t, j);
+        const int jr = j - j0;
+        const int st = jr % KV_STAGES;
+        if (!wait_all(&p_full[t], jr & 1) || !wait_all(&v_full[st], (jr / KV_STAGES) & 1)) {
           ok = false;
           break;
         }
@@ -406,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk)
           umma_bf16_ss_elect(tmem + 384 + t * DH, p0 + ((kk >> 2) * (BQ * 128) + (kk & 3) * 32) / 16,
-                             v0 + (kk * 16 * C::SWB) / 16, idO, (j > 0 || kk > 0) ? 1u : 0u);
+                             v0 + (kk * 16 * C::SWB) / 16, idO, (jr > 0 || kk > 0) ? 1u : 0u);
         umma_commit_elect(&o_done[t]);
         if (t == 1 || !has_b) umma_commit_elect(&kv_empty[st]);  // last reader of K_j, V_j
         // S(m+3) follows PV(m): with one tile it needs K_{j+3}, which shares a
@@ -419,17 +466,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- softmax
     const int t = warp >> 2;            // 0: tile a, 1: tile b
     const int i = threadIdx.x & 127;    // row in tile = TMEM lane
-    const int n_t = t == 0 ? nkv_a : nkv_b;
-    const int qi = (qt0 + t) * BQ + i;
+    const int jt1 = t == 0 ? ja1 : jb1;  // this tile's KV tiles: [j0, jt1)
+    const int n_t = (t == 0 || has_b) ? jt1 - j0 : 0;
+    const int qt = qt0 + t;
+    const int qi = qt * BQ + i;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tO = tmem + 384 + t * DH + lane_off;
     uint8_t* prow = sP + t * C::P_BYTES + i * 128;
     const float sc = p.scale_log2;
     float m = -INFINITY, l = 0.0f;
     bool ok = n_t > 0;
-    for (int j = 0; ok && j < n_t; ++j) {
+    for (int jr = 0; ok && jr < n_t; ++jr) {
+      const int j = j0 + jr;
       // This tile's S for KV tile j is sequence item n, in TMEM buffer n % 3.
-      const int n = has_b ? (j < nkv_a ? 2 * j + t : 2 * nkv_a) : j;
+      const int n = has_b ? (j < ja1 ? 2 * jr + t : 2 * na) : jr;
       const uint32_t tS = tmem + (n % 3) * 128 + lane_off;
       // Waits are made warp-uniform: tcgen05.ld/st below are .sync.aligned.
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[n % 3], (n / 3) & 1, abort_flag))) {
@@ -440,14 +490,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // PV of the previous KV tile must be complete before O is rescaled and
       // before this tile's single P buffer is overwritten; softmax_tile waits
       // for it after its max pass.
-      uint64_t* pv_prev = j > 0 ? &o_done[t] : nullptr;
+      uint64_t* pv_prev = jr > 0 ? &o_done[t] : nullptr;
       bool w_ok = true;
-      if (j == n_t - 1)
-        w_ok = softmax_tile<DH, true>(tS, tO, prow, i, qi - j * BKV, sc, j == 0, m, l, pv_prev,
-                                      (j - 1) & 1, abort_flag);
+      if (j == qt)  // the diagonal tile
+        w_ok = softmax_tile<DH, true>(tS, tO, prow, i, qi - j * BKV, sc, jr == 0, m, l, pv_prev,
+                                      (jr - 1) & 1, abort_flag);
       else
-        w_ok = softmax_tile<DH, false>(tS, tO, prow, i, BKV, sc, j == 0, m, l, pv_prev,
-                                       (j - 1) & 1, abort_flag);
+        w_ok = softmax_tile<DH, false>(tS, tO, prow, i, BKV, sc, jr == 0, m, l, pv_prev,
+                                       (jr - 1) & 1, abort_flag);
       if (!w_ok) {
         ok = false;
         break;
@@ -456,26 +506,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&o_done[t], (n_t - 1) & 1, abort_flag))) {
-      tc_fence_after();
-      const float inv = 1.0f / l;
-      uint16_t* dst = p.out + (static_cast<size_t>(b) * p.T + qi) * p.ldo + slot * DH;
+    const bool fin =
+        ok && n_t > 0 && __all_sync(0xffffffffu, mbar_wait(&o_done[t], (n_t - 1) & 1, abort_flag));
+    if (n_chunks == 1) {
+      if (fin) {
+        tc_fence_after();
+        const float inv = 1.0f / l;
+        uint16_t* dst = p.out + (static_cast<size_t>(b) * p.T + qi) * p.ldo + slot * DH;
 #pragma unroll
-      for (int c = 0; c < DH / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tO + c * 32, v);
-        if (qi < p.T) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tO + c * 32, v);
+          if (qi < p.T) store_row32(dst + c * 32, v, inv);
+        }
+      }
+    } else {
+      // Split-KV: publish this chunk's unnormalised rows (O relative to the
+      // row's m, and l); the last CTA of the pair to arrive merges all chunks:
+      // O = sum_c 2^(m_c - m*) O_c, l = sum_c 2^(m_c - m*) l_c, out = O / l.
+      const size_t row_id = ((static_cast<size_t>(bh) * p.items + item_base + chunk_id) * 2 + t) * BQ + i;
+      if (fin) {
+        tc_fence_after();
+        float4* dst = reinterpret_cast<float4*>(p.part + row_id * DH);
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv);
-            o.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv);
-            o.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv);
-            o.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv);
-            d4[q4] = o;
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tO + c * 32, v);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[c * 8 + q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                         __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+        }
+        p.part_ml[row_id] = make_float2(m, l);
+      }
+      named_bar_sync(1, 256);
+      if (threadIdx.x == 0) {
+        __threadfence();
+        const int old = atomicAdd(&p.counters[bh * p.n_pairs + pair], 1);
+        *s_last = old == n_chunks - 1;
+      }
+      named_bar_sync(1, 256);
+      if (*s_last) {
+        __threadfence();
+        if (n_t > 0 && qi < p.T) {
+          const size_t r0 = (static_cast<size_t>(bh) * p.items + item_base) * 2 * BQ + t * BQ + i;
+          float ms = -INFINITY;
+          for (int c = 0; c < n_chunks; ++c) ms = fmaxf(ms, __ldcg(&p.part_ml[r0 + c * 2 * BQ]).x);
+          float acc[DH];
+#pragma unroll
+          for (int x = 0; x < DH; ++x) acc[x] = 0.0f;
+          float lt = 0.0f;
+          for (int c = 0; c < n_chunks; ++c) {
+            const float2 ml = __ldcg(&p.part_ml[r0 + c * 2 * BQ]);
+            const float w = ex2(ml.x - ms);
+            lt += w * ml.y;
+            const float4* src = reinterpret_cast<const float4*>(p.part + (r0 + c * 2 * BQ) * DH);
+#pragma unroll
+            for (int q = 0; q < DH / 4; ++q) {
+              const float4 o = __ldcg(src + q);
+              acc[4 * q] += w * o.x;
+              acc[4 * q + 1] += w * o.y;
+              acc[4 * q + 2] += w * o.z;
+              acc[4 * q + 3] += w * o.w;
+            }
+          }
+          uint16_t* dst = p.out + (static_cast<size_t>(b) * p.T + qi) * p.ldo + slot * DH;
+          const float inv = 1.0f / lt;
+#pragma unroll
+          for (int c = 0; c < DH / 32; ++c) {
+            uint32_t v[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(acc[c * 32 + x]);
+            store_row32(dst + c * 32, v, inv);
           }
         }
+        if (threadIdx.x == 0) p.counters[bh * p.n_pairs + pair] = 0;  // ready for the next call
       }
     }
   }
@@ -495,7 +600,7 @@ int launch_attn(const CUtensorMap& q, const CUtensorMap& qs, const CUtensorMap& 
   using C = AttnCfg<DH>;
   const int e = ensure_smem<attn_kernel<DH>>(static_cast<int>(C::SMEM));
   if (e != cudaSuccess) return e;
-  const long long grid = static_cast<long long>(p.n_pairs) * p.B * p.H;
+  const long long grid = static_cast<long long>(p.items) * p.B * p.H;
   if (grid <= 0) return cudaSuccess;
   attn_kernel<DH><<<static_cast<unsigned>(grid), kThreads, C::SMEM, static_cast<cudaStream_t>(stream)>>>(
       q, qs, k, v, p);
@@ -503,9 +608,11 @@ int launch_attn(const CUtensorMap& q, const CUtensorMap& qs, const CUtensorMap& 
 }
 
 int run(const gqe_config& c, const uint16_t* Q, uint64_t nq_streams, const uint16_t* Qs,
-        const uint16_t* K, const uint16_t* V, uint16_t* out, int ldo, int H, int dense,
-        void* stream) {
+        const uint16_t* K, const uint16_t* V, uint16_t* out, int ldo, int H, int dense, void* ws,
+        size_t ws_bytes, void* stream) {
   const int dh = c.d_head;
+  const AttnPlan plan = attention_plan(c, H);
+  if (plan.total > 0 && (ws == nullptr || ws_bytes < plan.total)) return cudaErrorInvalidValue;
   CUtensorMap tq, tqs, tk, tv;
   if (!make_tmap_bf16_3d(&tq, Q, dh, c.T, nq_streams, dh, BQ)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_3d(&tqs, Qs ? Qs : Q, dh, c.T, Qs ? c.B : nq_streams, dh, BQ))
@@ -522,11 +629,22 @@ int run(const gqe_config& c, const uint16_t* Q, uint64_t nq_streams, const uint1
   p.k = c.k;
   p.M = c.M;
   p.dense = dense;
-  p.n_qt = (c.T + BQ - 1) / BQ;
-  p.n_pairs = (p.n_qt + 1) / 2;
+  p.n_qt = plan.n_qt;
+  p.n_pairs = plan.n_pairs;
+  p.chunk = plan.chunk;
+  p.items = plan.items;
   p.out = out;
   p.ldo = ldo;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(dh)));
+  char* w = static_cast<char*>(ws);
+  p.part = plan.total ? reinterpret_cast<float*>(w + plan.part) : nullptr;
+  p.part_ml = plan.total ? reinterpret_cast<float2*>(w + plan.ml) : nullptr;
+  p.counters = plan.total ? reinterpret_cast<int*>(w + plan.counters) : nullptr;
+  if (plan.total) {
+    const cudaError_t e = cudaMemsetAsync(p.counters, 0, plan.counter_bytes,
+                                          static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return e;
+  }
   if (dh == 64) return launch_attn<64>(tq, tqs, tk, tv, p, stream);
   return launch_attn<32>(tq, tqs, tk, tv, p, stream);
 }
@@ -534,17 +652,54 @@ int run(const gqe_config& c, const uint16_t* Q, uint64_t nq_streams, const uint1
 }  // namespace attn_impl
 using namespace attn_impl;
 
+AttnPlan attention_plan(const gqe_config& c, int H) {
+  AttnPlan pl{};
+  pl.n_qt = (c.T + BQ - 1) / BQ;
+  pl.n_pairs = (pl.n_qt + 1) / 2;
+  const long long streams = static_cast<long long>(c.B) * H;
+  // One CTA per SM: with fewer pair-CTAs than SMs, the longest pair (2 query
+  // tiles x n_qt KV tiles) sets the time. Split the pairs' KV ranges into the
+  // smallest chunks that still fit one wave.
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  pl.chunk = pl.n_qt;
+  pl.items = pl.n_pairs;
+  if (static_cast<long long>(pl.n_pairs) * streams < sms) {
+    for (int ch = 2; ch < pl.n_qt; ++ch) {
+      int items = 0;
+      for (int q = 0; q < pl.n_pairs; ++q) items += (2 * q + 1 + ch - 1) / ch;
+      if (static_cast<long long>(items) * streams <= sms) {
+        pl.chunk = ch;
+        pl.items = items;
+        break;
+      }
+    }
+  }
+  if (pl.chunk < pl.n_qt) {
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    const size_t rows = static_cast<size_t>(streams) * pl.items * 2 * BQ;
+    pl.part = 0;
+    pl.ml = up(rows * c.d_head * 4);
+    pl.counters = up(pl.ml + rows * 8);
+    pl.counter_bytes = static_cast<size_t>(streams) * pl.n_pairs * 4;
+    pl.total = up(pl.counters + pl.counter_bytes);
+  }
+  return pl;
+}
+
 int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
-                  const uint16_t* V, uint16_t* slots, void* stream) {
+                  const uint16_t* V, uint16_t* slots, void* ws, size_t ws_bytes, void* stream) {
   const int H = c.G * c.k + 1;
   return run(c, Qv, static_cast<uint64_t>(c.B) * c.G * c.k, Qs, K, V, slots,
-             (c.G * c.k + 2) * c.d_head, H, 0, stream);
+             (c.G * c.k + 2) * c.d_head, H, 0, ws, ws_bytes, stream);
 }
 
 int attention_dense(const gqe_config& c, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
-                    uint16_t* O, void* stream) {
+                    uint16_t* O, void* ws, size_t ws_bytes, void* stream) {
   const int N = c.G * c.M;
-  return run(c, Q, static_cast<uint64_t>(c.B) * N, nullptr, K, V, O, N * c.d_head, N, 1, stream);
+  return run(c, Q, static_cast<uint64_t>(c.B) * N, nullptr, K, V, O, N * c.d_head, N, 1, ws,
+             ws_bytes, stream);
 }
 
 }  // namespace gqe

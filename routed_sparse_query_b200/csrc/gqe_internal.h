@@ -78,10 +78,17 @@ int gemm_q_dense(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, ui
 int gemm_rowmajor(const uint16_t* A, int rows, int K, const uint16_t* W, int N, uint16_t* out,
                   void* stream);
 
-// Attention front ends (tcgen05).
+// Attention front ends (tcgen05). Split-KV plan: small problems cut each
+// query-tile pair's KV range into chunks; the scratch (partial rows and
+// per-pair counters) comes from the workspace (total == 0: no scratch).
+struct AttnPlan {
+  int n_qt, n_pairs, chunk, items;
+  size_t part, ml, counters, counter_bytes, total;
+};
+AttnPlan attention_plan(const gqe_config& c, int H);
 int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
-                  const uint16_t* V, uint16_t* slots, void* stream);
+                  const uint16_t* V, uint16_t* slots, void* ws, size_t ws_bytes, void* stream);
 int attention_dense(const gqe_config& c, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
-                    uint16_t* O, void* stream);
+                    uint16_t* O, void* ws, size_t ws_bytes, void* stream);
 
 }  // namespace gqe

@@ -78,7 +78,8 @@ def run_steps(rsq, shape: synth.LayerShape, d: dict) -> dict:
     o["V"] = torch.empty(B, G, T, dh, dtype=torch.bfloat16, device=dev)
     rsq.gqe_kv_proj(cfg, d["x"], d["W_k"], d["W_v"], o["K"], o["V"])
     o["slots"] = torch.zeros(R, (k * G + 2) * dh, dtype=torch.bfloat16, device=dev)
-    rsq.gqe_attention_fwd(cfg, o["Qv"], o["Qs"], o["K"], o["V"], o["slots"])
+    wsa = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_ATTENTION), dtype=torch.uint8, device=dev)
+    rsq.gqe_attention_fwd(cfg, o["Qv"], o["Qs"], o["K"], o["V"], o["slots"], wsa)
     o["y"] = torch.empty(R, shape.d_model, dtype=torch.bfloat16, device=dev)
     rsq.gqe_output_proj(cfg, o["slots"], o["omega"], d["W_o"], o["y"])
     torch.cuda.synchronize()

@@ -76,6 +76,18 @@ def test_seq2k_layer_matches_oracle(rsq):
     _check_float_parts(o, ref, shape)
     y, ws = run_layer(rsq, shape, d)
     assert torch.equal(y, o["y"]), "gqe_layer_fwd differs from the step calls"
+    # T = 2048 runs the split-KV attention; a second call on the same scratch
+    # (merge counters reset by the previous call) gives the same slots.
+    cfg = rsq.GQEConfig.of(shape)
+    wsa = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_ATTENTION), dtype=torch.uint8,
+                      device="cuda")
+    assert wsa.numel() > 256
+    for _ in range(2):
+        slots = torch.zeros_like(o["slots"])
+        rsq.gqe_attention_fwd(cfg, o["Qv"], o["Qs"], o["K"], o["V"], slots, wsa)
+        torch.cuda.synchronize()
+        assert torch.equal(slots[:, :(shape.k * shape.G + 1) * shape.d_head],
+                           o["slots"][:, :(shape.k * shape.G + 1) * shape.d_head])
 
 
 def test_dense_gqa_matches_oracle(rsq):
