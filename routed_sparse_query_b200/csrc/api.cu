@@ -195,10 +195,9 @@ gqe_status gqe_dispatch(const gqe_config* cfg, const int32_t* idx, const gqe_bf1
   int e = launch_dispatch_lists(*cfg, idx, counts, offsets, tok, slot_pos, ws, L, stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
   char* w = static_cast<char*>(ws);
-  e = gemm_q_routed(*cfg, x, W_q, idx, offsets, tok, w + L.qtiles,
-                    reinterpret_cast<const int32_t*>(w + L.n_qtiles), L.max_qtiles, Qv, stream);
-  if (e != cudaSuccess) return GQE_ERR_CUDA;
-  return cuda_status(gemm_q_shared(*cfg, x, W_qs, Qs, stream));
+  return cuda_status(gemm_q_routed(*cfg, x, W_q, W_qs, idx, offsets, tok, w + L.qtiles,
+                                   reinterpret_cast<const int32_t*>(w + L.n_qtiles), L.max_qtiles,
+                                   Qv, Qs, stream));
 }
 
 gqe_status gqe_kv_proj(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16* W_k,

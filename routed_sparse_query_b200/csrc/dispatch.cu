@@ -212,6 +212,106 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ListArgs a) {
   }
 }
 
+// Single-CTA dispatch for small batches (kSmallRows rows or fewer): counts,
+// (expert, sequence) prefix sums, stable scatter and the grouped-GEMM tile
+// table in one kernel, with the same results as the three-pass path. Rows are
+// visited sequence by sequence, kSmallThreads at a time (one per thread), so
+// ranks within an (expert, sequence) list follow the positions t.
+constexpr int kSmallThreads = 1024;
+
+__global__ void __launch_bounds__(kSmallThreads) small_dispatch_kernel(ListArgs a) {
+  __shared__ int wcnt[kSmallThreads / 32][kMaxExperts];
+  __shared__ int run[kMaxExperts];
+  extern __shared__ int eb_counts[];  // [N*B] counts, then exclusive offsets
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  const int EB = a.N * a.B;
+  for (int i = threadIdx.x; i < EB; i += blockDim.x) eb_counts[i] = 0;
+  __syncthreads();
+  // Pass 1: counts per (e, b).
+  bool bad = false;
+  for (int row = threadIdx.x; row < a.B * a.T; row += blockDim.x) {
+    uint64_t m;
+    bad |= !token_mask(a, row, m);
+    const int b = row / a.T;
+    while (m) {
+      const int e = __ffsll(static_cast<long long>(m)) - 1;
+      m &= m - 1;
+      atomicAdd(&eb_counts[e * a.B + b], 1);
+    }
+  }
+  if (bad) set_status(GQE_ERR_DEVICE_CHECK);
+  __syncthreads();
+  // Exclusive scan in (e, b) order; counts and offsets out; tile counts.
+  int total;
+  const int per = (EB + blockDim.x - 1) / blockDim.x;
+  const int lo = min(EB, threadIdx.x * per), hi = min(EB, lo + per);
+  int sum = 0, nq = 0;
+  for (int i = lo; i < hi; ++i) {
+    sum += eb_counts[i];
+    nq += (eb_counts[i] + kQTileRows - 1) / kQTileRows;
+  }
+  int base = block_exclusive_scan(sum, &total);
+  int nq_total;
+  int qbase = block_exclusive_scan(nq, &nq_total);
+  for (int i = lo; i < hi; ++i) {
+    const int c = eb_counts[i];
+    a.counts[i] = c;
+    a.offsets[i] = base;
+    const int e = i / a.B, b = i % a.B;
+    for (int s = 0; s < c; s += kQTileRows) {
+      if (qbase < a.max_qtiles) a.qtiles[qbase] = make_int4(e, b, s, min(kQTileRows, c - s));
+      ++qbase;
+    }
+    eb_counts[i] = base;  // becomes the list start
+    base += c;
+  }
+  if (threadIdx.x == 0) {
+    a.offsets[EB] = total;
+    *a.n_qtiles = min(nq_total, a.max_qtiles);
+    if (nq_total > a.max_qtiles || total != a.k * a.G * a.B * a.T) set_status(GQE_ERR_DEVICE_CHECK);
+  }
+  __syncthreads();
+  // Pass 2: stable ranks, sequence by sequence.
+  for (int b = 0; b < a.B; ++b) {
+    for (int e = threadIdx.x; e < a.N; e += blockDim.x) run[e] = 0;
+    __syncthreads();
+    for (int c0 = 0; c0 < a.T; c0 += blockDim.x) {
+      const int t = c0 + threadIdx.x;
+      const size_t row = static_cast<size_t>(b) * a.T + t;
+      uint64_t m = 0;
+      if (t < a.T) token_mask(a, row, m);
+      for (int e = 0; e < a.N; ++e) {
+        const unsigned bal = __ballot_sync(0xffffffffu, (m >> e) & 1ull);
+        if (lane == 0) wcnt[warp][e] = __popc(bal);
+      }
+      __syncthreads();
+      for (int e = threadIdx.x; e < a.N; e += blockDim.x) {
+        int pre = run[e];
+        for (int w = 0; w < kSmallThreads / 32; ++w) {
+          const int c = wcnt[w][e];
+          wcnt[w][e] = pre;
+          pre += c;
+        }
+        run[e] = pre;
+      }
+      __syncthreads();
+      for (int e = 0; e < a.N; ++e) {
+        const bool f = (m >> e) & 1ull;
+        const unsigned bal = __ballot_sync(0xffffffffu, f);
+        if (f) {
+          const int pos = eb_counts[e * a.B + b] + wcnt[warp][e] + __popc(bal & lt);
+          a.tok[pos] = t;
+          const int g = e / a.M, j = e % a.M;
+          const uint64_t gm = (m >> (g * a.M)) & ((1ull << j) - 1ull);
+          a.slot_pos[(row * a.G + g) * a.k + __popcll(static_cast<long long>(gm))] = pos;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
 // Weighted slot: one thread per 8 columns of one row.
 __global__ void __launch_bounds__(256) weighted_slot_kernel(uint16_t* slots, const float* omega,
                                                             int R, int G, int k, int dh) {
@@ -291,6 +391,12 @@ int launch_dispatch_lists(const gqe_config& c, const int32_t* idx, int32_t* coun
   a.num_tiles = L.num_tiles;
   a.tiles_per_seq = L.tiles_per_seq;
   a.max_qtiles = L.max_qtiles;
+  const long long R = static_cast<long long>(c.B) * c.T;
+  if (R <= kSmallRows && static_cast<long long>(a.N) * c.B <= 8192) {
+    const size_t smem = static_cast<size_t>(a.N) * c.B * 4;
+    small_dispatch_kernel<<<1, kSmallThreads, smem, st>>>(a);
+    return cudaGetLastError();
+  }
   count_kernel<<<L.num_tiles, kThreads, 0, st>>>(a);
   scan_kernel<<<1, 1024, 0, st>>>(a);
   scatter_kernel<<<L.num_tiles, kThreads, 0, st>>>(a);

@@ -39,7 +39,9 @@ struct GemmCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BK * BN * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (200 * 1024 / STAGE_BYTES) > 8 ? 8 : (200 * 1024 / STAGE_BYTES);
+  // Tiles up to 128 wide keep two CTAs per SM (<= ~113 KB of shared memory
+  // each): small projections are latency-bound and the second CTA hides it.
+  static constexpr int STAGES = BN <= 128 ? (110 * 1024) / STAGE_BYTES : 4;
   static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 256;
 };
@@ -60,6 +62,8 @@ struct Gather {
   const int32_t* n_qtiles;
   const int32_t* idx;
   uint16_t* Qv;
+  uint16_t* Qs;     // shared-head output [B*T, dh] (tiles after the routed ones)
+  int max_qtiles;   // CTAs reserved for routed tiles
   int d, T, G, M, k, B, dh;
 };
 
@@ -77,7 +81,7 @@ __device__ __forceinline__ void store32_bf16(uint16_t* dst, const uint32_t (&v)[
 }
 
 template <int BN, bool GATHER>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                 const __grid_constant__ CUtensorMap tmB1, const Epi epi0, const Epi epi1,
                 const Gather ga, const int K) {
@@ -95,20 +99,30 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool z1 = blockIdx.z == 1;
+  const bool z1 = blockIdx.z == 1 || (GATHER && blockIdx.x >= static_cast<unsigned>(ga.max_qtiles));
   const CUtensorMap* tmB = z1 ? &tmB1 : &tmB0;
   const Epi& epi = z1 ? epi1 : epi0;
 
   int m0 = 0, n0 = 0, e = 0, b = 0, list0 = 0, rows = 0;
+  bool shared_tile = false;
   if (GATHER) {
     const int q = blockIdx.x;
-    if (q >= *ga.n_qtiles) return;  // uniform: this tile slot is unused
-    const int4 qt = ga.qtiles[q];
-    e = qt.x;
-    b = qt.y;
-    list0 = ga.offsets[e * ga.B + b] + qt.z;
-    rows = qt.w;
-    n0 = e * ga.dh;
+    if (q < ga.max_qtiles) {
+      // Routed tile: up to 128 consecutive entries of one (expert, sequence)
+      // token list.
+      if (q >= *ga.n_qtiles) return;  // uniform: this tile slot is unused
+      const int4 qt = ga.qtiles[q];
+      e = qt.x;
+      b = qt.y;
+      list0 = ga.offsets[e * ga.B + b] + qt.z;
+      rows = qt.w;
+      n0 = e * ga.dh;
+    } else {
+      // Shared-head tile: 128 consecutive rows of x (all tokens).
+      shared_tile = true;
+      m0 = (q - ga.max_qtiles) * BM;
+      rows = min(BM, ga.B * ga.T - m0);
+    }
   } else {
     m0 = blockIdx.x * BM;
     n0 = blockIdx.y * BN;
@@ -174,11 +188,23 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     const int q = warp & 3;
     if (GATHER) {
-      // Thread i gathers row i of the A tile (zeros past the list's end).
+      // 128 threads gather the A tile: in pass r, thread i copies 16-byte
+      // chunk (i % 8) of row 16 r + i / 8, so each warp instruction moves four
+      // whole 128-byte row segments. Rows past the tile's end are zero-filled.
       const int i = threadIdx.x - 64;
-      const bool valid = i < rows;
-      const int t = valid ? ga.tok[list0 + i] : 0;
-      const uint16_t* src = ga.x + (static_cast<size_t>(b) * ga.T + t) * ga.d;
+      const int chunk = i & 7;
+      const uint16_t* src[8];
+      uint32_t nbytes[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int row = r * 16 + (i >> 3);
+        const bool valid = row < rows;
+        size_t xrow = 0;
+        if (valid) xrow = shared_tile ? static_cast<size_t>(m0 + row)
+                                      : static_cast<size_t>(b) * ga.T + ga.tok[list0 + row];
+        src[r] = ga.x + xrow * ga.d + chunk * 8;
+        nbytes[r] = valid ? 16u : 0u;
+      }
       const uint32_t a0 = smem_u32(sA);
       constexpr int LA = C::STAGES - 1;
       int kb = 0;
@@ -186,10 +212,12 @@ __global__ void __launch_bounds__(192, 1)
         const int s = kb % C::STAGES;
         const uint32_t ph = (kb / C::STAGES) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) break;
-        const uint32_t dst = a0 + s * C::A_BYTES + i * 128;
+        const uint32_t dst = a0 + s * C::A_BYTES;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          cp_async_16(dst + ((c ^ (i & 7)) << 4), src + kb * BK + c * 8, valid ? 16u : 0u);
+        for (int r = 0; r < 8; ++r) {
+          const int row = r * 16 + (i >> 3);
+          cp_async_16(dst + row * 128 + ((chunk ^ (row & 7)) << 4), src[r] + kb * BK, nbytes[r]);
+        }
         cp_async_commit();
         if (kb >= LA) {
           cp_async_wait<LA>();
@@ -208,7 +236,9 @@ __global__ void __launch_bounds__(192, 1)
     if (GATHER) {
       const bool valid = have && r < rows;
       size_t obase = 0;
-      if (valid) {
+      if (valid && shared_tile) {
+        obase = static_cast<size_t>(m0 + r) * ga.dh;
+      } else if (valid) {
         const int t = ga.tok[list0 + r];
         const int g = e / ga.M, j = e % ga.M;
         const int32_t* ip = ga.idx + ((static_cast<size_t>(b) * ga.T + t) * ga.G + g) * ga.k;
@@ -221,7 +251,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t v[32];
         tmem_ld32(trow + cc * 32, v);
-        if (valid) store32_bf16(ga.Qv + obase + cc * 32, v);
+        if (valid) store32_bf16((shared_tile ? ga.Qs : ga.Qv) + obase + cc * 32, v);
       }
     } else {
       const int row = m0 + r;
@@ -311,13 +341,6 @@ int gemm_kv(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const u
   return dense_gemm(x, R, c.d_model, W_k, W_v, c.G * c.d_head, ek, ev, 2, stream);
 }
 
-int gemm_q_shared(const gqe_config& c, const uint16_t* x, const uint16_t* W_qs, uint16_t* Qs,
-                  void* stream) {
-  const int R = c.B * c.T;
-  const Epi e = head_split(Qs, c.T, 1, c.d_head, R);
-  return dense_gemm(x, R, c.d_model, W_qs, nullptr, c.d_head, e, e, 1, stream);
-}
-
 int gemm_q_dense(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, uint16_t* Q,
                  void* stream) {
   const int R = c.B * c.T;
@@ -340,15 +363,17 @@ int gemm_rowmajor(const uint16_t* A, int rows, int K, const uint16_t* W, int N, 
   return dense_gemm(A, rows, K, W, nullptr, N, e, e, 1, stream);
 }
 
-int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const int32_t* idx,
-                  const int32_t* offsets, const int32_t* tok, const void* qtiles,
-                  const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, void* stream) {
+int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const uint16_t* W_qs,
+                  const int32_t* idx, const int32_t* offsets, const int32_t* tok, const void* qtiles,
+                  const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, uint16_t* Qs,
+                  void* stream) {
   const int N = c.G * c.M;
   const int dh = c.d_head;
-  CUtensorMap tb;
+  CUtensorMap tb, tbs;
   if (!make_tmap_bf16_2d(&tb, W_q, static_cast<uint64_t>(N) * dh, c.d_model,
                          static_cast<uint64_t>(N) * dh, dh, BK))
     return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tbs, W_qs, dh, c.d_model, dh, dh, BK)) return cudaErrorInvalidValue;
   Gather g;
   g.x = x;
   g.tok = tok;
@@ -357,6 +382,8 @@ int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, c
   g.n_qtiles = n_qtiles;
   g.idx = idx;
   g.Qv = Qv;
+  g.Qs = Qs;
+  g.max_qtiles = max_qtiles;
   g.d = c.d_model;
   g.T = c.T;
   g.G = c.G;
@@ -365,9 +392,10 @@ int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, c
   g.B = c.B;
   g.dh = dh;
   Epi e{};
-  const dim3 grid(static_cast<unsigned>(max_qtiles), 1, 1);
-  if (dh == 64) return launch<64, true>(tb, tb, tb, e, e, g, c.d_model, grid, stream);
-  return launch<32, true>(tb, tb, tb, e, e, g, c.d_model, grid, stream);
+  const long long R = static_cast<long long>(c.B) * c.T;
+  const dim3 grid(static_cast<unsigned>(max_qtiles + (R + BM - 1) / BM), 1, 1);
+  if (dh == 64) return launch<64, true>(tb, tb, tbs, e, e, g, c.d_model, grid, stream);
+  return launch<32, true>(tb, tb, tbs, e, e, g, c.d_model, grid, stream);
 }
 
 }  // namespace gqe

@@ -27,6 +27,9 @@ constexpr size_t kRouterSmemLimit = 200 * 1024;
 // Dispatch tiling: tokens of one sequence are cut into tiles of this size.
 constexpr int kDispatchTile = 256;  // == dispatch CTA size: one token per thread
 constexpr int kQTileRows = 128;  // rows of one grouped-GEMM tile
+// Batches of at most this many rows (and N*B*4 bytes of counts within the
+// 48 KiB static shared-memory limit) take the single-CTA dispatch.
+constexpr long long kSmallRows = 16384;
 
 struct DispatchWs {
   // Byte offsets inside the dispatch workspace.
@@ -68,11 +71,11 @@ int launch_weighted_slot(const gqe_config& c, uint16_t* slots, const float* omeg
 // GEMM front ends (tcgen05). out layouts are described in gemm.cu.
 int gemm_kv(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
             uint16_t* K, uint16_t* V, void* stream);
-int gemm_q_shared(const gqe_config& c, const uint16_t* x, const uint16_t* W_qs, uint16_t* Qs,
-                  void* stream);
-int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const int32_t* idx,
-                  const int32_t* offsets, const int32_t* tok, const void* qtiles,
-                  const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, void* stream);
+// Routed query projection over the token lists plus the shared-head query
+// projection, in one launch.
+int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const uint16_t* W_qs,
+                  const int32_t* idx, const int32_t* offsets, const int32_t* tok, const void* qtiles,
+                  const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, uint16_t* Qs, void* stream);
 int gemm_q_dense(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, uint16_t* Q,
                  void* stream);
 int gemm_rowmajor(const uint16_t* A, int rows, int K, const uint16_t* W, int N, uint16_t* out,

@@ -66,6 +66,20 @@ def test_layer_steps_match_oracle(rsq, name):
     _check_float_parts(o, ref, shape)
 
 
+def test_large_batch_dispatch_is_bit_exact(rsq):
+    # More than 16384 rows: the three-pass (count, scan, scatter) dispatch;
+    # smaller batches take the single-CTA path. Both must give the oracle's lists.
+    shape = LayerShape(B=3, T=7000, d_model=128, G=4, M=3, k=2, d_head=32)
+    inp = synth.make_layer_inputs(shape, seed=23)
+    import oracle as orc
+    f = orc._f64_inputs(inp)
+    rt = orc.router(f["x"], f["W_r"], f["b_r"], shape.G, shape.M, shape.k)
+    ref = dict(rt)
+    ref.update(orc.dispatch(rt["idx"], shape.B, shape.T, shape.G, shape.M))
+    o = run_steps(rsq, shape, device_inputs(inp))
+    _check_integer_parts(o, ref, shape)
+
+
 def test_seq2k_layer_matches_oracle(rsq):
     shape = synth.SEQ2K
     inp = synth.make_layer_inputs(shape)
