@@ -217,7 +217,7 @@ gqe_status gqe_attention_fwd(const gqe_config* cfg, const gqe_bf16* Qv, const gq
   const size_t need = attention_plan(*cfg, cfg->G * cfg->k + 1).total;
   if (need > 0 && (ws == nullptr || !aligned16(ws))) return GQE_ERR_INVALID;
   if (ws_bytes < need) return GQE_ERR_WORKSPACE;
-  return cuda_status(attention_gqe(*cfg, Qv, Qs, K, V, slots, ws, ws_bytes, stream));
+  return cuda_status(attention_gqe(*cfg, Qv, Qs, K, V, slots, ws, ws_bytes, false, stream));
 }
 
 gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* omega,
@@ -246,6 +246,10 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
   auto I = [&](size_t o) { return reinterpret_cast<int32_t*>(w + o); };
   auto F = [&](size_t o) { return reinterpret_cast<float*>(w + o); };
   auto H = [&](size_t o) { return reinterpret_cast<gqe_bf16*>(w + o); };
+  // The split-KV counters are zeroed first, so that the kernels of the layer
+  // follow each other directly (programmatic dependent launch).
+  if (zero_attention_counters(*cfg, cfg->G * cfg->k + 1, w + L.aws, stream) != cudaSuccess)
+    return GQE_ERR_CUDA;
   gqe_status st = gqe_router_topk(cfg, x, W_r, b_r, I(L.idx), F(L.r), F(L.omega), stream);
   if (st != GQE_OK) return st;
   st = gqe_dispatch(cfg, I(L.idx), x, W_q, W_qs, I(L.counts), I(L.offsets), I(L.tok),
@@ -253,9 +257,9 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
   if (st != GQE_OK) return st;
   st = gqe_kv_proj(cfg, x, W_k, W_v, H(L.K), H(L.V), stream);
   if (st != GQE_OK) return st;
-  st = gqe_attention_fwd(cfg, H(L.Qv), H(L.Qs), H(L.K), H(L.V), H(L.slots), w + L.aws,
-                         L.total - L.aws, stream);
-  if (st != GQE_OK) return st;
+  if (attention_gqe(*cfg, H(L.Qv), H(L.Qs), H(L.K), H(L.V), H(L.slots), w + L.aws,
+                    L.total - L.aws, true, stream) != cudaSuccess)
+    return GQE_ERR_CUDA;
   return gqe_output_proj(cfg, H(L.slots), F(L.omega), W_o, y, stream);
 }
 
@@ -273,11 +277,12 @@ gqe_status gqa_dense_fwd(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf1
   if (ws_bytes < L.total) return GQE_ERR_WORKSPACE;
   char* w = static_cast<char*>(ws);
   auto H = [&](size_t o) { return reinterpret_cast<gqe_bf16*>(w + o); };
-  int e = gemm_q_dense(c, x, W_q, H(L.Q), stream);
+  int e = zero_attention_counters(c, c.G * c.M, w + L.aws, stream);
+  if (e == cudaSuccess) e = gemm_q_dense(c, x, W_q, H(L.Q), stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
   e = gemm_kv(c, x, W_k, W_v, H(L.K), H(L.V), stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
-  e = attention_dense(c, H(L.Q), H(L.K), H(L.V), H(L.O), w + L.aws, L.total - L.aws, stream);
+  e = attention_dense(c, H(L.Q), H(L.K), H(L.V), H(L.O), w + L.aws, L.total - L.aws, true, stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
   const int N = c.G * c.M;
   return cuda_status(gemm_rowmajor(H(L.O), c.B * c.T, N * c.d_head, W_o_dense, c.d_model, y, stream));

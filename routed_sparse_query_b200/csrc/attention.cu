@@ -382,6 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  pdl_wait();  // every input (Q, K, V) is read after this point
+  pdl_launch_dependents();
 
   if (warp == kTmaWarp) {
     // ---------------------------------------------------------- TMA producer
@@ -602,14 +604,13 @@ int launch_attn(const CUtensorMap& q, const CUtensorMap& qs, const CUtensorMap& 
   if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(p.items) * p.B * p.H;
   if (grid <= 0) return cudaSuccess;
-  attn_kernel<DH><<<static_cast<unsigned>(grid), kThreads, C::SMEM, static_cast<cudaStream_t>(stream)>>>(
-      q, qs, k, v, p);
-  return cudaGetLastError();
+  return launch_pdl(attn_kernel<DH>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), C::SMEM,
+                    stream, q, qs, k, v, p);
 }
 
 int run(const gqe_config& c, const uint16_t* Q, uint64_t nq_streams, const uint16_t* Qs,
         const uint16_t* K, const uint16_t* V, uint16_t* out, int ldo, int H, int dense, void* ws,
-        size_t ws_bytes, void* stream) {
+        size_t ws_bytes, bool counters_zeroed, void* stream) {
   const int dh = c.d_head;
   const AttnPlan plan = attention_plan(c, H);
   if (plan.total > 0 && (ws == nullptr || ws_bytes < plan.total)) return cudaErrorInvalidValue;
@@ -640,7 +641,7 @@ int run(const gqe_config& c, const uint16_t* Q, uint64_t nq_streams, const uint1
   p.part = plan.total ? reinterpret_cast<float*>(w + plan.part) : nullptr;
   p.part_ml = plan.total ? reinterpret_cast<float2*>(w + plan.ml) : nullptr;
   p.counters = plan.total ? reinterpret_cast<int*>(w + plan.counters) : nullptr;
-  if (plan.total) {
+  if (plan.total && !counters_zeroed) {
     const cudaError_t e = cudaMemsetAsync(p.counters, 0, plan.counter_bytes,
                                           static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return e;
@@ -689,17 +690,25 @@ AttnPlan attention_plan(const gqe_config& c, int H) {
 }
 
 int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
-                  const uint16_t* V, uint16_t* slots, void* ws, size_t ws_bytes, void* stream) {
+                  const uint16_t* V, uint16_t* slots, void* ws, size_t ws_bytes,
+                  bool counters_zeroed, void* stream) {
   const int H = c.G * c.k + 1;
   return run(c, Qv, static_cast<uint64_t>(c.B) * c.G * c.k, Qs, K, V, slots,
-             (c.G * c.k + 2) * c.d_head, H, 0, ws, ws_bytes, stream);
+             (c.G * c.k + 2) * c.d_head, H, 0, ws, ws_bytes, counters_zeroed, stream);
 }
 
 int attention_dense(const gqe_config& c, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
-                    uint16_t* O, void* ws, size_t ws_bytes, void* stream) {
+                    uint16_t* O, void* ws, size_t ws_bytes, bool counters_zeroed, void* stream) {
   const int N = c.G * c.M;
   return run(c, Q, static_cast<uint64_t>(c.B) * N, nullptr, K, V, O, N * c.d_head, N, 1, ws,
-             ws_bytes, stream);
+             ws_bytes, counters_zeroed, stream);
+}
+
+int zero_attention_counters(const gqe_config& c, int H, void* ws, void* stream) {
+  const AttnPlan plan = attention_plan(c, H);
+  if (plan.total == 0) return cudaSuccess;
+  return cudaMemsetAsync(static_cast<char*>(ws) + plan.counters, 0, plan.counter_bytes,
+                         static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace gqe

@@ -67,6 +67,8 @@ __device__ __forceinline__ bool token_mask(const ListArgs& a, size_t row, uint64
 // One CTA per tile of kDispatchTile (= kThreads) tokens, one token per
 // thread; per-expert counts by warp ballots, summed over the CTA's warps.
 __global__ void __launch_bounds__(kThreads) count_kernel(ListArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ int wc[kThreads / 32][kMaxExperts];
   const int tile = blockIdx.x;
   const int b = tile / a.tiles_per_seq;
@@ -118,6 +120,8 @@ __device__ int block_exclusive_scan(int v, int* total) {
 }
 
 __global__ void __launch_bounds__(1024) scan_kernel(ListArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int L = a.N * a.num_tiles;
   const int per = (L + blockDim.x - 1) / blockDim.x;
   const int lo = min(L, threadIdx.x * per), hi = min(L, lo + per);
@@ -162,6 +166,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(ListArgs a) {
 }
 
 __global__ void __launch_bounds__(kThreads) scatter_kernel(ListArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ int wcnt[kThreads / 32][kMaxExperts];
   __shared__ int run[kMaxExperts];
   __shared__ int base[kMaxExperts];
@@ -220,6 +226,8 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ListArgs a) {
 constexpr int kSmallThreads = 1024;
 
 __global__ void __launch_bounds__(kSmallThreads) small_dispatch_kernel(ListArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ int wcnt[kSmallThreads / 32][kMaxExperts];
   __shared__ int run[kMaxExperts];
   extern __shared__ int eb_counts[];  // [N*B] counts, then exclusive offsets
@@ -315,6 +323,8 @@ __global__ void __launch_bounds__(kSmallThreads) small_dispatch_kernel(ListArgs 
 // Weighted slot: one thread per 8 columns of one row.
 __global__ void __launch_bounds__(256) weighted_slot_kernel(uint16_t* slots, const float* omega,
                                                             int R, int G, int k, int dh) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int per_row = dh / 8;
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (gid >= static_cast<long long>(R) * per_row) return;
@@ -394,22 +404,20 @@ int launch_dispatch_lists(const gqe_config& c, const int32_t* idx, int32_t* coun
   const long long R = static_cast<long long>(c.B) * c.T;
   if (R <= kSmallRows && static_cast<long long>(a.N) * c.B <= 8192) {
     const size_t smem = static_cast<size_t>(a.N) * c.B * 4;
-    small_dispatch_kernel<<<1, kSmallThreads, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(small_dispatch_kernel, dim3(1), dim3(kSmallThreads), smem, st, a);
   }
-  count_kernel<<<L.num_tiles, kThreads, 0, st>>>(a);
-  scan_kernel<<<1, 1024, 0, st>>>(a);
-  scatter_kernel<<<L.num_tiles, kThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(count_kernel, dim3(L.num_tiles), dim3(kThreads), 0, st, a);
+  if (e == cudaSuccess) e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, a);
+  if (e == cudaSuccess) e = launch_pdl(scatter_kernel, dim3(L.num_tiles), dim3(kThreads), 0, st, a);
+  return e;
 }
 
 int launch_weighted_slot(const gqe_config& c, uint16_t* slots, const float* omega, void* stream) {
   const long long R = static_cast<long long>(c.B) * c.T;
   const long long n = R * (c.d_head / 8);
   const int grid = static_cast<int>((n + 255) / 256);
-  weighted_slot_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      slots, omega, static_cast<int>(R), c.G, c.k, c.d_head);
-  return cudaGetLastError();
+  return launch_pdl(weighted_slot_kernel, dim3(grid), dim3(256), 0, stream, slots, omega,
+                    static_cast<int>(R), c.G, c.k, c.d_head);
 }
 
 }  // namespace gqe

@@ -103,30 +103,6 @@ __global__ void __launch_bounds__(192, 2)
   const CUtensorMap* tmB = z1 ? &tmB1 : &tmB0;
   const Epi& epi = z1 ? epi1 : epi0;
 
-  int m0 = 0, n0 = 0, e = 0, b = 0, list0 = 0, rows = 0;
-  bool shared_tile = false;
-  if (GATHER) {
-    const int q = blockIdx.x;
-    if (q < ga.max_qtiles) {
-      // Routed tile: up to 128 consecutive entries of one (expert, sequence)
-      // token list.
-      if (q >= *ga.n_qtiles) return;  // uniform: this tile slot is unused
-      const int4 qt = ga.qtiles[q];
-      e = qt.x;
-      b = qt.y;
-      list0 = ga.offsets[e * ga.B + b] + qt.z;
-      rows = qt.w;
-      n0 = e * ga.dh;
-    } else {
-      // Shared-head tile: 128 consecutive rows of x (all tokens).
-      shared_tile = true;
-      m0 = (q - ga.max_qtiles) * BM;
-      rows = min(BM, ga.B * ga.T - m0);
-    }
-  } else {
-    m0 = blockIdx.x * BM;
-    n0 = blockIdx.y * BN;
-  }
   const int nk = (K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
@@ -148,8 +124,42 @@ __global__ void __launch_bounds__(192, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  pdl_wait();
+  pdl_launch_dependents();
 
-  if (warp == 0) {
+  // Tile of this CTA (read after pdl_wait: the routed tile table is produced
+  // by the dispatch kernels).
+  int m0 = 0, n0 = 0, e = 0, b = 0, list0 = 0, rows = 0;
+  bool shared_tile = false, skip = false;
+  if (GATHER) {
+    const int q = blockIdx.x;
+    if (q < ga.max_qtiles) {
+      // Routed tile: up to 128 consecutive entries of one (expert, sequence)
+      // token list; slots past the table's length have nothing to do.
+      if (q >= *ga.n_qtiles) {
+        skip = true;
+      } else {
+        const int4 qt = ga.qtiles[q];
+        e = qt.x;
+        b = qt.y;
+        list0 = ga.offsets[e * ga.B + b] + qt.z;
+        rows = qt.w;
+        n0 = e * ga.dh;
+      }
+    } else {
+      // Shared-head tile: 128 consecutive rows of x (all tokens).
+      shared_tile = true;
+      m0 = (q - ga.max_qtiles) * BM;
+      rows = min(BM, ga.B * ga.T - m0);
+    }
+  } else {
+    m0 = blockIdx.x * BM;
+    n0 = blockIdx.y * BN;
+  }
+
+  if (skip) {
+    // nothing to compute: fall through to the teardown
+  } else if (warp == 0) {
     if (lane == 0) {
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % C::STAGES;
@@ -288,9 +298,8 @@ int launch(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, c
   using C = GemmCfg<BN>;
   const int e = ensure_smem<gemm_kernel<BN, GATHER>>(static_cast<int>(C::SMEM));
   if (e != cudaSuccess) return e;
-  gemm_kernel<BN, GATHER><<<grid, 192, C::SMEM, static_cast<cudaStream_t>(stream)>>>(
-      A, B0, B1, e0, e1, g, K);
-  return cudaGetLastError();
+  return launch_pdl(gemm_kernel<BN, GATHER>, grid, dim3(192), C::SMEM, stream, A, B0, B1, e0, e1,
+                    g, K);
 }
 
 // Dense GEMM with a head-split epilogue; chooses the tile width.

@@ -5,6 +5,8 @@
 
 #include <cuda_runtime.h>
 
+#include <utility>
+
 #include "gqe.h"
 
 namespace gqe {
@@ -49,6 +51,24 @@ size_t router_smem_bytes(const gqe_config& c);
 // Raises the dynamic shared-memory limit of kernel K to `bytes`, once per
 // device (the attribute is per device; re-setting it on every launch costs
 // host time on short layers).
+// Launches `kern` with programmatic dependent launch allowed (the kernel
+// overlaps the tail of the previous kernel on the stream; see pdl_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              void* stream, Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <auto K>
 inline int ensure_smem(int bytes) {
   static int done[64] = {0};
@@ -89,9 +109,13 @@ struct AttnPlan {
   size_t part, ml, counters, counter_bytes, total;
 };
 AttnPlan attention_plan(const gqe_config& c, int H);
+// counters_zeroed: the caller has zeroed the split-KV arrival counters of ws
+// earlier on the stream (zero_attention_counters); otherwise the call does.
 int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
-                  const uint16_t* V, uint16_t* slots, void* ws, size_t ws_bytes, void* stream);
+                  const uint16_t* V, uint16_t* slots, void* ws, size_t ws_bytes,
+                  bool counters_zeroed, void* stream);
 int attention_dense(const gqe_config& c, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
-                    uint16_t* O, void* ws, size_t ws_bytes, void* stream);
+                    uint16_t* O, void* ws, size_t ws_bytes, bool counters_zeroed, void* stream);
+int zero_attention_counters(const gqe_config& c, int H, void* ws, void* stream);
 
 }  // namespace gqe

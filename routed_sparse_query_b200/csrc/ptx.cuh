@@ -30,6 +30,19 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---------------------------------------------------------------- PDL
+// Programmatic dependent launch. A kernel launched with the programmatic
+// stream-serialisation attribute may start while the previous kernel of the
+// stream still runs; pdl_wait() blocks until every prerequisite grid has
+// completed and its memory is visible, so each kernel calls it before its
+// first read of any input (only barrier set-up, TMEM allocation and
+// tensor-map prefetch come before it). pdl_launch_dependents() lets the next
+// kernel be scheduled early. Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -82,6 +82,8 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_kernel(RouterArgs a)
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
+  pdl_wait();
+  pdl_launch_dependents();
 
   // Stage W_r (zero padded to S columns) and the bias. Rows of 4k floats are
   // copied with 16-byte cp.async so that all loads are in flight at once.
@@ -279,8 +281,7 @@ int launch_np(const gqe_config& c, const RouterArgs& a, cudaStream_t st) {
   int grid = (R + kRouterWarps - 1) / kRouterWarps;
   if (grid > 4 * 148) grid = 4 * 148;
   if (grid < 1) grid = 1;
-  router_kernel<NP><<<grid, kRouterWarps * 32, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(router_kernel<NP>, dim3(grid), dim3(kRouterWarps * 32), smem, st, a);
 }
 
 }  // namespace router_impl
