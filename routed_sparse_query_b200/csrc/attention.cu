@@ -526,20 +526,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Split-KV: publish this chunk's unnormalised rows (O relative to the
       // row's m, and l); the last CTA of the pair to arrive merges all chunks:
       // O = sum_c 2^(m_c - m*) O_c, l = sum_c 2^(m_c - m*) l_c, out = O / l.
-      const size_t row_id = ((static_cast<size_t>(bh) * p.items + item_base + chunk_id) * 2 + t) * BQ + i;
+      // Partial rows are stored column-major by 16-byte word ([chunk][tile]
+      // [dh/4][128 rows] float4): the 32 lanes of a warp (32 consecutive rows)
+      // touch 32 consecutive words.
+      const size_t blk = (static_cast<size_t>(bh) * p.items + item_base + chunk_id) * 2 + t;
       if (fin) {
         tc_fence_after();
-        float4* dst = reinterpret_cast<float4*>(p.part + row_id * DH);
+        float4* dst = reinterpret_cast<float4*>(p.part) + blk * (BQ * DH / 4) + i;
 #pragma unroll
         for (int c = 0; c < DH / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(tO + c * 32, v);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            dst[c * 8 + q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                         __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+            dst[(c * 8 + q) * BQ] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
         }
-        p.part_ml[row_id] = make_float2(m, l);
+        p.part_ml[blk * BQ + i] = make_float2(m, l);
       }
       named_bar_sync(1, 256);
       if (threadIdx.x == 0) {
@@ -551,21 +554,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*s_last) {
         __threadfence();
         if (n_t > 0 && qi < p.T) {
-          const size_t r0 = (static_cast<size_t>(bh) * p.items + item_base) * 2 * BQ + t * BQ + i;
+          const size_t blk0 = (static_cast<size_t>(bh) * p.items + item_base) * 2 + t;
           float ms = -INFINITY;
-          for (int c = 0; c < n_chunks; ++c) ms = fmaxf(ms, __ldcg(&p.part_ml[r0 + c * 2 * BQ]).x);
+          for (int c = 0; c < n_chunks; ++c) ms = fmaxf(ms, __ldcg(&p.part_ml[(blk0 + 2 * c) * BQ + i]).x);
           float acc[DH];
 #pragma unroll
           for (int x = 0; x < DH; ++x) acc[x] = 0.0f;
           float lt = 0.0f;
           for (int c = 0; c < n_chunks; ++c) {
-            const float2 ml = __ldcg(&p.part_ml[r0 + c * 2 * BQ]);
+            const float2 ml = __ldcg(&p.part_ml[(blk0 + 2 * c) * BQ + i]);
             const float w = ex2(ml.x - ms);
             lt += w * ml.y;
-            const float4* src = reinterpret_cast<const float4*>(p.part + (r0 + c * 2 * BQ) * DH);
+            const float4* src = reinterpret_cast<const float4*>(p.part) + (blk0 + 2 * c) * (BQ * DH / 4) + i;
 #pragma unroll
             for (int q = 0; q < DH / 4; ++q) {
-              const float4 o = __ldcg(src + q);
+              const float4 o = __ldcg(src + q * BQ);
               acc[4 * q] += w * o.x;
               acc[4 * q + 1] += w * o.y;
               acc[4 * q + 2] += w * o.z;

@@ -1,13 +1,18 @@
 // Dispatch (step a5): token lists per (expert, sequence), built from the
-// router's selections in three deterministic passes with no inter-CTA waits:
-//   1. count   one CTA per tile of kDispatchTile tokens of one sequence; a
-//              shared-memory histogram gives the tile's count per expert;
-//   2. scan    one CTA: exclusive prefix sum of the tile counts in
-//              (expert, sequence, tile) order -> each tile's base in the lists,
-//              counts, offsets, and the grouped-GEMM tile table;
+// router's selections in deterministic passes with no inter-CTA waits:
+//   1. masks   one CTA per tile of kDispatchTile tokens of one sequence: each
+//              token's selections become a bitmask over the N experts (kept
+//              in the workspace), and warp ballots give the tile's count per
+//              expert;
+//   2. scan    exclusive prefix sum of the tile counts in (expert, sequence,
+//              tile) order -> each tile's base in the lists, counts, offsets
+//              and the grouped-GEMM tile table;
 //   3. scatter one CTA per tile; warp ballots give every token its rank among
 //              the tile's tokens of the same expert (ascending t), so the
 //              lists are stable and bit-exact.
+// When the tile counts are few (kFusedScanMax), every scatter CTA computes
+// the prefix sum it needs itself and CTA 0 also writes the shared outputs, so
+// steps 2 and 3 are one launch.
 // Only the selected experts receive rows ("a router selects a sparse subset
 // of k query-head experts from each GQA group": gist.science Technical
 // Summary, Methodology), and every group gets exactly k entries per token.
@@ -36,6 +41,7 @@ struct ListArgs {
   int32_t* offsets;
   int32_t* tok;
   int32_t* slot_pos;
+  uint64_t* masks;       // [R] selection bitmask per token
   int32_t* tile_counts;  // [N][num_tiles]
   int32_t* tile_base;    // [N][num_tiles]
   int4* qtiles;
@@ -43,30 +49,47 @@ struct ListArgs {
   int B, T, G, M, k, N, num_tiles, tiles_per_seq, max_qtiles;
 };
 
-// Selection bitmask of one token over the N experts (bit e = g*M + j);
-// returns false if the row is not a valid top-k selection.
-__device__ __forceinline__ bool token_mask(const ListArgs& a, size_t row, uint64_t& mask) {
-  const int32_t* p = a.idx + row * a.G * a.k;
+// Selection bitmask of one token row over the N experts (bit e = g*M + j);
+// returns false if the row is not a valid top-k selection (k strictly
+// increasing expert indices below M in every group). The row's G*k entries
+// are loaded 16 bytes at a time when G*k is a multiple of 4.
+__device__ __forceinline__ bool row_mask(const ListArgs& a, size_t row, uint64_t& mask) {
+  const int GK = a.G * a.k;
+  const int32_t* p = a.idx + row * GK;
   mask = 0;
   bool ok = true;
-  for (int g = 0; g < a.G; ++g) {
-    int prev = -1;
-    for (int s = 0; s < a.k; ++s) {
-      const int j = p[g * a.k + s];
-      if (j <= prev || j >= a.M) {
-        ok = false;
-        continue;
-      }
-      prev = j;
-      mask |= 1ull << (g * a.M + j);
+  int g = 0, s = 0, prev = -1;
+  auto take = [&](int j) {
+    if (s == 0) prev = -1;
+    if (j > prev && j < a.M) mask |= 1ull << (g * a.M + j);
+    else ok = false;
+    prev = j;
+    if (++s == a.k) {
+      s = 0;
+      ++g;
     }
+  };
+  if ((GK & 3) == 0) {
+    const int4* p4 = reinterpret_cast<const int4*>(p);
+#pragma unroll 4
+    for (int q = 0; q < GK / 4; ++q) {
+      const int4 v = __ldg(p4 + q);
+      take(v.x);
+      take(v.y);
+      take(v.z);
+      take(v.w);
+    }
+  } else {
+#pragma unroll 4
+    for (int q = 0; q < GK; ++q) take(__ldg(p + q));
   }
   return ok;
 }
 
-// One CTA per tile of kDispatchTile (= kThreads) tokens, one token per
-// thread; per-expert counts by warp ballots, summed over the CTA's warps.
-__global__ void __launch_bounds__(kThreads) count_kernel(ListArgs a) {
+// Step 1: one CTA per tile of kDispatchTile (= kThreads) tokens, one token
+// per thread; the masks go to the workspace, per-expert counts by warp
+// ballots summed over the CTA's warps.
+__global__ void __launch_bounds__(kThreads) mask_count_kernel(ListArgs a) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ int wc[kThreads / 32][kMaxExperts];
@@ -75,22 +98,29 @@ __global__ void __launch_bounds__(kThreads) count_kernel(ListArgs a) {
   const int t = (tile % a.tiles_per_seq) * kDispatchTile + threadIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint64_t m = 0;
-  bool ok = true;
-  if (t < a.T) ok = token_mask(a, static_cast<size_t>(b) * a.T + t, m);
-  if (!ok) set_status(GQE_ERR_DEVICE_CHECK);
-  for (int e = 0; e < a.N; ++e) {
-    const unsigned bal = __ballot_sync(0xffffffffu, (m >> e) & 1ull);
-    if (lane == 0) wc[warp][e] = __popc(bal);
+  if (t < a.T) {
+    const size_t row = static_cast<size_t>(b) * a.T + t;
+    if (!row_mask(a, row, m)) set_status(GQE_ERR_DEVICE_CHECK);
+    a.masks[row] = m;
   }
+  int c0 = 0, c1 = 0;  // lane e (e + 32): this warp's count of expert e (e + 32)
+  for (int e = 0; e < a.N; ++e) {
+    const int n = __popc(__ballot_sync(0xffffffffu, (m >> e) & 1ull));
+    if (e == lane) c0 = n;
+    if (e == lane + 32) c1 = n;
+  }
+  if (lane < a.N) wc[warp][lane] = c0;
+  if (lane + 32 < a.N) wc[warp][lane + 32] = c1;
   __syncthreads();
   for (int e = threadIdx.x; e < a.N; e += blockDim.x) {
     int c = 0;
+#pragma unroll
     for (int w = 0; w < kThreads / 32; ++w) c += wc[w][e];
     a.tile_counts[static_cast<size_t>(e) * a.num_tiles + tile] = c;
   }
 }
 
-// Block-wide exclusive scan of one int per thread (1024 threads).
+// Block-wide exclusive scan of one int per thread.
 __device__ int block_exclusive_scan(int v, int* total) {
   __shared__ int warp_sums[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -119,38 +149,46 @@ __device__ int block_exclusive_scan(int v, int* total) {
   return before;
 }
 
-__global__ void __launch_bounds__(1024) scan_kernel(ListArgs a) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const int L = a.N * a.num_tiles;
-  const int per = (L + blockDim.x - 1) / blockDim.x;
-  const int lo = min(L, threadIdx.x * per), hi = min(L, lo + per);
+// Exclusive prefix of the flat tile counts [N][num_tiles] (= (expert,
+// sequence, tile) order). Every thread sums a contiguous run; the prefix at
+// each index is passed to visit(i, prefix). Returns the total.
+template <typename Visit>
+__device__ int tile_prefix(const ListArgs& a, Visit visit) {
+  const int F = a.N * a.num_tiles;
+  const int per = (F + blockDim.x - 1) / blockDim.x;
+  const int lo = min(F, static_cast<int>(threadIdx.x) * per), hi = min(F, lo + per);
   int sum = 0;
+#pragma unroll 4
   for (int i = lo; i < hi; ++i) sum += a.tile_counts[i];
   int total;
   int run = block_exclusive_scan(sum, &total);
   for (int i = lo; i < hi; ++i) {
-    a.tile_base[i] = run;
+    visit(i, run);
     run += a.tile_counts[i];
   }
-  __syncthreads();
-  // counts / offsets per (e, b); grouped-GEMM tiles per (e, b).
+  return total;
+}
+
+// Counts, offsets and the grouped-GEMM tile table from the tile bases (all
+// of tile_base written and visible to the calling CTA).
+__device__ void write_list_meta(const ListArgs& a, int total) {
   const int EB = a.N * a.B;
-  const int per2 = (EB + blockDim.x - 1) / blockDim.x;
-  const int lo2 = min(EB, threadIdx.x * per2), hi2 = min(EB, lo2 + per2);
+  const int F = a.N * a.num_tiles;
+  const int per = (EB + blockDim.x - 1) / blockDim.x;
+  const int lo = min(EB, static_cast<int>(threadIdx.x) * per), hi = min(EB, lo + per);
   int nq = 0;
-  for (int i = lo2; i < hi2; ++i) {
+  for (int i = lo; i < hi; ++i) {
     const int e = i / a.B, b = i % a.B;
-    const size_t f0 = static_cast<size_t>(e) * a.num_tiles + static_cast<size_t>(b) * a.tiles_per_seq;
-    int c = 0;
-    for (int tb = 0; tb < a.tiles_per_seq; ++tb) c += a.tile_counts[f0 + tb];
+    const int f0 = e * a.num_tiles + b * a.tiles_per_seq, f1 = f0 + a.tiles_per_seq;
+    const int start = a.tile_base[f0];
+    const int c = (f1 < F ? a.tile_base[f1] : total) - start;
     a.counts[i] = c;
-    a.offsets[i] = a.tile_base[f0];
+    a.offsets[i] = start;
     nq += (c + kQTileRows - 1) / kQTileRows;
   }
   int nq_total;
   int qbase = block_exclusive_scan(nq, &nq_total);
-  for (int i = lo2; i < hi2; ++i) {
+  for (int i = lo; i < hi; ++i) {
     const int e = i / a.B, b = i % a.B;
     const int c = a.counts[i];
     for (int s = 0; s < c; s += kQTileRows) {
@@ -165,159 +203,107 @@ __global__ void __launch_bounds__(1024) scan_kernel(ListArgs a) {
   }
 }
 
-__global__ void __launch_bounds__(kThreads) scatter_kernel(ListArgs a) {
+// Step 2 on its own (many tiles): one CTA of 1024 threads.
+__global__ void __launch_bounds__(1024) scan_kernel(ListArgs a) {
   pdl_wait();
   pdl_launch_dependents();
+  const int total = tile_prefix(a, [&](int i, int pre) { a.tile_base[i] = pre; });
+  __syncthreads();
+  write_list_meta(a, total);
+}
+
+// Step 3 for one tile, given the tile's list bases per expert in shared
+// memory (base[e]).
+__device__ void scatter_tile(const ListArgs& a, int tile, const int* base) {
   __shared__ int wcnt[kThreads / 32][kMaxExperts];
-  __shared__ int run[kMaxExperts];
-  __shared__ int base[kMaxExperts];
-  const int tile = blockIdx.x;
   const int b = tile / a.tiles_per_seq;
-  const int t0 = (tile % a.tiles_per_seq) * kDispatchTile;
-  const int t1 = min(a.T, t0 + kDispatchTile);
+  const int t = (tile % a.tiles_per_seq) * kDispatchTile + threadIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned lt = (1u << lane) - 1u;
+  const size_t row = static_cast<size_t>(b) * a.T + t;
+  const uint64_t m = t < a.T ? a.masks[row] : 0ull;
+  int c0 = 0, c1 = 0;
+  for (int e = 0; e < a.N; ++e) {
+    const int n = __popc(__ballot_sync(0xffffffffu, (m >> e) & 1ull));
+    if (e == lane) c0 = n;
+    if (e == lane + 32) c1 = n;
+  }
+  if (lane < a.N) wcnt[warp][lane] = c0;
+  if (lane + 32 < a.N) wcnt[warp][lane + 32] = c1;
+  __syncthreads();
+  // Exclusive prefix over the warps, per expert (one thread per expert).
   for (int e = threadIdx.x; e < a.N; e += blockDim.x) {
-    run[e] = 0;
-    base[e] = a.tile_base[static_cast<size_t>(e) * a.num_tiles + tile];
+    int pre = base[e];
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) {
+      const int c = wcnt[w][e];
+      wcnt[w][e] = pre;
+      pre += c;
+    }
   }
   __syncthreads();
-  for (int c0 = t0; c0 < t1; c0 += blockDim.x) {
-    const int t = c0 + threadIdx.x;
-    const size_t row = static_cast<size_t>(b) * a.T + t;
-    uint64_t m = 0;
-    if (t < t1) token_mask(a, row, m);
-    for (int e = 0; e < a.N; ++e) {
-      const unsigned bal = __ballot_sync(0xffffffffu, (m >> e) & 1ull);
-      if (lane == 0) wcnt[warp][e] = __popc(bal);
+  int g = 0, j = 0;  // e = g * M + j, stepped with e
+  for (int e = 0; e < a.N; ++e) {
+    const bool f = (m >> e) & 1ull;
+    const unsigned bal = __ballot_sync(0xffffffffu, f);
+    if (f) {
+      const int pos = wcnt[warp][e] + __popc(bal & lt);
+      a.tok[pos] = t;
+      const uint64_t gm = (m >> (g * a.M)) & ((1ull << j) - 1ull);
+      a.slot_pos[(row * a.G + g) * a.k + __popcll(static_cast<long long>(gm))] = pos;
     }
-    __syncthreads();
-    for (int e = threadIdx.x; e < a.N; e += blockDim.x) {
-      int pre = run[e];
-      for (int w = 0; w < kThreads / 32; ++w) {
-        const int c = wcnt[w][e];
-        wcnt[w][e] = pre;
-        pre += c;
-      }
-      run[e] = pre;
+    if (++j == a.M) {
+      j = 0;
+      ++g;
     }
-    __syncthreads();
-    for (int e = 0; e < a.N; ++e) {
-      const bool f = (m >> e) & 1ull;
-      const unsigned bal = __ballot_sync(0xffffffffu, f);
-      if (f) {
-        const int pos = base[e] + wcnt[warp][e] + __popc(bal & lt);
-        a.tok[pos] = t;
-        const int g = e / a.M, j = e % a.M;
-        const uint64_t gm = (m >> (g * a.M)) & ((1ull << j) - 1ull);
-        const int s = __popcll(static_cast<long long>(gm));
-        a.slot_pos[(row * a.G + g) * a.k + s] = pos;
-      }
-    }
-    __syncthreads();
   }
 }
 
-// Single-CTA dispatch for small batches (kSmallRows rows or fewer): counts,
-// (expert, sequence) prefix sums, stable scatter and the grouped-GEMM tile
-// table in one kernel, with the same results as the three-pass path. Rows are
-// visited sequence by sequence, kSmallThreads at a time (one per thread), so
-// ranks within an (expert, sequence) list follow the positions t.
-constexpr int kSmallThreads = 1024;
-
-__global__ void __launch_bounds__(kSmallThreads) small_dispatch_kernel(ListArgs a) {
+__global__ void __launch_bounds__(kThreads) scatter_kernel(ListArgs a) {
   pdl_wait();
   pdl_launch_dependents();
-  __shared__ int wcnt[kSmallThreads / 32][kMaxExperts];
-  __shared__ int run[kMaxExperts];
-  extern __shared__ int eb_counts[];  // [N*B] counts, then exclusive offsets
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned lt = (1u << lane) - 1u;
-  const int EB = a.N * a.B;
-  for (int i = threadIdx.x; i < EB; i += blockDim.x) eb_counts[i] = 0;
+  __shared__ int base[kMaxExperts];
+  for (int e = threadIdx.x; e < a.N; e += blockDim.x)
+    base[e] = a.tile_base[static_cast<size_t>(e) * a.num_tiles + blockIdx.x];
   __syncthreads();
-  // Pass 1: counts per (e, b).
-  bool bad = false;
-  for (int row = threadIdx.x; row < a.B * a.T; row += blockDim.x) {
-    uint64_t m;
-    bad |= !token_mask(a, row, m);
-    const int b = row / a.T;
-    while (m) {
-      const int e = __ffsll(static_cast<long long>(m)) - 1;
-      m &= m - 1;
-      atomicAdd(&eb_counts[e * a.B + b], 1);
-    }
-  }
-  if (bad) set_status(GQE_ERR_DEVICE_CHECK);
-  __syncthreads();
-  // Exclusive scan in (e, b) order; counts and offsets out; tile counts.
+  scatter_tile(a, blockIdx.x, base);
+}
+
+// Steps 2 and 3 in one launch (few tiles): every CTA scans the tile counts
+// for its own bases; CTA 0 also writes tile_base, counts, offsets and the
+// tile table.
+constexpr int kFusedScanMax = 16384;  // N * num_tiles
+
+__global__ void __launch_bounds__(kThreads) scan_scatter_kernel(ListArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ int base[kMaxExperts];
+  const int tile = blockIdx.x;
+  const bool lead = blockIdx.x == 0;
+  const int F = a.N * a.num_tiles;
+  const int per = (F + kThreads - 1) / kThreads;
+  const int lo = min(F, static_cast<int>(threadIdx.x) * per), hi = min(F, lo + per);
+  int sum = 0;
+#pragma unroll 4
+  for (int i = lo; i < hi; ++i) sum += a.tile_counts[i];
   int total;
-  const int per = (EB + blockDim.x - 1) / blockDim.x;
-  const int lo = min(EB, threadIdx.x * per), hi = min(EB, lo + per);
-  int sum = 0, nq = 0;
+  int run = block_exclusive_scan(sum, &total);
+  int e = lo / a.num_tiles, tl = lo - e * a.num_tiles;  // index i = e * num_tiles + tl
   for (int i = lo; i < hi; ++i) {
-    sum += eb_counts[i];
-    nq += (eb_counts[i] + kQTileRows - 1) / kQTileRows;
-  }
-  int base = block_exclusive_scan(sum, &total);
-  int nq_total;
-  int qbase = block_exclusive_scan(nq, &nq_total);
-  for (int i = lo; i < hi; ++i) {
-    const int c = eb_counts[i];
-    a.counts[i] = c;
-    a.offsets[i] = base;
-    const int e = i / a.B, b = i % a.B;
-    for (int s = 0; s < c; s += kQTileRows) {
-      if (qbase < a.max_qtiles) a.qtiles[qbase] = make_int4(e, b, s, min(kQTileRows, c - s));
-      ++qbase;
+    if (tl == tile) base[e] = run;
+    if (lead) a.tile_base[i] = run;
+    run += a.tile_counts[i];
+    if (++tl == a.num_tiles) {
+      tl = 0;
+      ++e;
     }
-    eb_counts[i] = base;  // becomes the list start
-    base += c;
-  }
-  if (threadIdx.x == 0) {
-    a.offsets[EB] = total;
-    *a.n_qtiles = min(nq_total, a.max_qtiles);
-    if (nq_total > a.max_qtiles || total != a.k * a.G * a.B * a.T) set_status(GQE_ERR_DEVICE_CHECK);
   }
   __syncthreads();
-  // Pass 2: stable ranks, sequence by sequence.
-  for (int b = 0; b < a.B; ++b) {
-    for (int e = threadIdx.x; e < a.N; e += blockDim.x) run[e] = 0;
+  if (lead) {
+    write_list_meta(a, total);
     __syncthreads();
-    for (int c0 = 0; c0 < a.T; c0 += blockDim.x) {
-      const int t = c0 + threadIdx.x;
-      const size_t row = static_cast<size_t>(b) * a.T + t;
-      uint64_t m = 0;
-      if (t < a.T) token_mask(a, row, m);
-      for (int e = 0; e < a.N; ++e) {
-        const unsigned bal = __ballot_sync(0xffffffffu, (m >> e) & 1ull);
-        if (lane == 0) wcnt[warp][e] = __popc(bal);
-      }
-      __syncthreads();
-      for (int e = threadIdx.x; e < a.N; e += blockDim.x) {
-        int pre = run[e];
-        for (int w = 0; w < kSmallThreads / 32; ++w) {
-          const int c = wcnt[w][e];
-          wcnt[w][e] = pre;
-          pre += c;
-        }
-        run[e] = pre;
-      }
-      __syncthreads();
-      for (int e = 0; e < a.N; ++e) {
-        const bool f = (m >> e) & 1ull;
-        const unsigned bal = __ballot_sync(0xffffffffu, f);
-        if (f) {
-          const int pos = eb_counts[e * a.B + b] + wcnt[warp][e] + __popc(bal & lt);
-          a.tok[pos] = t;
-          const int g = e / a.M, j = e % a.M;
-          const uint64_t gm = (m >> (g * a.M)) & ((1ull << j) - 1ull);
-          a.slot_pos[(row * a.G + g) * a.k + __popcll(static_cast<long long>(gm))] = pos;
-        }
-      }
-      __syncthreads();
-    }
   }
+  scatter_tile(a, tile, base);
 }
 
 // Weighted slot: one thread per 8 columns of one row.
@@ -365,6 +351,8 @@ DispatchWs dispatch_ws_layout(const gqe_config& c) {
   const long long R = static_cast<long long>(c.B) * c.T;
   L.max_qtiles = static_cast<int>((static_cast<long long>(c.k) * c.G * R) / kQTileRows + N * c.B + 1);
   size_t o = 0;
+  L.masks = o;
+  o = align_up(o + static_cast<size_t>(R) * 8, 256);
   L.tile_counts = o;
   o = align_up(o + static_cast<size_t>(N) * L.num_tiles * 4, 256);
   L.tile_base = o;
@@ -388,6 +376,7 @@ int launch_dispatch_lists(const gqe_config& c, const int32_t* idx, int32_t* coun
   a.offsets = offsets;
   a.tok = tok;
   a.slot_pos = slot_pos;
+  a.masks = reinterpret_cast<uint64_t*>(w + L.masks);
   a.tile_counts = reinterpret_cast<int32_t*>(w + L.tile_counts);
   a.tile_base = reinterpret_cast<int32_t*>(w + L.tile_base);
   a.qtiles = reinterpret_cast<int4*>(w + L.qtiles);
@@ -401,13 +390,11 @@ int launch_dispatch_lists(const gqe_config& c, const int32_t* idx, int32_t* coun
   a.num_tiles = L.num_tiles;
   a.tiles_per_seq = L.tiles_per_seq;
   a.max_qtiles = L.max_qtiles;
-  const long long R = static_cast<long long>(c.B) * c.T;
-  if (R <= kSmallRows && static_cast<long long>(a.N) * c.B <= 8192) {
-    const size_t smem = static_cast<size_t>(a.N) * c.B * 4;
-    return launch_pdl(small_dispatch_kernel, dim3(1), dim3(kSmallThreads), smem, st, a);
-  }
-  cudaError_t e = launch_pdl(count_kernel, dim3(L.num_tiles), dim3(kThreads), 0, st, a);
-  if (e == cudaSuccess) e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, a);
+  cudaError_t e = launch_pdl(mask_count_kernel, dim3(L.num_tiles), dim3(kThreads), 0, st, a);
+  if (e != cudaSuccess) return e;
+  if (static_cast<long long>(a.N) * L.num_tiles <= kFusedScanMax)
+    return launch_pdl(scan_scatter_kernel, dim3(L.num_tiles), dim3(kThreads), 0, st, a);
+  e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, a);
   if (e == cudaSuccess) e = launch_pdl(scatter_kernel, dim3(L.num_tiles), dim3(kThreads), 0, st, a);
   return e;
 }

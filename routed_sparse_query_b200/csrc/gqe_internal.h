@@ -29,12 +29,10 @@ constexpr size_t kRouterSmemLimit = 200 * 1024;
 // Dispatch tiling: tokens of one sequence are cut into tiles of this size.
 constexpr int kDispatchTile = 256;  // == dispatch CTA size: one token per thread
 constexpr int kQTileRows = 128;  // rows of one grouped-GEMM tile
-// Batches of at most this many rows (and N*B*4 bytes of counts within the
-// 48 KiB static shared-memory limit) take the single-CTA dispatch.
-constexpr long long kSmallRows = 16384;
 
 struct DispatchWs {
   // Byte offsets inside the dispatch workspace.
+  size_t masks;        // uint64 [R]: selection bitmask per token
   size_t tile_counts;  // int32 [N][num_tiles]
   size_t tile_base;    // int32 [N][num_tiles]
   size_t qtiles;       // int4  [max_qtiles]: (e, b, start, rows)

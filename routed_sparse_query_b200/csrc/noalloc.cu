@@ -6,8 +6,9 @@
 // start-up, or a plugin interface that passes the library only its input and
 // output buffers), so they cannot call cudaMalloc, or any routine that
 // allocates, for each call. This entry point serves them: the caller passes
-// inputs and outputs only, and the dispatch scratch (per-tile counts and
-// bases, the grouped-GEMM tile table and its length) lives in kScratchBytes of
+// inputs and outputs only, and the dispatch scratch (per-token selection
+// masks, per-tile counts and bases, the grouped-GEMM tile table and its
+// length) lives in kScratchBytes of
 // statically allocated device memory that every GPU loading the library holds
 // until the process exits.
 //

@@ -6,15 +6,18 @@
 // gist.science Technical Summary, Methodology; softmax before top-k inside
 // the group, pptc.cn blog section 7.)
 //
-// One warp per token row. W_r is staged once per CTA in shared memory.
-// Lane l owns rows l, l+32, l+64, ... of the dot products and keeps NP
-// partial sums; a shuffle reduce-scatter leaves every logit complete on one
-// or more lanes, in a fixed order (the result is deterministic).
+// The logits are a small fp32 GEMM on the CUDA cores. A CTA takes a block of
+// TB tokens (TB * NP = 256 logits); W_r (zero padded to NP columns) and the
+// block's x rows sit in shared memory. Warp w sums rows [w d/8, (w+1) d/8)
+// of the dot products; each thread keeps 2 tokens x 4 experts, reading a W_r
+// row once per 2 tokens (broadcast over the warp's token lanes). The 8 warp
+// partials are then added in warp order, so every logit is one fixed
+// sequence of roundings (the result is deterministic).
 //
 // Exact selection: each fp32 logit carries the bound
 //   |z_fp32 - z| <= gamma_h * (||x||_1 * max_i |W_r[i,e]| + |b_e|),
-// h = d/32 + 6 roundings on its longest path (d/32 FMAs per lane, 5 shuffle
-// adds, the bias add), gamma_h = h u / (1 - h u), u = 2^-24 (Higham,
+// h = d/8 + 8 roundings on its longest path (d/8 FMAs in one warp, 7 adds
+// of the warp partials, the bias add), gamma_h = h u / (1 - h u), u = 2^-24 (Higham,
 // "Accuracy and Stability of Numerical Algorithms", 2nd ed., sec. 3.1). A
 // group whose top-k decision is not certain under these intervals (computed
 // with directed rounding) recomputes its logits in fp64 (products of a bf16
@@ -30,34 +33,19 @@ namespace gqe {
 
 namespace router_impl {
 
-constexpr int kRouterWarps = 8;
+constexpr int kRouterThreads = 256;
+constexpr int kRouterWarps = kRouterThreads / 32;  // warp w sums rows [w d/8, (w+1) d/8)
+constexpr int kTPT = 2;                            // tokens per thread
+
+// Tokens per CTA block: lanes are (token lane tt, expert quad et) with NP/4
+// quads, so a warp covers 128/NP token lanes of kTPT tokens each.
+__host__ __device__ constexpr int router_tb(int NP) { return kTPT * 128 / NP; }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t v) {
   return __uint_as_float(static_cast<uint32_t>(v) << 16);
 }
-
-template <int NP>
-__device__ __forceinline__ void reduce_scatter(float (&v)[NP], int lane) {
-#pragma unroll
-  for (int lvl = 0; lvl < 5; ++lvl) {
-    const int off = 16 >> lvl;
-    const int cnt = NP >> lvl;
-    if (cnt > 1) {
-      const int h = cnt / 2;
-      const bool upper = (lane & off) != 0;
-#pragma unroll
-      for (int i = 0; i < NP / 2; ++i) {
-        if (i < h) {
-          const float keep = upper ? v[i + h] : v[i];
-          const float send = upper ? v[i] : v[i + h];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
-      }
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
-    }
-  }
-}
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
 struct RouterArgs {
   const uint16_t* x;
@@ -69,185 +57,268 @@ struct RouterArgs {
   int R, d, G, M, k, N;
 };
 
+// Dynamic shared memory of one CTA (byte offsets).
+struct RouterLayout {
+  size_t w, xs, part, zd, zf, wmax, bsm, nx, ps, list, total;
+};
+__host__ __device__ inline RouterLayout router_layout(int d, int NP) {
+  const int TB = router_tb(NP);
+  RouterLayout L;
+  size_t o = 0;
+  L.w = o;     o += static_cast<size_t>(d) * NP * 4;                     // W_r [d][NP]
+  L.xs = o;    o += static_cast<size_t>(TB) * (d + 8) * 2;               // x [TB][d + 8]
+  L.part = o;  o += static_cast<size_t>(kRouterWarps) * TB * NP * 4;     // [warp][TB][NP]
+  L.zd = o;    o += static_cast<size_t>(TB) * NP * 8;                    // fp64 logits
+  L.zf = o;    o += static_cast<size_t>(TB) * NP * 4;                    // fp32 logits
+  L.wmax = o;  o += NP * 4;                                               // max_i |W_r[i, e]|
+  L.bsm = o;   o += NP * 4;                                               // bias
+  L.nx = o;    o += TB * 4;                                               // ||x||_1
+  L.ps = o;    o += static_cast<size_t>(TB) * NP * 4;                    // selected mass per pair
+  L.list = o;  o += static_cast<size_t>(TB) * NP * 4;                    // uncertain pairs
+  L.total = (o + 15) & ~static_cast<size_t>(15);
+  return L;
+}
+
+// Top-k of one group's M logits (descending, ties to the lower index) as a
+// bitmask over j.
+template <typename V>
+__device__ __forceinline__ uint64_t group_topk(const V* zg, int M, int k) {
+  uint64_t sel = 0;
+  for (int s = 0; s < k; ++s) {
+    V best = -INFINITY;
+    int bj = -1;
+    for (int j = 0; j < M; ++j) {
+      if (!((sel >> j) & 1ull) && (bj < 0 || zg[j] > best)) {
+        best = zg[j];
+        bj = j;
+      }
+    }
+    sel |= 1ull << bj;
+  }
+  return sel;
+}
+
 template <int NP>
-__global__ void __launch_bounds__(kRouterWarps * 32) router_kernel(RouterArgs a) {
-  constexpr int S = router_row_floats(NP);
+__global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
+  constexpr int TB = router_tb(NP);
+  constexpr int EG = NP / 4;   // expert quads
+  constexpr int TG = 32 / EG;  // token lanes per warp; TB == kTPT * TG
+  static_assert(TB == kTPT * TG, "block shape");
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* Wsm = reinterpret_cast<float*>(smem_raw);                 // [d][S]
-  float* wmax = Wsm + static_cast<size_t>(a.d) * S;                 // [NP]
-  float* bsm = wmax + NP;                                           // [NP]
-  double* zd_all = reinterpret_cast<double*>(bsm + NP);             // [warps][NP]
-  float* zf_all = reinterpret_cast<float*>(zd_all + kRouterWarps * NP);  // [max(warps*NP, 256)]
+  __shared__ int n_uncertain;
+  const RouterLayout L = router_layout(a.d, NP);
+  float* Ws = reinterpret_cast<float*>(smem_raw + L.w);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw + L.xs);
+  float* part = reinterpret_cast<float*>(smem_raw + L.part);
+  double* zd = reinterpret_cast<double*>(smem_raw + L.zd);
+  float* zf = reinterpret_cast<float*>(smem_raw + L.zf);
+  float* wmax = reinterpret_cast<float*>(smem_raw + L.wmax);
+  float* bsm = reinterpret_cast<float*>(smem_raw + L.bsm);
+  float* nxs = reinterpret_cast<float*>(smem_raw + L.nx);
+  float* ps = reinterpret_cast<float*>(smem_raw + L.ps);
+  int* list = reinterpret_cast<int*>(smem_raw + L.list);
 
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int et = lane % EG, tt = lane / EG;
+  const int XS = a.d + 8;  // x row stride in shared memory (16-byte pad: no bank conflicts)
+  const int cpr = a.d / 8;  // 16-byte chunks per x row
+  const int n_blk = (a.R + TB - 1) / TB;
+
+  // Stages the TB rows of a block (rows past R repeat the last row); always
+  // commits one cp.async group (empty past the end).
+  auto stage_x = [&](int blk) {
+    if (blk < n_blk) {
+      for (int t = warp; t < TB; t += kRouterWarps) {
+        const uint16_t* src = a.x + static_cast<size_t>(min(blk * TB + t, a.R - 1)) * a.d;
+        for (int c = lane; c < cpr; c += 32) cp_async_16(smem_u32(xs + t * XS + c * 8), src + c * 8, 16u);
+      }
+    }
+    cp_async_commit();
+  };
+
   pdl_wait();
   pdl_launch_dependents();
 
-  // Stage W_r (zero padded to S columns) and the bias. Rows of 4k floats are
-  // copied with 16-byte cp.async so that all loads are in flight at once.
-  if ((a.N & 3) == 0) {
-    const int cpr = a.N >> 2;  // 16-byte chunks per row
-    for (int i = tid; i < a.d * cpr; i += blockDim.x) {
-      const int row = i / cpr, c = i - row * cpr;
-      cp_async_16(smem_u32(Wsm + row * S + 4 * c), a.W_r + static_cast<size_t>(row) * a.N + 4 * c, 16u);
+  // W_r into shared memory. Each CTA starts at a different chunk so that the
+  // CTAs do not all read the same L2 lines at once.
+  if (a.N == NP) {
+    const int total = a.d * NP / 4;  // 16-byte chunks
+    const int rot = static_cast<int>((static_cast<long long>(blockIdx.x) * 256) % total);
+    for (int i = tid; i < total; i += kRouterThreads) {
+      int j = i + rot;
+      if (j >= total) j -= total;
+      cp_async_16(smem_u32(Ws + 4 * j), a.W_r + 4 * static_cast<size_t>(j), 16u);
     }
-    cp_async_commit();
   } else {
-    for (int i = tid; i < a.d * a.N; i += blockDim.x) {
-      const int row = i / a.N, col = i - row * a.N;
-      Wsm[row * S + col] = a.W_r[i];
+    for (int i = tid; i < a.d * NP; i += kRouterThreads) {
+      const int row = i / NP, col = i % NP;
+      Ws[i] = col < a.N ? a.W_r[static_cast<size_t>(row) * a.N + col] : 0.0f;
     }
   }
-  for (int i = tid; i < a.d * (S - a.N); i += blockDim.x) {
-    const int row = i / (S - a.N), col = a.N + i % (S - a.N);
-    Wsm[row * S + col] = 0.0f;
-  }
-  cp_async_wait<0>();
-  for (int e = tid; e < NP; e += blockDim.x) bsm[e] = (e < a.N && a.b_r != nullptr) ? a.b_r[e] : 0.0f;
+  cp_async_commit();
+  int blk = blockIdx.x;
+  stage_x(blk);
+  cp_async_wait<1>();  // this thread's part of W_r is in
+  for (int e = tid; e < NP; e += kRouterThreads) bsm[e] = (e < a.N && a.b_r != nullptr) ? a.b_r[e] : 0.0f;
   __syncthreads();
-  // max_i |W_r[i, e]|: thread t scans column t % NP over rows t / NP (mod
-  // the number of parts), then one thread per column combines the parts.
+  // max_i |W_r[i, e]|: thread t scans column t % NP over every (256/NP)-th
+  // row, then one thread per column combines the parts.
   {
-    constexpr int parts = kRouterWarps * 32 / NP;
-    float mx = 0.0f;
-    const int col = tid % NP, part = tid / NP;
-    for (int row = part; row < a.d; row += parts) mx = fmaxf(mx, fabsf(Wsm[row * S + col]));
-    zf_all[tid] = mx;  // zf_all has room for kRouterWarps * 32 floats
+    constexpr int parts = kRouterThreads / NP;
+    const int col = tid % NP, p0 = tid / NP;
+    float m0 = 0.0f, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
+    int row = p0;
+    for (; row + 3 * parts < a.d; row += 4 * parts) {
+      m0 = fmaxf(m0, fabsf(Ws[row * NP + col]));
+      m1 = fmaxf(m1, fabsf(Ws[(row + parts) * NP + col]));
+      m2 = fmaxf(m2, fabsf(Ws[(row + 2 * parts) * NP + col]));
+      m3 = fmaxf(m3, fabsf(Ws[(row + 3 * parts) * NP + col]));
+    }
+    for (; row < a.d; row += parts) m0 = fmaxf(m0, fabsf(Ws[row * NP + col]));
+    part[tid] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
     __syncthreads();
     if (tid < NP) {
-      float m2 = 0.0f;
-      for (int p = 0; p < parts; ++p) m2 = fmaxf(m2, zf_all[p * NP + tid]);
-      wmax[tid] = m2;
+      float mx = 0.0f;
+      for (int p = 0; p < parts; ++p) mx = fmaxf(mx, part[p * NP + tid]);
+      wmax[tid] = mx;
     }
-    __syncthreads();
   }
 
-  double* zd = zd_all + warp * NP;
-  float* zf = zf_all + warp * NP;
-  const int h = a.d / 32 + 6;
+  const int h = a.d / kRouterWarps + kRouterWarps;
   const float u = 5.9604644775390625e-08f;  // 2^-24
   const float gam = (h * u) / (1.0f - h * u);
   const float gam_ru = __fmul_ru(gam, 1.01f);
+  const int slice = a.d / kRouterWarps;
+  const int P = TB * a.G;  // (token, group) pairs of a block
 
-  const int nwarps_total = gridDim.x * kRouterWarps;
-  for (int row = blockIdx.x * kRouterWarps + warp; row < a.R; row += nwarps_total) {
-    const uint16_t* xr = a.x + static_cast<size_t>(row) * a.d;
-    float acc[NP];
-#pragma unroll
-    for (int e = 0; e < NP; ++e) acc[e] = 0.0f;
-    float nx = 0.0f;
-#pragma unroll 8
-    for (int m = lane; m < a.d; m += 32) {
-      const float xi = bf16_to_f32(xr[m]);
-      nx += fabsf(xi);
-      const float4* w4 = reinterpret_cast<const float4*>(Wsm + m * S);
-#pragma unroll
-      for (int q = 0; q < NP / 4; ++q) {
-        const float4 w = w4[q];
-        acc[4 * q + 0] = fmaf(xi, w.x, acc[4 * q + 0]);
-        acc[4 * q + 1] = fmaf(xi, w.y, acc[4 * q + 1]);
-        acc[4 * q + 2] = fmaf(xi, w.z, acc[4 * q + 2]);
-        acc[4 * q + 3] = fmaf(xi, w.w, acc[4 * q + 3]);
-      }
-    }
-    reduce_scatter<NP>(acc, lane);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) nx += __shfl_xor_sync(0xffffffffu, nx, off);
+  for (; blk < n_blk; blk += gridDim.x) {
+    cp_async_wait<0>();
+    __syncthreads();  // x rows in; the previous block's decisions are done
 
-    // Owner lanes write the logits (+ bias) to the warp's scratch.
-    if constexpr (NP >= 32) {
+    // Partial logits over this warp's rows, in ascending row order.
+    float acc[kTPT][4];
 #pragma unroll
-      for (int i = 0; i < NP / 32; ++i) {
-        const int e = lane * (NP / 32) + i;
-        zf[e] = acc[i] + bsm[e];
-      }
-    } else {
-      constexpr int per = 32 / NP;
-      if (lane % per == 0) {
-        const int e = lane / per;
-        zf[e] = acc[0] + bsm[e];
-      }
-    }
-    __syncwarp();
-
-    // Lane g decides group g.
-    const int g = lane;
-    bool certain = true;
-    uint64_t selmask = 0;
-    if (g < a.G) {
-      const float* zg = zf + g * a.M;
-      for (int s = 0; s < a.k; ++s) {
-        float best = -INFINITY;
-        int bj = -1;
-        for (int j = 0; j < a.M; ++j) {
-          if (!((selmask >> j) & 1ull) && (bj < 0 || zg[j] > best)) {
-            best = zg[j];
-            bj = j;
-          }
+    for (int i = 0; i < kTPT; ++i)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[i][q] = 0.0f;
+    const int m_lo = warp * slice;
+#pragma unroll 2
+    for (int m = m_lo; m < m_lo + slice; m += 8) {
+      uint4 xv[kTPT];
+#pragma unroll
+      for (int i = 0; i < kTPT; ++i) xv[i] = *reinterpret_cast<const uint4*>(xs + (tt + TG * i) * XS + m);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 w = *reinterpret_cast<const float4*>(Ws + (m + q) * NP + 4 * et);
+#pragma unroll
+        for (int i = 0; i < kTPT; ++i) {
+          const uint32_t word = q < 2 ? xv[i].x : q < 4 ? xv[i].y : q < 6 ? xv[i].z : xv[i].w;
+          const float xf = (q & 1) ? bf16_hi(word) : bf16_lo(word);
+          acc[i][0] = fmaf(xf, w.x, acc[i][0]);
+          acc[i][1] = fmaf(xf, w.y, acc[i][1]);
+          acc[i][2] = fmaf(xf, w.z, acc[i][2]);
+          acc[i][3] = fmaf(xf, w.w, acc[i][3]);
         }
-        selmask |= 1ull << bj;
       }
+    }
+#pragma unroll
+    for (int i = 0; i < kTPT; ++i)
+      *reinterpret_cast<float4*>(part + (warp * TB + tt + TG * i) * NP + 4 * et) =
+          make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    // ||x||_1 per token (warp-strided tokens, lane-strided chunks).
+    for (int t = warp; t < TB; t += kRouterWarps) {
+      float sx = 0.0f;
+      for (int c = lane; c < cpr; c += 32) {
+        const uint4 v = *reinterpret_cast<const uint4*>(xs + t * XS + c * 8);
+        sx += fabsf(bf16_lo(v.x)) + fabsf(bf16_hi(v.x)) + fabsf(bf16_lo(v.y)) + fabsf(bf16_hi(v.y)) +
+              fabsf(bf16_lo(v.z)) + fabsf(bf16_hi(v.z)) + fabsf(bf16_lo(v.w)) + fabsf(bf16_hi(v.w));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, off);
+      if (lane == 0) nxs[t] = sx;
+    }
+    if (tid == 0) n_uncertain = 0;
+    __syncthreads();
+    // The x rows are consumed: fetch the next block while this one is decided.
+    stage_x(blk + gridDim.x);
+
+    // Logits: warp partials added in warp order, then the bias.
+    for (int i = tid; i < TB * NP; i += kRouterThreads) {
+      float z = part[i];
+#pragma unroll
+      for (int w = 1; w < kRouterWarps; ++w) z += part[w * TB * NP + i];
+      zf[i] = z + bsm[i % NP];
+    }
+    __syncthreads();
+
+    // Top-k per (token, group) on the fp32 logits, certified by the bound.
+    for (int p = tid; p < P; p += kRouterThreads) {
+      const int t = p / a.G, g = p - t * a.G;
+      if (blk * TB + t >= a.R) continue;
+      const float* zg = zf + t * NP + g * a.M;
+      bool certain = true;
       if (a.k < a.M) {
+        const uint64_t sel = group_topk(zg, a.M, a.k);
+        const float nx = nxs[t];
         float lo = INFINITY, hi = -INFINITY;
         for (int j = 0; j < a.M; ++j) {
           const int e = g * a.M + j;
           const float bd = __fmul_ru(gam_ru, __fmaf_ru(nx, wmax[e], fabsf(bsm[e])));
-          if ((selmask >> j) & 1ull) lo = fminf(lo, __fsub_rd(zg[j], bd));
+          if ((sel >> j) & 1ull) lo = fminf(lo, __fsub_rd(zg[j], bd));
           else hi = fmaxf(hi, __fadd_ru(zg[j], bd));
         }
         certain = lo > hi;
       }
+      for (int j = 0; j < a.M; ++j) zd[t * NP + g * a.M + j] = static_cast<double>(zg[j]);
+      if (!certain) list[atomicAdd(&n_uncertain, 1)] = p;
     }
-    for (int e = lane; e < a.N; e += 32) zd[e] = static_cast<double>(zf[e]);
-    unsigned todo = __ballot_sync(0xffffffffu, !certain);
-    __syncwarp();
-    // fp64 re-evaluation of the groups whose decision was not certain.
-    while (todo) {
-      const int gg = __ffs(todo) - 1;
-      todo &= todo - 1;
+    __syncthreads();
+    // fp64 logits of the uncertain groups, one warp per group (products of a
+    // bf16 and an fp32 value are exact in fp64).
+    const int nu = n_uncertain;
+    for (int v = warp; v < nu; v += kRouterWarps) {
+      const int p = list[v];
+      const int t = p / a.G, g = p - t * a.G;
+      const uint16_t* xr = a.x + static_cast<size_t>(blk * TB + t) * a.d;
       for (int j = 0; j < a.M; ++j) {
-        const int e = gg * a.M + j;
+        const int e = g * a.M + j;
         double s64 = 0.0;
         for (int m = lane; m < a.d; m += 32)
-          s64 = fma(static_cast<double>(bf16_to_f32(xr[m])), static_cast<double>(Wsm[m * S + e]), s64);
+          s64 = fma(static_cast<double>(bf16_to_f32(xr[m])), static_cast<double>(Ws[m * NP + e]), s64);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) s64 += __shfl_xor_sync(0xffffffffu, s64, off);
-        if (lane == 0) zd[e] = s64 + static_cast<double>(bsm[e]);
+        if (lane == 0) zd[t * NP + e] = s64 + static_cast<double>(bsm[e]);
       }
     }
-    __syncwarp();
-
-    float psel_sum = 0.0f;
-    if (g < a.G) {
-      const double* zg = zd + g * a.M;
-      if (!certain) {  // re-select on the fp64 logits
-        selmask = 0;
-        for (int s = 0; s < a.k; ++s) {
-          double best = -INFINITY;
-          int bj = -1;
-          for (int j = 0; j < a.M; ++j) {
-            if (!((selmask >> j) & 1ull) && (bj < 0 || zg[j] > best)) {
-              best = zg[j];
-              bj = j;
-            }
-          }
-          selmask |= 1ull << bj;
-        }
-      }
+    __syncthreads();
+    // Group softmax; selected mass per pair. (The fp64 values of certain
+    // groups are their fp32 logits, so the selection is the one made above.)
+    for (int p = tid; p < P; p += kRouterThreads) {
+      const int t = p / a.G, g = p - t * a.G;
+      if (blk * TB + t >= a.R) continue;
+      const double* zg = zd + t * NP + g * a.M;
+      const uint64_t sel = group_topk(zg, a.M, a.k);
       double zmax = zg[0];
       for (int j = 1; j < a.M; ++j) zmax = fmax(zmax, zg[j]);
       float den = 0.0f;
       for (int j = 0; j < a.M; ++j) den += expf(static_cast<float>(zg[j] - zmax));
+      float psel = 0.0f;
       for (int j = 0; j < a.M; ++j)
-        if ((selmask >> j) & 1ull) psel_sum += expf(static_cast<float>(zg[j] - zmax)) / den;
+        if ((sel >> j) & 1ull) psel += expf(static_cast<float>(zg[j] - zmax)) / den;
+      ps[p] = psel;
     }
-    float tot = psel_sum;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
-    if (g < a.G) {
-      const double* zg = zd + g * a.M;
+    __syncthreads();
+    // idx, r (renormalised in the group) and omega (over the token's groups).
+    for (int p = tid; p < P; p += kRouterThreads) {
+      const int t = p / a.G, g = p - t * a.G;
+      const int row = blk * TB + t;
+      if (row >= a.R) continue;
+      const double* zg = zd + t * NP + g * a.M;
+      const uint64_t sel = group_topk(zg, a.M, a.k);
+      float tot = 0.0f;
+      for (int g2 = 0; g2 < a.G; ++g2) tot += ps[t * a.G + g2];
+      const float psel = ps[p];
       double zmax = zg[0];
       for (int j = 1; j < a.M; ++j) zmax = fmax(zmax, zg[j]);
       float den = 0.0f;
@@ -255,43 +326,38 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_kernel(RouterArgs a)
       const size_t o = (static_cast<size_t>(row) * a.G + g) * a.k;
       int s = 0;
       for (int j = 0; j < a.M; ++j) {
-        if ((selmask >> j) & 1ull) {
-          const float p = expf(static_cast<float>(zg[j] - zmax)) / den;
+        if ((sel >> j) & 1ull) {
+          const float pj = expf(static_cast<float>(zg[j] - zmax)) / den;
           a.idx[o + s] = j;
-          a.r[o + s] = p / psel_sum;
-          a.omega[o + s] = p / tot;
+          a.r[o + s] = pj / psel;
+          a.omega[o + s] = pj / tot;
           ++s;
         }
       }
     }
-    __syncwarp();
   }
+  cp_async_wait<0>();
 }
-
 
 template <int NP>
 int launch_np(const gqe_config& c, const RouterArgs& a, cudaStream_t st) {
-  constexpr int S = router_row_floats(NP);
   const size_t smem = router_smem_bytes(c);
   if (smem > kRouterSmemLimit) return cudaErrorInvalidConfiguration;
   const int e = ensure_smem<router_kernel<NP>>(static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  // One token per warp while that fills the GPU; larger batches loop.
-  const int R = a.R;
-  int grid = (R + kRouterWarps - 1) / kRouterWarps;
-  if (grid > 4 * 148) grid = 4 * 148;
+  // One block per CTA while that fills the GPU; larger batches loop.
+  const int n_blk = (a.R + router_tb(NP) - 1) / router_tb(NP);
+  const int per_sm = smem <= 112 * 1024 ? 2 : 1;
+  int grid = n_blk < per_sm * 148 ? n_blk : per_sm * 148;
   if (grid < 1) grid = 1;
-  return launch_pdl(router_kernel<NP>, dim3(grid), dim3(kRouterWarps * 32), smem, st, a);
+  return launch_pdl(router_kernel<NP>, dim3(grid), dim3(kRouterThreads), smem, st, a);
 }
 
 }  // namespace router_impl
 using namespace router_impl;
 
 size_t router_smem_bytes(const gqe_config& c) {
-  const int NP = router_np(c.G * c.M);
-  const size_t zf = kRouterWarps * NP > kRouterWarps * 32 ? kRouterWarps * NP : kRouterWarps * 32;
-  return static_cast<size_t>(c.d_model) * router_row_floats(NP) * 4 + 2 * NP * 4 +
-         kRouterWarps * NP * 8 + zf * 4;
+  return router_layout(c.d_model, router_np(c.G * c.M)).total;
 }
 
 int launch_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r,
