@@ -10,17 +10,19 @@
 // chatpaper / hotpaper abstract; 9 of 16 heads active: gist.science Technical
 // Summary, Experimental Results).
 //
-// One CTA = one 128-row query tile of one stream; KV tiles of 128 keys up to
-// the diagonal (fully masked tiles are never loaded). Warp roles (192
+// One CTA = two consecutive 128-row query tiles (a, b) of one stream, or a
+// KV chunk of them (split-KV for short sequences); KV tiles of 128 keys up to
+// the diagonal (fully masked tiles are never loaded). Warp roles (320
 // threads):
-//   warps 0-3  softmax: thread i owns query row i (TMEM lane i); online
-//              softmax in fp32 (exp2 with the 1/sqrt(dh)*log2(e) scale folded
-//              in), P written to shared memory as bf16 in the UMMA K-major
-//              128B-swizzled layout, O rescaled in TMEM, final O / l stored;
-//   warp 4     TMA loads of Q and of K/V tiles (3-stage ring);
-//   warp 5     one thread issues S = Q K^T into one of two TMEM S buffers
-//              (S_{j+1} overlaps the softmax of S_j) and O += P V.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+dh).
+//   warps 0-7  softmax, warpgroup t for tile t: thread i owns query row i
+//              (TMEM lane i); online softmax in fp32 (exp2 with the
+//              1/sqrt(dh)*log2(e) scale folded in); P is written back over S
+//              in tensor memory as bf16 pairs; O is rescaled in TMEM only when
+//              the row max grows by more than 2^8; final O / l stored;
+//   warp 8     TMA loads of Q and of K/V tiles (4-stage ring);
+//   warp 9     issues S = Q K^T into three rotating TMEM S buffers and
+//              O += P V with P read from tensor memory.
+// TMEM columns: S buffers [0,128), [128,256), [256,384); O_a, O_b at 384.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -36,7 +38,7 @@ namespace attn_impl {
 
 constexpr int BQ = 128;
 constexpr int BKV = 128;
-constexpr int KV_STAGES = 3;
+constexpr int KV_STAGES = 4;
 constexpr int kThreads = 320;  // 2 softmax warpgroups + TMA warp + UMMA warp
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -49,9 +51,7 @@ struct AttnCfg {
   static constexpr int SWB = DH * 2;  // bytes per Q/K/V row = swizzle width
   static constexpr uint32_t LAYOUT = SWB == 128 ? kLayoutSW128 : kLayoutSW64;
   static constexpr int TILE_BYTES = BQ * DH * 2;
-  static constexpr int P_BYTES = BQ * BKV * 2;
-  static constexpr size_t SMEM =
-      1024 + static_cast<size_t>(TILE_BYTES) * (2 + 2 * KV_STAGES) + 2 * P_BYTES + 512;
+  static constexpr size_t SMEM = 1024 + static_cast<size_t>(TILE_BYTES) * (2 + 2 * KV_STAGES) + 512;
   static constexpr uint32_t TMEM_COLS = 512;  // 3 rotating S buffers (128 each), O_a, O_b (DH each)
 };
 
@@ -123,16 +123,17 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 }
 
 // Online softmax of one query row against one 128-key tile held in TMEM
-// (tS): pass 1 takes the row max, pass 2 writes P = 2^(s*scale - m) as bf16
-// into the UMMA K-major 128B-swizzled layout at prow and adds it to l. Only
-// the diagonal tile (MASK) tests keys against the row's position: key x is
-// visible iff x <= lim. O (tO) is rescaled only when the max grows by more
-// than kRescaleLog2.
+// (tS): pass 1 takes the row max, pass 2 computes P = 2^(s*scale - m), adds
+// it to l and writes it as bf16 pairs over the first 64 columns of the same
+// S buffer (the A operand of the PV product; each 32-column chunk of S is
+// read before the P columns over it are written). Only the diagonal tile
+// (MASK) tests keys against the row's position: key x is visible iff
+// x <= lim. O (tO) is rescaled only when the max grows by more than
+// kRescaleLog2; the rescale first waits for the previous PV (pv_prev).
 template <int DH, bool MASK>
-__device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, uint8_t* prow, int i,
-                                             int lim, float sc, bool first, float& m, float& l,
-                                             uint64_t* pv_prev, uint32_t pv_parity,
-                                             volatile int* abort_flag) {
+__device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int lim, float sc,
+                                             bool first, float& m, float& l, uint64_t* pv_prev,
+                                             uint32_t pv_parity, volatile int* abort_flag) {
   // TMEM loads are software-pipelined: chunk c+1 (32 columns) is in flight
   // while chunk c is processed.
   float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -167,14 +168,15 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, uint8_t* 
   row_max(vb, 3);
 
   const float mc = fmaxf(max3(mx[0], mx[1], mx[2]), mx[3]) * sc;
-  if (pv_prev != nullptr &&
-      !__all_sync(0xffffffffu, mbar_wait(pv_prev, pv_parity, abort_flag))) {
-    tmem_ld_wait(va);
-    return false;
-  }
-  tc_fence_after();
   const bool need = mc > m + kRescaleLog2;
   if (__any_sync(0xffffffffu, need)) {
+    if (pv_prev != nullptr) {  // O holds earlier tiles: their PV must be complete
+      if (!__all_sync(0xffffffffu, mbar_wait(pv_prev, pv_parity, abort_flag))) {
+        tmem_ld_wait(va);
+        return false;
+      }
+      tc_fence_after();
+    }
     const float m_new = need ? mc : m;
     const float alpha = ex2(m - m_new);
     if (!first) {
@@ -195,6 +197,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, uint8_t* 
   float2 lsum[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
                     make_float2(0.0f, 0.0f)};  // independent partial sums (no serial chain)
   auto exp_chunk = [&](const uint32_t (&v)[32], int c) {
+    uint32_t pw[16];
 #pragma unroll
     for (int c8 = 0; c8 < 4; ++c8) {
       const int c16 = c * 4 + c8;  // 8-key chunk index in the row
@@ -221,14 +224,12 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, uint8_t* 
         e8[x + 1] = e.y;
         lsum[x >> 1] = fadd2(lsum[x >> 1], e);
       }
-      uint4 o;
-      o.x = pack_bf16x2(e8[0], e8[1]);
-      o.y = pack_bf16x2(e8[2], e8[3]);
-      o.z = pack_bf16x2(e8[4], e8[5]);
-      o.w = pack_bf16x2(e8[6], e8[7]);
-      const int kc = c16 >> 3, cw = c16 & 7;
-      *reinterpret_cast<uint4*>(prow + kc * (BQ * 128) + ((cw ^ (i & 7)) << 4)) = o;
+      pw[4 * c8 + 0] = pack_bf16x2(e8[0], e8[1]);
+      pw[4 * c8 + 1] = pack_bf16x2(e8[2], e8[3]);
+      pw[4 * c8 + 2] = pack_bf16x2(e8[4], e8[5]);
+      pw[4 * c8 + 3] = pack_bf16x2(e8[6], e8[7]);
     }
+    tmem_st16(tS + c * 16, pw);  // keys 32c..32c+31 -> columns 16c..16c+15
   };
   tmem_ld_wait(va);
   tmem_ld32_nowait(tS + 32, vb);
@@ -241,6 +242,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, uint8_t* 
   exp_chunk(va, 2);
   tmem_ld_wait(vb);
   exp_chunk(vb, 3);
+  tmem_st_wait();
   const float2 l01 = fadd2(lsum[0], lsum[1]), l23 = fadd2(lsum[2], lsum[3]);
   const float2 l4 = fadd2(l01, l23);
   l += l4.x + l4.y;
@@ -293,15 +295,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = sp;                                // [2][TILE]
   uint8_t* sK = sQ + 2 * C::TILE_BYTES;            // [KV_STAGES][TILE]
   uint8_t* sV = sK + KV_STAGES * C::TILE_BYTES;    // [KV_STAGES][TILE]
-  uint8_t* sP = sV + KV_STAGES * C::TILE_BYTES;    // [2][P]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sP + 2 * C::P_BYTES);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sV + KV_STAGES * C::TILE_BYTES);
   uint64_t* q_full = bar;
   uint64_t* k_full = bar + 1;
   uint64_t* v_full = k_full + KV_STAGES;
   uint64_t* kv_empty = v_full + KV_STAGES;
   uint64_t* s_full = kv_empty + KV_STAGES;  // [3] one per S buffer
   uint64_t* p_full = s_full + 3;            // [2] one per query tile
-  uint64_t* o_done = p_full + 2;            // [2]
+  uint64_t* o_done = p_full + 2;            // [2] one per query tile
   uint64_t* drain = o_done + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
@@ -418,7 +419,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dQ = smem_desc(smem_u32(sQ), 16, 8 * C::SWB, C::LAYOUT);
       const uint64_t dK = smem_desc(smem_u32(sK), 16, 8 * C::SWB, C::LAYOUT);
       const uint64_t dV = smem_desc(smem_u32(sV), C::TILE_BYTES, 8 * C::SWB, C::LAYOUT);
-      const uint64_t dP = smem_desc(smem_u32(sP), 16, 1024, kLayoutSW128);
       auto wait_all = [&](uint64_t* b, uint32_t par) {
         return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag));
       };
@@ -450,12 +450,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint64_t p0 = dP + static_cast<uint64_t>((t * C::P_BYTES) >> 4);
+        // P(m) sits over the first 64 columns of S buffer m % 3.
+        const uint32_t aP = tmem + (m % 3) * 128;
         const uint64_t v0 = dV + static_cast<uint64_t>((st * C::TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk)
-          umma_bf16_ss_elect(tmem + 384 + t * DH, p0 + ((kk >> 2) * (BQ * 128) + (kk & 3) * 32) / 16,
-                             v0 + (kk * 16 * C::SWB) / 16, idO, (jr > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts_elect(tmem + 384 + t * DH, aP + kk * 8, v0 + (kk * 16 * C::SWB) / 16, idO,
+                             (jr > 0 || kk > 0) ? 1u : 0u);
         umma_commit_elect(&o_done[t]);
         if (t == 1 || !has_b) umma_commit_elect(&kv_empty[st]);  // last reader of K_j, V_j
         // S(m+3) follows PV(m): with one tile it needs K_{j+3}, which shares a
@@ -474,7 +475,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qi = qt * BQ + i;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tO = tmem + 384 + t * DH + lane_off;
-    uint8_t* prow = sP + t * C::P_BYTES + i * 128;
     const float sc = p.scale_log2;
     float m = -INFINITY, l = 0.0f;
     bool ok = n_t > 0;
@@ -489,22 +489,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      // PV of the previous KV tile must be complete before O is rescaled and
-      // before this tile's single P buffer is overwritten; softmax_tile waits
-      // for it after its max pass.
+      // PV(jr - 1) must be complete before O is rescaled (softmax_tile waits
+      // for it only then) and before P(jr) is published: the issuer waits for
+      // the phases of p_full[t] one at a time, so this tile may run at most
+      // one phase ahead of it. The exp pass overlaps PV(jr - 1).
       uint64_t* pv_prev = jr > 0 ? &o_done[t] : nullptr;
+      const uint32_t pv_par = static_cast<uint32_t>(jr - 1) & 1u;
       bool w_ok = true;
       if (j == qt)  // the diagonal tile
-        w_ok = softmax_tile<DH, true>(tS, tO, prow, i, qi - j * BKV, sc, jr == 0, m, l, pv_prev,
-                                      (jr - 1) & 1, abort_flag);
+        w_ok = softmax_tile<DH, true>(tS, tO, qi - j * BKV, sc, jr == 0, m, l, pv_prev, pv_par,
+                                      abort_flag);
       else
-        w_ok = softmax_tile<DH, false>(tS, tO, prow, i, BKV, sc, jr == 0, m, l, pv_prev,
-                                       (jr - 1) & 1, abort_flag);
+        w_ok = softmax_tile<DH, false>(tS, tO, BKV, sc, jr == 0, m, l, pv_prev, pv_par, abort_flag);
+      if (w_ok && jr >= 1) w_ok = __all_sync(0xffffffffu, mbar_wait(pv_prev, pv_par, abort_flag));
       if (!w_ok) {
         ok = false;
         break;
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }

@@ -196,30 +196,46 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
     cp_async_wait<0>();
     __syncthreads();  // x rows in; the previous block's decisions are done
 
-    // Partial logits over this warp's rows, in ascending row order.
+    // Partial logits over this warp's rows, in ascending row order. The
+    // shared-memory reads of the next 8 rows are issued before the FMAs of
+    // the current 8.
     float acc[kTPT][4];
 #pragma unroll
     for (int i = 0; i < kTPT; ++i)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[i][q] = 0.0f;
-    const int m_lo = warp * slice;
-#pragma unroll 2
-    for (int m = m_lo; m < m_lo + slice; m += 8) {
-      uint4 xv[kTPT];
+    auto load8 = [&](int m, uint4 (&xv)[kTPT], float4 (&wv)[8]) {
 #pragma unroll
       for (int i = 0; i < kTPT; ++i) xv[i] = *reinterpret_cast<const uint4*>(xs + (tt + TG * i) * XS + m);
 #pragma unroll
+      for (int q = 0; q < 8; ++q) wv[q] = *reinterpret_cast<const float4*>(Ws + (m + q) * NP + 4 * et);
+    };
+    auto fma8 = [&](const uint4 (&xv)[kTPT], const float4 (&wv)[8]) {
+#pragma unroll
       for (int q = 0; q < 8; ++q) {
-        const float4 w = *reinterpret_cast<const float4*>(Ws + (m + q) * NP + 4 * et);
 #pragma unroll
         for (int i = 0; i < kTPT; ++i) {
           const uint32_t word = q < 2 ? xv[i].x : q < 4 ? xv[i].y : q < 6 ? xv[i].z : xv[i].w;
           const float xf = (q & 1) ? bf16_hi(word) : bf16_lo(word);
-          acc[i][0] = fmaf(xf, w.x, acc[i][0]);
-          acc[i][1] = fmaf(xf, w.y, acc[i][1]);
-          acc[i][2] = fmaf(xf, w.z, acc[i][2]);
-          acc[i][3] = fmaf(xf, w.w, acc[i][3]);
+          acc[i][0] = fmaf(xf, wv[q].x, acc[i][0]);
+          acc[i][1] = fmaf(xf, wv[q].y, acc[i][1]);
+          acc[i][2] = fmaf(xf, wv[q].z, acc[i][2]);
+          acc[i][3] = fmaf(xf, wv[q].w, acc[i][3]);
         }
+      }
+    };
+    {
+      const int m_lo = warp * slice, m_hi = m_lo + slice;
+      uint4 xa[kTPT], xb[kTPT];
+      float4 wa[8], wb[8];
+      load8(m_lo, xa, wa);
+      for (int m = m_lo; m < m_hi; m += 16) {
+        const bool two = m + 8 < m_hi;
+        if (two) load8(m + 8, xb, wb);
+        fma8(xa, wa);
+        if (!two) break;
+        if (m + 16 < m_hi) load8(m + 16, xa, wa);
+        fma8(xb, wb);
       }
     }
 #pragma unroll
@@ -243,20 +259,20 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
     // The x rows are consumed: fetch the next block while this one is decided.
     stage_x(blk + gridDim.x);
 
-    // Logits: warp partials added in warp order, then the bias.
-    for (int i = tid; i < TB * NP; i += kRouterThreads) {
-      float z = part[i];
-#pragma unroll
-      for (int w = 1; w < kRouterWarps; ++w) z += part[w * TB * NP + i];
-      zf[i] = z + bsm[i % NP];
-    }
-    __syncthreads();
-
-    // Top-k per (token, group) on the fp32 logits, certified by the bound.
+    // One thread per (token, group) pair: the group's logits (warp partials
+    // added in warp order, then the bias), top-k on them, certified by the
+    // bound.
     for (int p = tid; p < P; p += kRouterThreads) {
       const int t = p / a.G, g = p - t * a.G;
       if (blk * TB + t >= a.R) continue;
-      const float* zg = zf + t * NP + g * a.M;
+      float* zg = zf + t * NP + g * a.M;
+      for (int j = 0; j < a.M; ++j) {
+        const int i = t * NP + g * a.M + j;
+        float z = part[i];
+#pragma unroll
+        for (int w = 1; w < kRouterWarps; ++w) z += part[w * TB * NP + i];
+        zg[j] = z + bsm[g * a.M + j];
+      }
       bool certain = true;
       if (a.k < a.M) {
         const uint64_t sel = group_topk(zg, a.M, a.k);
@@ -276,7 +292,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
     __syncthreads();
     // fp64 logits of the uncertain groups, one warp per group (products of a
     // bf16 and an fp32 value are exact in fp64).
-    const int nu = n_uncertain;
+    const int nu = n_uncertain;  // the same value in every thread: skip the barrier when 0
     for (int v = warp; v < nu; v += kRouterWarps) {
       const int p = list[v];
       const int t = p / a.G, g = p - t * a.G;
@@ -291,7 +307,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
         if (lane == 0) zd[t * NP + e] = s64 + static_cast<double>(bsm[e]);
       }
     }
-    __syncthreads();
+    if (nu > 0) __syncthreads();
     // Group softmax; selected mass per pair. (The fp64 values of certain
     // groups are their fp32 logits, so the selection is the one made above.)
     for (int p = tid; p < P; p += kRouterThreads) {

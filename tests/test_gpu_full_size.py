@@ -1,0 +1,70 @@
+"""Parity at the measured workloads' full sizes, in the launch configuration the
+benchmark times (the five step entry points on one stream), on a B200.
+
+The oracle evaluates the router, the token lists and K/V in full and the
+attention, slots and y at sampled rows: the first and last rows of each
+sequence, rows on both sides of 128-row tile boundaries (the first tile, the
+middle, the last full and the ragged last tile) and a few seeded random rows.
+Integer outputs must be bit-exact; floating-point outputs within the layer
+tolerance (max-abs 2e-2, mean-abs 2e-3).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_common import assert_close, device_inputs, run_layer, run_steps
+
+pytestmark = pytest.mark.gpu
+
+WORKLOADS = {
+    "b4x8k": (synth.BATCH4_8K, {}),
+    "seq32k": (synth.SEQ32K, {}),
+    "pool4_k1_skew": (synth.POOL4_K1, {"skew": True}),
+    "pool4_k2_skew": (synth.POOL4_K2, {"skew": True}),
+    "pool4_k2_balanced": (synth.POOL4_K2, {}),
+}
+
+
+@pytest.fixture(scope="module")
+def rsq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import routed_sparse_query_b200 as m
+    return m
+
+
+def sample_rows(shape: synth.LayerShape, seed: int = 7) -> np.ndarray:
+    T = shape.T
+    pos = {0, 1, 127, 128, 129, T // 2 - 1, T // 2, T - 129, T - 128, T - 2, T - 1}
+    rng = np.random.default_rng(seed)
+    pos |= set(int(v) for v in rng.integers(0, T, 5))
+    pos = sorted(p for p in pos if 0 <= p < T)
+    return np.array([b * T + p for b in range(shape.B) for p in pos], dtype=np.int64)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_full_size_sampled_rows(rsq, name):
+    shape, kw = WORKLOADS[name]
+    inp = synth.make_layer_inputs(shape, seed=2024, with_dense=False, **kw)
+    rows = sample_rows(shape)
+    ref = oracle.gqe_layer(inp, rows=rows)
+    o = run_steps(rsq, shape, device_inputs(inp))
+    # Router and lists: bit-exact in full.
+    assert np.array_equal(o["idx"].cpu().numpy(), ref["idx"]), "router indices differ"
+    assert np.array_equal(o["counts"].cpu().numpy().reshape(shape.N, shape.B), ref["counts"])
+    assert np.array_equal(o["offsets"].cpu().numpy(), ref["offsets"])
+    assert np.array_equal(o["tok"].cpu().numpy(), ref["tok"]), "token lists differ"
+    assert np.array_equal(o["slot_pos"].cpu().numpy(), ref["slot_pos"])
+    np.testing.assert_allclose(o["r"].cpu().numpy(), ref["r"], rtol=0, atol=2e-6)
+    np.testing.assert_allclose(o["omega"].cpu().numpy(), ref["omega"], rtol=0, atol=2e-6)
+    assert_close(o["K"], ref["K"], "K")
+    assert_close(o["V"], ref["V"], "V")
+    # Attention, slots and y at the sampled rows.
+    sel = torch.from_numpy(rows).cuda()
+    assert_close(o["slots"].index_select(0, sel), ref["slots"], "slots")
+    assert_close(o["y"].index_select(0, sel), ref["y"], "y")
+    # The fused entry point gives the same y.
+    y, _ = run_layer(rsq, shape, device_inputs(inp))
+    assert torch.equal(y, o["y"]), "gqe_layer_fwd differs from the step calls"

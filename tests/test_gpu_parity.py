@@ -67,8 +67,9 @@ def test_layer_steps_match_oracle(rsq, name):
 
 
 def test_large_batch_dispatch_is_bit_exact(rsq):
-    # More than 16384 rows: the three-pass (count, scan, scatter) dispatch;
-    # smaller batches take the single-CTA path. Both must give the oracle's lists.
+    # 21000 rows in three sequences with a ragged last dispatch tile, 12
+    # experts, k = 2; the last query tile of each stream is alone in its CTA
+    # with 55 KV tiles (a long single-tile loop of the attention kernel).
     shape = LayerShape(B=3, T=7000, d_model=128, G=4, M=3, k=2, d_head=32)
     inp = synth.make_layer_inputs(shape, seed=23)
     import oracle as orc
