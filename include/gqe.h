@@ -52,8 +52,15 @@ typedef struct gqe_config {
   int32_t M;       /* query-head experts per group; N = G*M <= 64 */
   int32_t k;       /* experts selected per group per token, 1 <= k <= M */
   int32_t d_head;  /* head dim: 32 or 64 */
-  uint32_t flags;  /* reserved, must be 0 */
+  uint32_t flags;  /* 0 or GQE_FLAG_WS_CLEAN; other bits must be 0 */
 } gqe_config;
+
+/* gqe_attention_fwd, gqe_layer_fwd, gqa_dense_fwd: the caller promises that
+ * the workspace holds zeroed split-KV arrival counters -- it was zero-filled
+ * before its first use and every earlier call on it completed with GQE_OK and
+ * a zero device status (each call leaves the counters zero) -- so the call
+ * does not clear them itself. Other entry points ignore the flag. */
+#define GQE_FLAG_WS_CLEAN 1u
 
 typedef enum gqe_status {
   GQE_OK = 0,
@@ -176,7 +183,9 @@ gqe_status gqe_kv_proj(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16*
  * Short sequences are split along the keys (each CTA takes a chunk of KV
  * tiles; the last CTA of a query-tile pair merges the chunks' unnormalised
  * rows), which needs scratch from ws: >= gqe_workspace_bytes(cfg,
- * GQE_WS_ATTENTION). Calls sharing one ws must not overlap on the GPU.
+ * GQE_WS_ATTENTION). Calls sharing one ws must not overlap on the GPU. The
+ * call clears the scratch's arrival counters first unless cfg->flags has
+ * GQE_FLAG_WS_CLEAN.
  * Qv [B, G, k, T, d_head]; Qs [B, T, d_head]; K, V [B, G, T, d_head];
  * slots [B*T, (k*G+2)*d_head].
  */

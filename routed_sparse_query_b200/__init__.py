@@ -25,6 +25,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 GQE_OK, GQE_ERR_INVALID, GQE_ERR_UNSUPPORTED, GQE_ERR_WORKSPACE = 0, 1, 2, 3
 GQE_ERR_CUDA, GQE_ERR_TIMEOUT, GQE_ERR_DEVICE_CHECK = 4, 5, 6
 GQE_WS_DISPATCH, GQE_WS_LAYER, GQE_WS_DENSE, GQE_WS_ATTENTION = 1, 2, 3, 4
+GQE_FLAG_WS_CLEAN = 1
 ITEMS = {"idx": 1, "r": 2, "omega": 3, "counts": 4, "offsets": 5, "tok": 6, "slot_pos": 7,
          "Qv": 8, "Qs": 9, "K": 10, "V": 11, "slots": 12, "dispatch_ws": 13, "attention_ws": 14,
          "dense_Q": 32, "dense_O": 33}
@@ -41,8 +42,8 @@ class GQEConfig(ctypes.Structure):
                 ("d_head", ctypes.c_int32), ("flags", ctypes.c_uint32)]
 
     @classmethod
-    def of(cls, shape) -> "GQEConfig":
-        return cls(shape.B, shape.T, shape.d_model, shape.G, shape.M, shape.k, shape.d_head, 0)
+    def of(cls, shape, flags: int = 0) -> "GQEConfig":
+        return cls(shape.B, shape.T, shape.d_model, shape.G, shape.M, shape.k, shape.d_head, flags)
 
 
 class GQEError(RuntimeError):

@@ -26,7 +26,7 @@ bool all_aligned(const P*... ps) {
 gqe_status check_cfg(const gqe_config* c) {
   if (c == nullptr) return GQE_ERR_INVALID;
   if (c->B < 1 || c->T < 1 || c->G < 1 || c->M < 1 || c->k < 1 || c->k > c->M) return GQE_ERR_INVALID;
-  if (c->d_model < 64 || c->d_model % 64 != 0 || c->flags != 0) return GQE_ERR_INVALID;
+  if (c->d_model < 64 || c->d_model % 64 != 0 || (c->flags & ~GQE_FLAG_WS_CLEAN) != 0u) return GQE_ERR_INVALID;
   if (c->G * c->M > kMaxExperts || c->G > 32) return GQE_ERR_UNSUPPORTED;
   if (c->d_head != 32 && c->d_head != 64) return GQE_ERR_UNSUPPORTED;
   // Index arithmetic of the kernels stays within int32 for these extents.
@@ -217,7 +217,8 @@ gqe_status gqe_attention_fwd(const gqe_config* cfg, const gqe_bf16* Qv, const gq
   const size_t need = attention_plan(*cfg, cfg->G * cfg->k + 1).total;
   if (need > 0 && (ws == nullptr || !aligned16(ws))) return GQE_ERR_INVALID;
   if (ws_bytes < need) return GQE_ERR_WORKSPACE;
-  return cuda_status(attention_gqe(*cfg, Qv, Qs, K, V, slots, ws, ws_bytes, false, stream));
+  const bool clean = (cfg->flags & GQE_FLAG_WS_CLEAN) != 0u;
+  return cuda_status(attention_gqe(*cfg, Qv, Qs, K, V, slots, ws, ws_bytes, clean, stream));
 }
 
 gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* omega,
@@ -246,9 +247,11 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
   auto I = [&](size_t o) { return reinterpret_cast<int32_t*>(w + o); };
   auto F = [&](size_t o) { return reinterpret_cast<float*>(w + o); };
   auto H = [&](size_t o) { return reinterpret_cast<gqe_bf16*>(w + o); };
-  // The split-KV counters are zeroed first, so that the kernels of the layer
-  // follow each other directly (programmatic dependent launch).
-  if (zero_attention_counters(*cfg, cfg->G * cfg->k + 1, w + L.aws, stream) != cudaSuccess)
+  // The split-KV counters are zeroed first (unless the caller vouches that
+  // they are), so that the kernels of the layer follow each other directly
+  // (programmatic dependent launch).
+  if ((cfg->flags & GQE_FLAG_WS_CLEAN) == 0u &&
+      zero_attention_counters(*cfg, cfg->G * cfg->k + 1, w + L.aws, stream) != cudaSuccess)
     return GQE_ERR_CUDA;
   gqe_status st = gqe_router_topk(cfg, x, W_r, b_r, I(L.idx), F(L.r), F(L.omega), stream);
   if (st != GQE_OK) return st;
@@ -277,7 +280,8 @@ gqe_status gqa_dense_fwd(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf1
   if (ws_bytes < L.total) return GQE_ERR_WORKSPACE;
   char* w = static_cast<char*>(ws);
   auto H = [&](size_t o) { return reinterpret_cast<gqe_bf16*>(w + o); };
-  int e = zero_attention_counters(c, c.G * c.M, w + L.aws, stream);
+  int e = (c.flags & GQE_FLAG_WS_CLEAN) != 0u ? cudaSuccess
+                                                : zero_attention_counters(c, c.G * c.M, w + L.aws, stream);
   if (e == cudaSuccess) e = gemm_q_dense(c, x, W_q, H(L.Q), stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
   e = gemm_kv(c, x, W_k, W_v, H(L.K), H(L.V), stream);

@@ -103,6 +103,25 @@ def test_seq2k_layer_matches_oracle(rsq):
         torch.cuda.synchronize()
         assert torch.equal(slots[:, :(shape.k * shape.G + 1) * shape.d_head],
                            o["slots"][:, :(shape.k * shape.G + 1) * shape.d_head])
+    # GQE_FLAG_WS_CLEAN: a zero-filled scratch, not cleared by the calls, stays
+    # valid from call to call (every call leaves the counters zero).
+    cfg_c = rsq.GQEConfig.of(shape, rsq.GQE_FLAG_WS_CLEAN)
+    wsz = torch.zeros_like(wsa)
+    for _ in range(3):
+        slots = torch.zeros_like(o["slots"])
+        rsq.gqe_attention_fwd(cfg_c, o["Qv"], o["Qs"], o["K"], o["V"], slots, wsz)
+        torch.cuda.synchronize()
+        assert rsq.gqe_read_status() == 0
+        assert torch.equal(slots[:, :(shape.k * shape.G + 1) * shape.d_head],
+                           o["slots"][:, :(shape.k * shape.G + 1) * shape.d_head])
+    wsl = torch.zeros(rsq.gqe_workspace_bytes(cfg_c, rsq.GQE_WS_LAYER), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        y2 = torch.empty_like(y)
+        rsq.gqe_layer_fwd(cfg_c, d["x"], d["W_r"], d["b_r"], d["W_q"], d["W_qs"], d["W_k"], d["W_v"],
+                          d["W_o"], y2, wsl)
+        torch.cuda.synchronize()
+        assert rsq.gqe_read_status() == 0
+        assert torch.equal(y2, y)
 
 
 def test_dense_gqa_matches_oracle(rsq):
