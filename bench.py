@@ -54,7 +54,9 @@ def launches(s: synth.LayerShape) -> dict:
     tiles = s.B * -(-s.T // DISPATCH_TILE)
     fused = s.N * tiles <= FUSED_SCAN_MAX
     # dispatch: masks+counts, scan+scatter (one launch or two), the grouped Q GEMM
-    return {"router": 1, "dispatch": 3 if fused else 4, "kv": 1, "attention": 1, "output": 2}
+    # output: the W_O GEMM, with the weighted slot fused in when d_head = 64
+    return {"router": 1, "dispatch": 3 if fused else 4, "kv": 1, "attention": 1,
+            "output": 1 if s.d_head == 64 else 2}
 
 
 FLUSH_BYTES = 256 << 20

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "gqe_internal.h"
 #include "ptx.cuh"
@@ -110,6 +111,34 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
   __syncwarp();
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, limit_ns);
   __syncwarp();
+}
+
+// Per-device side stream for the K/V projection of gqe_layer_fwd: it reads
+// only x and the weights, so it runs beside the dispatch and the Q
+// projection (fork on the caller's stream after the router, join before the
+// attention). Created on first use; the enqueue sequence is serialised by
+// the mutex so that concurrent callers on one device do not interleave
+// their event records. Captured into CUDA graphs like any fork/join.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool ok = false;
+};
+std::mutex g_side_mu;
+SideStream g_side[64];
+
+SideStream* side_stream_locked() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SideStream& ss = g_side[dev];
+  if (!ss.ok) {
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+    ss.ok = true;
+  }
+  return &ss;
 }
 
 }  // namespace api_impl
@@ -226,11 +255,7 @@ gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* 
   const gqe_status s = check_cfg(cfg);
   if (s != GQE_OK) return s;
   if (!all_aligned(slots, omega, W_o, y)) return GQE_ERR_INVALID;
-  int e = launch_weighted_slot(*cfg, slots, omega, stream);
-  if (e != cudaSuccess) return GQE_ERR_CUDA;
-  const int R = cfg->B * cfg->T;
-  return cuda_status(gemm_rowmajor(slots, R, (cfg->G * cfg->k + 2) * cfg->d_head, W_o,
-                                   cfg->d_model, y, stream));
+  return cuda_status(gemm_output(*cfg, slots, omega, W_o, y, stream));
 }
 
 gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
@@ -253,13 +278,27 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
   if ((cfg->flags & GQE_FLAG_WS_CLEAN) == 0u &&
       zero_attention_counters(*cfg, cfg->G * cfg->k + 1, w + L.aws, stream) != cudaSuccess)
     return GQE_ERR_CUDA;
-  gqe_status st = gqe_router_topk(cfg, x, W_r, b_r, I(L.idx), F(L.r), F(L.omega), stream);
-  if (st != GQE_OK) return st;
-  st = gqe_dispatch(cfg, I(L.idx), x, W_q, W_qs, I(L.counts), I(L.offsets), I(L.tok),
-                    I(L.slot_pos), H(L.Qv), H(L.Qs), w + L.dws, L.total - L.dws, stream);
-  if (st != GQE_OK) return st;
-  st = gqe_kv_proj(cfg, x, W_k, W_v, H(L.K), H(L.V), stream);
-  if (st != GQE_OK) return st;
+  // K/V projection on the side stream (falls back to the caller's stream).
+  cudaStream_t main_st = static_cast<cudaStream_t>(stream);
+  {
+    std::lock_guard<std::mutex> guard(g_side_mu);
+    // The router goes first (it heads the critical path); the K/V projection
+    // forks after it and runs beside the dispatch and the Q projection.
+    gqe_status st = gqe_router_topk(cfg, x, W_r, b_r, I(L.idx), F(L.r), F(L.omega), stream);
+    if (st != GQE_OK) return st;
+    SideStream* side = side_stream_locked();
+    if (side != nullptr && (cudaEventRecord(side->fork, main_st) != cudaSuccess ||
+                            cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess))
+      return GQE_ERR_CUDA;
+    const gqe_status kv = gqe_kv_proj(cfg, x, W_k, W_v, H(L.K), H(L.V), side ? side->s : stream);
+    if (kv != GQE_OK) return kv;
+    if (side != nullptr && cudaEventRecord(side->join, side->s) != cudaSuccess) return GQE_ERR_CUDA;
+    st = gqe_dispatch(cfg, I(L.idx), x, W_q, W_qs, I(L.counts), I(L.offsets), I(L.tok),
+                      I(L.slot_pos), H(L.Qv), H(L.Qs), w + L.dws, L.total - L.dws, stream);
+    if (st != GQE_OK) return st;
+    if (side != nullptr && cudaStreamWaitEvent(main_st, side->join, 0) != cudaSuccess)
+      return GQE_ERR_CUDA;
+  }
   if (attention_gqe(*cfg, H(L.Qv), H(L.Qs), H(L.K), H(L.V), H(L.slots), w + L.aws,
                     L.total - L.aws, true, stream) != cudaSuccess)
     return GQE_ERR_CUDA;
@@ -282,10 +321,21 @@ gqe_status gqa_dense_fwd(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf1
   auto H = [&](size_t o) { return reinterpret_cast<gqe_bf16*>(w + o); };
   int e = (c.flags & GQE_FLAG_WS_CLEAN) != 0u ? cudaSuccess
                                                 : zero_attention_counters(c, c.G * c.M, w + L.aws, stream);
-  if (e == cudaSuccess) e = gemm_q_dense(c, x, W_q, H(L.Q), stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
-  e = gemm_kv(c, x, W_k, W_v, H(L.K), H(L.V), stream);
-  if (e != cudaSuccess) return GQE_ERR_CUDA;
+  {
+    // K/V projection beside the Q projection (side stream, as in gqe_layer_fwd).
+    std::lock_guard<std::mutex> guard(g_side_mu);
+    cudaStream_t main_st = static_cast<cudaStream_t>(stream);
+    SideStream* side = side_stream_locked();
+    if (side != nullptr && (cudaEventRecord(side->fork, main_st) != cudaSuccess ||
+                            cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess))
+      return GQE_ERR_CUDA;
+    e = gemm_kv(c, x, W_k, W_v, H(L.K), H(L.V), side ? side->s : stream);
+    if (e == cudaSuccess && side != nullptr) e = cudaEventRecord(side->join, side->s);
+    if (e == cudaSuccess) e = gemm_q_dense(c, x, W_q, H(L.Q), stream);
+    if (e == cudaSuccess && side != nullptr) e = cudaStreamWaitEvent(main_st, side->join, 0);
+    if (e != cudaSuccess) return GQE_ERR_CUDA;
+  }
   e = attention_dense(c, H(L.Q), H(L.K), H(L.V), H(L.O), w + L.aws, L.total - L.aws, true, stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
   const int N = c.G * c.M;

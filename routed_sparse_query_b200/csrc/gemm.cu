@@ -10,7 +10,12 @@
 //    list; the A rows are gathered by four warps with cp.async into the same
 //    swizzled layout TMA would produce, and the epilogue writes each row to its
 //    slot-major stream Qv[b][g][s][t][:].
-//  - W_O projection (step a11): plain row-major output.
+//  - W_O projection (step a11): plain row-major output. With d_head = 64 the
+//    weighted slot (step a10) is exactly one K block of A: the epilogue warps,
+//    idle during the main loop, compute it from the routed slots and omega,
+//    write it into that K block's stage in the swizzled layout (and, in the
+//    CTAs of the first column tile, back to the slot buffer), and the TMA warp
+//    loads only B for that block.
 //
 // Warp roles (192 threads): warp 0 issues TMA loads, warp 1 issues the UMMAs
 // (one thread) and owns the TMEM allocation, warps 2-5 gather A rows (routed
@@ -52,6 +57,14 @@ struct Epi {
   int T;                 // rows per sequence
   int hd;                // columns per head
   int rows, cols;        // valid extent of C
+  // Weighted-slot fusion (W_O projection): K block kb_w of A is
+  // sum_gs omega[row, gs] * A[row, gs*BK ...] over gs < gk, computed in the
+  // kernel (kb_w < 0: off).
+  int kb_w = -1;
+  int gk = 0;
+  const float* omega = nullptr;
+  uint16_t* wslots = nullptr;  // A itself, written back by the blockIdx.y == 0 CTAs
+  int lda = 0;                 // A row length (elements)
 };
 
 struct Gather {
@@ -95,7 +108,9 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* empty = full + C::STAGES;
   uint64_t* accb = empty + C::STAGES;
   uint64_t* drain = accb + 1;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* wfree = drain + 1;   // weighted slot: its stage is free (producer arrives)
+  uint64_t* wready = wfree + 1;  // weighted slot: its tile is in shared memory (128 arrivals)
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(wready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -112,6 +127,8 @@ __global__ void __launch_bounds__(192, 2)
     }
     mbar_init(accb, 1u);
     mbar_init(drain, 1u);
+    mbar_init(wfree, 1u);
+    mbar_init(wready, 128u);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -165,8 +182,13 @@ __global__ void __launch_bounds__(192, 2)
         const int s = kb % C::STAGES;
         const uint32_t ph = (kb / C::STAGES) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) break;
-        mbar_arrive_expect_tx(&full[s], (GATHER ? 0 : C::A_BYTES) + C::B_BYTES);
-        if (!GATHER) tma_load_2d(sA + s * C::A_BYTES, &tmA, &full[s], kb * BK, m0);
+        const bool wblk = !GATHER && kb == epi.kb_w;
+        if (wblk) {  // A of this block is computed by the epilogue warps
+          mbar_arrive(wfree);
+          if (!mbar_wait(wready, 0, abort_flag)) break;
+        }
+        mbar_arrive_expect_tx(&full[s], (GATHER || wblk ? 0 : C::A_BYTES) + C::B_BYTES);
+        if (!GATHER && !wblk) tma_load_2d(sA + s * C::A_BYTES, &tmA, &full[s], kb * BK, m0);
 #pragma unroll
         for (int c = 0; c < BN / C::B_ATOM; ++c)
           tma_load_2d(sB + s * C::B_BYTES + c * (BK * C::B_SWB), tmB, &full[s],
@@ -238,6 +260,55 @@ __global__ void __launch_bounds__(192, 2)
       cp_async_wait<0>();
       fence_proxy_async_smem();
       for (int k2 = (kb - LA > 0 ? kb - LA : 0); k2 < kb; ++k2) mbar_arrive(&full[k2 % C::STAGES]);
+    }
+    if (!GATHER && epi.kb_w >= 0) {
+      // Weighted slot: the same fp32 sum, in the same order, as the
+      // stand-alone weighted-slot kernel, rounded to bf16. Thread i takes
+      // 16-byte chunk i % 8 of rows i / 8, i / 8 + 16, ... (8 threads read one
+      // slot row segment together), writes it into the block's stage once the
+      // stage is free, and (first column tile) into the slot buffer.
+      const int i = threadIdx.x - 64;
+      const int c = i & 7;
+      uint4 o[8];
+#pragma unroll 2
+      for (int pass = 0; pass < 8; ++pass) {
+        const int row = m0 + pass * 16 + (i >> 3);
+        if (row < epi.rows) {
+          const uint16_t* base = epi.wslots + static_cast<size_t>(row) * epi.lda + c * 8;
+          const float* w = epi.omega + static_cast<size_t>(row) * epi.gk;
+          float acc[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) acc[x] = 0.0f;
+#pragma unroll 4
+          for (int gs = 0; gs < epi.gk; ++gs) {
+            const float wi = __ldg(w + gs);
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + gs * BK));
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i2 = 0; i2 < 4; ++i2) {
+              acc[2 * i2] = fmaf(wi, __uint_as_float(u[i2] << 16), acc[2 * i2]);
+              acc[2 * i2 + 1] = fmaf(wi, __uint_as_float(u[i2] & 0xffff0000u), acc[2 * i2 + 1]);
+            }
+          }
+          o[pass] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                               pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+          if (blockIdx.y == 0)
+            *reinterpret_cast<uint4*>(epi.wslots + static_cast<size_t>(row) * epi.lda + epi.kb_w * BK +
+                                      c * 8) = o[pass];
+        } else {
+          o[pass] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      if (mbar_wait(wfree, 0, abort_flag)) {
+        uint8_t* stage = sA + (epi.kb_w % C::STAGES) * C::A_BYTES;
+#pragma unroll
+        for (int pass = 0; pass < 8; ++pass) {
+          const int r = pass * 16 + (i >> 3);
+          *reinterpret_cast<uint4*>(stage + r * 128 + ((c ^ (r & 7)) << 4)) = o[pass];
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(wready);
+      }
     }
     const bool have = mbar_wait(accb, 0, abort_flag);
     tc_fence_after();
@@ -370,6 +441,33 @@ int gemm_rowmajor(const uint16_t* A, int rows, int K, const uint16_t* W, int N, 
   e.rows = rows;
   e.cols = N;
   return dense_gemm(A, rows, K, W, nullptr, N, e, e, 1, stream);
+}
+
+int gemm_output(const gqe_config& c, uint16_t* slots, const float* omega, const uint16_t* W_o,
+                uint16_t* y, void* stream) {
+  const int R = c.B * c.T;
+  const int gk = c.G * c.k;
+  const int K = (gk + 2) * c.d_head;
+  if (c.d_head != BK) {  // the weighted slot is not one K block: separate kernel
+    const int e = launch_weighted_slot(c, slots, omega, stream);
+    if (e != cudaSuccess) return e;
+    return gemm_rowmajor(slots, R, K, W_o, c.d_model, y, stream);
+  }
+  Epi e;
+  e.out = y;
+  e.T = R;
+  e.hd = c.d_model;
+  e.sb = 0;
+  e.sh = 0;
+  e.st = c.d_model;
+  e.rows = R;
+  e.cols = c.d_model;
+  e.kb_w = gk + 1;
+  e.gk = gk;
+  e.omega = omega;
+  e.wslots = slots;
+  e.lda = K;
+  return dense_gemm(slots, R, K, W_o, nullptr, c.d_model, e, e, 1, stream);
 }
 
 int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const uint16_t* W_qs,

@@ -98,6 +98,11 @@ int gemm_q_dense(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, ui
                  void* stream);
 int gemm_rowmajor(const uint16_t* A, int rows, int K, const uint16_t* W, int N, uint16_t* out,
                   void* stream);
+// Weighted slot + W_O projection (steps a10, a11): y = slots @ W_o, with
+// the weighted slot written into slots first (fused into the GEMM when
+// d_head is one K block).
+int gemm_output(const gqe_config& c, uint16_t* slots, const float* omega, const uint16_t* W_o,
+                uint16_t* y, void* stream);
 
 // Attention front ends (tcgen05). Split-KV plan: small problems cut each
 // query-tile pair's KV range into chunks; the scratch (partial rows and
