@@ -562,6 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int x = 0; x < DH; ++x) acc[x] = 0.0f;
           float lt = 0.0f;
+#pragma unroll 2
           for (int c = 0; c < n_chunks; ++c) {
             const float2 ml = __ldcg(&p.part_ml[(blk0 + 2 * c) * BQ + i]);
             const float w = ex2(ml.x - ms);

@@ -8,16 +8,17 @@
 //
 // The logits are a small fp32 GEMM on the CUDA cores. A CTA takes a block of
 // TB tokens (TB * NP = 256 logits); W_r (zero padded to NP columns) and the
-// block's x rows sit in shared memory. Warp w sums rows [w d/8, (w+1) d/8)
-// of the dot products; each thread keeps 2 tokens x 4 experts, reading a W_r
-// row once per 2 tokens (broadcast over the warp's token lanes). The 8 warp
-// partials are then added in warp order, so every logit is one fixed
-// sequence of roundings (the result is deterministic).
+// block's x rows sit in shared memory. Warp w of W (16, or 8 when d is not a
+// multiple of 128) sums rows [w d/W, (w+1) d/W) of the dot products; each
+// thread keeps 2 tokens x 4 experts, reading a W_r row once per 2 tokens
+// (broadcast over the warp's token lanes). The W warp partials are then added
+// in warp order, so every logit is one fixed sequence of roundings (the
+// result is deterministic). One thread per (token, group) pair then decides.
 //
 // Exact selection: each fp32 logit carries the bound
 //   |z_fp32 - z| <= gamma_h * (||x||_1 * max_i |W_r[i,e]| + |b_e|),
-// h = d/8 + 8 roundings on its longest path (d/8 FMAs in one warp, 7 adds
-// of the warp partials, the bias add), gamma_h = h u / (1 - h u), u = 2^-24 (Higham,
+// h = d/W + W roundings on its longest path (d/W FMAs in one warp, W - 1
+// adds of the warp partials, the bias add), gamma_h = h u / (1 - h u), u = 2^-24 (Higham,
 // "Accuracy and Stability of Numerical Algorithms", 2nd ed., sec. 3.1). A
 // group whose top-k decision is not certain under these intervals (computed
 // with directed rounding) recomputes its logits in fp64 (products of a bf16
@@ -33,13 +34,14 @@ namespace gqe {
 
 namespace router_impl {
 
-constexpr int kRouterThreads = 256;
-constexpr int kRouterWarps = kRouterThreads / 32;  // warp w sums rows [w d/8, (w+1) d/8)
-constexpr int kTPT = 2;                            // tokens per thread
+constexpr int kMaxRouterWarps = 16;
+constexpr int kTPT = 2;  // tokens per thread
 
 // Tokens per CTA block: lanes are (token lane tt, expert quad et) with NP/4
 // quads, so a warp covers 128/NP token lanes of kTPT tokens each.
 __host__ __device__ constexpr int router_tb(int NP) { return kTPT * 128 / NP; }
+// Warps per CTA: warp w sums rows [w d/W, (w+1) d/W), a multiple of 8 rows.
+__host__ __device__ constexpr int router_warps(int d) { return d % 128 == 0 ? 16 : 8; }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t v) {
   return __uint_as_float(static_cast<uint32_t>(v) << 16);
@@ -59,22 +61,24 @@ struct RouterArgs {
 
 // Dynamic shared memory of one CTA (byte offsets).
 struct RouterLayout {
-  size_t w, xs, part, zd, zf, wmax, bsm, nx, ps, list, total;
+  size_t w, xs, part, zd, zf, ez, wmax, bsm, nx, ps, dn, list, total;
 };
 __host__ __device__ inline RouterLayout router_layout(int d, int NP) {
-  const int TB = router_tb(NP);
+  const int TB = router_tb(NP), W = router_warps(d);
   RouterLayout L;
   size_t o = 0;
-  L.w = o;     o += static_cast<size_t>(d) * NP * 4;                     // W_r [d][NP]
-  L.xs = o;    o += static_cast<size_t>(TB) * (d + 8) * 2;               // x [TB][d + 8]
-  L.part = o;  o += static_cast<size_t>(kRouterWarps) * TB * NP * 4;     // [warp][TB][NP]
-  L.zd = o;    o += static_cast<size_t>(TB) * NP * 8;                    // fp64 logits
-  L.zf = o;    o += static_cast<size_t>(TB) * NP * 4;                    // fp32 logits
-  L.wmax = o;  o += NP * 4;                                               // max_i |W_r[i, e]|
-  L.bsm = o;   o += NP * 4;                                               // bias
-  L.nx = o;    o += TB * 4;                                               // ||x||_1
-  L.ps = o;    o += static_cast<size_t>(TB) * NP * 4;                    // selected mass per pair
-  L.list = o;  o += static_cast<size_t>(TB) * NP * 4;                    // uncertain pairs
+  L.w = o;     o += static_cast<size_t>(d) * NP * 4;                  // W_r [d][NP]
+  L.xs = o;    o += static_cast<size_t>(TB) * (d + 8) * 2;            // x [TB][d + 8]
+  L.part = o;  o += static_cast<size_t>(W) * TB * NP * 4;             // [warp][TB][NP]
+  L.zd = o;    o += static_cast<size_t>(TB) * NP * 8;                 // fp64 logits
+  L.zf = o;    o += static_cast<size_t>(TB) * NP * 4;                 // fp32 logits
+  L.ez = o;    o += static_cast<size_t>(TB) * NP * 4;                 // exp(z - group max)
+  L.wmax = o;  o += NP * 4;                                            // max_i |W_r[i, e]|
+  L.bsm = o;   o += NP * 4;                                            // bias
+  L.nx = o;    o += TB * 4;                                            // ||x||_1
+  L.ps = o;    o += static_cast<size_t>(TB) * NP * 4;                 // selected mass per pair
+  L.dn = o;    o += static_cast<size_t>(TB) * NP * 4;                 // softmax denominator per pair
+  L.list = o;  o += static_cast<size_t>(TB) * NP * 4;                 // uncertain pairs
   L.total = (o + 15) & ~static_cast<size_t>(15);
   return L;
 }
@@ -98,12 +102,34 @@ __device__ __forceinline__ uint64_t group_topk(const V* zg, int M, int k) {
   return sel;
 }
 
-template <int NP>
-__global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
+// Group softmax of pair (t, g) from its logits zg (fp32, or fp64 for a
+// group decided in fp64): exp(z - max) into ez, the denominator into *den,
+// and the selected mass (sum of the selected probabilities) returned.
+template <typename V>
+__device__ __forceinline__ float group_softmax(const V* zg, int M, uint64_t sel, float* ez, float* den) {
+  V zmax = zg[0];
+  for (int j = 1; j < M; ++j) zmax = zg[j] > zmax ? zg[j] : zmax;
+  float dsum = 0.0f;
+  for (int j = 0; j < M; ++j) {
+    const float e = expf(static_cast<float>(zg[j] - zmax));
+    ez[j] = e;
+    dsum += e;
+  }
+  float psel = 0.0f;
+  for (int j = 0; j < M; ++j)
+    if ((sel >> j) & 1ull) psel += ez[j] / dsum;
+  *den = dsum;
+  return psel;
+}
+
+template <int NP, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
+  constexpr int THREADS = WARPS * 32;
   constexpr int TB = router_tb(NP);
   constexpr int EG = NP / 4;   // expert quads
   constexpr int TG = 32 / EG;  // token lanes per warp; TB == kTPT * TG
   static_assert(TB == kTPT * TG, "block shape");
+  static_assert(TB * NP <= THREADS, "one (token, group) pair per thread");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int n_uncertain;
   const RouterLayout L = router_layout(a.d, NP);
@@ -112,10 +138,12 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   float* part = reinterpret_cast<float*>(smem_raw + L.part);
   double* zd = reinterpret_cast<double*>(smem_raw + L.zd);
   float* zf = reinterpret_cast<float*>(smem_raw + L.zf);
+  float* ez = reinterpret_cast<float*>(smem_raw + L.ez);
   float* wmax = reinterpret_cast<float*>(smem_raw + L.wmax);
   float* bsm = reinterpret_cast<float*>(smem_raw + L.bsm);
   float* nxs = reinterpret_cast<float*>(smem_raw + L.nx);
   float* ps = reinterpret_cast<float*>(smem_raw + L.ps);
+  float* dn = reinterpret_cast<float*>(smem_raw + L.dn);
   int* list = reinterpret_cast<int*>(smem_raw + L.list);
 
   const int tid = threadIdx.x;
@@ -129,7 +157,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   // commits one cp.async group (empty past the end).
   auto stage_x = [&](int blk) {
     if (blk < n_blk) {
-      for (int t = warp; t < TB; t += kRouterWarps) {
+      for (int t = warp; t < TB; t += WARPS) {
         const uint16_t* src = a.x + static_cast<size_t>(min(blk * TB + t, a.R - 1)) * a.d;
         for (int c = lane; c < cpr; c += 32) cp_async_16(smem_u32(xs + t * XS + c * 8), src + c * 8, 16u);
       }
@@ -145,13 +173,13 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   if (a.N == NP) {
     const int total = a.d * NP / 4;  // 16-byte chunks
     const int rot = static_cast<int>((static_cast<long long>(blockIdx.x) * 256) % total);
-    for (int i = tid; i < total; i += kRouterThreads) {
+    for (int i = tid; i < total; i += THREADS) {
       int j = i + rot;
       if (j >= total) j -= total;
       cp_async_16(smem_u32(Ws + 4 * j), a.W_r + 4 * static_cast<size_t>(j), 16u);
     }
   } else {
-    for (int i = tid; i < a.d * NP; i += kRouterThreads) {
+    for (int i = tid; i < a.d * NP; i += THREADS) {
       const int row = i / NP, col = i % NP;
       Ws[i] = col < a.N ? a.W_r[static_cast<size_t>(row) * a.N + col] : 0.0f;
     }
@@ -160,12 +188,12 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   int blk = blockIdx.x;
   stage_x(blk);
   cp_async_wait<1>();  // this thread's part of W_r is in
-  for (int e = tid; e < NP; e += kRouterThreads) bsm[e] = (e < a.N && a.b_r != nullptr) ? a.b_r[e] : 0.0f;
+  for (int e = tid; e < NP; e += THREADS) bsm[e] = (e < a.N && a.b_r != nullptr) ? a.b_r[e] : 0.0f;
   __syncthreads();
-  // max_i |W_r[i, e]|: thread t scans column t % NP over every (256/NP)-th
+  // max_i |W_r[i, e]|: thread t scans column t % NP over every (THREADS/NP)-th
   // row, then one thread per column combines the parts.
   {
-    constexpr int parts = kRouterThreads / NP;
+    constexpr int parts = THREADS / NP;
     const int col = tid % NP, p0 = tid / NP;
     float m0 = 0.0f, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
     int row = p0;
@@ -180,17 +208,17 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
     __syncthreads();
     if (tid < NP) {
       float mx = 0.0f;
-      for (int p = 0; p < parts; ++p) mx = fmaxf(mx, part[p * NP + tid]);
+      for (int q = 0; q < parts; ++q) mx = fmaxf(mx, part[q * NP + tid]);
       wmax[tid] = mx;
     }
   }
 
-  const int h = a.d / kRouterWarps + kRouterWarps;
+  const int h = a.d / WARPS + WARPS;  // d/W FMAs, W - 1 partial additions, the bias
   const float u = 5.9604644775390625e-08f;  // 2^-24
   const float gam = (h * u) / (1.0f - h * u);
   const float gam_ru = __fmul_ru(gam, 1.01f);
-  const int slice = a.d / kRouterWarps;
-  const int P = TB * a.G;  // (token, group) pairs of a block
+  const int slice = a.d / WARPS;
+  const int P = TB * a.G;  // (token, group) pairs of a block: pair p is thread p
 
   for (; blk < n_blk; blk += gridDim.x) {
     cp_async_wait<0>();
@@ -243,7 +271,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
       *reinterpret_cast<float4*>(part + (warp * TB + tt + TG * i) * NP + 4 * et) =
           make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
     // ||x||_1 per token (warp-strided tokens, lane-strided chunks).
-    for (int t = warp; t < TB; t += kRouterWarps) {
+    for (int t = warp; t < TB; t += WARPS) {
       float sx = 0.0f;
       for (int c = lane; c < cpr; c += 32) {
         const uint4 v = *reinterpret_cast<const uint4*>(xs + t * XS + c * 8);
@@ -259,23 +287,24 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
     // The x rows are consumed: fetch the next block while this one is decided.
     stage_x(blk + gridDim.x);
 
-    // One thread per (token, group) pair: the group's logits (warp partials
-    // added in warp order, then the bias), top-k on them, certified by the
-    // bound.
-    for (int p = tid; p < P; p += kRouterThreads) {
-      const int t = p / a.G, g = p - t * a.G;
-      if (blk * TB + t >= a.R) continue;
-      float* zg = zf + t * NP + g * a.M;
+    // Thread p = pair (t, g): the group's logits (warp partials added in warp
+    // order, then the bias), top-k, certified by the bound; certain groups
+    // go straight on to their softmax.
+    const int t = tid / a.G, g = tid - t * a.G;
+    const bool mine = tid < P && blk * TB + t < a.R;
+    const int zo = t * NP + g * a.M;  // the group's logits in zf / zd / ez
+    bool certain = true;
+    uint64_t sel = 0;
+    if (mine) {
+      float* zg = zf + zo;
       for (int j = 0; j < a.M; ++j) {
-        const int i = t * NP + g * a.M + j;
-        float z = part[i];
+        float z = part[zo + j];
 #pragma unroll
-        for (int w = 1; w < kRouterWarps; ++w) z += part[w * TB * NP + i];
+        for (int w = 1; w < WARPS; ++w) z += part[w * TB * NP + zo + j];
         zg[j] = z + bsm[g * a.M + j];
       }
-      bool certain = true;
+      sel = group_topk(zg, a.M, a.k);
       if (a.k < a.M) {
-        const uint64_t sel = group_topk(zg, a.M, a.k);
         const float nx = nxs[t];
         float lo = INFINITY, hi = -INFINITY;
         for (int j = 0; j < a.M; ++j) {
@@ -286,64 +315,60 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
         }
         certain = lo > hi;
       }
-      for (int j = 0; j < a.M; ++j) zd[t * NP + g * a.M + j] = static_cast<double>(zg[j]);
-      if (!certain) list[atomicAdd(&n_uncertain, 1)] = p;
+      if (certain) ps[tid] = group_softmax(zg, a.M, sel, ez + zo, dn + tid);
+      else list[atomicAdd(&n_uncertain, 1)] = tid;
     }
     __syncthreads();
-    // fp64 logits of the uncertain groups, one warp per group (products of a
-    // bf16 and an fp32 value are exact in fp64).
-    const int nu = n_uncertain;  // the same value in every thread: skip the barrier when 0
-    for (int v = warp; v < nu; v += kRouterWarps) {
-      const int p = list[v];
-      const int t = p / a.G, g = p - t * a.G;
-      const uint16_t* xr = a.x + static_cast<size_t>(blk * TB + t) * a.d;
-      for (int j = 0; j < a.M; ++j) {
-        const int e = g * a.M + j;
-        double s64 = 0.0;
-        for (int m = lane; m < a.d; m += 32)
-          s64 = fma(static_cast<double>(bf16_to_f32(xr[m])), static_cast<double>(Ws[m * NP + e]), s64);
+    const int nu = n_uncertain;  // the same value in every thread: the barriers below are uniform
+    if (nu > 0) {
+      // fp64 logits of the uncertain groups, one warp per group (products of
+      // a bf16 and an fp32 value are exact in fp64).
+      for (int v = warp; v < nu; v += WARPS) {
+        const int pv = list[v];
+        const int tv = pv / a.G, gv = pv - tv * a.G;
+        const uint16_t* xr = a.x + static_cast<size_t>(blk * TB + tv) * a.d;
+        // Lane l takes columns 2l, 2l+1 (+64, ...): bf16 pairs, four
+        // independent fp64 sums per expert.
+        for (int j = 0; j < a.M; ++j) {
+          const int e = gv * a.M + j;
+          double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+          int m = 2 * lane;
+          for (; m + 64 < a.d; m += 128) {
+            const uint32_t p0 = *reinterpret_cast<const uint32_t*>(xr + m);
+            const uint32_t p1 = *reinterpret_cast<const uint32_t*>(xr + m + 64);
+            s0 = fma(static_cast<double>(bf16_lo(p0)), static_cast<double>(Ws[m * NP + e]), s0);
+            s1 = fma(static_cast<double>(bf16_hi(p0)), static_cast<double>(Ws[(m + 1) * NP + e]), s1);
+            s2 = fma(static_cast<double>(bf16_lo(p1)), static_cast<double>(Ws[(m + 64) * NP + e]), s2);
+            s3 = fma(static_cast<double>(bf16_hi(p1)), static_cast<double>(Ws[(m + 65) * NP + e]), s3);
+          }
+          for (; m < a.d; m += 64) {
+            const uint32_t p0 = *reinterpret_cast<const uint32_t*>(xr + m);
+            s0 = fma(static_cast<double>(bf16_lo(p0)), static_cast<double>(Ws[m * NP + e]), s0);
+            s1 = fma(static_cast<double>(bf16_hi(p0)), static_cast<double>(Ws[(m + 1) * NP + e]), s1);
+          }
+          double s64 = (s0 + s1) + (s2 + s3);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s64 += __shfl_xor_sync(0xffffffffu, s64, off);
-        if (lane == 0) zd[t * NP + e] = s64 + static_cast<double>(bsm[e]);
+          for (int off = 16; off > 0; off >>= 1) s64 += __shfl_xor_sync(0xffffffffu, s64, off);
+          if (lane == 0) zd[tv * NP + e] = s64 + static_cast<double>(bsm[e]);
+        }
       }
+      __syncthreads();
+      if (mine && !certain) {
+        sel = group_topk(zd + zo, a.M, a.k);
+        ps[tid] = group_softmax(zd + zo, a.M, sel, ez + zo, dn + tid);
+      }
+      __syncthreads();
     }
-    if (nu > 0) __syncthreads();
-    // Group softmax; selected mass per pair. (The fp64 values of certain
-    // groups are their fp32 logits, so the selection is the one made above.)
-    for (int p = tid; p < P; p += kRouterThreads) {
-      const int t = p / a.G, g = p - t * a.G;
-      if (blk * TB + t >= a.R) continue;
-      const double* zg = zd + t * NP + g * a.M;
-      const uint64_t sel = group_topk(zg, a.M, a.k);
-      double zmax = zg[0];
-      for (int j = 1; j < a.M; ++j) zmax = fmax(zmax, zg[j]);
-      float den = 0.0f;
-      for (int j = 0; j < a.M; ++j) den += expf(static_cast<float>(zg[j] - zmax));
-      float psel = 0.0f;
-      for (int j = 0; j < a.M; ++j)
-        if ((sel >> j) & 1ull) psel += expf(static_cast<float>(zg[j] - zmax)) / den;
-      ps[p] = psel;
-    }
-    __syncthreads();
     // idx, r (renormalised in the group) and omega (over the token's groups).
-    for (int p = tid; p < P; p += kRouterThreads) {
-      const int t = p / a.G, g = p - t * a.G;
-      const int row = blk * TB + t;
-      if (row >= a.R) continue;
-      const double* zg = zd + t * NP + g * a.M;
-      const uint64_t sel = group_topk(zg, a.M, a.k);
-      float tot = 0.0f;
+    if (mine) {
+      float tot = 0.0f;  // selected mass of the token over its groups
       for (int g2 = 0; g2 < a.G; ++g2) tot += ps[t * a.G + g2];
-      const float psel = ps[p];
-      double zmax = zg[0];
-      for (int j = 1; j < a.M; ++j) zmax = fmax(zmax, zg[j]);
-      float den = 0.0f;
-      for (int j = 0; j < a.M; ++j) den += expf(static_cast<float>(zg[j] - zmax));
-      const size_t o = (static_cast<size_t>(row) * a.G + g) * a.k;
+      const float psel = ps[tid], den = dn[tid];
+      const size_t o = (static_cast<size_t>(blk * TB + t) * a.G + g) * a.k;
       int s = 0;
       for (int j = 0; j < a.M; ++j) {
         if ((sel >> j) & 1ull) {
-          const float pj = expf(static_cast<float>(zg[j] - zmax)) / den;
+          const float pj = ez[zo + j] / den;
           a.idx[o + s] = j;
           a.r[o + s] = pj / psel;
           a.omega[o + s] = pj / tot;
@@ -355,18 +380,23 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   cp_async_wait<0>();
 }
 
-template <int NP>
+template <int NP, int WARPS>
 int launch_np(const gqe_config& c, const RouterArgs& a, cudaStream_t st) {
   const size_t smem = router_smem_bytes(c);
   if (smem > kRouterSmemLimit) return cudaErrorInvalidConfiguration;
-  const int e = ensure_smem<router_kernel<NP>>(static_cast<int>(smem));
+  const int e = ensure_smem<router_kernel<NP, WARPS>>(static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   // One block per CTA while that fills the GPU; larger batches loop.
   const int n_blk = (a.R + router_tb(NP) - 1) / router_tb(NP);
   const int per_sm = smem <= 112 * 1024 ? 2 : 1;
   int grid = n_blk < per_sm * 148 ? n_blk : per_sm * 148;
   if (grid < 1) grid = 1;
-  return launch_pdl(router_kernel<NP>, dim3(grid), dim3(kRouterThreads), smem, st, a);
+  return launch_pdl(router_kernel<NP, WARPS>, dim3(grid), dim3(WARPS * 32), smem, st, a);
+}
+
+template <int NP>
+int launch_w(const gqe_config& c, const RouterArgs& a, cudaStream_t st) {
+  return router_warps(c.d_model) == 16 ? launch_np<NP, 16>(c, a, st) : launch_np<NP, 8>(c, a, st);
 }
 
 }  // namespace router_impl
@@ -381,11 +411,11 @@ int launch_router(const gqe_config& c, const uint16_t* x, const float* W_r, cons
   RouterArgs a{x, W_r, b_r, idx, r, omega, c.B * c.T, c.d_model, c.G, c.M, c.k, c.G * c.M};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (router_np(a.N)) {
-    case 4: return launch_np<4>(c, a, st);
-    case 8: return launch_np<8>(c, a, st);
-    case 16: return launch_np<16>(c, a, st);
-    case 32: return launch_np<32>(c, a, st);
-    default: return launch_np<64>(c, a, st);
+    case 4: return launch_w<4>(c, a, st);
+    case 8: return launch_w<8>(c, a, st);
+    case 16: return launch_w<16>(c, a, st);
+    case 32: return launch_w<32>(c, a, st);
+    default: return launch_w<64>(c, a, st);
   }
 }
 
