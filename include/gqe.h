@@ -62,6 +62,13 @@ typedef struct gqe_config {
  * does not clear them itself. Other entry points ignore the flag. */
 #define GQE_FLAG_WS_CLEAN 1u
 
+/* Expert-major routed queries: gqe_dispatch writes Qv in token-list order
+ * ([k*G*B*T, d_head], row r = entry r of tok, i.e. (expert, sequence) lists
+ * one after another, positions ascending) instead of slot-major; the layer
+ * (gqe_layer_fwd) then runs gqe_attention_fwd_compact. Results are the same;
+ * only the layout of Qv and the attention's tiling differ. */
+#define GQE_FLAG_EXPERT_MAJOR 2u
+
 typedef enum gqe_status {
   GQE_OK = 0,
   GQE_ERR_INVALID = 1,      /* bad shape, k > M, null or misaligned pointer */
@@ -192,6 +199,29 @@ gqe_status gqe_kv_proj(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16*
 gqe_status gqe_attention_fwd(const gqe_config* cfg, const gqe_bf16* Qv, const gqe_bf16* Qs,
                              const gqe_bf16* K, const gqe_bf16* V, gqe_bf16* slots, void* ws,
                              size_t ws_bytes, gqe_stream_t stream);
+
+/*
+ * The same attention (steps a8, a9) over compacted, expert-major query
+ * tiles: the routed causal attention streams tiles of 128 consecutive entries
+ * of one (expert, sequence) token list against the group's dense K/V, masks
+ * each row causally by its original position tok[r], and never loads a K/V
+ * tile that lies entirely after a tile's last position; empty lists take no
+ * work ("only the selected query experts, plus one always-on shared head,
+ * run causal attention against their group's dense, unchanged KV head":
+ * gist.science "Technical Summary", Conditional activation and Dense KV
+ * path). The shared head runs as in gqe_attention_fwd.
+ *   slots[b*T + tok[r], (g*k+s)*dh ...] = o of list entry r, where the entry
+ *   belongs to expert e = g*M + j of sequence b and s is the rank of j among
+ *   the token's k selections in group g (from idx).
+ * Qe [k*G*B*T, d_head] in list order (gqe_dispatch with GQE_FLAG_EXPERT_MAJOR);
+ * Qs [B, T, d_head]; K, V [B, G, T, d_head]; idx, offsets, tok as written by
+ * gqe_router_topk and gqe_dispatch; slots [B*T, (k*G+2)*d_head]. No
+ * workspace. Slot kG+1 is not touched.
+ */
+gqe_status gqe_attention_fwd_compact(const gqe_config* cfg, const gqe_bf16* Qe, const gqe_bf16* Qs,
+                                     const gqe_bf16* K, const gqe_bf16* V, const int32_t* idx,
+                                     const int32_t* offsets, const int32_t* tok, gqe_bf16* slots,
+                                     gqe_stream_t stream);
 
 /*
  * Weighted slot and output projection (steps a10, a11): the renormalised

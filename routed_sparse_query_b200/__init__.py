@@ -25,7 +25,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 GQE_OK, GQE_ERR_INVALID, GQE_ERR_UNSUPPORTED, GQE_ERR_WORKSPACE = 0, 1, 2, 3
 GQE_ERR_CUDA, GQE_ERR_TIMEOUT, GQE_ERR_DEVICE_CHECK = 4, 5, 6
 GQE_WS_DISPATCH, GQE_WS_LAYER, GQE_WS_DENSE, GQE_WS_ATTENTION = 1, 2, 3, 4
-GQE_FLAG_WS_CLEAN = 1
+GQE_FLAG_WS_CLEAN, GQE_FLAG_EXPERT_MAJOR = 1, 2
 ITEMS = {"idx": 1, "r": 2, "omega": 3, "counts": 4, "offsets": 5, "tok": 6, "slot_pos": 7,
          "Qv": 8, "Qs": 9, "K": 10, "V": 11, "slots": 12, "dispatch_ws": 13, "attention_ws": 14,
          "dense_Q": 32, "dense_O": 33}
@@ -33,7 +33,7 @@ ITEMS = {"idx": 1, "r": 2, "omega": 3, "counts": 4, "offsets": 5, "tok": 6, "slo
 EXPORTED = ("gqe_workspace_bytes", "gqe_workspace_offset", "gqe_router_topk", "gqe_dispatch",
             "gqe_kv_proj", "gqe_attention_fwd", "gqe_output_proj", "gqe_layer_fwd",
             "gqa_dense_fwd", "gqe_read_status", "gqe_selftest_wait_timeout",
-            "gqe_status_string", "gqe_version", "gqe_dispatch_noalloc")
+            "gqe_status_string", "gqe_version", "gqe_dispatch_noalloc", "gqe_attention_fwd_compact")
 
 
 class GQEConfig(ctypes.Structure):
@@ -64,6 +64,7 @@ _sig = {
     "gqe_dispatch_noalloc": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "gqe_kv_proj": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),
     "gqe_attention_fwd": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "gqe_attention_fwd_compact": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "gqe_output_proj": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P]),
     "gqe_layer_fwd": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                      ctypes.c_size_t, _P]),
@@ -145,6 +146,12 @@ def gqe_attention_fwd(cfg, Qv, Qs, K, V, slots, ws, stream=None):
     _check(_lib.gqe_attention_fwd(_cfg(cfg), _ptr(Qv), _ptr(Qs), _ptr(K), _ptr(V), _ptr(slots),
                                   _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "gqe_attention_fwd")
+
+
+def gqe_attention_fwd_compact(cfg, Qe, Qs, K, V, idx, offsets, tok, slots, stream=None):
+    _check(_lib.gqe_attention_fwd_compact(_cfg(cfg), _ptr(Qe), _ptr(Qs), _ptr(K), _ptr(V), _ptr(idx),
+                                          _ptr(offsets), _ptr(tok), _ptr(slots), _stream(stream)),
+           "gqe_attention_fwd_compact")
 
 
 def gqe_output_proj(cfg, slots, omega, W_o, y, stream=None):

@@ -27,7 +27,7 @@ bool all_aligned(const P*... ps) {
 gqe_status check_cfg(const gqe_config* c) {
   if (c == nullptr) return GQE_ERR_INVALID;
   if (c->B < 1 || c->T < 1 || c->G < 1 || c->M < 1 || c->k < 1 || c->k > c->M) return GQE_ERR_INVALID;
-  if (c->d_model < 64 || c->d_model % 64 != 0 || (c->flags & ~GQE_FLAG_WS_CLEAN) != 0u) return GQE_ERR_INVALID;
+  if (c->d_model < 64 || c->d_model % 64 != 0 || (c->flags & ~(GQE_FLAG_WS_CLEAN | GQE_FLAG_EXPERT_MAJOR)) != 0u) return GQE_ERR_INVALID;
   if (c->G * c->M > kMaxExperts || c->G > 32) return GQE_ERR_UNSUPPORTED;
   if (c->d_head != 32 && c->d_head != 64) return GQE_ERR_UNSUPPORTED;
   // Index arithmetic of the kernels stays within int32 for these extents.
@@ -226,7 +226,7 @@ gqe_status gqe_dispatch(const gqe_config* cfg, const int32_t* idx, const gqe_bf1
   char* w = static_cast<char*>(ws);
   return cuda_status(gemm_q_routed(*cfg, x, W_q, W_qs, idx, offsets, tok, w + L.qtiles,
                                    reinterpret_cast<const int32_t*>(w + L.n_qtiles), L.max_qtiles,
-                                   Qv, Qs, stream));
+                                   Qv, Qs, (cfg->flags & GQE_FLAG_EXPERT_MAJOR) != 0u, stream));
 }
 
 gqe_status gqe_kv_proj(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16* W_k,
@@ -248,6 +248,16 @@ gqe_status gqe_attention_fwd(const gqe_config* cfg, const gqe_bf16* Qv, const gq
   if (ws_bytes < need) return GQE_ERR_WORKSPACE;
   const bool clean = (cfg->flags & GQE_FLAG_WS_CLEAN) != 0u;
   return cuda_status(attention_gqe(*cfg, Qv, Qs, K, V, slots, ws, ws_bytes, clean, stream));
+}
+
+gqe_status gqe_attention_fwd_compact(const gqe_config* cfg, const gqe_bf16* Qe, const gqe_bf16* Qs,
+                                     const gqe_bf16* K, const gqe_bf16* V, const int32_t* idx,
+                                     const int32_t* offsets, const int32_t* tok, gqe_bf16* slots,
+                                     gqe_stream_t stream) {
+  const gqe_status s = check_cfg(cfg);
+  if (s != GQE_OK) return s;
+  if (!all_aligned(Qe, Qs, K, V, idx, offsets, tok, slots)) return GQE_ERR_INVALID;
+  return cuda_status(attention_gqe_em(*cfg, Qe, Qs, K, V, idx, offsets, tok, slots, stream));
 }
 
 gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* omega,
@@ -275,7 +285,7 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
   // The split-KV counters are zeroed first (unless the caller vouches that
   // they are), so that the kernels of the layer follow each other directly
   // (programmatic dependent launch).
-  if ((cfg->flags & GQE_FLAG_WS_CLEAN) == 0u &&
+  if ((cfg->flags & (GQE_FLAG_WS_CLEAN | GQE_FLAG_EXPERT_MAJOR)) == 0u &&
       zero_attention_counters(*cfg, cfg->G * cfg->k + 1, w + L.aws, stream) != cudaSuccess)
     return GQE_ERR_CUDA;
   // K/V projection on the side stream (falls back to the caller's stream).
@@ -299,9 +309,12 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
     if (side != nullptr && cudaStreamWaitEvent(main_st, side->join, 0) != cudaSuccess)
       return GQE_ERR_CUDA;
   }
-  if (attention_gqe(*cfg, H(L.Qv), H(L.Qs), H(L.K), H(L.V), H(L.slots), w + L.aws,
-                    L.total - L.aws, true, stream) != cudaSuccess)
-    return GQE_ERR_CUDA;
+  const int ea = (cfg->flags & GQE_FLAG_EXPERT_MAJOR) != 0u
+                     ? attention_gqe_em(*cfg, H(L.Qv), H(L.Qs), H(L.K), H(L.V), I(L.idx), I(L.offsets),
+                                        I(L.tok), H(L.slots), stream)
+                     : attention_gqe(*cfg, H(L.Qv), H(L.Qs), H(L.K), H(L.V), H(L.slots), w + L.aws,
+                                     L.total - L.aws, true, stream);
+  if (ea != cudaSuccess) return GQE_ERR_CUDA;
   return gqe_output_proj(cfg, H(L.slots), F(L.omega), W_o, y, stream);
 }
 

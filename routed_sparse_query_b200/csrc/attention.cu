@@ -69,7 +69,55 @@ struct AttnParams {
   float* part;       // split-KV partial O: [B*H][items][2][128][dh] fp32
   float2* part_ml;   // split-KV partial (m, l): [B*H][items][2][128]
   int* counters;     // split-KV arrivals per (stream, pair), zero between calls
+  // Expert-major routed tiles (em = 1): a query tile is 128 consecutive
+  // entries of one (expert, sequence) token list, the Q rows in list order
+  // (row r of the layer's routed queries = list entry r); each row is masked
+  // by its own original position tok[r]. The first em_units CTAs take pairs
+  // of such tiles (an upper bound: CTAs past the last pair exit); the rest
+  // take the shared head's stream, as in the slot-major layout.
+  int em;
+  int em_units;
+  int N;
+  const int32_t* offsets;  // [N*B + 1]: list starts in (expert, sequence) order
+  const int32_t* tok;      // list entries: positions t
+  const int32_t* idx;      // [B*T, G, k]: selections (the output slot of a row)
 };
+
+// Expert-major decode: routed unit u -> (list l = e*B + b, pair q of its
+// tiles). Units are counted list by list; inside a list the pair with the
+// largest positions (the longest KV range) comes first. Warp-cooperative;
+// every lane returns the same values. False past the last unit.
+__device__ __forceinline__ bool em_find_unit(const AttnParams& p, int u, int lane, int& l_out,
+                                             int& list0, int& cnt, int& q) {
+  const int NB = p.N * p.B;
+  int base = 0;
+  for (int l0 = 0; l0 < NB; l0 += 32) {
+    const int l = l0 + lane;
+    int c = 0;
+    if (l < NB) c = p.offsets[l + 1] - p.offsets[l];
+    const int pairs = (c + 2 * BQ - 1) / (2 * BQ);
+    int incl = pairs;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (u < base + total) {
+      const unsigned m = __ballot_sync(0xffffffffu, u < base + incl);
+      const int src = __ffs(m) - 1;
+      const int src_pairs = __shfl_sync(0xffffffffu, pairs, src);
+      const int src_excl = __shfl_sync(0xffffffffu, incl, src) - src_pairs;
+      cnt = __shfl_sync(0xffffffffu, c, src);
+      l_out = l0 + src;
+      q = src_pairs - 1 - (u - base - src_excl);
+      list0 = __ldg(p.offsets + l_out) + 2 * BQ * q;
+      return true;
+    }
+    base += total;
+  }
+  return false;
+}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -268,7 +316,8 @@ __device__ __forceinline__ void store_row32(uint16_t* dst, const uint32_t (&v)[3
 }
 
 // Item n of a CTA's S sequence over its KV tiles j0..: (a,j0), (b,j0),
-// (a,j0+1), (b,j0+1), ..., and tile b's extra diagonal tile last; tile a
+// (a,j0+1), (b,j0+1), ..., then tile b's further tiles (one diagonal tile in
+// the slot-major layout, possibly more with expert-major tiles); tile a
 // alone when the CTA has no tile b. na = tile a's KV tiles in the CTA.
 __device__ __forceinline__ void seq_item(int n, bool has_b, int j0, int na, int& t, int& j) {
   if (!has_b) {
@@ -279,7 +328,7 @@ __device__ __forceinline__ void seq_item(int n, bool has_b, int j0, int na, int&
     j = j0 + (n >> 1);
   } else {
     t = 1;
-    j = j0 + na;
+    j = j0 + na + (n - 2 * na);
   }
 }
 
@@ -310,52 +359,76 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
-  // Work item: (stream bh, query-tile pair, KV chunk), longest pairs first.
-  int ord = static_cast<int>(blockIdx.x) / BH;
-  int pair, chunk_id = 0, n_chunks = 1, item_base = ord;
-  if (p.chunk >= p.n_qt) {
-    pair = p.n_pairs - 1 - ord;
-  } else {
-    item_base = 0;
-    for (pair = p.n_pairs - 1; pair > 0; --pair) {
-      const int nc = (2 * pair + 1 + p.chunk - 1) / p.chunk;
-      if (ord < nc) break;
-      ord -= nc;
-      item_base += nc;
-    }
-    n_chunks = (2 * pair + 1 + p.chunk - 1) / p.chunk;
-    chunk_id = ord;
-  }
-  const int b = bh / p.H, h = bh % p.H;
-  int zq, grp, slot;
+  // Work of this CTA. Slot-major (and the shared head of an expert-major
+  // launch): (stream, query-tile pair, KV chunk), longest pairs first, decoded
+  // from the launch parameters. Expert-major routed tiles: decoded after
+  // pdl_wait from the token lists (below).
+  const bool em_routed = p.em != 0 && static_cast<int>(blockIdx.x) < p.em_units;
+  int bh = 0, b = 0, zq = 0, grp = 0, slot = 0, pair = 0, chunk_id = 0, n_chunks = 1, item_base = 0;
+  int qa = 0, qb = 0;    // Q rows (TMA coordinate) of tiles a and b
+  int mfa = 0, mfb = 0;  // first KV tile that needs the causal mask, per tile
+  int j0 = 0, ja1 = 0, jb1 = 0;
+  bool has_b = false;
+  int em_e = 0, em_list0 = 0, em_rows_a = 0, em_rows_b = 0;
   const CUtensorMap* tq = &tmQ;
-  if (p.dense) {
-    zq = b * p.H + h;
-    grp = h / p.M;
-    slot = h;
-  } else if (h < p.G * p.k) {
-    zq = b * p.G * p.k + h;
-    grp = h / p.k;
-    slot = h;
-  } else {
-    zq = b;
-    grp = 0;
-    slot = p.G * p.k;
-    tq = &tmQs;
+  if (!em_routed) {
+    int ord, h;
+    if (p.em) {  // the shared head of an expert-major launch: B streams
+      const int u2 = static_cast<int>(blockIdx.x) - p.em_units;
+      b = u2 % p.B;
+      ord = u2 / p.B;
+      h = p.G * p.k;
+      bh = b * p.H + h;
+    } else {
+      bh = static_cast<int>(blockIdx.x) % BH;
+      ord = static_cast<int>(blockIdx.x) / BH;
+      b = bh / p.H;
+      h = bh % p.H;
+    }
+    item_base = ord;
+    if (p.chunk >= p.n_qt) {
+      pair = p.n_pairs - 1 - ord;
+    } else {
+      item_base = 0;
+      for (pair = p.n_pairs - 1; pair > 0; --pair) {
+        const int nc = (2 * pair + 1 + p.chunk - 1) / p.chunk;
+        if (ord < nc) break;
+        ord -= nc;
+        item_base += nc;
+      }
+      n_chunks = (2 * pair + 1 + p.chunk - 1) / p.chunk;
+      chunk_id = ord;
+    }
+    if (p.dense) {
+      zq = b * p.H + h;
+      grp = h / p.M;
+      slot = h;
+    } else if (h < p.G * p.k) {
+      zq = b * p.G * p.k + h;
+      grp = h / p.k;
+      slot = h;
+    } else {
+      zq = b;
+      grp = 0;
+      slot = p.G * p.k;
+      tq = &tmQs;
+    }
+    const int qt0 = 2 * pair;
+    has_b = qt0 + 1 < p.n_qt;
+    // Causal: query tile qt needs KV tiles 0..qt (tile a = qt0, tile b =
+    // qt0+1). This CTA takes KV tiles [j0, ja1) for tile a and [j0, jb1) for
+    // tile b; the last chunk also holds tile b's extra diagonal tile.
+    j0 = chunk_id * (p.chunk < p.n_qt ? p.chunk : 0);
+    const bool last_chunk = chunk_id == n_chunks - 1;
+    ja1 = last_chunk ? qt0 + 1 : j0 + p.chunk;
+    jb1 = has_b ? (last_chunk ? qt0 + 2 : ja1) : j0;
+    qa = qt0 * BQ;
+    qb = qa + BQ;
+    mfa = qt0;  // only the diagonal tile is masked
+    mfb = qt0 + 1;
   }
-  const int zkv = b * p.G + grp;
-  const int qt0 = 2 * pair;
-  const bool has_b = qt0 + 1 < p.n_qt;
-  // Causal: query tile qt needs KV tiles 0..qt (tile a = qt0, tile b = qt0+1).
-  // This CTA takes KV tiles [j0, ja1) for tile a and [j0, jb1) for tile b;
-  // the last chunk also holds tile b's extra diagonal tile.
-  const int j0 = chunk_id * (p.chunk < p.n_qt ? p.chunk : 0);
-  const bool last_chunk = chunk_id == n_chunks - 1;
-  const int ja1 = last_chunk ? qt0 + 1 : j0 + p.chunk;
-  const int jb1 = has_b ? (last_chunk ? qt0 + 2 : ja1) : j0;
-  const int na = ja1 - j0;
-  const int jend = has_b ? jb1 : ja1;
+  int na = ja1 - j0;
+  int jend = has_b ? jb1 : ja1;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -385,13 +458,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tslot;
   pdl_wait();  // every input (Q, K, V) is read after this point
   pdl_launch_dependents();
+  if (em_routed) {
+    // Expert-major routed pair: tiles of 128 consecutive list entries; the KV
+    // range of a tile ends at the tile containing its last (largest)
+    // position, and the mask starts at the first tile not entirely below its
+    // first (smallest) position. A CTA past the last pair loads one Q tile
+    // and exits.
+    int l = 0, cnt = 0, q = 0, list0 = 0;
+    if (em_find_unit(p, static_cast<int>(blockIdx.x), lane, l, list0, cnt, q)) {
+      em_e = l / p.B;
+      b = l % p.B;
+      grp = em_e / p.M;
+      em_list0 = list0;
+      const int rem = cnt - 2 * BQ * q;
+      em_rows_a = rem < BQ ? rem : BQ;
+      em_rows_b = rem - BQ < BQ ? rem - BQ : BQ;
+      has_b = em_rows_b > 0;
+      const int pa0 = __ldg(p.tok + list0), pa1 = __ldg(p.tok + list0 + em_rows_a - 1);
+      qa = list0;
+      qb = list0 + BQ;
+      mfa = (pa0 + 1) / BKV;
+      ja1 = pa1 / BKV + 1;
+      if (has_b) {
+        const int pb0 = __ldg(p.tok + list0 + BQ), pb1 = __ldg(p.tok + list0 + BQ + em_rows_b - 1);
+        mfb = (pb0 + 1) / BKV;
+        jb1 = pb1 / BKV + 1;
+      } else {
+        jb1 = 0;
+      }
+    }
+    na = ja1 - j0;
+    jend = has_b ? jb1 : ja1;
+  }
+  const int zkv = b * p.G + grp;
 
   if (warp == kTmaWarp) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, C::TILE_BYTES * (has_b ? 2 : 1));
-      tma_load_3d(sQ, tq, q_full, 0, qt0 * BQ, zq);
-      if (has_b) tma_load_3d(sQ + C::TILE_BYTES, tq, q_full, 0, (qt0 + 1) * BQ, zq);
+      tma_load_3d(sQ, tq, q_full, 0, qa, zq);
+      if (has_b) tma_load_3d(sQ + C::TILE_BYTES, tq, q_full, 0, qb, zq);
       for (int j = j0; j < jend; ++j) {
         const int st = (j - j0) % KV_STAGES;
         const uint32_t ph = ((j - j0) / KV_STAGES) & 1;
@@ -471,8 +577,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = threadIdx.x & 127;    // row in tile = TMEM lane
     const int jt1 = t == 0 ? ja1 : jb1;  // this tile's KV tiles: [j0, jt1)
     const int n_t = (t == 0 || has_b) ? jt1 - j0 : 0;
-    const int qt = qt0 + t;
-    const int qi = qt * BQ + i;
+    const int mask_from = t == 0 ? mfa : mfb;
+    // The row's original position (qi) and whether it holds a query.
+    int qi;
+    bool row_ok;
+    if (em_routed) {
+      const int rows = t == 0 ? em_rows_a : em_rows_b;
+      row_ok = i < rows;
+      qi = rows > 0 ? __ldg(p.tok + em_list0 + t * BQ + (row_ok ? i : rows - 1)) : 0;
+    } else {
+      qi = (qa / BQ + t) * BQ + i;
+      row_ok = qi < p.T;
+    }
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tO = tmem + 384 + t * DH + lane_off;
     const float sc = p.scale_log2;
@@ -481,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int jr = 0; ok && jr < n_t; ++jr) {
       const int j = j0 + jr;
       // This tile's S for KV tile j is sequence item n, in TMEM buffer n % 3.
-      const int n = has_b ? (j < ja1 ? 2 * jr + t : 2 * na) : jr;
+      const int n = has_b ? (j < ja1 ? 2 * jr + t : 2 * na + (j - ja1)) : jr;
       const uint32_t tS = tmem + (n % 3) * 128 + lane_off;
       // Waits are made warp-uniform: tcgen05.ld/st below are .sync.aligned.
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[n % 3], (n / 3) & 1, abort_flag))) {
@@ -496,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t* pv_prev = jr > 0 ? &o_done[t] : nullptr;
       const uint32_t pv_par = static_cast<uint32_t>(jr - 1) & 1u;
       bool w_ok = true;
-      if (j == qt)  // the diagonal tile
+      if (j >= mask_from)  // a tile with keys after some row's position
         w_ok = softmax_tile<DH, true>(tS, tO, qi - j * BKV, sc, jr == 0, m, l, pv_prev, pv_par,
                                       abort_flag);
       else
@@ -515,12 +631,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (fin) {
         tc_fence_after();
         const float inv = 1.0f / l;
-        uint16_t* dst = p.out + (static_cast<size_t>(b) * p.T + qi) * p.ldo + slot * DH;
+        int col = slot;
+        if (em_routed && row_ok) {
+          // The row's slot: rank of its expert among its selections in the group.
+          const int g = em_e / p.M, jj = em_e % p.M;
+          const int32_t* ip = p.idx + (static_cast<size_t>(b) * p.T + qi) * p.G * p.k + g * p.k;
+          int s2 = 0;
+          for (int s3 = 0; s3 < p.k; ++s3)
+            if (__ldg(ip + s3) == jj) s2 = s3;
+          col = g * p.k + s2;
+        }
+        uint16_t* dst = p.out + (static_cast<size_t>(b) * p.T + qi) * p.ldo + col * DH;
 #pragma unroll
         for (int c = 0; c < DH / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(tO + c * 32, v);
-          if (qi < p.T) store_row32(dst + c * 32, v, inv);
+          if (row_ok) store_row32(dst + c * 32, v, inv);
         }
       }
     } else {
@@ -554,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_sync(1, 256);
       if (*s_last) {
         __threadfence();
-        if (n_t > 0 && qi < p.T) {
+        if (n_t > 0 && row_ok) {
           const size_t blk0 = (static_cast<size_t>(bh) * p.items + item_base) * 2 + t;
           float ms = -INFINITY;
           for (int c = 0; c < n_chunks; ++c) ms = fmaxf(ms, __ldcg(&p.part_ml[(blk0 + 2 * c) * BQ + i]).x);
@@ -603,12 +729,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int DH>
 int launch_attn(const CUtensorMap& q, const CUtensorMap& qs, const CUtensorMap& k,
-                const CUtensorMap& v, const AttnParams& p, void* stream) {
+                const CUtensorMap& v, const AttnParams& p, long long grid, void* stream) {
   using C = AttnCfg<DH>;
   const int e = ensure_smem<attn_kernel<DH>>(static_cast<int>(C::SMEM));
   if (e != cudaSuccess) return e;
-  const long long grid = static_cast<long long>(p.items) * p.B * p.H;
   if (grid <= 0) return cudaSuccess;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   return launch_pdl(attn_kernel<DH>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), C::SMEM,
                     stream, q, qs, k, v, p);
 }
@@ -627,7 +753,7 @@ int run(const gqe_config& c, const uint16_t* Q, uint64_t nq_streams, const uint1
     return cudaErrorInvalidValue;
   if (!make_tmap_bf16_3d(&tv, V, dh, c.T, static_cast<uint64_t>(c.B) * c.G, dh, BKV))
     return cudaErrorInvalidValue;
-  AttnParams p;
+  AttnParams p{};
   p.T = c.T;
   p.B = c.B;
   p.H = H;
@@ -651,8 +777,51 @@ int run(const gqe_config& c, const uint16_t* Q, uint64_t nq_streams, const uint1
                                           static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return e;
   }
-  if (dh == 64) return launch_attn<64>(tq, tqs, tk, tv, p, stream);
-  return launch_attn<32>(tq, tqs, tk, tv, p, stream);
+  const long long grid = static_cast<long long>(p.items) * p.B * p.H;
+  if (dh == 64) return launch_attn<64>(tq, tqs, tk, tv, p, grid, stream);
+  return launch_attn<32>(tq, tqs, tk, tv, p, grid, stream);
+}
+
+// Expert-major routed attention plus the shared head (one launch, no split).
+int run_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const uint16_t* K,
+           const uint16_t* V, const int32_t* idx, const int32_t* offsets, const int32_t* tok,
+           uint16_t* slots, void* stream) {
+  const int dh = c.d_head;
+  const long long R = static_cast<long long>(c.B) * c.T;
+  const long long rows = R * c.G * c.k;  // routed query rows, in list order
+  CUtensorMap tq, tqs, tk, tv;
+  if (!make_tmap_bf16_3d(&tq, Qe, dh, static_cast<uint64_t>(rows), 1, dh, BQ)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_3d(&tqs, Qs, dh, c.T, c.B, dh, BQ)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_3d(&tk, K, dh, c.T, static_cast<uint64_t>(c.B) * c.G, dh, BKV))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_3d(&tv, V, dh, c.T, static_cast<uint64_t>(c.B) * c.G, dh, BKV))
+    return cudaErrorInvalidValue;
+  AttnParams p{};
+  p.T = c.T;
+  p.B = c.B;
+  p.H = c.G * c.k + 1;
+  p.G = c.G;
+  p.k = c.k;
+  p.M = c.M;
+  p.dense = 0;
+  p.n_qt = (c.T + BQ - 1) / BQ;
+  p.n_pairs = (p.n_qt + 1) / 2;
+  p.chunk = p.n_qt;  // no split
+  p.items = p.n_pairs;
+  p.out = slots;
+  p.ldo = (c.G * c.k + 2) * dh;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(dh)));
+  p.em = 1;
+  p.N = c.G * c.M;
+  // Pairs of 128-row tiles over all lists: at most rows / 256 + one partial
+  // pair per list.
+  p.em_units = static_cast<int>(rows / (2 * BQ) + static_cast<long long>(p.N) * c.B + 1);
+  p.offsets = offsets;
+  p.tok = tok;
+  p.idx = idx;
+  const long long grid = static_cast<long long>(p.em_units) + static_cast<long long>(p.n_pairs) * c.B;
+  if (dh == 64) return launch_attn<64>(tq, tqs, tk, tv, p, grid, stream);
+  return launch_attn<32>(tq, tqs, tk, tv, p, grid, stream);
 }
 
 }  // namespace attn_impl
@@ -700,6 +869,12 @@ int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, c
   const int H = c.G * c.k + 1;
   return run(c, Qv, static_cast<uint64_t>(c.B) * c.G * c.k, Qs, K, V, slots,
              (c.G * c.k + 2) * c.d_head, H, 0, ws, ws_bytes, counters_zeroed, stream);
+}
+
+int attention_gqe_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const uint16_t* K,
+                     const uint16_t* V, const int32_t* idx, const int32_t* offsets, const int32_t* tok,
+                     uint16_t* slots, void* stream) {
+  return run_em(c, Qe, Qs, K, V, idx, offsets, tok, slots, stream);
 }
 
 int attention_dense(const gqe_config& c, const uint16_t* Q, const uint16_t* K, const uint16_t* V,

@@ -78,6 +78,7 @@ struct Gather {
   uint16_t* Qs;     // shared-head output [B*T, dh] (tiles after the routed ones)
   int max_qtiles;   // CTAs reserved for routed tiles
   int d, T, G, M, k, B, dh;
+  int expert_major;  // routed rows go to Qv[list entry] (token-list order)
 };
 
 __device__ __forceinline__ void store32_bf16(uint16_t* dst, const uint32_t (&v)[32]) {
@@ -319,6 +320,8 @@ __global__ void __launch_bounds__(192, 2)
       size_t obase = 0;
       if (valid && shared_tile) {
         obase = static_cast<size_t>(m0 + r) * ga.dh;
+      } else if (valid && ga.expert_major) {
+        obase = static_cast<size_t>(list0 + r) * ga.dh;
       } else if (valid) {
         const int t = ga.tok[list0 + r];
         const int g = e / ga.M, j = e % ga.M;
@@ -473,7 +476,7 @@ int gemm_output(const gqe_config& c, uint16_t* slots, const float* omega, const 
 int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const uint16_t* W_qs,
                   const int32_t* idx, const int32_t* offsets, const int32_t* tok, const void* qtiles,
                   const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, uint16_t* Qs,
-                  void* stream) {
+                  bool expert_major, void* stream) {
   const int N = c.G * c.M;
   const int dh = c.d_head;
   CUtensorMap tb, tbs;
@@ -498,6 +501,7 @@ int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, c
   g.k = c.k;
   g.B = c.B;
   g.dh = dh;
+  g.expert_major = expert_major ? 1 : 0;
   Epi e{};
   const long long R = static_cast<long long>(c.B) * c.T;
   const dim3 grid(static_cast<unsigned>(max_qtiles + (R + BM - 1) / BM), 1, 1);

@@ -91,9 +91,12 @@ int gemm_kv(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const u
             uint16_t* K, uint16_t* V, void* stream);
 // Routed query projection over the token lists plus the shared-head query
 // projection, in one launch.
+// expert_major: Qv is written in token-list order ([k*G*B*T, dh], row = list
+// entry) instead of slot-major [B, G, k, T, dh].
 int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const uint16_t* W_qs,
                   const int32_t* idx, const int32_t* offsets, const int32_t* tok, const void* qtiles,
-                  const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, uint16_t* Qs, void* stream);
+                  const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, uint16_t* Qs,
+                  bool expert_major, void* stream);
 int gemm_q_dense(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, uint16_t* Q,
                  void* stream);
 int gemm_rowmajor(const uint16_t* A, int rows, int K, const uint16_t* W, int N, uint16_t* out,
@@ -117,6 +120,11 @@ AttnPlan attention_plan(const gqe_config& c, int H);
 int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
                   const uint16_t* V, uint16_t* slots, void* ws, size_t ws_bytes,
                   bool counters_zeroed, void* stream);
+// Expert-major routed attention (Qe in token-list order, rows masked by
+// their positions tok[]) plus the shared head, one launch, no scratch.
+int attention_gqe_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const uint16_t* K,
+                     const uint16_t* V, const int32_t* idx, const int32_t* offsets, const int32_t* tok,
+                     uint16_t* slots, void* stream);
 int attention_dense(const gqe_config& c, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                     uint16_t* O, void* ws, size_t ws_bytes, bool counters_zeroed, void* stream);
 int zero_attention_counters(const gqe_config& c, int H, void* ws, void* stream);

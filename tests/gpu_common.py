@@ -106,3 +106,54 @@ def run_dense(rsq, shape, d: dict):
     torch.cuda.synchronize()
     assert rsq.gqe_read_status() == 0
     return y, ws
+
+
+def run_expert_major(rsq, shape: synth.LayerShape, d: dict, o: dict) -> dict:
+    """The expert-major layout on the outputs `o` of run_steps: dispatch with
+    GQE_FLAG_EXPERT_MAJOR (Q rows in token-list order), compact attention,
+    output projection. Returns Qe, slots and y."""
+    cfg = rsq.GQEConfig.of(shape, rsq.GQE_FLAG_EXPERT_MAJOR)
+    B, T, G, M, k, dh = shape.B, shape.T, shape.G, shape.M, shape.k, shape.d_head
+    R, N = B * T, G * M
+    dev = torch.device("cuda")
+    e = {}
+    e["Qe"] = torch.empty(k * G * R, dh, dtype=torch.bfloat16, device=dev)
+    e["Qs"] = torch.empty(B, T, dh, dtype=torch.bfloat16, device=dev)
+    counts = torch.empty(N * B, dtype=torch.int32, device=dev)
+    offsets = torch.empty(N * B + 1, dtype=torch.int32, device=dev)
+    tok = torch.empty(k * G * R, dtype=torch.int32, device=dev)
+    slot_pos = torch.empty(R, G, k, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_DISPATCH), 16), dtype=torch.uint8,
+                     device=dev)
+    rsq.gqe_dispatch(cfg, o["idx"], d["x"], d["W_q"], d["W_qs"], counts, offsets, tok, slot_pos,
+                     e["Qe"], e["Qs"], ws)
+    assert torch.equal(offsets, o["offsets"]) and torch.equal(tok, o["tok"])
+    e["slots"] = torch.zeros(R, (k * G + 2) * dh, dtype=torch.bfloat16, device=dev)
+    rsq.gqe_attention_fwd_compact(cfg, e["Qe"], e["Qs"], o["K"], o["V"], o["idx"], offsets, tok,
+                                  e["slots"])
+    e["y"] = torch.empty(R, shape.d_model, dtype=torch.bfloat16, device=dev)
+    rsq.gqe_output_proj(cfg, e["slots"], o["omega"], d["W_o"], e["y"])
+    torch.cuda.synchronize()
+    assert rsq.gqe_read_status() == 0
+    return e
+
+
+def qv_in_list_order(o: dict, shape: synth.LayerShape) -> torch.Tensor:
+    """Slot-major Qv gathered into token-list order (list entry r of expert
+    e = g*M + j, sequence b, position t -> Qv[b, g, s, t] with s the rank of j
+    among the token's selections in group g)."""
+    B, T, G, M, k = shape.B, shape.T, shape.G, shape.M, shape.k
+    N = G * M
+    offs = o["offsets"].cpu().numpy()
+    tok = o["tok"].cpu().numpy()
+    idx = o["idx"].cpu().numpy()
+    rows = []
+    for e in range(N):
+        g, j = divmod(e, M)
+        for b in range(B):
+            for r in range(offs[e * B + b], offs[e * B + b + 1]):
+                t = int(tok[r])
+                s = int(np.nonzero(idx[b * T + t, g] == j)[0][0])
+                rows.append(((b * G + g) * k + s) * T + t)
+    flat = o["Qv"].reshape(B * G * k * T, -1)
+    return flat[torch.tensor(rows, dtype=torch.long, device=flat.device)]

@@ -13,7 +13,8 @@ import torch
 import oracle
 import synth
 from synth import LayerShape
-from gpu_common import (assert_close, device_inputs, run_dense, run_layer, run_steps, to_f64)
+from gpu_common import (assert_close, device_inputs, qv_in_list_order, run_dense, run_expert_major,
+                        run_layer, run_steps, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -193,3 +194,44 @@ def test_device_wait_timeout_is_reported_and_recoverable(rsq):
     ref = oracle.gqe_layer(inp)
     y, _ = run_layer(rsq, shape, device_inputs(inp))
     assert_close(y, ref["y"], "y after timeout self-test")
+
+
+EM_CASES = ["tiny", "ragged_b2", "pool4_k2_skew", "k_equals_m", "t5_dh32"]
+
+
+@pytest.mark.parametrize("name", EM_CASES)
+def test_expert_major_layout_matches_oracle(rsq, name):
+    # Compacted, expert-major query tiles (rows masked by their positions):
+    # the same Q rows, and slots and y within the layer tolerance.
+    shape, kw = CASES[name]
+    inp = synth.make_layer_inputs(shape, seed=101, **kw)
+    ref = oracle.gqe_layer(inp)
+    d = device_inputs(inp)
+    o = run_steps(rsq, shape, d)
+    e = run_expert_major(rsq, shape, d, o)
+    assert torch.equal(e["Qe"], qv_in_list_order(o, shape)), "Q rows differ between layouts"
+    assert torch.equal(e["Qs"], o["Qs"])
+    assert_close(e["slots"], ref["slots"], "slots (expert-major)")
+    assert_close(e["y"], ref["y"], "y (expert-major)")
+
+
+def test_expert_major_long_sequences_equal_slot_major(rsq):
+    # No split-KV at this size (27 streams x 28 tile pairs): both layouts run
+    # the same online softmax over the same K/V tiles for every row, so the
+    # slots are bitwise equal; three sequences, 12 experts, k = 2, ragged tiles.
+    shape = LayerShape(B=3, T=7000, d_model=128, G=4, M=3, k=2, d_head=32)
+    inp = synth.make_layer_inputs(shape, seed=23)
+    d = device_inputs(inp)
+    o = run_steps(rsq, shape, d)
+    e = run_expert_major(rsq, shape, d, o)
+    assert torch.equal(e["slots"], o["slots"]), "expert-major slots differ from slot-major"
+    assert torch.equal(e["y"], o["y"])
+    # The whole layer with the flag gives the same y.
+    cfg = rsq.GQEConfig.of(shape, rsq.GQE_FLAG_EXPERT_MAJOR)
+    ws = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_LAYER), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(o["y"])
+    rsq.gqe_layer_fwd(cfg, d["x"], d["W_r"], d["b_r"], d["W_q"], d["W_qs"], d["W_k"], d["W_v"],
+                      d["W_o"], y, ws)
+    torch.cuda.synchronize()
+    assert rsq.gqe_read_status() == 0
+    assert torch.equal(y, o["y"])
