@@ -1,4 +1,5 @@
-"""fp64 CPU oracle of one Grouped Query Experts (GQE) prefill layer.
+"""fp64 CPU oracle of one Grouped Query Experts (GQE) prefill layer (and of one
+decode step against its dense K/V cache).
 
 TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
 baseline / reference arm of ``bench.py`` may import or call this package. The
@@ -388,3 +389,67 @@ def gqa_dense_layer(inp: LayerInputs, rows=None) -> dict:
 def active_query_heads(shape: LayerShape) -> int:
     """Query heads that run attention per token: k per group plus the shared head."""
     return shape.k * shape.G + 1
+
+
+# ---------------------------------------------------------------- decode step
+def _decode_attention(q: np.ndarray, K_cache: np.ndarray, V_cache: np.ndarray,
+                      k_new: np.ndarray, v_new: np.ndarray) -> np.ndarray:
+    """Attention of one new query against its cache plus its own key: the
+    causal definition at position L = len(cache), all L+1 keys visible."""
+    K = np.concatenate([K_cache, k_new[None, :]], axis=0)
+    V = np.concatenate([V_cache, v_new[None, :]], axis=0)
+    L = K_cache.shape[0]
+    return causal_attention(q[None, :], K, V, rows=[L])[0]
+
+
+def gqe_decode_step(x_new: np.ndarray, K_cache: np.ndarray, V_cache: np.ndarray, W_r, b_r,
+                    W_q, W_qs, W_k, W_v, W_o, G: int, M: int, k: int, dh: int) -> dict:
+    """One GQE decode step (the survey's next row f2): each sequence b appends
+    token x_new[b] at position L to its dense, unchanged K/V cache [B, G, L, dh]
+    ("the Key-Value projections and the KV cache stay dense and unchanged":
+    gist.science Technical Summary, Dense KV path) and the layer's output for
+    that token is the prefill definition (a1-a11) at position L: router on the
+    new token, only its selected experts' queries plus the shared head attend
+    to the cache and the new key, the (kG+2) slots, W_O.
+
+    All inputs are fp64 values of the bf16 / fp32 bits; returns idx, r, omega,
+    k_new, v_new [B, G, dh], slots and y.
+    """
+    B = x_new.shape[0]
+    rt = router(x_new, W_r, b_r, G, M, k)
+    idx = rt["idx"]
+    k_new = (x_new @ W_k).reshape(B, G, dh)
+    v_new = (x_new @ W_v).reshape(B, G, dh)
+    o_r = np.zeros((B, G, k, dh))
+    for b in range(B):
+        for g in range(G):
+            for s in range(k):
+                e = g * M + int(idx[b, g, s])
+                q = x_new[b] @ W_q[:, e * dh:(e + 1) * dh]
+                o_r[b, g, s] = _decode_attention(q, K_cache[b, g], V_cache[b, g], k_new[b, g],
+                                                 v_new[b, g])
+    q_s = x_new @ W_qs
+    o_s = np.stack([_decode_attention(q_s[b], K_cache[b, 0], V_cache[b, 0], k_new[b, 0], v_new[b, 0])
+                    for b in range(B)])
+    slots = assemble_slots(o_r, o_s, rt["omega"])
+    out = dict(rt)
+    out.update(k_new=k_new, v_new=v_new, slots=slots, y=output_proj(slots, W_o))
+    return out
+
+
+def gqa_dense_decode_step(x_new: np.ndarray, K_cache: np.ndarray, V_cache: np.ndarray, W_q, W_k,
+                          W_v, W_o_dense, G: int, M: int, dh: int) -> dict:
+    """Dense GQA decode step: all N = G*M heads, head h on group h // M."""
+    B = x_new.shape[0]
+    N = G * M
+    k_new = (x_new @ W_k).reshape(B, G, dh)
+    v_new = (x_new @ W_v).reshape(B, G, dh)
+    Q = x_new @ W_q
+    O = np.zeros((B, N, dh))
+    for b in range(B):
+        for h in range(N):
+            g = h // M
+            O[b, h] = _decode_attention(Q[b, h * dh:(h + 1) * dh], K_cache[b, g], V_cache[b, g],
+                                        k_new[b, g], v_new[b, g])
+    O = O.reshape(B, N * dh)
+    return {"k_new": k_new, "v_new": v_new, "O": O, "y": O @ W_o_dense}

@@ -436,3 +436,47 @@ def test_published_setting_counts():
     assert inp.W_o.shape == (shape.n_slots * shape.d_head, shape.d_model)
     # active (token, query-head) attention rows: one per selected expert + shared
     assert gq["idx"].size + shape.R == oracle.active_query_heads(shape) * shape.R
+
+
+def _decode_case(seed, B=2, T=9, G=2, M=3, k=2, dh=32):
+    s = LayerShape(B=B, T=T, d_model=64, G=G, M=M, k=k, d_head=dh)
+    inp = synth.make_layer_inputs(s, seed=seed)
+    f = oracle._f64_inputs(inp)
+    L = T - 1
+    K = oracle.kv_proj(f["x"], f["W_k"], B, T, G, dh)
+    V = oracle.kv_proj(f["x"], f["W_v"], B, T, G, dh)
+    rows = [b * T + L for b in range(B)]
+    return s, inp, f, K[:, :, :L], V[:, :, :L], rows
+
+
+def test_decode_step_is_the_prefill_layer_at_the_last_position():
+    # Decoding token L against the K/V cache of tokens 0..L-1 is the prefill
+    # definition evaluated at position L (causality): GQE and dense GQA.
+    s, inp, f, Kc, Vc, rows = _decode_case(seed=31)
+    ref = oracle.gqe_layer(inp, rows=rows)
+    d = oracle.gqe_decode_step(f["x"][rows], Kc, Vc, f["W_r"], f["b_r"], f["W_q"], f["W_qs"],
+                               f["W_k"], f["W_v"], f["W_o"], s.G, s.M, s.k, s.d_head)
+    np.testing.assert_array_equal(d["idx"], ref["idx"][rows])
+    np.testing.assert_allclose(d["slots"], ref["slots"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(d["y"], ref["y"], rtol=0, atol=1e-13)
+    dref = oracle.gqa_dense_layer(inp, rows=rows)
+    dd = oracle.gqa_dense_decode_step(f["x"][rows], Kc, Vc, f["W_q"], f["W_k"], f["W_v"],
+                                      f["W_o_dense"], s.G, s.M, s.d_head)
+    np.testing.assert_allclose(dd["y"], dref["y"], rtol=0, atol=1e-13)
+
+
+def test_decode_step_with_an_empty_cache_returns_the_new_values():
+    # L = 0: the only key is the token's own, so every head's output is v_new
+    # of its group (the shared head's of group 0), whatever the query.
+    s, inp, f, Kc, Vc, rows = _decode_case(seed=32)
+    x = f["x"][rows]
+    d = oracle.gqe_decode_step(x, Kc[:, :, :0], Vc[:, :, :0], f["W_r"], f["W_r"][0] * 0, f["W_q"],
+                               f["W_qs"], f["W_k"], f["W_v"], f["W_o"], s.G, s.M, s.k, s.d_head)
+    dh, G, k = s.d_head, s.G, s.k
+    v_new = (x @ f["W_v"]).reshape(len(rows), G, dh)
+    for g in range(G):
+        for si in range(k):
+            np.testing.assert_allclose(d["slots"][:, (g * k + si) * dh:(g * k + si + 1) * dh],
+                                       v_new[:, g], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(d["slots"][:, G * k * dh:(G * k + 1) * dh], v_new[:, 0], rtol=0,
+                               atol=1e-13)
