@@ -84,7 +84,9 @@ enum {
   GQE_WS_DISPATCH = 1, /* scratch of gqe_dispatch */
   GQE_WS_LAYER = 2,    /* everything gqe_layer_fwd keeps between its steps */
   GQE_WS_DENSE = 3,    /* everything gqa_dense_fwd keeps between its steps */
-  GQE_WS_ATTENTION = 4 /* scratch of gqe_attention_fwd (split-KV partials) */
+  GQE_WS_ATTENTION = 4, /* scratch of gqe_attention_fwd (split-KV partials) */
+  GQE_WS_DECODE = 5,    /* scratch of gqe_decode_step */
+  GQE_WS_DENSE_DECODE = 6 /* scratch of gqa_dense_decode_step */
 };
 
 /* Items inside the GQE_WS_LAYER / GQE_WS_DENSE workspaces (for inspection). */
@@ -275,6 +277,39 @@ const char* gqe_status_string(gqe_status s);
 
 /* Library ABI version (major*100 + minor). */
 int gqe_version(void);
+
+/*
+ * Decode step (one new token per sequence against its K/V cache). The K/V
+ * cache stays dense and unchanged ("the Key-Value projections and the KV
+ * cache stay dense and unchanged": gist.science "Technical Summary", Dense KV
+ * path); the new token's output is the prefill definition (steps a1-a11) at
+ * its position: the router picks k experts per group for it, only those
+ * experts' queries and the shared head attend to the cache and the token's
+ * own key, then the (kG+2) slots and W_O.
+ *   cfg->B   sequences, one new token each;
+ *   cfg->T   keys after the step: the new token is at position T - 1 and
+ *            the cache holds positions 0 .. T-2 on entry (T >= 1);
+ *   x        [B, d_model] the new tokens;
+ *   K_cache, V_cache [B, G, cache_capacity, d_head], cache_capacity >= T;
+ *            the call writes the new token's K and V at position T - 1;
+ *   y        [B, d_model].
+ * Scratch: >= gqe_workspace_bytes(cfg, GQE_WS_DECODE) (0 when unsupported:
+ * more than 16 query heads per group). Weights as in gqe_layer_fwd.
+ */
+gqe_status gqe_decode_step(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
+                           const float* b_r, const gqe_bf16* W_q, const gqe_bf16* W_qs,
+                           const gqe_bf16* W_k, const gqe_bf16* W_v, const gqe_bf16* W_o,
+                           gqe_bf16* K_cache, gqe_bf16* V_cache, int32_t cache_capacity, gqe_bf16* y,
+                           void* ws, size_t ws_bytes, gqe_stream_t stream);
+
+/* Dense-GQA decode step: every one of the N heads (head h on group h / M)
+ * against the same cache; W_o_dense [N*d_head, d_model]. cfg->k is ignored.
+ * Scratch: gqe_workspace_bytes(cfg, GQE_WS_DENSE_DECODE). */
+gqe_status gqa_dense_decode_step(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16* W_q,
+                                 const gqe_bf16* W_k, const gqe_bf16* W_v,
+                                 const gqe_bf16* W_o_dense, gqe_bf16* K_cache, gqe_bf16* V_cache,
+                                 int32_t cache_capacity, gqe_bf16* y, void* ws, size_t ws_bytes,
+                                 gqe_stream_t stream);
 
 #ifdef __cplusplus
 }

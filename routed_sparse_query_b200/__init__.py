@@ -25,6 +25,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 GQE_OK, GQE_ERR_INVALID, GQE_ERR_UNSUPPORTED, GQE_ERR_WORKSPACE = 0, 1, 2, 3
 GQE_ERR_CUDA, GQE_ERR_TIMEOUT, GQE_ERR_DEVICE_CHECK = 4, 5, 6
 GQE_WS_DISPATCH, GQE_WS_LAYER, GQE_WS_DENSE, GQE_WS_ATTENTION = 1, 2, 3, 4
+GQE_WS_DECODE, GQE_WS_DENSE_DECODE = 5, 6
 GQE_FLAG_WS_CLEAN, GQE_FLAG_EXPERT_MAJOR = 1, 2
 ITEMS = {"idx": 1, "r": 2, "omega": 3, "counts": 4, "offsets": 5, "tok": 6, "slot_pos": 7,
          "Qv": 8, "Qs": 9, "K": 10, "V": 11, "slots": 12, "dispatch_ws": 13, "attention_ws": 14,
@@ -33,7 +34,8 @@ ITEMS = {"idx": 1, "r": 2, "omega": 3, "counts": 4, "offsets": 5, "tok": 6, "slo
 EXPORTED = ("gqe_workspace_bytes", "gqe_workspace_offset", "gqe_router_topk", "gqe_dispatch",
             "gqe_kv_proj", "gqe_attention_fwd", "gqe_output_proj", "gqe_layer_fwd",
             "gqa_dense_fwd", "gqe_read_status", "gqe_selftest_wait_timeout",
-            "gqe_status_string", "gqe_version", "gqe_dispatch_noalloc", "gqe_attention_fwd_compact")
+            "gqe_status_string", "gqe_version", "gqe_dispatch_noalloc", "gqe_attention_fwd_compact",
+            "gqe_decode_step", "gqa_dense_decode_step")
 
 
 class GQEConfig(ctypes.Structure):
@@ -69,6 +71,10 @@ _sig = {
     "gqe_layer_fwd": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                      ctypes.c_size_t, _P]),
     "gqa_dense_fwd": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "gqe_decode_step": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int32,
+                                       _P, _P, ctypes.c_size_t, _P]),
+    "gqa_dense_decode_step": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P,
+                                             _P, ctypes.c_size_t, _P]),
     "gqe_read_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32)]),
     "gqe_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
     "gqe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -169,6 +175,24 @@ def gqa_dense_fwd(cfg, x, W_q, W_k, W_v, W_o_dense, y, ws, stream=None):
     _check(_lib.gqa_dense_fwd(_cfg(cfg), _ptr(x), _ptr(W_q), _ptr(W_k), _ptr(W_v),
                               _ptr(W_o_dense), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
                               _stream(stream)), "gqa_dense_fwd")
+
+
+def gqe_decode_step(cfg, x, W_r, b_r, W_q, W_qs, W_k, W_v, W_o, K_cache, V_cache, y, ws,
+                    stream=None):
+    """cfg.T = keys after the step (the new token at T - 1); the cache capacity
+    is K_cache.shape[2]."""
+    _check(_lib.gqe_decode_step(_cfg(cfg), _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(W_q), _ptr(W_qs),
+                                _ptr(W_k), _ptr(W_v), _ptr(W_o), _ptr(K_cache), _ptr(V_cache),
+                                int(K_cache.shape[2]), _ptr(y), _ptr(ws),
+                                ws.numel() * ws.element_size(), _stream(stream)), "gqe_decode_step")
+
+
+def gqa_dense_decode_step(cfg, x, W_q, W_k, W_v, W_o_dense, K_cache, V_cache, y, ws, stream=None):
+    _check(_lib.gqa_dense_decode_step(_cfg(cfg), _ptr(x), _ptr(W_q), _ptr(W_k), _ptr(W_v),
+                                      _ptr(W_o_dense), _ptr(K_cache), _ptr(V_cache),
+                                      int(K_cache.shape[2]), _ptr(y), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)),
+           "gqa_dense_decode_step")
 
 
 def gqe_read_status() -> int:

@@ -75,6 +75,41 @@ LayerWs layer_ws(const gqe_config& c) {
   return L;
 }
 
+// Decode step: the layer's per-token buffers for B rows (one new token per
+// sequence; K/V go to the caller's cache), then the decode attention scratch.
+gqe_config decode_rows_cfg(const gqe_config& c) {
+  gqe_config c1 = c;
+  c1.T = 1;
+  return c1;
+}
+
+struct DecodeWs {
+  LayerWs L1;
+  size_t daws, total;
+};
+
+DecodeWs decode_ws(const gqe_config& c) {
+  DecodeWs D{};
+  D.L1 = layer_ws(decode_rows_cfg(c));
+  D.daws = round256(D.L1.total);
+  D.total = D.daws + decode_attention_ws_bytes(c, false);
+  return D;
+}
+
+struct DenseDecodeWs {
+  size_t Q, O, daws, total;
+};
+
+DenseDecodeWs dense_decode_ws(const gqe_config& c) {
+  const size_t N = static_cast<size_t>(c.G) * c.M;
+  DenseDecodeWs D{};
+  D.Q = 0;
+  D.O = round256(static_cast<size_t>(c.B) * N * c.d_head * 2);
+  D.daws = round256(D.O + static_cast<size_t>(c.B) * N * c.d_head * 2);
+  D.total = D.daws + decode_attention_ws_bytes(c, true);
+  return D;
+}
+
 struct DenseWs {
   size_t Q, K, V, O, aws, total;
 };
@@ -156,6 +191,8 @@ size_t gqe_workspace_bytes(const gqe_config* cfg, int which) {
     case GQE_WS_DISPATCH: return dispatch_ws_layout(*cfg).total;
     case GQE_WS_LAYER: return layer_ws(*cfg).total;
     case GQE_WS_DENSE: return dense_ws(*cfg).total;
+    case GQE_WS_DECODE: return decode_heads(*cfg, false) > 16 ? 0 : decode_ws(*cfg).total;
+    case GQE_WS_DENSE_DECODE: return decode_heads(*cfg, true) > 16 ? 0 : dense_decode_ws(*cfg).total;
     case GQE_WS_ATTENTION: {
       const size_t t = attention_plan(*cfg, cfg->G * cfg->k + 1).total;
       return t > 256 ? t : 256;
@@ -388,3 +425,67 @@ const char* gqe_status_string(gqe_status s) {
 int gqe_version(void) { return 100; }
 
 }  // extern "C"
+
+gqe_status gqe_decode_step(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
+                           const float* b_r, const gqe_bf16* W_q, const gqe_bf16* W_qs,
+                           const gqe_bf16* W_k, const gqe_bf16* W_v, const gqe_bf16* W_o,
+                           gqe_bf16* K_cache, gqe_bf16* V_cache, int32_t cache_capacity, gqe_bf16* y,
+                           void* ws, size_t ws_bytes, gqe_stream_t stream) {
+  const gqe_status s = check_cfg(cfg);
+  if (s != GQE_OK) return s;
+  if (cache_capacity < cfg->T) return GQE_ERR_INVALID;
+  if (!all_aligned(x, W_r, W_q, W_qs, W_k, W_v, W_o, K_cache, V_cache, y) || ws == nullptr ||
+      !aligned16(ws))
+    return GQE_ERR_INVALID;
+  if (b_r != nullptr && (reinterpret_cast<uintptr_t>(b_r) & 3u)) return GQE_ERR_INVALID;
+  if (decode_heads(*cfg, false) > 16) return GQE_ERR_UNSUPPORTED;
+  const DecodeWs D = decode_ws(*cfg);
+  if (ws_bytes < D.total) return GQE_ERR_WORKSPACE;
+  const gqe_config c1 = decode_rows_cfg(*cfg);
+  const LayerWs& L = D.L1;
+  char* w = static_cast<char*>(ws);
+  auto I = [&](size_t o) { return reinterpret_cast<int32_t*>(w + o); };
+  auto F = [&](size_t o) { return reinterpret_cast<float*>(w + o); };
+  auto H = [&](size_t o) { return reinterpret_cast<gqe_bf16*>(w + o); };
+  gqe_status st = gqe_router_topk(&c1, x, W_r, b_r, I(L.idx), F(L.r), F(L.omega), stream);
+  if (st != GQE_OK) return st;
+  st = gqe_dispatch(&c1, I(L.idx), x, W_q, W_qs, I(L.counts), I(L.offsets), I(L.tok),
+                    I(L.slot_pos), H(L.Qv), H(L.Qs), w + L.dws, L.aws - L.dws, stream);
+  if (st != GQE_OK) return st;
+  if (gemm_kv_at(c1, x, W_k, W_v, K_cache, V_cache, cache_capacity, cfg->T - 1, stream) != cudaSuccess)
+    return GQE_ERR_CUDA;
+  if (decode_attention(*cfg, false, H(L.Qv), H(L.Qs), K_cache, V_cache, cache_capacity, H(L.slots),
+                       (cfg->G * cfg->k + 2) * cfg->d_head, w + D.daws, stream) != cudaSuccess)
+    return GQE_ERR_CUDA;
+  return gqe_output_proj(&c1, H(L.slots), F(L.omega), W_o, y, stream);
+}
+
+gqe_status gqa_dense_decode_step(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16* W_q,
+                                 const gqe_bf16* W_k, const gqe_bf16* W_v,
+                                 const gqe_bf16* W_o_dense, gqe_bf16* K_cache, gqe_bf16* V_cache,
+                                 int32_t cache_capacity, gqe_bf16* y, void* ws, size_t ws_bytes,
+                                 gqe_stream_t stream) {
+  if (cfg == nullptr) return GQE_ERR_INVALID;
+  gqe_config c = *cfg;
+  c.k = 1;  // not used by the dense layer
+  const gqe_status s = check_cfg(&c);
+  if (s != GQE_OK) return s;
+  if (cache_capacity < c.T) return GQE_ERR_INVALID;
+  if (!all_aligned(x, W_q, W_k, W_v, W_o_dense, K_cache, V_cache, y) || ws == nullptr ||
+      !aligned16(ws))
+    return GQE_ERR_INVALID;
+  if (decode_heads(c, true) > 16) return GQE_ERR_UNSUPPORTED;
+  const DenseDecodeWs D = dense_decode_ws(c);
+  if (ws_bytes < D.total) return GQE_ERR_WORKSPACE;
+  const gqe_config c1 = decode_rows_cfg(c);
+  char* w = static_cast<char*>(ws);
+  auto H = [&](size_t o) { return reinterpret_cast<gqe_bf16*>(w + o); };
+  const int N = c.G * c.M;
+  int e = gemm_q_dense(c1, x, W_q, H(D.Q), stream);
+  if (e == cudaSuccess) e = gemm_kv_at(c1, x, W_k, W_v, K_cache, V_cache, cache_capacity, c.T - 1, stream);
+  if (e == cudaSuccess)
+    e = decode_attention(c, true, H(D.Q), nullptr, K_cache, V_cache, cache_capacity, H(D.O),
+                         N * c.d_head, w + D.daws, stream);
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+  return cuda_status(gemm_rowmajor(H(D.O), c.B, N * c.d_head, W_o_dense, c.d_model, y, stream));
+}

@@ -424,6 +424,25 @@ int gemm_kv(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const u
   return dense_gemm(x, R, c.d_model, W_k, W_v, c.G * c.d_head, ek, ev, 2, stream);
 }
 
+int gemm_kv_at(const gqe_config& c1, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
+               uint16_t* Kc, uint16_t* Vc, int cap, int pos, void* stream) {
+  // Row b (one token of sequence b) -> cache[b][g][pos][:].
+  const int B = c1.B;
+  auto at = [&](uint16_t* cache) {
+    Epi e;
+    e.out = cache + static_cast<size_t>(pos) * c1.d_head;
+    e.T = 1;
+    e.hd = c1.d_head;
+    e.sb = static_cast<long long>(c1.G) * cap * c1.d_head;
+    e.sh = static_cast<long long>(cap) * c1.d_head;
+    e.st = c1.d_head;
+    e.rows = B;
+    e.cols = c1.G * c1.d_head;
+    return e;
+  };
+  return dense_gemm(x, B, c1.d_model, W_k, W_v, c1.G * c1.d_head, at(Kc), at(Vc), 2, stream);
+}
+
 int gemm_q_dense(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, uint16_t* Q,
                  void* stream) {
   const int R = c.B * c.T;

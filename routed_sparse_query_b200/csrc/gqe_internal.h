@@ -129,4 +129,18 @@ int attention_dense(const gqe_config& c, const uint16_t* Q, const uint16_t* K, c
                     uint16_t* O, void* ws, size_t ws_bytes, bool counters_zeroed, void* stream);
 int zero_attention_counters(const gqe_config& c, int H, void* ws, void* stream);
 
+// Decode step. cfg.T = keys after the step (the new token sits at T - 1),
+// cap = cache capacity per (sequence, group). K/V projection of the new
+// tokens (rows B, one per sequence) written into the cache at position pos.
+int gemm_kv_at(const gqe_config& c1, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
+               uint16_t* Kc, uint16_t* Vc, int cap, int pos, void* stream);
+// Heads per group of the decode attention: k + 1 (GQE, the shared head in
+// group 0) or M (dense).
+int decode_heads(const gqe_config& c, bool dense);
+size_t decode_attention_ws_bytes(const gqe_config& c, bool dense);
+// Q: GQE routed queries [B][G][k][dh] (Qs [B][dh]) or dense [B][G*M][dh].
+int decode_attention(const gqe_config& c, bool dense, const uint16_t* Q, const uint16_t* Qs,
+                     const uint16_t* Kc, const uint16_t* Vc, int cap, uint16_t* out, int ldo,
+                     void* ws, void* stream);
+
 }  // namespace gqe

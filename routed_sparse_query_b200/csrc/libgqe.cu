@@ -4,5 +4,6 @@
 #include "dispatch.cu"
 #include "gemm.cu"
 #include "attention.cu"
+#include "decode.cu"
 #include "api.cu"
 #include "noalloc.cu"
