@@ -196,6 +196,23 @@ class Layer:
     def attention(self):
         self.rsq.gqe_attention_fwd(self.cfg_clean, self.Qv, self.Qs, self.K, self.V, self.slots, self.wsa)
 
+    def attention_expert_major_fn(self):
+        """The same attention over compacted expert-major tiles (the routed
+        queries rewritten in token-list order once, outside any timing)."""
+        import torch
+        rsq, s, d = self.rsq, self.s, self.d
+        cfg = rsq.GQEConfig.of(s, rsq.GQE_FLAG_EXPERT_MAJOR)
+        Qe = torch.empty(s.k * s.G * s.R, s.d_head, dtype=torch.bfloat16, device="cuda")
+        Qs = torch.empty_like(self.Qs)
+        rsq.gqe_dispatch(cfg, self.idx, d["x"], d["W_q"], d["W_qs"], self.counts, self.offsets,
+                         self.tok, self.slot_pos, Qe, Qs, self.wsd)
+        slots = torch.zeros_like(self.slots)
+
+        def f():
+            rsq.gqe_attention_fwd_compact(cfg, Qe, Qs, self.K, self.V, self.idx, self.offsets,
+                                          self.tok, slots)
+        return f
+
     def output(self):
         self.rsq.gqe_output_proj(self.cfg, self.slots, self.omega, self.d["W_o"], self.y)
 
@@ -468,9 +485,55 @@ def run_ours(args, rank: int, world: int, dist):
     }
     if world == 1 and not args.no_sweep:
         out["sweep"] = sweep(rsq, pk, args)
+        out["decode"] = decode_bench(rsq, pk, args.steps)
     if world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(shape, min_seconds=10.0)
     return out
+
+
+DECODE = {"batch": 64, "cache": 32768}  # decode measurement: 64 sequences, 32k cached tokens
+
+
+def decode_bench(rsq, pk, steps: int) -> dict:
+    """One decode step (a new token per sequence against a 32k-token K/V cache)
+    through gqe_decode_step and gqa_dense_decode_step, CUDA-event timed. The
+    cache and weights are drawn on the device with the synth distributions
+    (K, V ~ N(0, 1) like x W with x ~ N(0, 1), W ~ N(0, 1/d))."""
+    import torch
+    B, T = DECODE["batch"], DECODE["cache"] + 1
+    s = synth.LayerShape(B, T, 1024, 8, 2, 1, 64)
+    g = torch.Generator(device="cuda").manual_seed(4321)
+    d = device_inputs_seeded(synth.LayerShape(B, 1, s.d_model, s.G, s.M, s.k, s.d_head), 4321)
+    cap = T
+    Kc = torch.randn(B, s.G, cap, s.d_head, device="cuda", generator=g).to(torch.bfloat16)
+    Vc = torch.randn(B, s.G, cap, s.d_head, device="cuda", generator=g).to(torch.bfloat16)
+    cfg = rsq.GQEConfig.of(s)
+    ws = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_DECODE), dtype=torch.uint8, device="cuda")
+    wsd = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_DENSE_DECODE), dtype=torch.uint8,
+                      device="cuda")
+    y = torch.empty(B, s.d_model, dtype=torch.bfloat16, device="cuda")
+
+    def f():
+        rsq.gqe_decode_step(cfg, d["x"], d["W_r"], d["b_r"], d["W_q"], d["W_qs"], d["W_k"], d["W_v"],
+                            d["W_o"], Kc, Vc, y, ws)
+
+    def fd():
+        rsq.gqa_dense_decode_step(cfg, d["x"], d["W_q"], d["W_k"], d["W_v"], d["W_o_dense"], Kc, Vc,
+                                  y, wsd)
+
+    n = max(3, min(steps, 50))
+    ms = _time_calls(f, n, 3, None) / n
+    dms = _time_calls(fd, n, 3, None) / n
+    if rsq.gqe_read_status() != 0:
+        raise RuntimeError("device-side status set in the decode measurement")
+    kv_bytes = 2 * B * s.G * T * s.d_head * 2  # the cache is read once per step
+    return {"workload": f"decode: {B} sequences, {T - 1} cached tokens each, one new token "
+                        f"(d_model=1024, G=8, M=2, k=1, d_head=64)",
+            "steps": n, "gqe_ms": ms, "gqe_tokens_per_s": B / (ms / 1e3),
+            "dense_ms": dms, "dense_tokens_per_s": B / (dms / 1e3), "speedup": dms / ms,
+            "kv_cache_bytes": kv_bytes, "kv_gbs": kv_bytes / (ms / 1e3) / 1e9,
+            "kv_frac_of_hbm_peak": kv_bytes / (ms / 1e3) / 1e9 / pk["hbm"],
+            "l2": "cache (4.3 GB) larger than L2, not flushed"}
 
 
 def sweep(rsq, pk, args):
@@ -489,11 +552,14 @@ def sweep(rsq, pk, args):
         gq_ms = time_layer(rsq, s, d, steps, 1, None) / steps
         attn_s = res["per_call_ms"]["attention"] / steps / 1e3
         ach = flops(s)["attention"] / attn_s / 1e12
+        em_s = _time_calls(layer.attention_expert_major_fn(), steps, 1, None) / steps / 1e3
         rows.append({"workload": f"{name}: {describe(s)}", "T": s.T, "B": s.B, "steps": steps,
                      "gqe_ms": gq_ms, "gqe_tokens_per_s": s.R / (gq_ms / 1e3),
                      "dense_ms": dense_ms, "dense_tokens_per_s": s.R / (dense_ms / 1e3),
                      "speedup": dense_ms / gq_ms, "attn_tflops": ach,
                      "attn_frac_of_bf16_peak": ach / pk["bf16"],
+                     "attn_expert_major_ms": em_s * 1e3,
+                     "attn_expert_major_frac_of_bf16_peak": flops(s)["attention"] / em_s / 1e12 / pk["bf16"],
                      "l2": "inputs larger than L2, not flushed",
                      "breakdown_ms": {c: v / steps for c, v in res["per_call_ms"].items()}})
         if rsq.gqe_read_status() != 0:

@@ -294,7 +294,9 @@ int gqe_version(void);
  *            the call writes the new token's K and V at position T - 1;
  *   y        [B, d_model].
  * Scratch: >= gqe_workspace_bytes(cfg, GQE_WS_DECODE) (0 when unsupported:
- * more than 16 query heads per group). Weights as in gqe_layer_fwd.
+ * more than 16 query heads per group). GQE_ERR_UNSUPPORTED also for B >
+ * 65535. The extent limits of the other calls apply to the B new rows, not
+ * to the cache length. Weights as in gqe_layer_fwd.
  */
 gqe_status gqe_decode_step(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
                            const float* b_r, const gqe_bf16* W_q, const gqe_bf16* W_qs,

@@ -186,13 +186,21 @@ using namespace gqe;
 extern "C" {
 
 size_t gqe_workspace_bytes(const gqe_config* cfg, int which) {
+  if (cfg != nullptr && (which == GQE_WS_DECODE || which == GQE_WS_DENSE_DECODE)) {
+    // Decode: the per-token buffers have B rows; T is the cache length.
+    gqe_config c1 = decode_rows_cfg(*cfg);
+    if (which == GQE_WS_DENSE_DECODE) c1.k = 1;
+    if (cfg->T < 1 || check_cfg(&c1) != GQE_OK) return 0;
+    if (which == GQE_WS_DECODE) return decode_heads(*cfg, false) > 16 ? 0 : decode_ws(*cfg).total;
+    gqe_config cd = *cfg;
+    cd.k = 1;
+    return decode_heads(cd, true) > 16 ? 0 : dense_decode_ws(cd).total;
+  }
   if (check_cfg(cfg) != GQE_OK) return 0;
   switch (which) {
     case GQE_WS_DISPATCH: return dispatch_ws_layout(*cfg).total;
     case GQE_WS_LAYER: return layer_ws(*cfg).total;
     case GQE_WS_DENSE: return dense_ws(*cfg).total;
-    case GQE_WS_DECODE: return decode_heads(*cfg, false) > 16 ? 0 : decode_ws(*cfg).total;
-    case GQE_WS_DENSE_DECODE: return decode_heads(*cfg, true) > 16 ? 0 : dense_decode_ws(*cfg).total;
     case GQE_WS_ATTENTION: {
       const size_t t = attention_plan(*cfg, cfg->G * cfg->k + 1).total;
       return t > 256 ? t : 256;
@@ -431,17 +439,18 @@ gqe_status gqe_decode_step(const gqe_config* cfg, const gqe_bf16* x, const float
                            const gqe_bf16* W_k, const gqe_bf16* W_v, const gqe_bf16* W_o,
                            gqe_bf16* K_cache, gqe_bf16* V_cache, int32_t cache_capacity, gqe_bf16* y,
                            void* ws, size_t ws_bytes, gqe_stream_t stream) {
-  const gqe_status s = check_cfg(cfg);
+  if (cfg == nullptr || cfg->T < 1) return GQE_ERR_INVALID;
+  const gqe_config c1 = decode_rows_cfg(*cfg);
+  const gqe_status s = check_cfg(&c1);  // B rows; the long extent is the cache
   if (s != GQE_OK) return s;
   if (cache_capacity < cfg->T) return GQE_ERR_INVALID;
   if (!all_aligned(x, W_r, W_q, W_qs, W_k, W_v, W_o, K_cache, V_cache, y) || ws == nullptr ||
       !aligned16(ws))
     return GQE_ERR_INVALID;
   if (b_r != nullptr && (reinterpret_cast<uintptr_t>(b_r) & 3u)) return GQE_ERR_INVALID;
-  if (decode_heads(*cfg, false) > 16) return GQE_ERR_UNSUPPORTED;
+  if (decode_heads(*cfg, false) > 16 || cfg->B > 65535) return GQE_ERR_UNSUPPORTED;
   const DecodeWs D = decode_ws(*cfg);
   if (ws_bytes < D.total) return GQE_ERR_WORKSPACE;
-  const gqe_config c1 = decode_rows_cfg(*cfg);
   const LayerWs& L = D.L1;
   char* w = static_cast<char*>(ws);
   auto I = [&](size_t o) { return reinterpret_cast<int32_t*>(w + o); };
@@ -468,16 +477,17 @@ gqe_status gqa_dense_decode_step(const gqe_config* cfg, const gqe_bf16* x, const
   if (cfg == nullptr) return GQE_ERR_INVALID;
   gqe_config c = *cfg;
   c.k = 1;  // not used by the dense layer
-  const gqe_status s = check_cfg(&c);
+  if (c.T < 1) return GQE_ERR_INVALID;
+  const gqe_config c1 = decode_rows_cfg(c);
+  const gqe_status s = check_cfg(&c1);  // B rows; the long extent is the cache
   if (s != GQE_OK) return s;
   if (cache_capacity < c.T) return GQE_ERR_INVALID;
   if (!all_aligned(x, W_q, W_k, W_v, W_o_dense, K_cache, V_cache, y) || ws == nullptr ||
       !aligned16(ws))
     return GQE_ERR_INVALID;
-  if (decode_heads(c, true) > 16) return GQE_ERR_UNSUPPORTED;
+  if (decode_heads(c, true) > 16 || c.B > 65535) return GQE_ERR_UNSUPPORTED;
   const DenseDecodeWs D = dense_decode_ws(c);
   if (ws_bytes < D.total) return GQE_ERR_WORKSPACE;
-  const gqe_config c1 = decode_rows_cfg(c);
   char* w = static_cast<char*>(ws);
   auto H = [&](size_t o) { return reinterpret_cast<gqe_bf16*>(w + o); };
   const int N = c.G * c.M;

@@ -65,17 +65,27 @@ __device__ __forceinline__ int column_of(const DecodeArgs& a, int g, int h) {
 
 __device__ __forceinline__ float bf16f(uint16_t v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
 
+// O phase: thread t takes 16-byte column chunk t % (DH/8) of the rows of row
+// group t / (DH/8) (8 rows of a KV tile per pass for DH = 64).
+template <int DH>
+struct OShape {
+  static constexpr int CPR = DH / 8;            // 16-byte chunks per row
+  static constexpr int NG = kThreads / CPR;     // row groups (32 for DH = 64)
+  static constexpr int PASSES = kCh / NG;       // rows per thread
+};
+
 // Dynamic shared memory: q [H][DH], scores / probabilities [H][kCh], warp
-// partials [kWarps][H] (max, then sum), O partials [key groups][H][DH].
+// partials [kWarps][H] (max, then sum), O partials [row groups][H][DH].
 template <int DH>
 size_t partial_smem(int H) {
-  constexpr int NG = kThreads / (DH / 2);
-  return static_cast<size_t>(H) * (DH + kCh + 2 * kWarps + NG * DH) * 4 + 2 * H * 4;
+  return static_cast<size_t>(H) * (DH + kCh + 2 * kWarps + OShape<DH>::NG * DH) * 4 + 2 * H * 4;
 }
 
-template <int DH>
+// HM: a bound on the heads per group (2, 4, 8 or 16) sizing the registers.
+template <int DH, int HM>
 __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) {
-  constexpr int NG = kThreads / (DH / 2);  // key groups in the O phase
+  using OS = OShape<DH>;
+  constexpr int NG = OS::NG;
   pdl_wait();
   pdl_launch_dependents();
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -118,9 +128,10 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
     for (int h = 0; h < H; ++h) {
       float s = -INFINITY;
       if (valid) {
-        s = 0.0f;
+        float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int d = 0; d < DH; ++d) s = fmaf(qsm[h * DH + d], kr[d], s);
+        for (int d = 0; d < DH; ++d) s4[d & 3] = fmaf(qsm[h * DH + d], kr[d], s4[d & 3]);
+        s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       }
       sc[h * kCh + tid] = s;
       float m = s;
@@ -148,29 +159,47 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
     lh[tid] = s;
   }
 
-  // O: thread t takes dims 2*(t % (DH/2)) and +1 over keys kg, kg + NG, ...
-  const int dp = tid % (DH / 2), kg = tid / (DH / 2);
-  float acc[2 * 16];
-#pragma unroll
-  for (int i = 0; i < 2 * 16; ++i) acc[i] = 0.0f;
+  // O: thread t takes columns 8*cc .. 8*cc+7 (cc = t % CPR) of rows rg,
+  // rg + NG, ... (rg = t / CPR): 16-byte loads, all rows of a thread in flight.
+  const int cc = tid % OS::CPR, rg = tid / OS::CPR;
   const int n_keys = min(kCh, a.T - c * kCh);
-  for (int ul = kg; ul < n_keys; ul += NG) {
-    const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(a.Vc + (kv0 + c * kCh + ul) * DH) + dp);
-    const float v0 = __uint_as_float(v << 16), v1 = __uint_as_float(v & 0xffff0000u);
+  uint4 vr[OS::PASSES];
 #pragma unroll
-    for (int h = 0; h < 16; ++h) {
+  for (int q = 0; q < OS::PASSES; ++q) {
+    const int ul = rg + q * NG;
+    vr[q] = ul < n_keys ? __ldg(reinterpret_cast<const uint4*>(a.Vc + (kv0 + c * kCh + ul) * DH) + cc)
+                        : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float acc[HM][8];
+#pragma unroll
+  for (int h = 0; h < HM; ++h)
+#pragma unroll
+    for (int x = 0; x < 8; ++x) acc[h][x] = 0.0f;
+#pragma unroll
+  for (int q = 0; q < OS::PASSES; ++q) {
+    const int ul = rg + q * NG;
+    const uint32_t w[4] = {vr[q].x, vr[q].y, vr[q].z, vr[q].w};
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+#pragma unroll
+    for (int h = 0; h < HM; ++h) {
       if (h < H) {
-        const float p = sc[h * kCh + ul];
-        acc[2 * h] = fmaf(p, v0, acc[2 * h]);
-        acc[2 * h + 1] = fmaf(p, v1, acc[2 * h + 1]);
+        const float p = ul < n_keys ? sc[h * kCh + ul] : 0.0f;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc[h][x] = fmaf(p, v[x], acc[h][x]);
       }
     }
   }
 #pragma unroll
-  for (int h = 0; h < 16; ++h) {
+  for (int h = 0; h < HM; ++h) {
     if (h < H) {
-      ored[(kg * a.H + h) * DH + 2 * dp] = acc[2 * h];
-      ored[(kg * a.H + h) * DH + 2 * dp + 1] = acc[2 * h + 1];
+      float4* dst = reinterpret_cast<float4*>(ored + (rg * a.H + h) * DH + 8 * cc);
+      dst[0] = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+      dst[1] = make_float4(acc[h][4], acc[h][5], acc[h][6], acc[h][7]);
     }
   }
   __syncthreads();
@@ -195,8 +224,10 @@ __global__ void __launch_bounds__(1024) decode_merge_kernel(DecodeArgs a) {
   if (h >= H) return;
   const size_t blk0 = (static_cast<size_t>(b) * a.G + g) * a.n_ch;
   float m = -INFINITY;
+#pragma unroll 8
   for (int c = 0; c < a.n_ch; ++c) m = fmaxf(m, a.part_ml[(blk0 + c) * a.H + h].x);
   float o = 0.0f, l = 0.0f;
+#pragma unroll 8
   for (int c = 0; c < a.n_ch; ++c) {
     const float2 ml = a.part_ml[(blk0 + c) * a.H + h];
     const float w = exp2f(ml.x - m);
@@ -208,12 +239,21 @@ __global__ void __launch_bounds__(1024) decode_merge_kernel(DecodeArgs a) {
       *reinterpret_cast<const uint16_t*>(&r);
 }
 
+template <int DH, int HM>
+int launch_partial(const DecodeArgs& a, void* stream) {
+  const size_t smem = partial_smem<DH>(a.H);
+  const int e = ensure_smem<decode_partial_kernel<DH, HM>>(static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(decode_partial_kernel<DH, HM>, dim3(a.n_ch, a.G, a.B), dim3(kThreads), smem,
+                    stream, a);
+}
+
 template <int DH>
 int launch(const DecodeArgs& a, void* stream) {
-  const size_t smem = partial_smem<DH>(a.H);
-  int e = ensure_smem<decode_partial_kernel<DH>>(static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  e = launch_pdl(decode_partial_kernel<DH>, dim3(a.n_ch, a.G, a.B), dim3(kThreads), smem, stream, a);
+  const int e = a.H <= 2   ? launch_partial<DH, 2>(a, stream)
+                : a.H <= 4 ? launch_partial<DH, 4>(a, stream)
+                : a.H <= 8 ? launch_partial<DH, 8>(a, stream)
+                           : launch_partial<DH, 16>(a, stream);
   if (e != cudaSuccess) return e;
   return launch_pdl(decode_merge_kernel<DH>, dim3(a.G, a.B), dim3(a.H * DH), 0, stream, a);
 }
