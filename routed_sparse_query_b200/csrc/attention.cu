@@ -380,8 +380,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       h = p.G * p.k;
       bh = b * p.H + h;
     } else {
-      bh = static_cast<int>(blockIdx.x) % BH;
-      ord = static_cast<int>(blockIdx.x) / BH;
+      if (p.chunk >= p.n_qt && p.n_pairs >= 1024) {
+        // Long sequences: stream-major, so that the CTAs in flight share one
+        // group's K/V in L2 (longest pairs first inside each stream).
+        bh = static_cast<int>(blockIdx.x) / p.items;
+        ord = static_cast<int>(blockIdx.x) % p.items;
+      } else {
+        // Longest pairs of every stream first (balanced tail).
+        bh = static_cast<int>(blockIdx.x) % BH;
+        ord = static_cast<int>(blockIdx.x) / BH;
+      }
       b = bh / p.H;
       h = bh % p.H;
     }
