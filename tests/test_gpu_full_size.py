@@ -68,3 +68,28 @@ def test_full_size_sampled_rows(rsq, name):
     # The fused entry point gives the same y.
     y, _ = run_layer(rsq, shape, device_inputs(inp))
     assert torch.equal(y, o["y"]), "gqe_layer_fwd differs from the step calls"
+
+
+def test_long_sequence_layouts_agree_bitwise(rsq):
+    # 256k tokens: the slot-major attention runs its stream-major CTA order
+    # (1024 tile pairs per stream) and no split-KV; the expert-major layout
+    # computes every row with the same online softmax over the same K/V
+    # tiles, so the slots must agree bitwise (and the lists stay valid).
+    from gpu_common import run_expert_major, run_steps
+    shape = synth.LayerShape(B=1, T=262144, d_model=1024, G=8, M=2, k=1, d_head=64)
+    g = torch.Generator(device="cuda").manual_seed(262144)
+    sd = shape.d_model ** -0.5
+    d = {"x": torch.randn(shape.R, shape.d_model, device="cuda", generator=g).to(torch.bfloat16),
+         "W_r": torch.randn(shape.d_model, shape.N, device="cuda", generator=g) * sd, "b_r": None}
+    for nm, shp in (("W_q", (shape.d_model, shape.N * shape.d_head)), ("W_qs", (shape.d_model, shape.d_head)),
+                    ("W_k", (shape.d_model, shape.G * shape.d_head)),
+                    ("W_v", (shape.d_model, shape.G * shape.d_head)),
+                    ("W_o", (shape.n_slots * shape.d_head, shape.d_model))):
+        d[nm] = (torch.randn(*shp, device="cuda", generator=g) * sd).to(torch.bfloat16)
+    o = run_steps(rsq, shape, d)
+    counts = o["counts"].view(shape.N, shape.B)
+    assert int(counts.sum()) == shape.k * shape.G * shape.R
+    e = run_expert_major(rsq, shape, d, o)
+    n = (shape.k * shape.G + 1) * shape.d_head
+    assert torch.equal(e["slots"][:, :n], o["slots"][:, :n]), "layouts differ at 256k"
+    assert torch.isfinite(o["y"].float()).all()
