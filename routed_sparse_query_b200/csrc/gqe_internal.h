@@ -5,6 +5,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <utility>
 
 #include "gqe.h"
@@ -46,9 +47,6 @@ DispatchWs dispatch_ws_layout(const gqe_config& c);
 
 size_t router_smem_bytes(const gqe_config& c);
 
-// Raises the dynamic shared-memory limit of kernel K to `bytes`, once per
-// device (the attribute is per device; re-setting it on every launch costs
-// host time on short layers).
 // Launches `kern` with programmatic dependent launch allowed (the kernel
 // overlaps the tail of the previous kernel on the stream; see pdl_wait).
 template <typename... KArgs, typename... Args>
@@ -67,14 +65,19 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// Raises the dynamic shared-memory limit of kernel K to `bytes`, once per
+// device (the attribute is per device; re-setting it on every launch costs
+// host time on short layers).
+// Safe to call from several host threads (the attribute may be set twice).
 template <auto K>
 inline int ensure_smem(int bytes) {
-  static int done[64] = {0};
+  static std::atomic<int> done[64];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) dev = 63;
-  if (dev >= 0 && dev < 64 && done[dev] >= bytes) return 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (done[dev].load(std::memory_order_relaxed) >= bytes) return 0;
   const cudaError_t e = cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = bytes;
+  if (e == cudaSuccess) done[dev].store(bytes, std::memory_order_relaxed);
   return e;
 }
 
