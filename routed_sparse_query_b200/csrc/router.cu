@@ -7,13 +7,17 @@
 // the group, pptc.cn blog section 7.)
 //
 // The logits are a small fp32 GEMM on the CUDA cores. A CTA takes a block of
-// TB tokens (TB * NP = 256 logits); W_r (zero padded to NP columns) and the
-// block's x rows sit in shared memory. Warp w of W (16, or 8 when d is not a
-// multiple of 128) sums rows [w d/W, (w+1) d/W) of the dot products; each
-// thread keeps 2 tokens x 4 experts, reading a W_r row once per 2 tokens
-// (broadcast over the warp's token lanes). The W warp partials are then added
-// in warp order, so every logit is one fixed sequence of roundings (the
-// result is deterministic). One thread per (token, group) pair then decides.
+// TB tokens (TB * NP = 128 * TPT logits); W_r (zero padded to NP columns) and
+// the block's x rows sit in shared memory. Warp w of W (16, or 8 when d is
+// not a multiple of 128) sums rows [w d/W, (w+1) d/W) of the dot products;
+// each thread keeps TPT tokens x 4 experts, so one 16-byte W_r read (one
+// shared-memory pass per quarter warp) feeds 4 TPT FMAs. Large batches take
+// the largest TPT of 8, 6, 4 whose block fits in shared memory (6 for
+// d = 1024 with 16 experts), small ones TPT = 2 so that the blocks spread
+// over the SMs. The W warp partials are then added in warp
+// order, so every logit is one fixed sequence of roundings (the result is
+// deterministic and the same for every TPT). The threads then take the
+// (token, group) pairs and decide.
 //
 // Exact selection: each fp32 logit carries the bound
 //   |z_fp32 - z| <= gamma_h * (||x||_1 * max_i |W_r[i,e]| + |b_e|),
@@ -27,6 +31,8 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "gqe_internal.h"
 #include "ptx.cuh"
 
@@ -35,11 +41,10 @@ namespace gqe {
 namespace router_impl {
 
 constexpr int kMaxRouterWarps = 16;
-constexpr int kTPT = 2;  // tokens per thread
 
 // Tokens per CTA block: lanes are (token lane tt, expert quad et) with NP/4
-// quads, so a warp covers 128/NP token lanes of kTPT tokens each.
-__host__ __device__ constexpr int router_tb(int NP) { return kTPT * 128 / NP; }
+// quads, so a warp covers 128/NP token lanes of TPT tokens each.
+__host__ __device__ constexpr int router_tb(int NP, int TPT) { return TPT * 128 / NP; }
 // Warps per CTA: warp w sums rows [w d/W, (w+1) d/W), a multiple of 8 rows.
 __host__ __device__ constexpr int router_warps(int d) { return d % 128 == 0 ? 16 : 8; }
 
@@ -59,18 +64,23 @@ struct RouterArgs {
   int R, d, G, M, k, N;
 };
 
-// Dynamic shared memory of one CTA (byte offsets).
+// Dynamic shared memory of one CTA (byte offsets). The warp partials
+// [warp][TB][NP] share their space with the block's x rows: they are written
+// once every warp has finished reading x, and the next block's rows are
+// fetched once the partials have been summed.
 struct RouterLayout {
-  size_t w, xs, part, zd, zf, ez, wmax, bsm, nx, ps, dn, list, total;
+  size_t w, xs, zd, sel, zf, ez, wmax, bsm, nx, ps, dn, list, total;
 };
-__host__ __device__ inline RouterLayout router_layout(int d, int NP) {
-  const int TB = router_tb(NP), W = router_warps(d);
+__host__ __device__ inline RouterLayout router_layout(int d, int NP, int TPT) {
+  const int TB = router_tb(NP, TPT), W = router_warps(d);
+  const size_t xbytes = static_cast<size_t>(TB) * (d + 8) * 2;  // x [TB][d + 8]
+  const size_t pbytes = static_cast<size_t>(W) * TB * NP * 4;   // partials [warp][TB][NP]
   RouterLayout L;
   size_t o = 0;
   L.w = o;     o += static_cast<size_t>(d) * NP * 4;                  // W_r [d][NP]
-  L.xs = o;    o += static_cast<size_t>(TB) * (d + 8) * 2;            // x [TB][d + 8]
-  L.part = o;  o += static_cast<size_t>(W) * TB * NP * 4;             // [warp][TB][NP]
+  L.xs = o;    o += ((xbytes > pbytes ? xbytes : pbytes) + 15) & ~static_cast<size_t>(15);
   L.zd = o;    o += static_cast<size_t>(TB) * NP * 8;                 // fp64 logits
+  L.sel = o;   o += static_cast<size_t>(TB) * NP * 8;                 // selection mask per pair
   L.zf = o;    o += static_cast<size_t>(TB) * NP * 4;                 // fp32 logits
   L.ez = o;    o += static_cast<size_t>(TB) * NP * 4;                 // exp(z - group max)
   L.wmax = o;  o += NP * 4;                                            // max_i |W_r[i, e]|
@@ -122,21 +132,21 @@ __device__ __forceinline__ float group_softmax(const V* zg, int M, uint64_t sel,
   return psel;
 }
 
-template <int NP, int WARPS>
+template <int NP, int WARPS, int TPT>
 __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
   constexpr int THREADS = WARPS * 32;
-  constexpr int TB = router_tb(NP);
+  constexpr int TB = router_tb(NP, TPT);
   constexpr int EG = NP / 4;   // expert quads
-  constexpr int TG = 32 / EG;  // token lanes per warp; TB == kTPT * TG
-  static_assert(TB == kTPT * TG, "block shape");
-  static_assert(TB * NP <= THREADS, "one (token, group) pair per thread");
+  constexpr int TG = 32 / EG;  // token lanes per warp; TB == TPT * TG
+  static_assert(TB == TPT * TG, "block shape");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int n_uncertain;
-  const RouterLayout L = router_layout(a.d, NP);
+  const RouterLayout L = router_layout(a.d, NP, TPT);
   float* Ws = reinterpret_cast<float*>(smem_raw + L.w);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw + L.xs);
-  float* part = reinterpret_cast<float*>(smem_raw + L.part);
+  float* part = reinterpret_cast<float*>(smem_raw + L.xs);  // shares the x rows' space
   double* zd = reinterpret_cast<double*>(smem_raw + L.zd);
+  uint64_t* selp = reinterpret_cast<uint64_t*>(smem_raw + L.sel);
   float* zf = reinterpret_cast<float*>(smem_raw + L.zf);
   float* ez = reinterpret_cast<float*>(smem_raw + L.ez);
   float* wmax = reinterpret_cast<float*>(smem_raw + L.wmax);
@@ -204,11 +214,14 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
       m3 = fmaxf(m3, fabsf(Ws[(row + 3 * parts) * NP + col]));
     }
     for (; row < a.d; row += parts) m0 = fmaxf(m0, fabsf(Ws[row * NP + col]));
-    part[tid] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+    // Scratch: the fp64 logit space (THREADS floats fit in it; the x space
+    // is receiving the first block's rows).
+    float* scratch = reinterpret_cast<float*>(zd);
+    scratch[tid] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
     __syncthreads();
     if (tid < NP) {
       float mx = 0.0f;
-      for (int q = 0; q < parts; ++q) mx = fmaxf(mx, part[q * NP + tid]);
+      for (int q = 0; q < parts; ++q) mx = fmaxf(mx, scratch[q * NP + tid]);
       wmax[tid] = mx;
     }
   }
@@ -218,58 +231,41 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
   const float gam = (h * u) / (1.0f - h * u);
   const float gam_ru = __fmul_ru(gam, 1.01f);
   const int slice = a.d / WARPS;
-  const int P = TB * a.G;  // (token, group) pairs of a block: pair p is thread p
+  const int P = TB * a.G;  // (token, group) pairs of a block
 
   for (; blk < n_blk; blk += gridDim.x) {
     cp_async_wait<0>();
-    __syncthreads();  // x rows in; the previous block's decisions are done
+    __syncthreads();  // x rows in; the previous block's outputs are written
 
-    // Partial logits over this warp's rows, in ascending row order. The
-    // shared-memory reads of the next 8 rows are issued before the FMAs of
-    // the current 8.
-    float acc[kTPT][4];
+    // Partial logits over this warp's rows, in ascending row order: per 8
+    // rows, one 16-byte x read per token and one W_r row quad per row.
+    float acc[TPT][4];
 #pragma unroll
-    for (int i = 0; i < kTPT; ++i)
+    for (int i = 0; i < TPT; ++i)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[i][q] = 0.0f;
-    auto load8 = [&](int m, uint4 (&xv)[kTPT], float4 (&wv)[8]) {
-#pragma unroll
-      for (int i = 0; i < kTPT; ++i) xv[i] = *reinterpret_cast<const uint4*>(xs + (tt + TG * i) * XS + m);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) wv[q] = *reinterpret_cast<const float4*>(Ws + (m + q) * NP + 4 * et);
-    };
-    auto fma8 = [&](const uint4 (&xv)[kTPT], const float4 (&wv)[8]) {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-#pragma unroll
-        for (int i = 0; i < kTPT; ++i) {
-          const uint32_t word = q < 2 ? xv[i].x : q < 4 ? xv[i].y : q < 6 ? xv[i].z : xv[i].w;
-          const float xf = (q & 1) ? bf16_hi(word) : bf16_lo(word);
-          acc[i][0] = fmaf(xf, wv[q].x, acc[i][0]);
-          acc[i][1] = fmaf(xf, wv[q].y, acc[i][1]);
-          acc[i][2] = fmaf(xf, wv[q].z, acc[i][2]);
-          acc[i][3] = fmaf(xf, wv[q].w, acc[i][3]);
-        }
-      }
-    };
     {
       const int m_lo = warp * slice, m_hi = m_lo + slice;
-      uint4 xa[kTPT], xb[kTPT];
-      float4 wa[8], wb[8];
-      load8(m_lo, xa, wa);
-      for (int m = m_lo; m < m_hi; m += 16) {
-        const bool two = m + 8 < m_hi;
-        if (two) load8(m + 8, xb, wb);
-        fma8(xa, wa);
-        if (!two) break;
-        if (m + 16 < m_hi) load8(m + 16, xa, wa);
-        fma8(xb, wb);
+#pragma unroll 2
+      for (int m = m_lo; m < m_hi; m += 8) {
+        uint4 xv[TPT];
+#pragma unroll
+        for (int i = 0; i < TPT; ++i) xv[i] = *reinterpret_cast<const uint4*>(xs + (tt + TG * i) * XS + m);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 wv = *reinterpret_cast<const float4*>(Ws + (m + q) * NP + 4 * et);
+#pragma unroll
+          for (int i = 0; i < TPT; ++i) {
+            const uint32_t word = q < 2 ? xv[i].x : q < 4 ? xv[i].y : q < 6 ? xv[i].z : xv[i].w;
+            const float xf = (q & 1) ? bf16_hi(word) : bf16_lo(word);
+            acc[i][0] = fmaf(xf, wv.x, acc[i][0]);
+            acc[i][1] = fmaf(xf, wv.y, acc[i][1]);
+            acc[i][2] = fmaf(xf, wv.z, acc[i][2]);
+            acc[i][3] = fmaf(xf, wv.w, acc[i][3]);
+          }
+        }
       }
     }
-#pragma unroll
-    for (int i = 0; i < kTPT; ++i)
-      *reinterpret_cast<float4*>(part + (warp * TB + tt + TG * i) * NP + 4 * et) =
-          make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
     // ||x||_1 per token (warp-strided tokens, lane-strided chunks).
     for (int t = warp; t < TB; t += WARPS) {
       float sx = 0.0f;
@@ -283,19 +279,18 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
       if (lane == 0) nxs[t] = sx;
     }
     if (tid == 0) n_uncertain = 0;
+    __syncthreads();  // x is consumed: its space takes the partials
+#pragma unroll
+    for (int i = 0; i < TPT; ++i)
+      *reinterpret_cast<float4*>(part + (warp * TB + tt + TG * i) * NP + 4 * et) =
+          make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
     __syncthreads();
-    // The x rows are consumed: fetch the next block while this one is decided.
-    stage_x(blk + gridDim.x);
-
-    // Thread p = pair (t, g): the group's logits (warp partials added in warp
-    // order, then the bias), top-k, certified by the bound; certain groups
-    // go straight on to their softmax.
-    const int t = tid / a.G, g = tid - t * a.G;
-    const bool mine = tid < P && blk * TB + t < a.R;
-    const int zo = t * NP + g * a.M;  // the group's logits in zf / zd / ez
-    bool certain = true;
-    uint64_t sel = 0;
-    if (mine) {
+    // Every pair (t, g): the group's logits (warp partials added in warp
+    // order, then the bias), top-k, certified by the bound; certain groups go
+    // straight on to their softmax.
+    for (int p = tid; p < P; p += THREADS) {
+      const int t = p / a.G, g = p - t * a.G;
+      const int zo = t * NP + g * a.M;
       float* zg = zf + zo;
       for (int j = 0; j < a.M; ++j) {
         float z = part[zo + j];
@@ -303,7 +298,9 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
         for (int w = 1; w < WARPS; ++w) z += part[w * TB * NP + zo + j];
         zg[j] = z + bsm[g * a.M + j];
       }
-      sel = group_topk(zg, a.M, a.k);
+      if (blk * TB + t >= a.R) continue;
+      const uint64_t sel = group_topk(zg, a.M, a.k);
+      bool certain = true;
       if (a.k < a.M) {
         const float nx = nxs[t];
         float lo = INFINITY, hi = -INFINITY;
@@ -315,14 +312,23 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
         }
         certain = lo > hi;
       }
-      if (certain) ps[tid] = group_softmax(zg, a.M, sel, ez + zo, dn + tid);
-      else list[atomicAdd(&n_uncertain, 1)] = tid;
+      if (certain) {
+        ps[p] = group_softmax(zg, a.M, sel, ez + zo, dn + p);
+        selp[p] = sel;
+      } else {
+        list[atomicAdd(&n_uncertain, 1)] = p;
+      }
     }
     __syncthreads();
+    // The partials are consumed: fetch the next block's rows while this one
+    // is finished.
+    stage_x(blk + gridDim.x);
     const int nu = n_uncertain;  // the same value in every thread: the barriers below are uniform
     if (nu > 0) {
       // fp64 logits of the uncertain groups, one warp per group (products of
-      // a bf16 and an fp32 value are exact in fp64).
+      // a bf16 and an fp32 value are exact in fp64). The block's x rows are
+      // being replaced, so x is read from global memory, several loads in
+      // flight per lane.
       for (int v = warp; v < nu; v += WARPS) {
         const int pv = list[v];
         const int tv = pv / a.G, gv = pv - tv * a.G;
@@ -333,16 +339,17 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
           const int e = gv * a.M + j;
           double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
           int m = 2 * lane;
+#pragma unroll 4
           for (; m + 64 < a.d; m += 128) {
-            const uint32_t p0 = *reinterpret_cast<const uint32_t*>(xr + m);
-            const uint32_t p1 = *reinterpret_cast<const uint32_t*>(xr + m + 64);
+            const uint32_t p0 = __ldg(reinterpret_cast<const unsigned int*>(xr + m));
+            const uint32_t p1 = __ldg(reinterpret_cast<const unsigned int*>(xr + m + 64));
             s0 = fma(static_cast<double>(bf16_lo(p0)), static_cast<double>(Ws[m * NP + e]), s0);
             s1 = fma(static_cast<double>(bf16_hi(p0)), static_cast<double>(Ws[(m + 1) * NP + e]), s1);
             s2 = fma(static_cast<double>(bf16_lo(p1)), static_cast<double>(Ws[(m + 64) * NP + e]), s2);
             s3 = fma(static_cast<double>(bf16_hi(p1)), static_cast<double>(Ws[(m + 65) * NP + e]), s3);
           }
           for (; m < a.d; m += 64) {
-            const uint32_t p0 = *reinterpret_cast<const uint32_t*>(xr + m);
+            const uint32_t p0 = __ldg(reinterpret_cast<const unsigned int*>(xr + m));
             s0 = fma(static_cast<double>(bf16_lo(p0)), static_cast<double>(Ws[m * NP + e]), s0);
             s1 = fma(static_cast<double>(bf16_hi(p0)), static_cast<double>(Ws[(m + 1) * NP + e]), s1);
           }
@@ -353,17 +360,25 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
         }
       }
       __syncthreads();
-      if (mine && !certain) {
-        sel = group_topk(zd + zo, a.M, a.k);
-        ps[tid] = group_softmax(zd + zo, a.M, sel, ez + zo, dn + tid);
+      for (int v = tid; v < nu; v += THREADS) {
+        const int pv = list[v];
+        const int tv = pv / a.G, gv = pv - tv * a.G;
+        const int zo = tv * NP + gv * a.M;
+        const uint64_t sel = group_topk(zd + zo, a.M, a.k);
+        ps[pv] = group_softmax(zd + zo, a.M, sel, ez + zo, dn + pv);
+        selp[pv] = sel;
       }
       __syncthreads();
     }
     // idx, r (renormalised in the group) and omega (over the token's groups).
-    if (mine) {
+    for (int p = tid; p < P; p += THREADS) {
+      const int t = p / a.G, g = p - t * a.G;
+      if (blk * TB + t >= a.R) continue;
+      const int zo = t * NP + g * a.M;
       float tot = 0.0f;  // selected mass of the token over its groups
       for (int g2 = 0; g2 < a.G; ++g2) tot += ps[t * a.G + g2];
-      const float psel = ps[tid], den = dn[tid];
+      const float psel = ps[p], den = dn[p];
+      const uint64_t sel = selp[p];
       const size_t o = (static_cast<size_t>(blk * TB + t) * a.G + g) * a.k;
       int s = 0;
       for (int j = 0; j < a.M; ++j) {
@@ -380,18 +395,48 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
   cp_async_wait<0>();
 }
 
+// SMs of the current device and resident CTAs per SM of one router kernel.
+inline int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+template <int NP, int WARPS, int TPT>
+int launch_tpt(const gqe_config& c, const RouterArgs& a, cudaStream_t st) {
+  const size_t smem = router_layout(c.d_model, NP, TPT).total;
+  if (smem > kRouterSmemLimit) return cudaErrorInvalidConfiguration;
+  const int e = ensure_smem<router_kernel<NP, WARPS, TPT>>(static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  static std::atomic<int> per_sm{0};
+  int ps = per_sm.load(std::memory_order_relaxed);
+  if (ps <= 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ps, router_kernel<NP, WARPS, TPT>, WARPS * 32,
+                                                      smem) != cudaSuccess || ps < 1)
+      ps = 1;
+    per_sm.store(ps, std::memory_order_relaxed);
+  }
+  // One token block per CTA while that fills the GPU; larger batches loop.
+  const int n_blk = (a.R + router_tb(NP, TPT) - 1) / router_tb(NP, TPT);
+  const int slots = ps * device_sms();
+  const int grid = n_blk < slots ? n_blk : slots;
+  return launch_pdl(router_kernel<NP, WARPS, TPT>, dim3(grid > 0 ? grid : 1), dim3(WARPS * 32), smem, st, a);
+}
+
+// Rows from which a launch takes more tokens per thread: each W_r quad read
+// from shared memory then feeds 4 to 8 tokens instead of 2 (the widest block
+// that fits in shared memory), at the price of fewer, larger token blocks
+// (which small batches cannot spread over the SMs).
+constexpr int kRouterWideRows = 4096;
+
 template <int NP, int WARPS>
 int launch_np(const gqe_config& c, const RouterArgs& a, cudaStream_t st) {
-  const size_t smem = router_smem_bytes(c);
-  if (smem > kRouterSmemLimit) return cudaErrorInvalidConfiguration;
-  const int e = ensure_smem<router_kernel<NP, WARPS>>(static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  // One block per CTA while that fills the GPU; larger batches loop.
-  const int n_blk = (a.R + router_tb(NP) - 1) / router_tb(NP);
-  const int per_sm = smem <= 112 * 1024 ? 2 : 1;
-  int grid = n_blk < per_sm * 148 ? n_blk : per_sm * 148;
-  if (grid < 1) grid = 1;
-  return launch_pdl(router_kernel<NP, WARPS>, dim3(grid), dim3(WARPS * 32), smem, st, a);
+  if (a.R >= kRouterWideRows) {
+    if (router_layout(c.d_model, NP, 8).total <= kRouterSmemLimit) return launch_tpt<NP, WARPS, 8>(c, a, st);
+    if (router_layout(c.d_model, NP, 6).total <= kRouterSmemLimit) return launch_tpt<NP, WARPS, 6>(c, a, st);
+    if (router_layout(c.d_model, NP, 4).total <= kRouterSmemLimit) return launch_tpt<NP, WARPS, 4>(c, a, st);
+  }
+  return launch_tpt<NP, WARPS, 2>(c, a, st);
 }
 
 template <int NP>
@@ -402,8 +447,10 @@ int launch_w(const gqe_config& c, const RouterArgs& a, cudaStream_t st) {
 }  // namespace router_impl
 using namespace router_impl;
 
+// The narrowest block shape (2 tokens per thread) is the one every batch can
+// take.
 size_t router_smem_bytes(const gqe_config& c) {
-  return router_layout(c.d_model, router_np(c.G * c.M)).total;
+  return router_layout(c.d_model, router_np(c.G * c.M), 2).total;
 }
 
 int launch_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r,
