@@ -64,12 +64,15 @@ struct RouterArgs {
   int R, d, G, M, k, N;
 };
 
+// Uncertain groups per round of the fp64 fallback.
+__host__ __device__ constexpr int router_fb(int NP) { return NP >= 64 ? 1 : NP >= 32 ? 2 : 4; }
+
 // Dynamic shared memory of one CTA (byte offsets). The warp partials
 // [warp][TB][NP] share their space with the block's x rows: they are written
 // once every warp has finished reading x, and the next block's rows are
 // fetched once the partials have been summed.
 struct RouterLayout {
-  size_t w, xs, zd, sel, zf, ez, wmax, bsm, nx, ps, dn, list, total;
+  size_t w, xs, zd, sel, fb, zf, ez, wmax, bsm, nx, ps, dn, list, total;
 };
 __host__ __device__ inline RouterLayout router_layout(int d, int NP, int TPT) {
   const int TB = router_tb(NP, TPT), W = router_warps(d);
@@ -81,6 +84,7 @@ __host__ __device__ inline RouterLayout router_layout(int d, int NP, int TPT) {
   L.xs = o;    o += ((xbytes > pbytes ? xbytes : pbytes) + 15) & ~static_cast<size_t>(15);
   L.zd = o;    o += static_cast<size_t>(TB) * NP * 8;                 // fp64 logits
   L.sel = o;   o += static_cast<size_t>(TB) * NP * 8;                 // selection mask per pair
+  L.fb = o;    o += static_cast<size_t>(router_fb(NP)) * W * NP * 8;   // fp64 warp partials (fallback)
   L.zf = o;    o += static_cast<size_t>(TB) * NP * 4;                 // fp32 logits
   L.ez = o;    o += static_cast<size_t>(TB) * NP * 4;                 // exp(z - group max)
   L.wmax = o;  o += NP * 4;                                            // max_i |W_r[i, e]|
@@ -325,41 +329,70 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
     stage_x(blk + gridDim.x);
     const int nu = n_uncertain;  // the same value in every thread: the barriers below are uniform
     if (nu > 0) {
-      // fp64 logits of the uncertain groups, one warp per group (products of
-      // a bf16 and an fp32 value are exact in fp64). The block's x rows are
-      // being replaced, so x is read from global memory, several loads in
-      // flight per lane.
-      for (int v = warp; v < nu; v += WARPS) {
-        const int pv = list[v];
-        const int tv = pv / a.G, gv = pv - tv * a.G;
-        const uint16_t* xr = a.x + static_cast<size_t>(blk * TB + tv) * a.d;
-        // Lane l takes columns 2l, 2l+1 (+64, ...): bf16 pairs, four
-        // independent fp64 sums per expert.
-        for (int j = 0; j < a.M; ++j) {
-          const int e = gv * a.M + j;
-          double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-          int m = 2 * lane;
-#pragma unroll 4
-          for (; m + 64 < a.d; m += 128) {
-            const uint32_t p0 = __ldg(reinterpret_cast<const unsigned int*>(xr + m));
-            const uint32_t p1 = __ldg(reinterpret_cast<const unsigned int*>(xr + m + 64));
-            s0 = fma(static_cast<double>(bf16_lo(p0)), static_cast<double>(Ws[m * NP + e]), s0);
-            s1 = fma(static_cast<double>(bf16_hi(p0)), static_cast<double>(Ws[(m + 1) * NP + e]), s1);
-            s2 = fma(static_cast<double>(bf16_lo(p1)), static_cast<double>(Ws[(m + 64) * NP + e]), s2);
-            s3 = fma(static_cast<double>(bf16_hi(p1)), static_cast<double>(Ws[(m + 65) * NP + e]), s3);
-          }
-          for (; m < a.d; m += 64) {
-            const uint32_t p0 = __ldg(reinterpret_cast<const unsigned int*>(xr + m));
-            s0 = fma(static_cast<double>(bf16_lo(p0)), static_cast<double>(Ws[m * NP + e]), s0);
-            s1 = fma(static_cast<double>(bf16_hi(p0)), static_cast<double>(Ws[(m + 1) * NP + e]), s1);
-          }
-          double s64 = (s0 + s1) + (s2 + s3);
+      // fp64 logits of the uncertain groups (products of a bf16 and an fp32
+      // value are exact in fp64), up to FB groups per round. A round's logits
+      // (group vb, column j) are items; warp w sums rows [w d/W, (w+1) d/W)
+      // of every item, lanes 4i..4i+3 taking item i (8 per pass) and a
+      // quarter of the slice each, so that the fp64 work is one product and
+      // one add per row and item, and the lane sums are reduced in two
+      // shuffle steps. x comes from global memory in 16-byte loads (the
+      // block's x rows are being replaced), W_r from shared memory. Warp sums
+      // are then added in warp order, so every logit is one fixed sequence of
+      // roundings.
+      constexpr int FB = router_fb(NP);
+      double* fb = reinterpret_cast<double*>(smem_raw + L.fb);  // [FB][WARPS][NP]
+      const int quarter = slice / 4;                             // a multiple of 2
+      for (int v0 = 0; v0 < nu; v0 += FB) {
+        const int nv = min(FB, nu - v0);
+        const int items = nv * a.M;
+        for (int i0 = 0; i0 < items; i0 += 8) {
+          const int item = i0 + (lane >> 2);
+          const int it = item < items ? item : items - 1;
+          const int vb = it / a.M, j = it - vb * a.M;
+          const int pv = list[v0 + vb];
+          const int tv = pv / a.G;
+          const int e = (pv - tv * a.G) * a.M + j;
+          const int m0 = warp * slice + (lane & 3) * quarter;
+          const uint16_t* xp = a.x + static_cast<size_t>(blk * TB + tv) * a.d + m0;
+          const float* wp = Ws + m0 * NP + e;
+          double acc0 = 0.0, acc1 = 0.0;  // even and odd rows
+          if (quarter % 8 == 0) {
+            // 16-byte x loads (8 rows each; m0 is a multiple of 8).
+#pragma unroll 2
+            for (int r0 = 0; r0 < quarter; r0 += 8) {
+              const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xp + r0));
+              const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) s64 += __shfl_xor_sync(0xffffffffu, s64, off);
-          if (lane == 0) zd[tv * NP + e] = s64 + static_cast<double>(bsm[e]);
+              for (int q = 0; q < 4; ++q) {
+                acc0 = fma(static_cast<double>(bf16_lo(xw[q])), static_cast<double>(wp[(r0 + 2 * q) * NP]), acc0);
+                acc1 = fma(static_cast<double>(bf16_hi(xw[q])), static_cast<double>(wp[(r0 + 2 * q + 1) * NP]),
+                           acc1);
+              }
+            }
+          } else {
+            for (int r = 0; r < quarter; r += 2) {
+              acc0 = fma(static_cast<double>(bf16_to_f32(__ldg(xp + r))), static_cast<double>(wp[r * NP]), acc0);
+              acc1 = fma(static_cast<double>(bf16_to_f32(__ldg(xp + r + 1))), static_cast<double>(wp[(r + 1) * NP]),
+                         acc1);
+            }
+          }
+          double acc = acc0 + acc1;
+          acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+          acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+          if ((lane & 3) == 0 && item < items) fb[(vb * WARPS + warp) * NP + e] = acc;
         }
+        __syncthreads();
+        for (int u = tid; u < items; u += THREADS) {
+          const int vb = u / a.M, j = u - vb * a.M;
+          const int pv = list[v0 + vb];
+          const int tv = pv / a.G, gv = pv - tv * a.G;
+          const int e = gv * a.M + j;
+          double z = 0.0;
+          for (int w = 0; w < WARPS; ++w) z += fb[(vb * WARPS + w) * NP + e];
+          zd[tv * NP + e] = z + static_cast<double>(bsm[e]);
+        }
+        __syncthreads();
       }
-      __syncthreads();
       for (int v = tid; v < nu; v += THREADS) {
         const int pv = list[v];
         const int tv = pv / a.G, gv = pv - tv * a.G;

@@ -185,6 +185,35 @@ def test_router_zero_weights_ties_go_low(rsq):
     np.testing.assert_allclose(o["omega"].cpu().numpy(), 1.0 / 8, rtol=1e-6)
 
 
+@pytest.mark.parametrize("B,T,M,k", [(2, 300, 2, 1), (1, 4500, 2, 1), (1, 700, 4, 2)])
+def test_router_near_ties_decided_exactly(rsq, B, T, M, k):
+    # Every group's columns of W_r differ by a perturbation of ~1e-7, far
+    # below the certified fp32 bound, so nearly every group is decided by the
+    # fp64 path. The selection must still be the exact one (the oracle's);
+    # 4500 rows take the wide token blocks, 300 and 700 the narrow ones.
+    shape = LayerShape(B=B, T=T, d_model=1024, G=8, M=M, k=k, d_head=64)
+    inp = synth.make_layer_inputs(shape, seed=31)
+    rng = np.random.default_rng(3)
+    W = inp.W_r.copy()
+    for g in range(shape.G):
+        for j in range(1, M):
+            W[:, g * M + j] = W[:, g * M] + (rng.standard_normal(W.shape[0]) * 1e-7).astype(np.float32)
+    inp.W_r = W
+    f = oracle._f64_inputs(inp)
+    ref = oracle.router(f["x"], f["W_r"], f["b_r"], shape.G, M, k)
+    d = device_inputs(inp)
+    R = B * T
+    idx = torch.empty(R, shape.G, k, dtype=torch.int32, device="cuda")
+    r = torch.empty(R, shape.G, k, dtype=torch.float32, device="cuda")
+    om = torch.empty_like(r)
+    rsq.gqe_router_topk(rsq.GQEConfig.of(shape), d["x"], d["W_r"], d["b_r"], idx, r, om)
+    torch.cuda.synchronize()
+    assert rsq.gqe_read_status() == 0
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"]), "near-tie selection differs from the exact one"
+    np.testing.assert_allclose(r.cpu().numpy(), ref["r"], rtol=0, atol=2e-6)
+    np.testing.assert_allclose(om.cpu().numpy(), ref["omega"], rtol=0, atol=2e-6)
+
+
 def test_device_wait_timeout_is_reported_and_recoverable(rsq):
     rsq.gqe_selftest_wait_timeout(2_000_000)  # 2 ms bound on a barrier nothing completes
     assert rsq.gqe_read_status() == rsq.GQE_ERR_TIMEOUT
