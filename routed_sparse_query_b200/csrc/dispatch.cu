@@ -212,16 +212,22 @@ __global__ void __launch_bounds__(1024) scan_kernel(ListArgs a) {
   write_list_meta(a, total);
 }
 
+// The selection mask of this thread's token in tile `tile` (0 past T).
+__device__ __forceinline__ uint64_t tile_token_mask(const ListArgs& a, int tile) {
+  const int b = tile / a.tiles_per_seq;
+  const int t = (tile % a.tiles_per_seq) * kDispatchTile + threadIdx.x;
+  return t < a.T ? a.masks[static_cast<size_t>(b) * a.T + t] : 0ull;
+}
+
 // Step 3 for one tile, given the tile's list bases per expert in shared
-// memory (base[e]).
-__device__ void scatter_tile(const ListArgs& a, int tile, const int* base) {
+// memory (base[e]) and this thread's token mask m.
+__device__ void scatter_tile(const ListArgs& a, int tile, const int* base, uint64_t m) {
   __shared__ int wcnt[kThreads / 32][kMaxExperts];
   const int b = tile / a.tiles_per_seq;
   const int t = (tile % a.tiles_per_seq) * kDispatchTile + threadIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned lt = (1u << lane) - 1u;
   const size_t row = static_cast<size_t>(b) * a.T + t;
-  const uint64_t m = t < a.T ? a.masks[row] : 0ull;
   int c0 = 0, c1 = 0;
   for (int e = 0; e < a.N; ++e) {
     const int n = __popc(__ballot_sync(0xffffffffu, (m >> e) & 1ull));
@@ -266,12 +272,13 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ListArgs a) {
   for (int e = threadIdx.x; e < a.N; e += blockDim.x)
     base[e] = a.tile_base[static_cast<size_t>(e) * a.num_tiles + blockIdx.x];
   __syncthreads();
-  scatter_tile(a, blockIdx.x, base);
+  scatter_tile(a, blockIdx.x, base, tile_token_mask(a, blockIdx.x));
 }
 
-// Steps 2 and 3 in one launch (few tiles): every CTA scans the tile counts
-// for its own bases; CTA 0 also writes tile_base, counts, offsets and the
-// tile table.
+// Steps 2 and 3 in one launch (few tiles): every scatter CTA scans the tile
+// counts for its own bases (its tokens' masks are loaded first, so that load
+// overlaps the scan); one more CTA (the last) writes tile_base, counts,
+// offsets and the tile table.
 constexpr int kFusedScanMax = 16384;  // N * num_tiles
 
 __global__ void __launch_bounds__(kThreads) scan_scatter_kernel(ListArgs a) {
@@ -279,7 +286,8 @@ __global__ void __launch_bounds__(kThreads) scan_scatter_kernel(ListArgs a) {
   pdl_launch_dependents();
   __shared__ int base[kMaxExperts];
   const int tile = blockIdx.x;
-  const bool lead = blockIdx.x == 0;
+  const bool lead = blockIdx.x == static_cast<unsigned>(a.num_tiles);
+  const uint64_t m = lead ? 0ull : tile_token_mask(a, tile);
   const int F = a.N * a.num_tiles;
   const int per = (F + kThreads - 1) / kThreads;
   const int lo = min(F, static_cast<int>(threadIdx.x) * per), hi = min(F, lo + per);
@@ -301,9 +309,9 @@ __global__ void __launch_bounds__(kThreads) scan_scatter_kernel(ListArgs a) {
   __syncthreads();
   if (lead) {
     write_list_meta(a, total);
-    __syncthreads();
+    return;
   }
-  scatter_tile(a, tile, base);
+  scatter_tile(a, tile, base, m);
 }
 
 // Weighted slot: one thread per 8 columns of one row.
@@ -393,7 +401,7 @@ int launch_dispatch_lists(const gqe_config& c, const int32_t* idx, int32_t* coun
   cudaError_t e = launch_pdl(mask_count_kernel, dim3(L.num_tiles), dim3(kThreads), 0, st, a);
   if (e != cudaSuccess) return e;
   if (static_cast<long long>(a.N) * L.num_tiles <= kFusedScanMax)
-    return launch_pdl(scan_scatter_kernel, dim3(L.num_tiles), dim3(kThreads), 0, st, a);
+    return launch_pdl(scan_scatter_kernel, dim3(L.num_tiles + 1), dim3(kThreads), 0, st, a);
   e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, a);
   if (e == cudaSuccess) e = launch_pdl(scatter_kernel, dim3(L.num_tiles), dim3(kThreads), 0, st, a);
   return e;
