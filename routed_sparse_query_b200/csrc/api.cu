@@ -148,9 +148,9 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
   __syncwarp();
 }
 
-// Per-device side stream for the K/V projection of gqe_layer_fwd: it reads
-// only x and the weights, so it runs beside the dispatch and the Q
-// projection (fork on the caller's stream after the router, join before the
+// Per-device side stream for the K/V (and shared-head Q) projections of
+// gqe_layer_fwd: they read only x and the weights, so they run beside the
+// dispatch and the routed Q projection (fork on the caller's stream after the router, join before the
 // attention). Created on first use; the enqueue sequence is serialised by
 // the mutex so that concurrent callers on one device do not interleave
 // their event records. Captured into CUDA graphs like any fork/join.
@@ -174,6 +174,22 @@ SideStream* side_stream_locked() {
     ss.ok = true;
   }
   return &ss;
+}
+
+// Token lists and the routed query projection (plus the shared head unless
+// Qs is null), after the caller's checks.
+gqe_status dispatch_and_project(const gqe_config& c, const int32_t* idx, const gqe_bf16* x,
+                                const gqe_bf16* W_q, const gqe_bf16* W_qs, int32_t* counts,
+                                int32_t* offsets, int32_t* tok, int32_t* slot_pos, gqe_bf16* Qv,
+                                gqe_bf16* Qs, void* ws, size_t ws_bytes, gqe_stream_t stream) {
+  const DispatchWs L = dispatch_ws_layout(c);
+  if (ws_bytes < L.total) return GQE_ERR_WORKSPACE;
+  int e = launch_dispatch_lists(c, idx, counts, offsets, tok, slot_pos, ws, L, stream);
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+  char* w = static_cast<char*>(ws);
+  return cuda_status(gemm_q_routed(c, x, W_q, W_qs, idx, offsets, tok, w + L.qtiles,
+                                   reinterpret_cast<const int32_t*>(w + L.n_qtiles), L.max_qtiles,
+                                   Qv, Qs, (c.flags & GQE_FLAG_EXPERT_MAJOR) != 0u, stream));
 }
 
 }  // namespace api_impl
@@ -264,14 +280,8 @@ gqe_status gqe_dispatch(const gqe_config* cfg, const int32_t* idx, const gqe_bf1
   if (!all_aligned(idx, x, W_q, W_qs, counts, offsets, tok, slot_pos, Qv, Qs) || ws == nullptr ||
       !aligned16(ws))
     return GQE_ERR_INVALID;
-  const DispatchWs L = dispatch_ws_layout(*cfg);
-  if (ws_bytes < L.total) return GQE_ERR_WORKSPACE;
-  int e = launch_dispatch_lists(*cfg, idx, counts, offsets, tok, slot_pos, ws, L, stream);
-  if (e != cudaSuccess) return GQE_ERR_CUDA;
-  char* w = static_cast<char*>(ws);
-  return cuda_status(gemm_q_routed(*cfg, x, W_q, W_qs, idx, offsets, tok, w + L.qtiles,
-                                   reinterpret_cast<const int32_t*>(w + L.n_qtiles), L.max_qtiles,
-                                   Qv, Qs, (cfg->flags & GQE_FLAG_EXPERT_MAJOR) != 0u, stream));
+  return dispatch_and_project(*cfg, idx, x, W_q, W_qs, counts, offsets, tok, slot_pos, Qv, Qs, ws,
+                              ws_bytes, stream);
 }
 
 gqe_status gqe_kv_proj(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16* W_k,
@@ -345,11 +355,15 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
     if (side != nullptr && (cudaEventRecord(side->fork, main_st) != cudaSuccess ||
                             cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess))
       return GQE_ERR_CUDA;
+    // The side stream also takes the shared-head query projection (it reads
+    // only x), so the routed Q projection on the critical path has only the
+    // routed tiles.
     const gqe_status kv = gqe_kv_proj(cfg, x, W_k, W_v, H(L.K), H(L.V), side ? side->s : stream);
     if (kv != GQE_OK) return kv;
+    if (gemm_q_shared(*cfg, x, W_qs, H(L.Qs), side ? side->s : stream) != cudaSuccess) return GQE_ERR_CUDA;
     if (side != nullptr && cudaEventRecord(side->join, side->s) != cudaSuccess) return GQE_ERR_CUDA;
-    st = gqe_dispatch(cfg, I(L.idx), x, W_q, W_qs, I(L.counts), I(L.offsets), I(L.tok),
-                      I(L.slot_pos), H(L.Qv), H(L.Qs), w + L.dws, L.total - L.dws, stream);
+    st = dispatch_and_project(*cfg, I(L.idx), x, W_q, W_qs, I(L.counts), I(L.offsets), I(L.tok),
+                              I(L.slot_pos), H(L.Qv), nullptr, w + L.dws, L.total - L.dws, stream);
     if (st != GQE_OK) return st;
     if (side != nullptr && cudaStreamWaitEvent(main_st, side->join, 0) != cudaSuccess)
       return GQE_ERR_CUDA;

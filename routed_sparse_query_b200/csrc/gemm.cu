@@ -523,9 +523,18 @@ int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, c
   g.expert_major = expert_major ? 1 : 0;
   Epi e{};
   const long long R = static_cast<long long>(c.B) * c.T;
-  const dim3 grid(static_cast<unsigned>(max_qtiles + (R + BM - 1) / BM), 1, 1);
+  const long long shared_tiles = Qs != nullptr ? (R + BM - 1) / BM : 0;
+  const dim3 grid(static_cast<unsigned>(max_qtiles + shared_tiles), 1, 1);
+  if (grid.x == 0) return cudaSuccess;
   if (dh == 64) return launch<64, true>(tb, tb, tbs, e, e, g, c.d_model, grid, stream);
   return launch<32, true>(tb, tb, tbs, e, e, g, c.d_model, grid, stream);
+}
+
+int gemm_q_shared(const gqe_config& c, const uint16_t* x, const uint16_t* W_qs, uint16_t* Qs,
+                  void* stream) {
+  const int R = c.B * c.T;
+  const Epi e = head_split(Qs, c.T, 1, c.d_head, R);
+  return dense_gemm(x, R, c.d_model, W_qs, nullptr, c.d_head, e, e, 1, stream);
 }
 
 }  // namespace gqe

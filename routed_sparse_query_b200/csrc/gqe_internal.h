@@ -93,13 +93,17 @@ int launch_weighted_slot(const gqe_config& c, uint16_t* slots, const float* omeg
 int gemm_kv(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
             uint16_t* K, uint16_t* V, void* stream);
 // Routed query projection over the token lists plus the shared-head query
-// projection, in one launch.
+// projection, in one launch (Qs == nullptr: routed tiles only).
 // expert_major: Qv is written in token-list order ([k*G*B*T, dh], row = list
 // entry) instead of slot-major [B, G, k, T, dh].
 int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const uint16_t* W_qs,
                   const int32_t* idx, const int32_t* offsets, const int32_t* tok, const void* qtiles,
                   const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, uint16_t* Qs,
                   bool expert_major, void* stream);
+// The shared-head query projection alone (Qs [B, T, dh]); the same tiles and
+// accumulation order as the shared tiles of gemm_q_routed, so the same bits.
+int gemm_q_shared(const gqe_config& c, const uint16_t* x, const uint16_t* W_qs, uint16_t* Qs,
+                  void* stream);
 int gemm_q_dense(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, uint16_t* Q,
                  void* stream);
 int gemm_rowmajor(const uint16_t* A, int rows, int K, const uint16_t* W, int N, uint16_t* out,
