@@ -239,9 +239,14 @@ gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* 
                            const gqe_bf16* W_o, gqe_bf16* y, gqe_stream_t stream);
 
 /*
- * The whole GQE layer (a1-a11) on one stream; every intermediate lives in
- * `ws` (>= gqe_workspace_bytes(cfg, GQE_WS_LAYER); see gqe_workspace_offset).
- * Arguments as in the calls above.
+ * The whole GQE layer (a1-a11), ordered on `stream`; every intermediate
+ * lives in `ws` (>= gqe_workspace_bytes(cfg, GQE_WS_LAYER); see
+ * gqe_workspace_offset). The K/V and shared-head query projections run on a
+ * side stream owned by the library (one per device) that forks from `stream`
+ * after the router and joins it before the attention, so the call is still
+ * stream-ordered as a whole (and captures into a CUDA graph as a fork/join).
+ * The results are bitwise those of the step calls. Arguments as in the calls
+ * above.
  */
 gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
                          const float* b_r, const gqe_bf16* W_q, const gqe_bf16* W_qs,
