@@ -16,15 +16,13 @@ namespace gqe {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Router limits: N = G*M experts (<= 64, G <= 32). The logits are reduced
-// over NP = max(4, next power of two >= N) columns; W_r is staged in shared
-// memory with a row stride of router_row_floats(NP) floats, == 4 (mod 8), so
-// that the 16-byte reads of 8 consecutive lanes (consecutive rows) land in
-// distinct bank groups.
+// over NP = max(4, next power of two >= N) columns (W_r is staged in shared
+// memory zero-padded to NP columns); a configuration is supported when the
+// router's narrowest block (2 tokens per thread) fits in kRouterSmemLimit.
 constexpr int kMaxExperts = 64;
 __host__ __device__ constexpr int router_np(int N) {
   return N <= 4 ? 4 : N <= 8 ? 8 : N <= 16 ? 16 : N <= 32 ? 32 : 64;
 }
-__host__ __device__ constexpr int router_row_floats(int NP) { return NP == 4 ? 4 : NP + 4; }
 constexpr size_t kRouterSmemLimit = 200 * 1024;
 
 // Dispatch tiling: tokens of one sequence are cut into tiles of this size.
