@@ -91,3 +91,18 @@ def test_workspace_sizes_cover_items(rsq):
     assert slots + R * (k * G + 2) * dh * 2 <= total
     assert rsq.gqe_workspace_offset(c, rsq.GQE_WS_LAYER, "K") % 256 == 0
     assert rsq.gqe_workspace_bytes(c, rsq.GQE_WS_DENSE) >= R * 16 * dh * 2 * 2
+
+
+def test_router_staging_limit(rsq):
+    # The router stages W_r (fp32, zero-padded to a power-of-two column count)
+    # in shared memory: 32 experts at d_model = 1024 (the expert-pool
+    # workloads) fit, 64 experts at d_model = 1024 (256 KB of W_r) do not and
+    # are refused on the host, 64 experts at d_model = 256 fit again.
+    ws = rsq.GQE_WS_LAYER
+    assert rsq.gqe_workspace_bytes(_cfg(rsq, G=8, M=4, k=2), ws) > 0
+    assert rsq.gqe_workspace_bytes(_cfg(rsq, G=8, M=8), ws) == 0
+    assert rsq.gqe_workspace_bytes(_cfg(rsq, G=8, M=8, d_model=256), ws) > 0
+    lib = rsq.lib()
+    c = _cfg(rsq, G=8, M=8)
+    assert lib.gqe_router_topk(ctypes.byref(c), None, None, None, None, None, None,
+                               None) == rsq.GQE_ERR_UNSUPPORTED
