@@ -531,6 +531,8 @@ def run_ours(args, rank: int, world: int, dist):
     if world == 1 and not args.no_sweep:
         out["sweep"] = sweep(rsq, pk, args)
         out["decode"] = decode_bench(rsq, pk, args.steps)
+    if world == 1 and args.sweep_pool:
+        out["pool_sweep"] = sweep_pool(rsq, pk, args)
     if world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(shape, min_seconds=10.0)
     return out
@@ -614,6 +616,43 @@ def sweep(rsq, pk, args):
     return rows
 
 
+POOL_SWEEP = [("pool4_k1", True), ("pool4_k2", True), ("pool4_k2", False)]  # (workload, skewed)
+
+
+def sweep_pool(rsq, pk, args):
+    """GQE vs dense GQA on the expert-pool workloads (32 experts, T = 32k):
+    k = 1 and 2 with the skew bias (one expert per group takes ~80 % of the
+    tokens) and k = 2 balanced. Reports the measured hot-expert share."""
+    import torch
+    rows = []
+    for name, skew in POOL_SWEEP:
+        s = WORKLOADS[name]
+        d = device_inputs_seeded(s, 1234)
+        if skew:
+            b = np.zeros(s.N, dtype=np.float32)
+            b[0::s.M] = np.float32(synth.SKEW_BETA[(s.M, s.k)])
+            d["b_r"] = torch.from_numpy(b).cuda()
+        layer = Layer(rsq, s, d)
+        steps = max(2, min(args.steps, 20))
+        res = time_steps(layer, steps, 2, None, lambda: None)
+        dense_ms = time_dense(rsq, s, d, steps, 1, None) / steps
+        gq_ms = time_layer(rsq, s, d, steps, 1, None) / steps
+        counts = layer.counts.view(s.N, s.B).sum(dim=1).cpu().numpy().reshape(s.G, s.M)
+        attn_s = res["per_call_ms"]["attention"] / steps / 1e3
+        ach = flops(s)["attention"] / attn_s / 1e12
+        rows.append({"workload": f"{name} ({'skewed' if skew else 'balanced'}): {describe(s)}",
+                     "steps": steps, "gqe_ms": gq_ms, "dense_ms": dense_ms,
+                     "speedup": dense_ms / gq_ms,
+                     "hot_expert_share": float(counts[:, 0].sum()) / (s.G * s.R),
+                     "attn_tflops": ach, "attn_frac_of_bf16_peak": ach / pk["bf16"],
+                     "breakdown_ms": {c: v / steps for c, v in res["per_call_ms"].items()}})
+        if rsq.gqe_read_status() != 0:
+            raise RuntimeError(f"device-side status set in pool sweep {name}")
+        del layer, d
+        torch.cuda.empty_cache()
+    return rows
+
+
 def run_reference(args):
     """The fp64 oracle on the host cores, on prefixes of the workload sized so
     that warmup + steps end within about two minutes."""
@@ -658,6 +697,8 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--sweep-max", choices=SWEEP, default=None)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--sweep-pool", action="store_true",
+                    help="also time the expert-pool workloads (32 experts, k = 1, 2; skewed, balanced)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
