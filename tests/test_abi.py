@@ -106,3 +106,16 @@ def test_router_staging_limit(rsq):
     c = _cfg(rsq, G=8, M=8)
     assert lib.gqe_router_topk(ctypes.byref(c), None, None, None, None, None, None,
                                None) == rsq.GQE_ERR_UNSUPPORTED
+
+
+def test_attention_split_kv_plan(rsq):
+    # Split-KV (and its workspace of partial rows) only when the query-tile
+    # pairs of all streams are fewer than the SMs: 9 streams x 8 pairs at
+    # T = 2048 are split, 9 x 128 pairs at T = 32768 are not (the workspace is
+    # then the 256-byte minimum).
+    ws = rsq.GQE_WS_ATTENTION
+    small = rsq.gqe_workspace_bytes(_cfg(rsq, T=2048), ws)
+    large = rsq.gqe_workspace_bytes(_cfg(rsq, T=32768), ws)
+    assert large == 256
+    rows = 9 * 16 * 2 * 128  # streams x items (chunk of 5 KV tiles: 16 per stream) x 2 tiles x 128 rows
+    assert small >= rows * 64 * 4 + rows * 8  # fp32 partial O rows and (m, l) pairs
