@@ -12,9 +12,8 @@
 // not a multiple of 128) sums rows [w d/W, (w+1) d/W) of the dot products;
 // each thread keeps TPT tokens x 4 experts, so one 16-byte W_r read (one
 // shared-memory pass per quarter warp) feeds 4 TPT FMAs. Large batches take
-// the largest TPT of 8, 6, 4 whose block fits in shared memory (6 for
-// d = 1024 with 16 experts), small ones TPT = 2 so that the blocks spread
-// over the SMs. The W warp partials are then added in warp
+// TPT = 6 (4 where that block does not fit in shared memory, e.g. 32 experts
+// at d = 1024), small ones TPT = 2 so that the blocks spread over the SMs. The W warp partials are then added in warp
 // order, so every logit is one fixed sequence of roundings (the result is
 // deterministic and the same for every TPT). The threads then take the
 // (token, group) pairs and decide.
@@ -457,15 +456,14 @@ int launch_tpt(const gqe_config& c, const RouterArgs& a, cudaStream_t st) {
 }
 
 // Rows from which a launch takes more tokens per thread: each W_r quad read
-// from shared memory then feeds 4 to 8 tokens instead of 2 (the widest block
-// that fits in shared memory), at the price of fewer, larger token blocks
-// (which small batches cannot spread over the SMs).
+// from shared memory then feeds 6 (or 4, where shared memory is short)
+// tokens instead of 2, at the price of fewer, larger token blocks (which
+// small batches cannot spread over the SMs).
 constexpr int kRouterWideRows = 4096;
 
 template <int NP, int WARPS>
 int launch_np(const gqe_config& c, const RouterArgs& a, cudaStream_t st) {
   if (a.R >= kRouterWideRows) {
-    if (router_layout(c.d_model, NP, 8).total <= kRouterSmemLimit) return launch_tpt<NP, WARPS, 8>(c, a, st);
     if (router_layout(c.d_model, NP, 6).total <= kRouterSmemLimit) return launch_tpt<NP, WARPS, 6>(c, a, st);
     if (router_layout(c.d_model, NP, 4).total <= kRouterSmemLimit) return launch_tpt<NP, WARPS, 4>(c, a, st);
   }
