@@ -214,6 +214,42 @@ def test_router_near_ties_decided_exactly(rsq, B, T, M, k):
     np.testing.assert_allclose(om.cpu().numpy(), ref["omega"], rtol=0, atol=2e-6)
 
 
+def test_dispatch_lists_with_separate_scan(rsq):
+    # 16 experts x 1026 tiles of 256 tokens = 16416 tile counts: more than one
+    # fused scan + scatter launch takes, so the lists come from the
+    # stand-alone scan kernel and the scatter kernel (the path of the 1M
+    # workload). Router output and lists must be bit-exact.
+    shape = LayerShape(B=1, T=262401, d_model=256, G=8, M=2, k=1, d_head=64)
+    assert shape.N * shape.B * -(-shape.T // 256) > 16384
+    inp = synth.make_layer_inputs(shape, seed=47, with_dense=False)
+    f = oracle._f64_inputs(inp)
+    ref = oracle.router(f["x"], f["W_r"], f["b_r"], shape.G, shape.M, shape.k)
+    lists = oracle.dispatch(ref["idx"], shape.B, shape.T, shape.G, shape.M)
+    d = device_inputs(inp)
+    cfg = rsq.GQEConfig.of(shape)
+    B, T, G, k, dh, R, N = shape.B, shape.T, shape.G, shape.k, shape.d_head, shape.R, shape.N
+    dev = torch.device("cuda")
+    idx = torch.empty(R, G, k, dtype=torch.int32, device=dev)
+    r = torch.empty(R, G, k, dtype=torch.float32, device=dev)
+    om = torch.empty_like(r)
+    rsq.gqe_router_topk(cfg, d["x"], d["W_r"], d["b_r"], idx, r, om)
+    counts = torch.empty(N * B, dtype=torch.int32, device=dev)
+    offsets = torch.empty(N * B + 1, dtype=torch.int32, device=dev)
+    tok = torch.empty(k * G * R, dtype=torch.int32, device=dev)
+    slot_pos = torch.empty(R, G, k, dtype=torch.int32, device=dev)
+    Qv = torch.empty(B, G, k, T, dh, dtype=torch.bfloat16, device=dev)
+    Qs = torch.empty(B, T, dh, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_DISPATCH), dtype=torch.uint8, device=dev)
+    rsq.gqe_dispatch(cfg, idx, d["x"], d["W_q"], d["W_qs"], counts, offsets, tok, slot_pos, Qv, Qs, ws)
+    torch.cuda.synchronize()
+    assert rsq.gqe_read_status() == 0
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"]), "router indices differ"
+    assert np.array_equal(counts.cpu().numpy().reshape(N, B), lists["counts"])
+    assert np.array_equal(offsets.cpu().numpy(), lists["offsets"])
+    assert np.array_equal(tok.cpu().numpy(), lists["tok"]), "token lists differ"
+    assert np.array_equal(slot_pos.cpu().numpy(), lists["slot_pos"])
+
+
 def test_device_wait_timeout_is_reported_and_recoverable(rsq):
     rsq.gqe_selftest_wait_timeout(2_000_000)  # 2 ms bound on a barrier nothing completes
     assert rsq.gqe_read_status() == rsq.GQE_ERR_TIMEOUT
