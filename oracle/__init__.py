@@ -76,6 +76,34 @@ def _exact_logit(xrow: np.ndarray, wcol: np.ndarray, b: float) -> float:
     return math.fsum(list(xrow * wcol) + [b])
 
 
+def _exact_sign_of_difference(xrow: np.ndarray, wa: np.ndarray, wb: np.ndarray, ba: float,
+                              bb: float) -> int:
+    """Sign of z_a - z_b computed exactly.
+
+    z_a - z_b = sum_i x_i W[i,a] - sum_i x_i W[i,b] + b_a - b_b. Every term is
+    an exact fp64 value (bf16 x fp32 products), and math.fsum returns the
+    correctly rounded value of their exact sum, which is zero exactly when the
+    sum is zero and otherwise has its sign.
+    """
+    s = math.fsum(list(xrow * wa) + list(-(xrow * wb)) + [ba, -bb])
+    return (s > 0) - (s < 0)
+
+
+def _exact_topk(xrow: np.ndarray, W: np.ndarray, bvec: np.ndarray, g: int, M: int, k: int):
+    """The k experts of group g with the largest exact logits, ties to the lower
+    index, ascending: expert j precedes i when z_j > z_i exactly, or z_j = z_i
+    and j < i."""
+    import functools
+
+    def before(j, i):
+        s = _exact_sign_of_difference(xrow, W[:, g * M + j], W[:, g * M + i], bvec[g * M + j],
+                                      bvec[g * M + i])
+        return -1 if s > 0 or (s == 0 and j < i) else 1
+
+    order = sorted(range(M), key=functools.cmp_to_key(before))
+    return sorted(order[:k])
+
+
 def router(x: np.ndarray, W_r: np.ndarray, b_r: np.ndarray | None, G: int, M: int, k: int):
     """Per-group softmax, top-k per group, renormalised weights.
 
@@ -88,8 +116,10 @@ def router(x: np.ndarray, W_r: np.ndarray, b_r: np.ndarray | None, G: int, M: in
 
     The selection is the one exact arithmetic gives: where the fp64 logits of
     a group are closer at the top-k boundary than a certified bound on their
-    rounding error, that group's logits are recomputed correctly rounded
-    (math.fsum of exact products) before selecting.
+    rounding error, that group's order is decided on the exact logits (the
+    exact sign of each difference, ``_exact_topk``) and its logits are
+    recomputed correctly rounded (math.fsum of exact products) for the
+    softmax.
     """
     if not (1 <= k <= M):
         raise ValueError("need 1 <= k <= M")
@@ -106,6 +136,7 @@ def router(x: np.ndarray, W_r: np.ndarray, b_r: np.ndarray | None, G: int, M: in
     bound = gam * (np.abs(x) @ np.abs(W_r) + np.abs(bvec)[None, :]) * 2.0
 
     zg = z.reshape(R, G, M)
+    exact_sel = {}
     if k < M:
         srt = -np.sort(-zg, axis=-1)
         margin = srt[..., k - 1] - srt[..., k]
@@ -114,6 +145,7 @@ def router(x: np.ndarray, W_r: np.ndarray, b_r: np.ndarray | None, G: int, M: in
             for j in range(M):
                 e = g * M + j
                 zg[t, g, j] = _exact_logit(x[t], W_r[:, e], bvec[e])
+            exact_sel[(int(t), int(g))] = _exact_topk(x[t], W_r, bvec, int(g), M, k)
         z = zg.reshape(R, N)
 
     # a2: softmax over the M logits of each group (softmax before top-k).
@@ -123,8 +155,11 @@ def router(x: np.ndarray, W_r: np.ndarray, b_r: np.ndarray | None, G: int, M: in
 
     # a3: top-k on the logits; a stable sort of -z keeps equal logits in index
     # order, so ties go to the lower j. Selected indices stored ascending.
+    # Groups without a certified fp64 margin take their exact selection.
     order = np.argsort(-zg, axis=-1, kind="stable")[..., :k]
     idx = np.sort(order, axis=-1).astype(np.int32)
+    for (t, g), sel in exact_sel.items():
+        idx[t, g] = sel
 
     # a4: renormalised weights.
     psel = np.take_along_axis(p, idx.astype(np.int64), axis=-1)
@@ -146,38 +181,39 @@ def dispatch(idx: np.ndarray, B: int, T: int, G: int, M: int):
     tok[...]       for each (e, b), the positions t (0..T-1) that selected e,
                    ascending;
     slot_pos[row, g, s] the index in ``tok`` of the entry for that selection.
+
+    For each (e, b): the positions whose selections in group g contain j
+    (e = g*M + j), in increasing order; a selection's entry is the list's
+    base plus the number of earlier positions in the same list.
     """
     R, G_, k = idx.shape
     assert G_ == G and R == B * T
     N = G * M
     counts = np.zeros((N, B), dtype=np.int64)
-    lists = [[[] for _ in range(B)] for _ in range(N)]
-    for row in range(R):
-        b, t = divmod(row, T)
-        for g in range(G):
-            for s in range(k):
-                e = g * M + int(idx[row, g, s])
-                lists[e][b].append(t)
-                counts[e, b] += 1
+    hits = {}
+    for e in range(N):
+        g, j = divmod(e, M)
+        for b in range(B):
+            sel = idx[b * T:(b + 1) * T, g, :] == j      # [T, k]: which slot took j
+            hits[(e, b)] = sel
+            counts[e, b] = int(sel.sum())
     offsets = np.zeros(N * B + 1, dtype=np.int64)
     offsets[1:] = np.cumsum(counts.reshape(-1))
     tok = np.zeros(int(offsets[-1]), dtype=np.int32)
-    slot_pos = np.zeros((R, G, k), dtype=np.int32)
-    where = {}
+    slot_pos = np.full((R, G, k), -1, dtype=np.int64)
     for e in range(N):
+        g, j = divmod(e, M)
         for b in range(B):
+            sel = hits[(e, b)]
             base = int(offsets[e * B + b])
-            for i, t in enumerate(lists[e][b]):
-                tok[base + i] = t
-                where[(e, b, t)] = base + i
-    for row in range(R):
-        b, t = divmod(row, T)
-        for g in range(G):
-            for s in range(k):
-                e = g * M + int(idx[row, g, s])
-                slot_pos[row, g, s] = where[(e, b, t)]
+            t_list = np.nonzero(sel.any(axis=1))[0]       # ascending positions
+            tok[base:base + t_list.size] = t_list
+            t_s, s_s = np.nonzero(sel)                    # (position, slot) of each hit
+            rank = np.searchsorted(t_list, t_s)           # earlier entries of the list
+            slot_pos[b * T + t_s, g, s_s] = base + rank
+    assert (slot_pos >= 0).all()
     return {"counts": counts.astype(np.int32), "offsets": offsets.astype(np.int32),
-            "tok": tok, "slot_pos": slot_pos}
+            "tok": tok, "slot_pos": slot_pos.astype(np.int32)}
 
 
 # --------------------------------------------------------------------------
@@ -194,30 +230,37 @@ def kv_proj(x: np.ndarray, W: np.ndarray, B: int, T: int, G: int, dh: int) -> np
     return y.reshape(B, T, G, dh).transpose(0, 2, 1, 3).copy()
 
 
-def q_routed(x: np.ndarray, W_q: np.ndarray, idx: np.ndarray, B: int, T: int, G: int,
-             M: int, dh: int) -> np.ndarray:
-    """Query of every selected expert only, slot-major: Qv[b, g, s, t, :].
+def q_routed_rows(x_rows: np.ndarray, W_q: np.ndarray, idx_rows: np.ndarray, G: int, M: int,
+                  dh: int) -> np.ndarray:
+    """Query of every selected expert of the given token rows: q[n, g, s, :].
 
-    Expert e = g*M + idx[row, g, s] computes q = x[row] @ W_q[:, e*dh:(e+1)*dh]
-    for the rows that selected it, and no other rows (conditional query
-    computation: chatpaper / hotpaper abstract).
+    Row n's selection (g, s) is expert e = g*M + idx_rows[n, g, s], and its
+    query is x_rows[n] @ W_q[:, e*dh:(e+1)*dh]; no other expert computes a
+    query for the row (conditional query computation: chatpaper / hotpaper
+    abstract).
     """
-    x = np.asarray(x, np.float64)
+    x_rows = np.asarray(x_rows, np.float64)
     W_q = np.asarray(W_q, np.float64)
-    R, _, k = idx.shape
-    Qv = np.zeros((B, G, k, T, dh))
-    rows = np.arange(R)
+    n, _, k = idx_rows.shape
+    q = np.zeros((n, G, k, dh))
     for g in range(G):
         for j in range(M):
             e = g * M + j
             We = W_q[:, e * dh:(e + 1) * dh]
             for s in range(k):
-                sel = rows[idx[:, g, s] == j]
-                if sel.size == 0:
-                    continue
-                q = x[sel] @ We
-                Qv[sel // T, g, s, sel % T, :] = q
-    return Qv
+                m = idx_rows[:, g, s] == j
+                if m.any():
+                    q[m, g, s] = x_rows[m] @ We
+    return q
+
+
+def q_routed(x: np.ndarray, W_q: np.ndarray, idx: np.ndarray, B: int, T: int, G: int,
+             M: int, dh: int) -> np.ndarray:
+    """The routed queries of every row, slot-major: Qv[b, g, s, t, :]
+    (``q_routed_rows`` of all rows, laid out by stream)."""
+    k = idx.shape[2]
+    q = q_routed_rows(x, W_q, idx, G, M, dh)             # [B*T, G, k, dh]
+    return q.reshape(B, T, G, k, dh).transpose(0, 2, 3, 1, 4).copy()
 
 
 def q_shared(x: np.ndarray, W_qs: np.ndarray, B: int, T: int, dh: int) -> np.ndarray:
@@ -230,12 +273,13 @@ def q_shared(x: np.ndarray, W_qs: np.ndarray, B: int, T: int, dh: int) -> np.nda
 # --------------------------------------------------------------------------
 
 def causal_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, rows=None,
-                     block: int = 512) -> np.ndarray:
+                     block: int | None = None) -> np.ndarray:
     """o[t] = sum_{u <= t} softmax_u(q[t] . K[u] / sqrt(dh)) V[u] for one head.
 
     ``q`` holds the queries of the rows ``rows`` (positions in the sequence;
     all positions 0..len(q)-1 when None). Each row is evaluated on its own
-    from the definition; ``block`` only groups rows to bound memory.
+    from the definition; ``block`` only groups rows to bound memory (by
+    default as many rows as keep one score block near 128 MB).
     """
     q = np.asarray(q, np.float64)
     K = np.asarray(K, np.float64)
@@ -244,6 +288,8 @@ def causal_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, rows=None,
     pos = np.arange(n) if rows is None else np.asarray(rows, np.int64)
     scale = 1.0 / math.sqrt(dh)
     out = np.empty((n, V.shape[1]))
+    if block is None:
+        block = max(1, min(512, (1 << 24) // max(1, int(pos.max(initial=0)) + 1)))
     for s in range(0, n, block):
         ps = pos[s:s + block]
         hi = int(ps.max()) + 1
@@ -261,18 +307,60 @@ def causal_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, rows=None,
 # a10-a11: slots and W_O
 # --------------------------------------------------------------------------
 
-def assemble_slots(o_routed: np.ndarray, o_shared: np.ndarray, omega: np.ndarray) -> np.ndarray:
-    """(kG+2) slots per token: [o_{g,s} for g, s] + [o_shared] + [sum w*o].
+# Output constructions. "gqe" is the layer (reading R3); the others are the
+# ablation variants of the pptc.cn blog's section 4.3 and Table 1 (reading R15:
+# that page's labels), and "group_mean" is the alternative weighted slot:
+#   gqe              [o_{g,s}] + [o_shared] + [sum_{g,s} omega_{g,s} o_{g,s}]
+#   group_mean       [o_{g,s}] + [o_shared] + [(1/G) sum_g sum_s r_{g,s} o_{g,s}]
+#                    (each group's selected outputs renormalised inside the
+#                    group, then the groups averaged)
+#   hard             [o_{g,s}] only: hard concatenation of the selected experts,
+#                    with neither the router-supervision slot nor the shared head
+#                    ("仅硬拼接")
+#   weighted_concat  [p_{g,s} o_{g,s}]: each selected output scaled by its
+#                    in-group softmax probability, with neither the supervision
+#                    slot nor the shared head ("加权拼接但无重归一化槽"; the page
+#                    says the weights are possibly the in-group softmax
+#                    probabilities, and that is the reading taken)
+OUTPUT_MODES = ("gqe", "group_mean", "hard", "weighted_concat")
 
-    o_routed [R, G, k, dh], o_shared [R, dh], omega [R, G, k] -> [R, (kG+2)*dh].
+
+def mode_slots(mode: str, G: int, k: int) -> int:
+    """Slots per token (W_O has this many d_head-row blocks)."""
+    return k * G + 2 if mode in ("gqe", "group_mean") else k * G
+
+
+def mode_has_shared_head(mode: str) -> bool:
+    return mode in ("gqe", "group_mean")
+
+
+def assemble_slots(o_routed: np.ndarray, o_shared: np.ndarray | None, rt_rows: dict,
+                   mode: str = "gqe") -> np.ndarray:
+    """Slots per token for an output construction (see OUTPUT_MODES).
+
+    o_routed [R, G, k, dh]; o_shared [R, dh] (None for the modes without the
+    shared head); rt_rows holds the router's omega, r, p and idx of the same
+    rows -> [R, mode_slots * dh].
     """
     R, G, k, dh = o_routed.shape
-    weighted = np.einsum("rgs,rgsd->rd", omega, o_routed)
-    return np.concatenate([o_routed.reshape(R, G * k * dh), o_shared, weighted], axis=1)
+    concat = o_routed.reshape(R, G * k * dh)
+    if mode == "gqe":
+        weighted = np.einsum("rgs,rgsd->rd", rt_rows["omega"], o_routed)
+        return np.concatenate([concat, o_shared, weighted], axis=1)
+    if mode == "group_mean":
+        weighted = np.einsum("rgs,rgsd->rd", rt_rows["r"], o_routed) / G
+        return np.concatenate([concat, o_shared, weighted], axis=1)
+    if mode == "hard":
+        return concat.copy()
+    if mode == "weighted_concat":
+        psel = np.take_along_axis(rt_rows["p"], rt_rows["idx"].astype(np.int64), axis=-1)
+        return (psel[..., None] * o_routed).reshape(R, G * k * dh)
+    raise ValueError(f"unknown output mode {mode!r}")
 
 
 def output_proj(slots: np.ndarray, W_o: np.ndarray) -> np.ndarray:
-    """y = slots @ W_O with W_O of shape [(kG+2)*dh, d] (reading R9)."""
+    """y = slots @ W_O with W_O of shape [slots*dh, d]: [(kG+2)*dh, d] for the
+    layer (reading R9)."""
     return np.asarray(slots, np.float64) @ np.asarray(W_o, np.float64)
 
 
@@ -280,9 +368,10 @@ def output_proj(slots: np.ndarray, W_o: np.ndarray) -> np.ndarray:
 # whole layers
 # --------------------------------------------------------------------------
 
-def _f64_inputs(inp: LayerInputs):
+def _f64_weights(inp: LayerInputs) -> dict:
+    """Exact fp64 values of every weight (x is widened row block by row block
+    where it is used)."""
     return {
-        "x": bf16_to_f64(inp.x),
         "W_r": inp.W_r.astype(np.float64),
         "b_r": None if inp.b_r is None else inp.b_r.astype(np.float64),
         "W_q": bf16_to_f64(inp.W_q),
@@ -294,57 +383,113 @@ def _f64_inputs(inp: LayerInputs):
     }
 
 
-def gqe_layer(inp: LayerInputs, rows=None, with_dispatch: bool = True) -> dict:
+def _f64_inputs(inp: LayerInputs) -> dict:
+    f = _f64_weights(inp)
+    f["x"] = bf16_to_f64(inp.x)
+    return f
+
+
+# Rows of x widened to fp64 at a time. Every output row of the router and of
+# the projections depends on its own x row only, so taking the rows block by
+# block changes no arithmetic; it only bounds host memory on long sequences.
+_ROW_BLOCK = 16384
+
+
+def _router_by_rows(inp: LayerInputs, f: dict) -> dict:
+    s = inp.shape
+    parts = [router(bf16_to_f64(inp.x[lo:lo + _ROW_BLOCK]), f["W_r"], f["b_r"], s.G, s.M, s.k)
+             for lo in range(0, s.R, _ROW_BLOCK)]
+    return {key: np.concatenate([p_[key] for p_ in parts]) for key in parts[0]}
+
+
+def _kv_group_prefix(inp: LayerInputs, W_k: np.ndarray, W_v: np.ndarray, b: int, g: int,
+                     hi: int):
+    """K and V of group g for positions 0..hi-1 of sequence b:
+    x[b*T + u] @ W[:, g*dh:(g+1)*dh], as in kv_proj."""
+    s = inp.shape
+    dh = s.d_head
+    Wg = np.concatenate([W_k[:, g * dh:(g + 1) * dh], W_v[:, g * dh:(g + 1) * dh]], axis=1)
+    out = np.empty((hi, 2 * dh))
+    for lo in range(0, hi, _ROW_BLOCK):
+        up = min(hi, lo + _ROW_BLOCK)
+        out[lo:up] = bf16_to_f64(inp.x[b * s.T + lo:b * s.T + up]) @ Wg
+    return out[:, :dh], out[:, dh:]
+
+
+def gqe_layer(inp: LayerInputs, rows=None, with_dispatch: bool = True,
+              full_kv: bool = True, mode: str = "gqe") -> dict:
     """GQE prefill forward (a1-a11).
 
+    ``mode`` selects the output construction (OUTPUT_MODES; "gqe" is the
+    layer); inp.W_o must then have mode_slots(mode, G, k) * d_head rows.
+
     ``rows`` (optional) is a list of global row indices b*T+t at which the
-    attention, slots and y are evaluated; router, dispatch, K and V are always
-    computed in full. Without ``rows`` every output is computed in full.
+    queries, attention, slots and y are evaluated; the router and dispatch
+    are always computed in full. Without ``rows`` every output is computed in
+    full. ``full_kv`` returns K and V for every row ([B, G, T, dh]);
+    otherwise only at the evaluated rows (``K_rows``, ``V_rows`` [n, G, dh]),
+    and each group's K/V is built only as far as the evaluated rows of a
+    sequence reach (long sequences).
     """
     s: LayerShape = inp.shape
     B, T, G, M, k, dh = s.B, s.T, s.G, s.M, s.k, s.d_head
-    f = _f64_inputs(inp)
-    rt = router(f["x"], f["W_r"], f["b_r"], G, M, k)
+    f = _f64_weights(inp)
+    rt = _router_by_rows(inp, f)
     out = dict(rt)
     if with_dispatch:
         out.update(dispatch(rt["idx"], B, T, G, M))
-    K = kv_proj(f["x"], f["W_k"], B, T, G, dh)
-    V = kv_proj(f["x"], f["W_v"], B, T, G, dh)
-    out["K"], out["V"] = K, V
     idx = rt["idx"]
     R = B * T
     sel_rows = np.arange(R) if rows is None else np.asarray(rows, np.int64)
+    if full_kv:
+        x_all = bf16_to_f64(inp.x)
+        K = kv_proj(x_all, f["W_k"], B, T, G, dh)
+        V = kv_proj(x_all, f["W_v"], B, T, G, dh)
+        out["K"], out["V"] = K, V
 
-    # Queries (only for the evaluated rows when sampling; same definition).
-    x_sel = f["x"][sel_rows]
-    idx_sel = idx[sel_rows]
-    n = sel_rows.size
-    q_r = np.zeros((n, G, k, dh))
-    for g in range(G):
-        for j in range(M):
-            e = g * M + j
-            We = f["W_q"][:, e * dh:(e + 1) * dh]
-            for si in range(k):
-                m = idx_sel[:, g, si] == j
-                if m.any():
-                    q_r[m, g, si] = x_sel[m] @ We
-    q_s = x_sel @ f["W_qs"]
+    # Queries of the evaluated rows (a7): routed experts and the shared head.
+    x_sel = bf16_to_f64(inp.x[sel_rows])
+    q_r = q_routed_rows(x_sel, f["W_q"], idx[sel_rows], G, M, dh)
+    q_s = q_shared(x_sel, f["W_qs"], 1, sel_rows.size, dh)[0]
     if rows is None:
         out["Qv"] = q_r.reshape(B, T, G, k, dh).transpose(0, 2, 3, 1, 4).copy()
         out["Qs"] = q_s.reshape(B, T, dh)
 
+    # a8-a9: causal attention of each evaluated row against its group's K/V.
+    n = sel_rows.size
     o_r = np.zeros((n, G, k, dh))
     o_s = np.zeros((n, dh))
-    for b in range(B):
+    if not full_kv:
+        out["K_rows"] = np.zeros((n, G, dh))
+        out["V_rows"] = np.zeros((n, G, dh))
+    def attend(b, g):
+        # Every evaluated row of sequence b, for every head on group g.
         m = (sel_rows // T) == b
-        if not m.any():
-            continue
         pos = sel_rows[m] % T
-        for g in range(G):
-            for si in range(k):
-                o_r[m, g, si] = causal_attention(q_r[m, g, si], K[b, g], V[b, g], rows=pos)
-        o_s[m] = causal_attention(q_s[m], K[b, 0], V[b, 0], rows=pos)
-    slots = assemble_slots(o_r, o_s, rt["omega"][sel_rows])
+        if full_kv:
+            Kg, Vg = K[b, g], V[b, g]
+        else:
+            Kg, Vg = _kv_group_prefix(inp, f["W_k"], f["W_v"], b, g, int(pos.max()) + 1)
+            out["K_rows"][m, g] = Kg[pos]
+            out["V_rows"][m, g] = Vg[pos]
+        for si in range(k):
+            o_r[m, g, si] = causal_attention(q_r[m, g, si], Kg, Vg, rows=pos)
+        if g == 0:  # the shared head attends to KV group 0 (reading R1)
+            o_s[m] = causal_attention(q_s[m], Kg, Vg, rows=pos)
+
+    work = [(b, g) for b in range(B) if ((sel_rows // T) == b).any() for g in range(G)]
+    if full_kv:
+        for b, g in work:
+            attend(b, g)
+    else:
+        # Groups are independent: several at a time (numpy's kernels release
+        # the GIL); each writes only its own outputs.
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=4) as ex:
+            list(ex.map(lambda bg: attend(*bg), work))
+    rt_rows = {key: rt[key][sel_rows] for key in ("omega", "r", "p", "idx")}
+    slots = assemble_slots(o_r, o_s if mode_has_shared_head(mode) else None, rt_rows, mode)
+    assert f["W_o"].shape[0] == slots.shape[1], "W_o rows do not match the output mode"
     out["slots"] = slots
     out["y"] = output_proj(slots, f["W_o"])
     out["rows"] = sel_rows
@@ -431,7 +576,7 @@ def gqe_decode_step(x_new: np.ndarray, K_cache: np.ndarray, V_cache: np.ndarray,
     q_s = x_new @ W_qs
     o_s = np.stack([_decode_attention(q_s[b], K_cache[b, 0], V_cache[b, 0], k_new[b, 0], v_new[b, 0])
                     for b in range(B)])
-    slots = assemble_slots(o_r, o_s, rt["omega"])
+    slots = assemble_slots(o_r, o_s, rt)
     out = dict(rt)
     out.update(k_new=k_new, v_new=v_new, slots=slots, y=output_proj(slots, W_o))
     return out

@@ -29,6 +29,7 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
 
 import numpy as np
 
@@ -52,9 +53,17 @@ STREAM_BR = 9
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
-    z = (z ^ (z >> np.uint64(30))) * _M1
-    z = (z ^ (z >> np.uint64(27))) * _M2
-    return z ^ (z >> np.uint64(31))
+    """splitmix64 finaliser, applied in place (z is overwritten and returned)."""
+    t = np.empty_like(z)
+    np.right_shift(z, np.uint64(30), out=t)
+    np.bitwise_xor(z, t, out=z)
+    np.multiply(z, _M1, out=z)
+    np.right_shift(z, np.uint64(27), out=t)
+    np.bitwise_xor(z, t, out=z)
+    np.multiply(z, _M2, out=z)
+    np.right_shift(z, np.uint64(31), out=t)
+    np.bitwise_xor(z, t, out=z)
+    return z
 
 
 def uniform_bits(seed: int, stream: int, n: int, start: int = 0) -> np.ndarray:
@@ -62,8 +71,10 @@ def uniform_bits(seed: int, stream: int, n: int, start: int = 0) -> np.ndarray:
     with np.errstate(over="ignore"):
         key = _mix(np.array([(seed ^ (stream * 0xD1B54A32D192ED03)) & 0xFFFFFFFFFFFFFFFF],
                             dtype=np.uint64))[0]
-        ctr = np.arange(start + 1, start + n + 1, dtype=np.uint64)
-        return _mix(key + ctr * _GOLDEN)
+        z = np.arange(start + 1, start + n + 1, dtype=np.uint64)
+        np.multiply(z, _GOLDEN, out=z)
+        np.add(z, key, out=z)
+        return _mix(z)
 
 
 def normal_f64(seed: int, stream: int, n: int, start: int = 0) -> np.ndarray:
@@ -85,7 +96,7 @@ def normal_f64(seed: int, stream: int, n: int, start: int = 0) -> np.ndarray:
     return out[:n]
 
 
-_CHUNK = 1 << 24
+_CHUNK = 1 << 22
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -95,10 +106,20 @@ def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     return rounded.astype(np.uint16)
 
 
+def _bf16_table() -> np.ndarray:
+    b = np.arange(65536, dtype=np.uint32) << np.uint32(16)
+    with np.errstate(invalid="ignore"):
+        return b.view(np.float32).astype(np.float64)
+
+
+_BF16_F64 = _bf16_table()
+
+
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
-    """Exact widening of bf16 bit patterns to fp64."""
-    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
-    return b.view(np.float32).astype(np.float64)
+    """Exact widening of bf16 bit patterns to fp64 (a bf16 value is the fp32
+    value whose upper 16 bits are the pattern; a 65536-entry table holds every
+    one of them widened)."""
+    return np.take(_BF16_F64, np.ascontiguousarray(bits, dtype=np.uint16))
 
 
 def bf16_bits_from_f64(a: np.ndarray) -> np.ndarray:
@@ -107,11 +128,25 @@ def bf16_bits_from_f64(a: np.ndarray) -> np.ndarray:
 
 
 def normal_bf16(seed: int, stream: int, shape, std: float = 1.0) -> np.ndarray:
+    """bf16 bits of N(0, std^2) draws 0..n-1 of a stream. Large tensors are
+    drawn in chunks on several threads (numpy releases the GIL in its
+    element-wise kernels); every element depends only on its index, so the
+    bits do not depend on the chunking."""
     n = int(np.prod(shape))
     out = np.empty(n, dtype=np.uint16)
-    for s in range(0, n, _CHUNK):
+
+    def fill(s):
         m = min(_CHUNK, n - s)
         out[s:s + m] = bf16_bits_from_f64(normal_f64(seed, stream, m, s) * std)
+
+    starts = range(0, n, _CHUNK)
+    if n <= _CHUNK:
+        for s in starts:
+            fill(s)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, starts))
     return out.reshape(shape)
 
 

@@ -163,6 +163,67 @@ def test_router_exact_tie_through_reordered_sum():
     assert (rt2["idx"][:, 0, 0] == (0 if z0 > z1 else 1)).all()
 
 
+def _bf16_value(v: float) -> float:
+    return float(bf16_to_f64(synth.f32_to_bf16_bits(np.array([v], dtype=np.float32)))[0])
+
+
+def _sub_ulp_pair(seed: int, tiny: float):
+    """Two router columns equal except one entry one fp32 ulp apart, and an x
+    row whose entry on that row is `tiny`: the exact logits differ by
+    tiny * ulp, far below one fp64 ulp of the logits themselves."""
+    rng = np.random.default_rng(seed)
+    d = 1024
+    w0 = (rng.standard_normal(d) / 32).astype(np.float32)
+    i0 = int(rng.integers(d))
+    w1 = w0.copy()
+    w1[i0] = np.nextafter(w0[i0], np.float32(np.inf))
+    x = bf16_to_f64(synth.f32_to_bf16_bits(rng.standard_normal(d).astype(np.float32)))
+    x[i0] = _bf16_value(tiny)
+    return x, np.stack([w0, w1], axis=1).astype(np.float64), i0
+
+
+@pytest.mark.parametrize("sign", [1.0, -1.0])
+def test_router_sub_ulp_difference_decided_exactly(sign):
+    # z_1 - z_0 = x[i0] * ulp(w0[i0]): about 2^-88, so the correctly rounded
+    # logits are equal and only the exact values order them. x[i0] > 0 makes
+    # expert 1 the larger (selected although it has the higher index);
+    # x[i0] < 0 makes expert 0 the larger.
+    x, W, i0 = _sub_ulp_pair(17, sign * 2.0 ** -60)
+    assert math.fsum(x * W[:, 0]) == math.fsum(x * W[:, 1])  # rounding alone cannot decide
+    rt = oracle.router(x[None, :], W, None, 1, 2, 1)
+    assert rt["idx"][0, 0, 0] == (1 if sign > 0 else 0)
+
+
+def test_router_exact_selection_matches_rational_arithmetic():
+    # Independent exact method: Fraction sums of the same terms. Near-tied
+    # groups of 4 experts (columns one ulp apart at one row, the x entry there
+    # between 2^-70 and 2^-10), k = 2; the oracle's selection must be the one
+    # the rational logits give (largest first, ties to the lower index).
+    from fractions import Fraction
+    rng = np.random.default_rng(41)
+    d, M, k = 256, 4, 2
+    for case in range(24):
+        w = (rng.standard_normal(d) / 16).astype(np.float32)
+        cols = []
+        rows_hit = rng.choice(d, size=M, replace=False)
+        for j in range(M):
+            c = w.copy()
+            steps = int(rng.integers(-1, 2))  # -1, 0 or +1 ulp at this column's row
+            for _ in range(abs(steps)):
+                c[rows_hit[j]] = np.nextafter(c[rows_hit[j]], np.float32(np.inf * steps))
+            cols.append(c)
+        W = np.stack(cols, axis=1).astype(np.float64)
+        x = bf16_to_f64(synth.f32_to_bf16_bits(rng.standard_normal(d).astype(np.float32)))
+        for r in rows_hit:
+            x[r] = _bf16_value(float(rng.choice([-1.0, 1.0])) * 2.0 ** -float(rng.integers(10, 71)))
+        b = np.zeros(M)
+        rt = oracle.router(x[None, :], W, b, 1, M, k)
+        zq = [sum((Fraction(float(xi)) * Fraction(float(wi)) for xi, wi in zip(x, W[:, j])), Fraction(0))
+              for j in range(M)]
+        want = sorted(sorted(range(M), key=lambda j: (-zq[j], j))[:k])
+        assert rt["idx"][0, 0].tolist() == want, (case, zq)
+
+
 def test_router_skew_bias_gives_80_percent():
     # Bias beta on expert 0 of each group: P(hot expert in top-k) = 0.80 for
     # iid N(0,1) logits (the load-skew workload).
@@ -423,6 +484,27 @@ def test_sampled_rows_equal_full_layer():
     np.testing.assert_allclose(part["slots"], full["slots"][rows], rtol=0, atol=1e-14)
 
 
+def test_row_blocked_sampled_layer_equals_full_layer(monkeypatch):
+    # The long-sequence evaluation (x widened 5 rows at a time, each group's
+    # K/V built only up to the last evaluated position) gives the full layer's
+    # values at the evaluated rows: router, lists, K/V, slots and y.
+    s = LayerShape(B=2, T=23, d_model=64, G=3, M=3, k=2, d_head=8)
+    inp = synth.make_layer_inputs(s, seed=44, skew=False)
+    full = oracle.gqe_layer(inp)
+    monkeypatch.setattr(oracle, "_ROW_BLOCK", 5)
+    rows = np.array([0, 4, 5, 11, 23, 27, 45])
+    part = oracle.gqe_layer(inp, rows=rows, full_kv=False)
+    for key in ("idx", "counts", "offsets", "tok", "slot_pos"):
+        assert np.array_equal(part[key], full[key]), key
+    for key in ("r", "omega", "p", "z"):
+        np.testing.assert_allclose(part[key], full[key], rtol=0, atol=1e-14)
+    b, t = rows // s.T, rows % s.T
+    np.testing.assert_allclose(part["K_rows"], full["K"][b, :, t], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(part["V_rows"], full["V"][b, :, t], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(part["slots"], full["slots"][rows], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(part["y"], full["y"][rows], rtol=0, atol=1e-13)
+
+
 def test_published_setting_counts():
     g = _golden("published_setting.json")
     ms = g["main_setting"]
@@ -480,3 +562,96 @@ def test_decode_step_with_an_empty_cache_returns_the_new_values():
                                        v_new[:, g], rtol=0, atol=1e-13)
     np.testing.assert_allclose(d["slots"][:, G * k * dh:(G * k + 1) * dh], v_new[:, 0], rtol=0,
                                atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# output constructions (the layer and the ablation variants)
+# --------------------------------------------------------------------------
+
+def _with_mode_wo(inp, mode):
+    """The instance with W_o cut to the mode's slot rows (the first ones)."""
+    import dataclasses
+    s = inp.shape
+    rows = oracle.mode_slots(mode, s.G, s.k) * s.d_head
+    return dataclasses.replace(inp, W_o=inp.W_o[:rows].copy())
+
+
+def test_hard_concat_with_k_equal_m_is_dense_gqa():
+    # k = M selects every expert of every group in ascending order, so the hard
+    # concatenation is the dense heads in head order; with W_O_dense = W_o it
+    # is the dense GQA layer.
+    s = LayerShape(B=2, T=9, d_model=32, G=2, M=3, k=3, d_head=8)
+    inp = _with_mode_wo(synth.make_layer_inputs(s, seed=90), "hard")
+    import dataclasses
+    dense = oracle.gqa_dense_layer(dataclasses.replace(inp, W_o_dense=inp.W_o))
+    hard = oracle.gqe_layer(inp, mode="hard")
+    np.testing.assert_allclose(hard["slots"], dense["O"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(hard["y"], dense["y"], rtol=0, atol=1e-12)
+
+
+def test_weighted_concat_uniform_router_scales_by_one_over_m():
+    # W_r = 0, no bias: every in-group probability is 1/M, so each selected
+    # output is scaled by 1/M; with k = M that is the dense layer over M.
+    s = LayerShape(B=1, T=11, d_model=32, G=2, M=2, k=2, d_head=8)
+    import dataclasses
+    inp = _with_mode_wo(synth.make_layer_inputs(s, seed=91), "weighted_concat")
+    inp = dataclasses.replace(inp, W_r=np.zeros_like(inp.W_r))
+    dense = oracle.gqa_dense_layer(dataclasses.replace(inp, W_o_dense=inp.W_o))
+    wc = oracle.gqe_layer(inp, mode="weighted_concat")
+    np.testing.assert_allclose(wc["y"], dense["y"] / s.M, rtol=0, atol=1e-13)
+
+
+def test_weighted_concat_hand_probabilities():
+    # Bias ln 3 on expert 0 of each group, W_r = 0: p = (3/4, 1/4), expert 0 is
+    # selected with weight 3/4 (k = 1).
+    s = LayerShape(B=1, T=7, d_model=32, G=3, M=2, k=1, d_head=8)
+    import dataclasses
+    base = synth.make_layer_inputs(s, seed=92)
+    b = np.zeros(s.N, dtype=np.float32)
+    b[0::2] = np.float32(math.log(3.0))
+    inp = dataclasses.replace(base, W_r=np.zeros_like(base.W_r), b_r=b)
+    hard = oracle.gqe_layer(_with_mode_wo(inp, "hard"), mode="hard")
+    wc = oracle.gqe_layer(_with_mode_wo(inp, "weighted_concat"), mode="weighted_concat")
+    assert (wc["idx"] == 0).all()
+    p0 = 3.0 / 4.0  # the fp32 bias ln 3 moves p by ~1e-8 only
+    np.testing.assert_allclose(wc["slots"], p0 * hard["slots"], rtol=1e-7, atol=1e-12)
+
+
+def test_group_mean_slot_with_k1_is_mean_of_routed_outputs():
+    # k = 1: r = 1 for every selection, so the slot is the mean of the G routed
+    # outputs whatever the router does.
+    s = LayerShape(B=2, T=10, d_model=32, G=4, M=3, k=1, d_head=8)
+    inp = synth.make_layer_inputs(s, seed=93)
+    gm = oracle.gqe_layer(inp, mode="group_mean")
+    dh, G = s.d_head, s.G
+    routed = gm["slots"][:, :G * dh].reshape(-1, G, dh)
+    np.testing.assert_allclose(gm["slots"][:, (G + 1) * dh:], routed.mean(axis=1), rtol=0, atol=1e-14)
+
+
+def test_group_mean_slot_hand_weights_k2():
+    # p proportional to (5, 3, 2, 1) in every group (bias ln of those, W_r = 0):
+    # the top 2 are experts 0 and 1 with r = (5/8, 3/8).
+    s = LayerShape(B=1, T=6, d_model=32, G=2, M=4, k=2, d_head=8)
+    import dataclasses
+    base = synth.make_layer_inputs(s, seed=94)
+    b = np.tile(np.log(np.array([5.0, 3.0, 2.0, 1.0])), s.G).astype(np.float32)
+    inp = dataclasses.replace(base, W_r=np.zeros_like(base.W_r), b_r=b)
+    gm = oracle.gqe_layer(inp, mode="group_mean")
+    assert (gm["idx"] == np.array([0, 1])).all()
+    dh, G, k = s.d_head, s.G, s.k
+    o = gm["slots"][:, :G * k * dh].reshape(-1, G, k, dh)
+    want = (5 / 8 * o[:, :, 0] + 3 / 8 * o[:, :, 1]).mean(axis=1)
+    np.testing.assert_allclose(gm["slots"][:, (G * k + 1) * dh:], want, rtol=1e-7, atol=1e-12)
+
+
+def test_group_mean_equals_layer_slot_under_uniform_router():
+    # With equal selected mass in every group (W_r = 0), omega = r / G, so the
+    # layer's weighted slot and the group mean coincide; the other slots are
+    # the same in both constructions.
+    s = LayerShape(B=1, T=8, d_model=32, G=3, M=3, k=2, d_head=8)
+    import dataclasses
+    base = synth.make_layer_inputs(s, seed=95)
+    inp = dataclasses.replace(base, W_r=np.zeros_like(base.W_r))
+    a = oracle.gqe_layer(inp)
+    b = oracle.gqe_layer(inp, mode="group_mean")
+    np.testing.assert_allclose(a["slots"], b["slots"], rtol=0, atol=1e-14)
