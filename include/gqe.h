@@ -52,7 +52,7 @@ typedef struct gqe_config {
   int32_t M;       /* query-head experts per group; N = G*M <= 64 */
   int32_t k;       /* experts selected per group per token, 1 <= k <= M */
   int32_t d_head;  /* head dim: 32 or 64 */
-  uint32_t flags;  /* 0 or GQE_FLAG_WS_CLEAN; other bits must be 0 */
+  uint32_t flags;  /* GQE_FLAG_* bits below; other bits must be 0 */
 } gqe_config;
 
 /* gqe_attention_fwd, gqe_layer_fwd, gqa_dense_fwd: the caller promises that
@@ -68,6 +68,38 @@ typedef struct gqe_config {
  * (gqe_layer_fwd) then runs gqe_attention_fwd_compact. Results are the same;
  * only the layout of Qv and the attention's tiling differ. */
 #define GQE_FLAG_EXPERT_MAJOR 2u
+
+/* Output construction (at most one of the three; none = the GQE layer). The
+ * layer builds S slots per token from its routed outputs o[g, s]:
+ *   default      S = kG+2: o[g, s] (hard concatenation), the shared head,
+ *                and the weighted slot sum_{g,s} omega[g, s] o[g, s] with
+ *                omega = p / (selected p of all groups);
+ *   GROUP_MEAN   S = kG+2, as the default but omega = r / G: each group's
+ *                selected outputs renormalised inside the group, the groups
+ *                averaged (the other reading of the weighted slot);
+ *   OUT_HARD     S = kG: the routed outputs only -- no weighted slot, no
+ *                shared head ("hard concatenation only": pptc.cn blog, section
+ *                4.3 and Table 1);
+ *   OUT_WEIGHTED_CONCAT
+ *                S = kG: p[g, s] * o[g, s] with p the in-group softmax
+ *                probability -- no weighted slot, no shared head ("weighted
+ *                concatenation without the renormalised slot": same section).
+ * The flag changes what gqe_router_topk writes to omega (the weights the
+ * output uses), the slot buffer ([B*T, S*d_head]), W_o ([S*d_head, d_model])
+ * and, for the last two, drops the shared head (Qs may be NULL). The decode
+ * step supports the default construction only. */
+#define GQE_FLAG_SLOT_GROUP_MEAN 4u
+#define GQE_FLAG_OUT_HARD 8u
+#define GQE_FLAG_OUT_WEIGHTED_CONCAT 16u
+
+/* A shard of the layer split over KV groups: the same construction without
+ * the shared head, S = kG+1 (routed slots, then the weighted slot); combines
+ * with the default or GROUP_MEAN. Each rank of a split runs its groups (G =
+ * its group count, W_q/W_k/W_v columns and W_o rows of those groups) on the
+ * routing of the whole layer; the rank holding group 0 keeps the shared head
+ * (no flag), the others set this one, and the partial y of the ranks sum to
+ * the layer's y (the weighted slot enters W_O linearly). */
+#define GQE_FLAG_NO_SHARED_HEAD 32u
 
 typedef enum gqe_status {
   GQE_OK = 0,
@@ -101,7 +133,9 @@ enum {
  * at least 256 otherwise). */
 size_t gqe_workspace_bytes(const gqe_config* cfg, int which);
 
-/* Byte offset of `item` inside workspace `which`, or (size_t)-1. */
+/* Byte offset of `item` inside workspace `which`, or (size_t)-1. Items of
+ * GQE_WS_LAYER: all above; of GQE_WS_DENSE: DENSE_Q, K, V, DENSE_O; of
+ * GQE_WS_DECODE (one row per sequence): IDX, R, OMEGA, SLOTS. */
 size_t gqe_workspace_offset(const gqe_config* cfg, int which, int item);
 
 /*
@@ -113,12 +147,17 @@ size_t gqe_workspace_offset(const gqe_config* cfg, int which, int item);
  *
  *   z[row, e]  = sum_i x[row, i] * W_r[i, e] + b_r[e]      (fp32, with a
  *                certified error bound; a top-k decision whose margin is
- *                below the bound is re-taken from fp64 logits, so idx is the
- *                exact-arithmetic selection)
+ *                below the bound is re-taken from fp64 logits under their
+ *                own certified bound, and one that bound does not settle
+ *                either from the exact logits (integer sums of the exact
+ *                products), so idx is the exact-arithmetic selection, ties
+ *                included)
  *   p          = softmax over the M logits of each group
  *   idx[row, g, s] = the k largest j of group g, ascending, ties to lower j
  *   r[row, g, s]     = p / sum of the selected p of group g
- *   omega[row, g, s] = p / sum of the selected p of all G groups
+ *   omega[row, g, s] = p / sum of the selected p of all G groups (the
+ *                      weighted slot's weights; with GQE_FLAG_SLOT_GROUP_MEAN
+ *                      r / G, with GQE_FLAG_OUT_WEIGHTED_CONCAT p itself)
  *
  * x [B*T, d_model] bf16; W_r [d_model, N] fp32; b_r [N] fp32 or NULL;
  * idx [B*T, G, k] int32; r, omega [B*T, G, k] fp32.
@@ -144,7 +183,8 @@ gqe_status gqe_router_topk(const gqe_config* cfg, const gqe_bf16* x, const float
  * idx [B*T, G, k] int32 (from gqe_router_topk); x [B*T, d_model];
  * W_q [d_model, N*d_head]; W_qs [d_model, d_head]; counts [N*B];
  * offsets [N*B + 1]; tok [k*G*B*T]; slot_pos [B*T, G, k];
- * Qv [B, G, k, T, d_head]; Qs [B, T, d_head].
+ * Qv [B, G, k, T, d_head]; Qs [B, T, d_head] (NULL allowed, and not
+ * written, when the output construction has no shared head).
  * ws: >= gqe_workspace_bytes(cfg, GQE_WS_DISPATCH) bytes.
  */
 gqe_status gqe_dispatch(const gqe_config* cfg, const int32_t* idx, const gqe_bf16* x,
@@ -161,7 +201,9 @@ gqe_status gqe_dispatch(const gqe_config* cfg, const int32_t* idx, const gqe_bf1
  * lives in a 4 MiB static device array of the library (held by every GPU that
  * loads it, until exit); arguments and results are those of gqe_dispatch.
  *  - The first call on a device looks up the array's address on that device;
- *    make it before any stream capture.
+ *    make it before any stream capture. The address is kept for the life of
+ *    the process: do not use this entry point after cudaDeviceReset (or any
+ *    other teardown of the device's primary context) in the same process.
  *  - All calls on a device share the array: calls that overlap on the GPU
  *    race. Each call writes every scratch word before reading it.
  *  - Configurations needing more than 4 MiB of dispatch scratch
@@ -195,8 +237,9 @@ gqe_status gqe_kv_proj(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16*
  * GQE_WS_ATTENTION). Calls sharing one ws must not overlap on the GPU. The
  * call clears the scratch's arrival counters first unless cfg->flags has
  * GQE_FLAG_WS_CLEAN.
- * Qv [B, G, k, T, d_head]; Qs [B, T, d_head]; K, V [B, G, T, d_head];
- * slots [B*T, (k*G+2)*d_head].
+ * Qv [B, G, k, T, d_head]; Qs [B, T, d_head] (unused, NULL allowed, when
+ * the output construction has no shared head); K, V [B, G, T, d_head];
+ * slots [B*T, S*d_head] (S of the output construction: kG+2 by default).
  */
 gqe_status gqe_attention_fwd(const gqe_config* cfg, const gqe_bf16* Qv, const gqe_bf16* Qs,
                              const gqe_bf16* K, const gqe_bf16* V, gqe_bf16* slots, void* ws,
@@ -234,6 +277,10 @@ gqe_status gqe_attention_fwd_compact(const gqe_config* cfg, const gqe_bf16* Qe, 
  *   y = slots @ W_o
  * slots [B*T, (k*G+2)*d_head] (updated in place); omega [B*T, G, k] fp32;
  * W_o [(k*G+2)*d_head, d_model]; y [B*T, d_model].
+ * With GQE_FLAG_OUT_HARD: y = slots @ W_o over the kG routed slots
+ * (slots [B*T, kG*d_head], W_o [kG*d_head, d_model]); with
+ * GQE_FLAG_OUT_WEIGHTED_CONCAT each routed slot is first scaled in place by
+ * omega (= its in-group probability, rounded to bf16 once).
  */
 gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* omega,
                            const gqe_bf16* W_o, gqe_bf16* y, gqe_stream_t stream);

@@ -27,6 +27,10 @@ GQE_ERR_CUDA, GQE_ERR_TIMEOUT, GQE_ERR_DEVICE_CHECK = 4, 5, 6
 GQE_WS_DISPATCH, GQE_WS_LAYER, GQE_WS_DENSE, GQE_WS_ATTENTION = 1, 2, 3, 4
 GQE_WS_DECODE, GQE_WS_DENSE_DECODE = 5, 6
 GQE_FLAG_WS_CLEAN, GQE_FLAG_EXPERT_MAJOR = 1, 2
+# Output constructions (at most one): see include/gqe.h.
+GQE_FLAG_SLOT_GROUP_MEAN, GQE_FLAG_OUT_HARD, GQE_FLAG_OUT_WEIGHTED_CONCAT = 4, 8, 16
+OUTPUT_MODE_FLAGS = {"gqe": 0, "group_mean": GQE_FLAG_SLOT_GROUP_MEAN, "hard": GQE_FLAG_OUT_HARD,
+                     "weighted_concat": GQE_FLAG_OUT_WEIGHTED_CONCAT}
 ITEMS = {"idx": 1, "r": 2, "omega": 3, "counts": 4, "offsets": 5, "tok": 6, "slot_pos": 7,
          "Qv": 8, "Qs": 9, "K": 10, "V": 11, "slots": 12, "dispatch_ws": 13, "attention_ws": 14,
          "dense_Q": 32, "dense_O": 33}

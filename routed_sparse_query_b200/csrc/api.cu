@@ -27,7 +27,14 @@ bool all_aligned(const P*... ps) {
 gqe_status check_cfg(const gqe_config* c) {
   if (c == nullptr) return GQE_ERR_INVALID;
   if (c->B < 1 || c->T < 1 || c->G < 1 || c->M < 1 || c->k < 1 || c->k > c->M) return GQE_ERR_INVALID;
-  if (c->d_model < 64 || c->d_model % 64 != 0 || (c->flags & ~(GQE_FLAG_WS_CLEAN | GQE_FLAG_EXPERT_MAJOR)) != 0u) return GQE_ERR_INVALID;
+  if (c->d_model < 64 || c->d_model % 64 != 0 ||
+      (c->flags & ~(GQE_FLAG_WS_CLEAN | GQE_FLAG_EXPERT_MAJOR | kOutFlags | GQE_FLAG_NO_SHARED_HEAD)) != 0u)
+    return GQE_ERR_INVALID;
+  const uint32_t out = c->flags & kOutFlags;
+  if ((out & (out - 1u)) != 0u) return GQE_ERR_INVALID;  // at most one output construction
+  // A shard without the shared head keeps the weighted slot.
+  if ((c->flags & GQE_FLAG_NO_SHARED_HEAD) && (out & (GQE_FLAG_OUT_HARD | GQE_FLAG_OUT_WEIGHTED_CONCAT)))
+    return GQE_ERR_INVALID;
   if (c->G * c->M > kMaxExperts || c->G > 32) return GQE_ERR_UNSUPPORTED;
   if (c->d_head != 32 && c->d_head != 64) return GQE_ERR_UNSUPPORTED;
   // Index arithmetic of the kernels stays within int32 for these extents.
@@ -68,9 +75,9 @@ LayerWs layer_ws(const gqe_config& c) {
   put(L.Qs, R * dh * 2);
   put(L.K, R * c.G * dh * 2);
   put(L.V, R * c.G * dh * 2);
-  put(L.slots, R * (c.G * c.k + 2) * dh * 2);
+  put(L.slots, R * n_slots(c) * dh * 2);
   put(L.dws, dispatch_ws_layout(c).total);
-  put(L.aws, attention_plan(c, c.G * c.k + 1).total);
+  put(L.aws, attention_plan(c, n_streams(c)).total);
   L.total = o;
   return L;
 }
@@ -206,7 +213,8 @@ size_t gqe_workspace_bytes(const gqe_config* cfg, int which) {
     // Decode: the per-token buffers have B rows; T is the cache length.
     gqe_config c1 = decode_rows_cfg(*cfg);
     if (which == GQE_WS_DENSE_DECODE) c1.k = 1;
-    if (cfg->T < 1 || check_cfg(&c1) != GQE_OK) return 0;
+    if (cfg->T < 1 || check_cfg(&c1) != GQE_OK || (cfg->flags & (kOutFlags | GQE_FLAG_NO_SHARED_HEAD)) != 0u)
+      return 0;
     if (which == GQE_WS_DECODE) return decode_heads(*cfg, false) > 16 ? 0 : decode_ws(*cfg).total;
     gqe_config cd = *cfg;
     cd.k = 1;
@@ -218,7 +226,7 @@ size_t gqe_workspace_bytes(const gqe_config* cfg, int which) {
     case GQE_WS_LAYER: return layer_ws(*cfg).total;
     case GQE_WS_DENSE: return dense_ws(*cfg).total;
     case GQE_WS_ATTENTION: {
-      const size_t t = attention_plan(*cfg, cfg->G * cfg->k + 1).total;
+      const size_t t = attention_plan(*cfg, n_streams(*cfg)).total;
       return t > 256 ? t : 256;
     }
     default: return 0;
@@ -227,6 +235,18 @@ size_t gqe_workspace_bytes(const gqe_config* cfg, int which) {
 
 size_t gqe_workspace_offset(const gqe_config* cfg, int which, int item) {
   const size_t bad = static_cast<size_t>(-1);
+  if (cfg != nullptr && which == GQE_WS_DECODE) {
+    // The decode step's per-token buffers (one row per sequence).
+    if (gqe_workspace_bytes(cfg, GQE_WS_DECODE) == 0) return bad;
+    const LayerWs& L = decode_ws(*cfg).L1;
+    switch (item) {
+      case GQE_ITEM_IDX: return L.idx;
+      case GQE_ITEM_R: return L.r;
+      case GQE_ITEM_OMEGA: return L.omega;
+      case GQE_ITEM_SLOTS: return L.slots;
+      default: return bad;
+    }
+  }
   if (check_cfg(cfg) != GQE_OK) return bad;
   if (which == GQE_WS_LAYER) {
     const LayerWs L = layer_ws(*cfg);
@@ -277,11 +297,12 @@ gqe_status gqe_dispatch(const gqe_config* cfg, const int32_t* idx, const gqe_bf1
                         gqe_bf16* Qs, void* ws, size_t ws_bytes, gqe_stream_t stream) {
   const gqe_status s = check_cfg(cfg);
   if (s != GQE_OK) return s;
-  if (!all_aligned(idx, x, W_q, W_qs, counts, offsets, tok, slot_pos, Qv, Qs) || ws == nullptr ||
-      !aligned16(ws))
+  const bool shared = has_shared_head(*cfg);
+  if (!all_aligned(idx, x, W_q, counts, offsets, tok, slot_pos, Qv) || ws == nullptr || !aligned16(ws) ||
+      (shared && !all_aligned(W_qs, Qs)))
     return GQE_ERR_INVALID;
-  return dispatch_and_project(*cfg, idx, x, W_q, W_qs, counts, offsets, tok, slot_pos, Qv, Qs, ws,
-                              ws_bytes, stream);
+  return dispatch_and_project(*cfg, idx, x, W_q, W_qs, counts, offsets, tok, slot_pos, Qv,
+                              shared ? Qs : nullptr, ws, ws_bytes, stream);
 }
 
 gqe_status gqe_kv_proj(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16* W_k,
@@ -297,8 +318,8 @@ gqe_status gqe_attention_fwd(const gqe_config* cfg, const gqe_bf16* Qv, const gq
                              size_t ws_bytes, gqe_stream_t stream) {
   const gqe_status s = check_cfg(cfg);
   if (s != GQE_OK) return s;
-  if (!all_aligned(Qv, Qs, K, V, slots)) return GQE_ERR_INVALID;
-  const size_t need = attention_plan(*cfg, cfg->G * cfg->k + 1).total;
+  if (!all_aligned(Qv, K, V, slots) || (has_shared_head(*cfg) && !all_aligned(Qs))) return GQE_ERR_INVALID;
+  const size_t need = attention_plan(*cfg, n_streams(*cfg)).total;
   if (need > 0 && (ws == nullptr || !aligned16(ws))) return GQE_ERR_INVALID;
   if (ws_bytes < need) return GQE_ERR_WORKSPACE;
   const bool clean = (cfg->flags & GQE_FLAG_WS_CLEAN) != 0u;
@@ -311,7 +332,8 @@ gqe_status gqe_attention_fwd_compact(const gqe_config* cfg, const gqe_bf16* Qe, 
                                      gqe_stream_t stream) {
   const gqe_status s = check_cfg(cfg);
   if (s != GQE_OK) return s;
-  if (!all_aligned(Qe, Qs, K, V, idx, offsets, tok, slots)) return GQE_ERR_INVALID;
+  if (!all_aligned(Qe, K, V, idx, offsets, tok, slots) || (has_shared_head(*cfg) && !all_aligned(Qs)))
+    return GQE_ERR_INVALID;
   return cuda_status(attention_gqe_em(*cfg, Qe, Qs, K, V, idx, offsets, tok, slots, stream));
 }
 
@@ -329,7 +351,9 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
                          gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream_t stream) {
   const gqe_status s = check_cfg(cfg);
   if (s != GQE_OK) return s;
-  if (!all_aligned(x, W_r, W_q, W_qs, W_k, W_v, W_o, y) || ws == nullptr || !aligned16(ws))
+  const bool shared = has_shared_head(*cfg);
+  if (!all_aligned(x, W_r, W_q, W_k, W_v, W_o, y) || ws == nullptr || !aligned16(ws) ||
+      (shared && !all_aligned(W_qs)))
     return GQE_ERR_INVALID;
   const LayerWs L = layer_ws(*cfg);
   if (ws_bytes < L.total) return GQE_ERR_WORKSPACE;
@@ -341,7 +365,7 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
   // they are), so that the kernels of the layer follow each other directly
   // (programmatic dependent launch).
   if ((cfg->flags & (GQE_FLAG_WS_CLEAN | GQE_FLAG_EXPERT_MAJOR)) == 0u &&
-      zero_attention_counters(*cfg, cfg->G * cfg->k + 1, w + L.aws, stream) != cudaSuccess)
+      zero_attention_counters(*cfg, n_streams(*cfg), w + L.aws, stream) != cudaSuccess)
     return GQE_ERR_CUDA;
   // K/V projection on the side stream (falls back to the caller's stream).
   cudaStream_t main_st = static_cast<cudaStream_t>(stream);
@@ -360,7 +384,8 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
     // routed tiles.
     const gqe_status kv = gqe_kv_proj(cfg, x, W_k, W_v, H(L.K), H(L.V), side ? side->s : stream);
     if (kv != GQE_OK) return kv;
-    if (gemm_q_shared(*cfg, x, W_qs, H(L.Qs), side ? side->s : stream) != cudaSuccess) return GQE_ERR_CUDA;
+    if (shared && gemm_q_shared(*cfg, x, W_qs, H(L.Qs), side ? side->s : stream) != cudaSuccess)
+      return GQE_ERR_CUDA;
     if (side != nullptr && cudaEventRecord(side->join, side->s) != cudaSuccess) return GQE_ERR_CUDA;
     st = dispatch_and_project(*cfg, I(L.idx), x, W_q, W_qs, I(L.counts), I(L.offsets), I(L.tok),
                               I(L.slot_pos), H(L.Qv), nullptr, w + L.dws, L.total - L.dws, stream);
@@ -457,6 +482,8 @@ gqe_status gqe_decode_step(const gqe_config* cfg, const gqe_bf16* x, const float
   const gqe_config c1 = decode_rows_cfg(*cfg);
   const gqe_status s = check_cfg(&c1);  // B rows; the long extent is the cache
   if (s != GQE_OK) return s;
+  if ((cfg->flags & (kOutFlags | GQE_FLAG_NO_SHARED_HEAD)) != 0u)
+    return GQE_ERR_UNSUPPORTED;  // default construction only
   if (cache_capacity < cfg->T) return GQE_ERR_INVALID;
   if (!all_aligned(x, W_r, W_q, W_qs, W_k, W_v, W_o, K_cache, V_cache, y) || ws == nullptr ||
       !aligned16(ws))

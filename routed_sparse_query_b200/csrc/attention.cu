@@ -799,7 +799,7 @@ int run_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const ui
   const long long rows = R * c.G * c.k;  // routed query rows, in list order
   CUtensorMap tq, tqs, tk, tv;
   if (!make_tmap_bf16_3d(&tq, Qe, dh, static_cast<uint64_t>(rows), 1, dh, BQ)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16_3d(&tqs, Qs, dh, c.T, c.B, dh, BQ)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_3d(&tqs, Qs ? Qs : Qe, dh, c.T, c.B, dh, BQ)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_3d(&tk, K, dh, c.T, static_cast<uint64_t>(c.B) * c.G, dh, BKV))
     return cudaErrorInvalidValue;
   if (!make_tmap_bf16_3d(&tv, V, dh, c.T, static_cast<uint64_t>(c.B) * c.G, dh, BKV))
@@ -807,7 +807,7 @@ int run_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const ui
   AttnParams p{};
   p.T = c.T;
   p.B = c.B;
-  p.H = c.G * c.k + 1;
+  p.H = n_streams(c);
   p.G = c.G;
   p.k = c.k;
   p.M = c.M;
@@ -817,7 +817,7 @@ int run_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const ui
   p.chunk = p.n_qt;  // no split
   p.items = p.n_pairs;
   p.out = slots;
-  p.ldo = (c.G * c.k + 2) * dh;
+  p.ldo = n_slots(c) * dh;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(dh)));
   p.em = 1;
   p.N = c.G * c.M;
@@ -827,7 +827,8 @@ int run_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const ui
   p.offsets = offsets;
   p.tok = tok;
   p.idx = idx;
-  const long long grid = static_cast<long long>(p.em_units) + static_cast<long long>(p.n_pairs) * c.B;
+  const long long grid =
+      static_cast<long long>(p.em_units) + (has_shared_head(c) ? static_cast<long long>(p.n_pairs) * c.B : 0);
   if (dh == 64) return launch_attn<64>(tq, tqs, tk, tv, p, grid, stream);
   return launch_attn<32>(tq, tqs, tk, tv, p, grid, stream);
 }
@@ -874,9 +875,8 @@ AttnPlan attention_plan(const gqe_config& c, int H) {
 int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
                   const uint16_t* V, uint16_t* slots, void* ws, size_t ws_bytes,
                   bool counters_zeroed, void* stream) {
-  const int H = c.G * c.k + 1;
-  return run(c, Qv, static_cast<uint64_t>(c.B) * c.G * c.k, Qs, K, V, slots,
-             (c.G * c.k + 2) * c.d_head, H, 0, ws, ws_bytes, counters_zeroed, stream);
+  return run(c, Qv, static_cast<uint64_t>(c.B) * c.G * c.k, Qs, K, V, slots, n_slots(c) * c.d_head,
+             n_streams(c), 0, ws, ws_bytes, counters_zeroed, stream);
 }
 
 int attention_gqe_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const uint16_t* K,

@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(kThreads) scan_scatter_kernel(ListArgs a) {
 
 // Weighted slot: one thread per 8 columns of one row.
 __global__ void __launch_bounds__(256) weighted_slot_kernel(uint16_t* slots, const float* omega,
-                                                            int R, int G, int k, int dh) {
+                                                            int R, int G, int k, int dh, int S) {
   pdl_wait();
   pdl_launch_dependents();
   const int per_row = dh / 8;
@@ -324,7 +324,7 @@ __global__ void __launch_bounds__(256) weighted_slot_kernel(uint16_t* slots, con
   if (gid >= static_cast<long long>(R) * per_row) return;
   const int row = static_cast<int>(gid / per_row);
   const int c8 = static_cast<int>(gid % per_row);
-  const int ld = (k * G + 2) * dh;
+  const int ld = S * dh;  // the weighted slot is the last of the S slots
   uint16_t* base = slots + static_cast<size_t>(row) * ld + c8 * 8;
   const float* w = omega + static_cast<size_t>(row) * G * k;
   float acc[8];
@@ -345,7 +345,28 @@ __global__ void __launch_bounds__(256) weighted_slot_kernel(uint16_t* slots, con
   o.y = pack_bf16x2(acc[2], acc[3]);
   o.z = pack_bf16x2(acc[4], acc[5]);
   o.w = pack_bf16x2(acc[6], acc[7]);
-  *reinterpret_cast<uint4*>(base + (k * G + 1) * dh) = o;
+  *reinterpret_cast<uint4*>(base + (S - 1) * dh) = o;
+}
+
+// Weighted concatenation: slots[row, gs*dh + c] *= omega[row, gs] (routed
+// slots only; one thread per 8 columns, one bf16 rounding of the product).
+__global__ void __launch_bounds__(256) scale_slots_kernel(uint16_t* slots, const float* omega, int R,
+                                                          int gk, int dh, int ld) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int per_row = gk * dh / 8;
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gid >= static_cast<long long>(R) * per_row) return;
+  const int row = static_cast<int>(gid / per_row);
+  const int c8 = static_cast<int>(gid % per_row);
+  uint16_t* p = slots + static_cast<size_t>(row) * ld + c8 * 8;
+  const float w = omega[static_cast<size_t>(row) * gk + (c8 * 8) / dh];
+  uint4 v = *reinterpret_cast<const uint4*>(p);
+  uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    u[i] = pack_bf16x2(w * __uint_as_float(u[i] << 16), w * __uint_as_float(u[i] & 0xffff0000u));
+  *reinterpret_cast<uint4*>(p) = make_uint4(u[0], u[1], u[2], u[3]);
 }
 
 }  // namespace dispatch_impl
@@ -412,7 +433,20 @@ int launch_weighted_slot(const gqe_config& c, uint16_t* slots, const float* omeg
   const long long n = R * (c.d_head / 8);
   const int grid = static_cast<int>((n + 255) / 256);
   return launch_pdl(weighted_slot_kernel, dim3(grid), dim3(256), 0, stream, slots, omega,
-                    static_cast<int>(R), c.G, c.k, c.d_head);
+                    static_cast<int>(R), c.G, c.k, c.d_head, n_slots(c));
+}
+
+}  // namespace gqe
+
+namespace gqe {
+
+int launch_scale_slots(const gqe_config& c, uint16_t* slots, const float* omega, void* stream) {
+  const long long R = static_cast<long long>(c.B) * c.T;
+  const int gk = c.G * c.k;
+  const long long n = R * gk * c.d_head / 8;
+  const int grid = static_cast<int>((n + 255) / 256);
+  return launch_pdl(scale_slots_kernel, dim3(grid), dim3(256), 0, stream, slots, omega,
+                    static_cast<int>(R), gk, c.d_head, n_slots(c) * c.d_head);
 }
 
 }  // namespace gqe

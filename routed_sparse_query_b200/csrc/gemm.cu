@@ -469,7 +469,14 @@ int gemm_output(const gqe_config& c, uint16_t* slots, const float* omega, const 
                 uint16_t* y, void* stream) {
   const int R = c.B * c.T;
   const int gk = c.G * c.k;
-  const int K = (gk + 2) * c.d_head;
+  const int K = n_slots(c) * c.d_head;
+  if (!has_weighted_slot(c)) {  // ablation constructions: the kG routed slots only
+    if (c.flags & GQE_FLAG_OUT_WEIGHTED_CONCAT) {
+      const int e = launch_scale_slots(c, slots, omega, stream);
+      if (e != cudaSuccess) return e;
+    }
+    return gemm_rowmajor(slots, R, K, W_o, c.d_model, y, stream);
+  }
   if (c.d_head != BK) {  // the weighted slot is not one K block: separate kernel
     const int e = launch_weighted_slot(c, slots, omega, stream);
     if (e != cudaSuccess) return e;
@@ -484,7 +491,7 @@ int gemm_output(const gqe_config& c, uint16_t* slots, const float* omega, const 
   e.st = c.d_model;
   e.rows = R;
   e.cols = c.d_model;
-  e.kb_w = gk + 1;
+  e.kb_w = n_slots(c) - 1;  // the weighted slot is the last one
   e.gk = gk;
   e.omega = omega;
   e.wslots = slots;

@@ -25,6 +25,26 @@ __host__ __device__ constexpr int router_np(int N) {
 }
 constexpr size_t kRouterSmemLimit = 200 * 1024;
 
+// Output construction (gqe.h, GQE_FLAG_OUT_* / GQE_FLAG_SLOT_GROUP_MEAN):
+// whether the layer has the shared head, its query streams (kG routed, plus
+// the shared head) and its slots per token (plus the weighted slot).
+constexpr uint32_t kOutFlags = GQE_FLAG_SLOT_GROUP_MEAN | GQE_FLAG_OUT_HARD | GQE_FLAG_OUT_WEIGHTED_CONCAT;
+inline bool has_weighted_slot(const gqe_config& c) {
+  return (c.flags & (GQE_FLAG_OUT_HARD | GQE_FLAG_OUT_WEIGHTED_CONCAT)) == 0u;
+}
+inline bool has_shared_head(const gqe_config& c) {
+  return has_weighted_slot(c) && (c.flags & GQE_FLAG_NO_SHARED_HEAD) == 0u;
+}
+inline int n_streams(const gqe_config& c) { return c.G * c.k + (has_shared_head(c) ? 1 : 0); }
+inline int n_slots(const gqe_config& c) {
+  return c.G * c.k + (has_shared_head(c) ? 1 : 0) + (has_weighted_slot(c) ? 1 : 0);
+}
+// What gqe_router_topk writes to omega: 0 = p over all selected, 1 = r / G,
+// 2 = p (the in-group probability).
+inline int omega_mode(const gqe_config& c) {
+  return (c.flags & GQE_FLAG_SLOT_GROUP_MEAN) ? 1 : (c.flags & GQE_FLAG_OUT_WEIGHTED_CONCAT) ? 2 : 0;
+}
+
 // Dispatch tiling: tokens of one sequence are cut into tiles of this size.
 constexpr int kDispatchTile = 256;  // == dispatch CTA size: one token per thread
 constexpr int kQTileRows = 128;  // rows of one grouped-GEMM tile
@@ -86,6 +106,8 @@ int launch_dispatch_lists(const gqe_config& c, const int32_t* idx, int32_t* coun
                           int32_t* offsets, int32_t* tok, int32_t* slot_pos, void* ws,
                           const DispatchWs& L, void* stream);
 int launch_weighted_slot(const gqe_config& c, uint16_t* slots, const float* omega, void* stream);
+// Weighted concatenation: routed slot (g, s) of every row times omega[row, g, s].
+int launch_scale_slots(const gqe_config& c, uint16_t* slots, const float* omega, void* stream);
 
 // GEMM front ends (tcgen05). out layouts are described in gemm.cu.
 int gemm_kv(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,

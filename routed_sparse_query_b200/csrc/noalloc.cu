@@ -15,7 +15,11 @@
 // Properties a caller must know:
 //  - The first call on a device looks up the array's device address on that
 //    device (cudaGetSymbolAddress, with the device current) and caches it;
-//    make that first call before any stream capture.
+//    make that first call before any stream capture. The cached address
+//    belongs to that device's context: do not call this entry point again
+//    after cudaDeviceReset (or any teardown of the primary context) in the
+//    same process, since the library's module, and the array with it, may
+//    then sit at another address.
 //  - Every call on a device shares the one array, which keeps the last call's
 //    contents. Each call writes every scratch word before reading it, so
 //    nothing needs clearing, but calls that overlap on the GPU (different

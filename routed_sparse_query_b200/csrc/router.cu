@@ -25,8 +25,14 @@
 // "Accuracy and Stability of Numerical Algorithms", 2nd ed., sec. 3.1). A
 // group whose top-k decision is not certain under these intervals (computed
 // with directed rounding) recomputes its logits in fp64 (products of a bf16
-// and an fp32 value are exact in fp64) and decides on those, so the selection
-// equals the exact-arithmetic one.
+// and an fp32 value are exact in fp64), and the fp64 decision is certified
+// the same way with its own path length and u = 2^-53. A group that even
+// the fp64 intervals do not settle (exact ties, or logits closer than about
+// 1e-15 of their size) is decided on the exact logits: every product is an
+// integer multiple of 2^-282, so the sum is accumulated exactly as a
+// 576-bit integer in 32-bit limbs (kept in 64-bit words so that no carry is
+// lost) and compared exactly. The selection therefore equals the
+// exact-arithmetic one in every case.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -61,6 +67,7 @@ struct RouterArgs {
   float* r;
   float* omega;
   int R, d, G, M, k, N;
+  int wmode;  // omega: 0 = p / selected p of all groups, 1 = r / G, 2 = p
 };
 
 // Uncertain groups per round of the fp64 fallback.
@@ -135,6 +142,115 @@ __device__ __forceinline__ float group_softmax(const V* zg, int M, uint64_t sel,
   return psel;
 }
 
+// Exact logits. A bf16 value is m * 2^(E' - 134) with an 8-bit integer m
+// and E' = max(E, 1) (E its biased exponent); an fp32 value is m * 2^(E' -
+// 150) with a 24-bit m. A product is therefore a 32-bit integer times 2^p,
+// p + 282 in [0, 508], and the bias a 24-bit integer times 2^p, p + 282 in
+// [133, 386]. W_r sits in shared memory, so d < 2^15, and the sum of d + 1
+// terms stays below 2^556 (in units of 2^-282): 18 limbs of 32 bits hold it,
+// the top one signed. The limbs are 64-bit words and each receives fewer
+// than 2^16 additions below 2^32, so nothing overflows before the carries
+// are propagated.
+constexpr int kExactLimbs = 18;
+
+// Adds sign * m * 2^bitpos (m < 2^32) to the shared limbs.
+__device__ __forceinline__ void exact_add(long long* limbs, uint32_t m, int bitpos, bool neg) {
+  const unsigned long long v = static_cast<unsigned long long>(m) << (bitpos & 31);
+  const int l = bitpos >> 5;
+  const unsigned long long lo = v & 0xffffffffull, hi = v >> 32;
+  auto* u = reinterpret_cast<unsigned long long*>(limbs);
+  if (lo) atomicAdd(u + l, neg ? 0ull - lo : lo);
+  if (hi) atomicAdd(u + l + 1, neg ? 0ull - hi : hi);
+}
+
+__device__ __forceinline__ void exact_add_product(long long* limbs, uint16_t xb, float w) {
+  const uint32_t wb = __float_as_uint(w);
+  const int ex = (xb >> 7) & 0xff, ew = (wb >> 23) & 0xff;
+  const uint32_t mx = ex ? (0x80u | (xb & 0x7fu)) : (xb & 0x7fu);
+  const uint32_t mw = ew ? (0x800000u | (wb & 0x7fffffu)) : (wb & 0x7fffffu);
+  const uint32_t m = mx * mw;
+  if (m == 0u) return;
+  // exponent (max(ex,1) - 134) + (max(ew,1) - 150), offset by +282
+  exact_add(limbs, m, (ex ? ex : 1) + (ew ? ew : 1) - 2, ((xb >> 15) ^ (wb >> 31)) & 1u);
+}
+
+__device__ __forceinline__ void exact_add_bias(long long* limbs, float b) {
+  const uint32_t bb = __float_as_uint(b);
+  const int eb = (bb >> 23) & 0xff;
+  const uint32_t m = eb ? (0x800000u | (bb & 0x7fffffu)) : (bb & 0x7fffffu);
+  if (m == 0u) return;
+  exact_add(limbs, m, (eb ? eb : 1) - 150 + 282, (bb >> 31) & 1u);
+}
+
+// Carries the limbs so that limbs 0..16 lie in [0, 2^32) and limb 17 holds
+// the signed rest: one canonical form per value.
+__device__ __forceinline__ void exact_normalize(long long* limbs) {
+  for (int l = 0; l + 1 < kExactLimbs; ++l) {
+    const long long c = limbs[l] >> 32;  // floor division by 2^32
+    limbs[l] -= c * 4294967296ll;
+    limbs[l + 1] += c;
+  }
+}
+
+// a > b for canonical limbs.
+__device__ __forceinline__ bool exact_greater(const long long* a, const long long* b) {
+  if (a[kExactLimbs - 1] != b[kExactLimbs - 1]) return a[kExactLimbs - 1] > b[kExactLimbs - 1];
+  for (int l = kExactLimbs - 2; l >= 0; --l)
+    if (a[l] != b[l]) return a[l] > b[l];
+  return false;
+}
+
+// Exact decisions of the ne pairs in list (exact ties and logits closer
+// than the fp64 bound only), one pair at a time; every thread of the CTA
+// calls it. The k selections are taken one by one: each pass computes the
+// exact logit of every unselected expert (the whole CTA adds the products
+// into shared limbs, cur) and keeps the largest (best), the lower index on
+// equality. Out of line: the rare path stays out of the main loop's
+// register allocation.
+__device__ __noinline__ void exact_decide(const uint16_t* x, int d, int G, int M, int k, const float* Ws,
+                                          int NP, const float* bsm, long long* cur, const int* list,
+                                          int ne, int row0, const double* zd, float* ez, float* dn,
+                                          float* ps, uint64_t* selp, unsigned long long* sel_sh,
+                                          int* best_sh) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  long long* best = cur + kExactLimbs;
+  for (int v = 0; v < ne; ++v) {
+    const int pv = list[v];
+    const int tv = pv / G, gv = pv - tv * G;
+    const uint16_t* xr = x + static_cast<size_t>(row0 + tv) * d;
+    if (tid == 0) *sel_sh = 0ull;
+    __syncthreads();
+    for (int s = 0; s < k; ++s) {
+      if (tid == 0) *best_sh = -1;
+      for (int j = 0; j < M; ++j) {
+        if ((*sel_sh >> j) & 1ull) continue;  // uniform (shared, set before a barrier)
+        const int e = gv * M + j;
+        if (tid < kExactLimbs) cur[tid] = 0;
+        __syncthreads();
+        for (int i = tid; i < d; i += nthr) exact_add_product(cur, __ldg(xr + i), Ws[i * NP + e]);
+        if (tid == 0) exact_add_bias(cur, bsm[e]);
+        __syncthreads();
+        if (tid == 0) {
+          exact_normalize(cur);
+          if (*best_sh < 0 || exact_greater(cur, best)) {
+            for (int l = 0; l < kExactLimbs; ++l) best[l] = cur[l];
+            *best_sh = j;
+          }
+        }
+        __syncthreads();
+      }
+      if (tid == 0) *sel_sh |= 1ull << *best_sh;
+      __syncthreads();
+    }
+    if (tid == 0) {
+      const int zo = tv * NP + gv * M;
+      ps[pv] = group_softmax(zd + zo, M, *sel_sh, ez + zo, dn + pv);
+      selp[pv] = *sel_sh;
+    }
+    __syncthreads();
+  }
+}
+
 template <int NP, int WARPS, int TPT>
 __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
   constexpr int THREADS = WARPS * 32;
@@ -143,7 +259,8 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
   constexpr int TG = 32 / EG;  // token lanes per warp; TB == TPT * TG
   static_assert(TB == TPT * TG, "block shape");
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  __shared__ int n_uncertain;
+  __shared__ int n_uncertain, n_exact, exact_best;
+  __shared__ unsigned long long exact_sel;
   const RouterLayout L = router_layout(a.d, NP, TPT);
   float* Ws = reinterpret_cast<float*>(smem_raw + L.w);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw + L.xs);
@@ -235,6 +352,11 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
   const float gam_ru = __fmul_ru(gam, 1.01f);
   const int slice = a.d / WARPS;
   const int P = TB * a.G;  // (token, group) pairs of a block
+  // fp64 fix-up path: slice/8 FMAs into each of two accumulators, their sum,
+  // two shuffle adds, W adds of the warp sums, the bias.
+  const int h64 = slice / 8 + WARPS + 4;
+  const double u64 = 1.1102230246251565e-16;  // 2^-53
+  const double gam64_ru = __dmul_ru((h64 * u64) / (1.0 - h64 * u64), 1.01);
 
   for (; blk < n_blk; blk += gridDim.x) {
     cp_async_wait<0>();
@@ -392,15 +514,43 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
         }
         __syncthreads();
       }
+      // fp64 decisions, certified by the fp64 bound (directed rounding; the
+      // 1 % in gam64_ru covers the fp32 rounding of ||x||_1). A pair that
+      // stays uncertain is marked with an empty selection.
       for (int v = tid; v < nu; v += THREADS) {
         const int pv = list[v];
         const int tv = pv / a.G, gv = pv - tv * a.G;
         const int zo = tv * NP + gv * a.M;
         const uint64_t sel = group_topk(zd + zo, a.M, a.k);
-        ps[pv] = group_softmax(zd + zo, a.M, sel, ez + zo, dn + pv);
-        selp[pv] = sel;
+        bool certain = true;
+        if (a.k < a.M) {
+          const double nx = static_cast<double>(nxs[tv]);
+          double lo = INFINITY, hi = -INFINITY;
+          for (int j = 0; j < a.M; ++j) {
+            const int e = gv * a.M + j;
+            const double bd =
+                __dmul_ru(gam64_ru, __fma_ru(nx, static_cast<double>(wmax[e]), fabs(static_cast<double>(bsm[e]))));
+            if ((sel >> j) & 1ull) lo = fmin(lo, __dsub_rd(zd[zo + j], bd));
+            else hi = fmax(hi, __dadd_ru(zd[zo + j], bd));
+          }
+          certain = lo > hi;
+        }
+        if (certain) ps[pv] = group_softmax(zd + zo, a.M, sel, ez + zo, dn + pv);
+        selp[pv] = certain ? sel : 0ull;
       }
       __syncthreads();
+      // Pairs left undecided, compacted in place (one thread).
+      if (tid == 0) {
+        int ne = 0;
+        for (int v = 0; v < nu; ++v)
+          if (selp[list[v]] == 0ull) list[ne++] = list[v];
+        n_exact = ne;
+      }
+      __syncthreads();
+      const int ne = n_exact;  // uniform: the call below holds barriers
+      if (ne > 0)
+        exact_decide(a.x, a.d, a.G, a.M, a.k, Ws, NP, bsm, reinterpret_cast<long long*>(smem_raw + L.fb),
+                     list, ne, blk * TB, zd, ez, dn, ps, selp, &exact_sel, &exact_best);
     }
     // idx, r (renormalised in the group) and omega (over the token's groups).
     for (int p = tid; p < P; p += THREADS) {
@@ -418,7 +568,7 @@ __global__ void __launch_bounds__(WARPS * 32) router_kernel(RouterArgs a) {
           const float pj = ez[zo + j] / den;
           a.idx[o + s] = j;
           a.r[o + s] = pj / psel;
-          a.omega[o + s] = pj / tot;
+          a.omega[o + s] = a.wmode == 0 ? pj / tot : a.wmode == 1 ? (pj / psel) / a.G : pj;
           ++s;
         }
       }
@@ -440,13 +590,16 @@ int launch_tpt(const gqe_config& c, const RouterArgs& a, cudaStream_t st) {
   if (smem > kRouterSmemLimit) return cudaErrorInvalidConfiguration;
   const int e = ensure_smem<router_kernel<NP, WARPS, TPT>>(static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  static std::atomic<int> per_sm{0};
-  int ps = per_sm.load(std::memory_order_relaxed);
+  // Resident CTAs per SM, looked up once per device (devices may differ).
+  static std::atomic<int> per_sm[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = -1;
+  int ps = dev >= 0 ? per_sm[dev].load(std::memory_order_relaxed) : 0;
   if (ps <= 0) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ps, router_kernel<NP, WARPS, TPT>, WARPS * 32,
                                                       smem) != cudaSuccess || ps < 1)
       ps = 1;
-    per_sm.store(ps, std::memory_order_relaxed);
+    if (dev >= 0) per_sm[dev].store(ps, std::memory_order_relaxed);
   }
   // One token block per CTA while that fills the GPU; larger batches loop.
   const int n_blk = (a.R + router_tb(NP, TPT) - 1) / router_tb(NP, TPT);
@@ -486,7 +639,7 @@ size_t router_smem_bytes(const gqe_config& c) {
 
 int launch_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r,
                   int32_t* idx, float* r, float* omega, void* stream) {
-  RouterArgs a{x, W_r, b_r, idx, r, omega, c.B * c.T, c.d_model, c.G, c.M, c.k, c.G * c.M};
+  RouterArgs a{x, W_r, b_r, idx, r, omega, c.B * c.T, c.d_model, c.G, c.M, c.k, c.G * c.M, omega_mode(c)};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (router_np(a.N)) {
     case 4: return launch_w<4>(c, a, st);
