@@ -421,25 +421,45 @@ def roofline_of(shape, per_call_ms: dict, steps: int, pk: dict, traffic=None):
             "avg_launch_ms": avg_s * 1e3}
 
 
+def router_bytes(s: synth.LayerShape) -> float:
+    """Algorithmic HBM bytes of the router: x read once, W_r, idx/r/omega written."""
+    return s.R * s.d_model * 2 + s.d_model * s.N * 4 + s.R * s.G * s.k * 12
+
+
+def call_fractions(s: synth.LayerShape, per_call_ms: dict, steps: int, pk: dict) -> dict:
+    """Each entry point's achieved rate against its roofline (of the measured
+    peaks): the router on HBM bytes; the K/V and W_O GEMMs, the dispatch call
+    (token-list kernels plus the grouped Q GEMM, FLOPs of the Q GEMM) and the
+    attention on bf16 tensor FLOPs (burst peak: each is timed alone)."""
+    fl = flops(s)
+    t = {c: per_call_ms[c] / steps / 1e3 for c in per_call_ms}
+    out = {"router_hbm_frac": router_bytes(s) / t["router"] / 1e9 / pk["hbm"]}
+    for call, key in (("kv", "kv"), ("output", "wo"), ("dispatch", "q"), ("attention", "attention")):
+        out[f"{call}_tensor_frac"] = fl[key] / t[call] / 1e12 / pk["bf16"]
+    return {k: round(v, 4) for k, v in out.items()}
+
+
 def cpu_baseline(shape: synth.LayerShape, max_tokens: int | None = None,
-                 min_seconds: float = 0.0) -> dict:
+                 min_seconds: float = 0.0, threads: int | None = None) -> dict:
     """The oracle as it stands, on this host: full layer passes over one
-    sequence (the first max_tokens tokens), repeated until min_seconds."""
+    sequence (the first max_tokens tokens), repeated until min_seconds.
+    `threads` limits the BLAS thread pool (None: as many as it has)."""
     import oracle
-    from threadpoolctl import threadpool_info
+    from threadpoolctl import threadpool_info, threadpool_limits
     T = shape.T if max_tokens is None else min(shape.T, max_tokens)
     s = synth.LayerShape(1, T, shape.d_model, shape.G, shape.M, shape.k, shape.d_head)
     inp = synth.make_layer_inputs(s, with_dense=False)
-    passes, dt = 0, 0.0
-    t0 = time.perf_counter()
-    while passes == 0 or (dt < min_seconds and passes < 1000):
-        oracle.gqe_layer(inp)
-        passes += 1
-        dt = time.perf_counter() - t0
-    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    with threadpool_limits(limits=threads):
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        passes, dt = 0, 0.0
+        t0 = time.perf_counter()
+        while passes == 0 or (dt < min_seconds and passes < 1000):
+            oracle.gqe_layer(inp)
+            passes += 1
+            dt = time.perf_counter() - t0
     return {"value": T * passes / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"{passes} full oracle layer passes over {T} tokens of one sequence "
-                      f"(fp64 numpy, {dt:.2f} s)", "seconds": dt / passes}
+                      f"(fp64 numpy, {dt:.2f} s, {cores} BLAS threads)", "seconds": dt / passes}
 
 
 def max_over_ranks(value: float, dist, device) -> float:
@@ -454,6 +474,29 @@ def max_over_ranks(value: float, dist, device) -> float:
 def job_throughput(tokens_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
     """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
     return tokens_per_rank_step * world * steps / (max_ms / 1e3)
+
+
+def summary_of(out: dict) -> dict:
+    """Short per-workload table (the last key of the line): T, B, GQE and
+    dense layer ms, speed-up, attention fraction of the bf16 peak, and the
+    other calls' fractions of their rooflines."""
+    def r4(v):
+        return None if v is None else round(float(v), 4)
+
+    rows = [{"workload": out["config"]["workload"].split(":")[0], "gqe_ms": r4(out["ms_per_step"]),
+             "dense_ms": r4(out["dense_gqa"]["ms_per_step"]),
+             "speedup": r4(out["dense_gqa"]["speedup_gqe_over_dense"]),
+             "attn_frac": r4(out["roofline"]["frac"]), **out.get("fractions", {})}]
+    for row in out.get("sweep", []):
+        rows.append({"workload": row["workload"].split(":")[0], "gqe_ms": r4(row["gqe_ms"]),
+                     "dense_ms": r4(row["dense_ms"]), "speedup": r4(row["speedup"]),
+                     "attn_frac": r4(row["attn_frac_of_bf16_peak"]), **row.get("fractions", {})})
+    for row in out.get("pool_sweep", []):
+        rows.append({"workload": row["workload"].split(":")[0], "gqe_ms": r4(row["gqe_ms"]),
+                     "dense_ms": r4(row["dense_ms"]), "speedup": r4(row["speedup"]),
+                     "attn_frac": r4(row["attn_frac_of_bf16_peak"]),
+                     "hot_expert_share": r4(row["hot_expert_share"]), **row.get("fractions", {})})
+    return {"per_workload": rows, "peaks": "fractions of the measured peaks (bf16 burst, HBM copy)"}
 
 
 def run_ours(args, rank: int, world: int, dist):
@@ -522,6 +565,7 @@ def run_ours(args, rank: int, world: int, dist):
                 "cuda_graph_stages": e2e["graph"]},
         "roofline": roof,
         "breakdown_ms_per_step": {c: v / args.steps for c, v in res["per_call_ms"].items()},
+        "fractions": call_fractions(shape, res["per_call_ms"], args.steps, pk),
         "breakdown_note": "per entry point, timed call by call in a second loop of the same steps",
         "dense_gqa": {"ms_per_step": dense_ms,
                       "tokens_per_s": shape.R * world / (dense_ms / 1e3),
@@ -531,10 +575,14 @@ def run_ours(args, rank: int, world: int, dist):
     if world == 1 and not args.no_sweep:
         out["sweep"] = sweep(rsq, pk, args)
         out["decode"] = decode_bench(rsq, pk, args.steps)
-    if world == 1 and args.sweep_pool:
+    if world == 1 and not args.no_pool:
         out["pool_sweep"] = sweep_pool(rsq, pk, args)
     if world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(shape, min_seconds=10.0)
+        one = cpu_baseline(shape, min_seconds=5.0, threads=1)
+        out["cpu_baseline"]["one_core"] = {k: one[k] for k in ("value", "unit", "cores", "sample")}
+        out["cpu_baseline"]["host_cores"] = os.cpu_count()
+    out["summary"] = summary_of(out)
     return out
 
 
@@ -608,7 +656,8 @@ def sweep(rsq, pk, args):
                      "attn_expert_major_ms": em_s * 1e3,
                      "attn_expert_major_frac_of_bf16_peak": flops(s)["attention"] / em_s / 1e12 / pk["bf16"],
                      "l2": "inputs larger than L2, not flushed",
-                     "breakdown_ms": {c: v / steps for c, v in res["per_call_ms"].items()}})
+                     "breakdown_ms": {c: v / steps for c, v in res["per_call_ms"].items()},
+                     "fractions": call_fractions(s, res["per_call_ms"], steps, pk)})
         if rsq.gqe_read_status() != 0:
             raise RuntimeError(f"device-side status set in sweep {name}")
         del layer, d
@@ -645,7 +694,8 @@ def sweep_pool(rsq, pk, args):
                      "speedup": dense_ms / gq_ms,
                      "hot_expert_share": float(counts[:, 0].sum()) / (s.G * s.R),
                      "attn_tflops": ach, "attn_frac_of_bf16_peak": ach / pk["bf16"],
-                     "breakdown_ms": {c: v / steps for c, v in res["per_call_ms"].items()}})
+                     "breakdown_ms": {c: v / steps for c, v in res["per_call_ms"].items()},
+                     "fractions": call_fractions(s, res["per_call_ms"], steps, pk)})
         if rsq.gqe_read_status() != 0:
             raise RuntimeError(f"device-side status set in pool sweep {name}")
         del layer, d
@@ -697,8 +747,8 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--sweep-max", choices=SWEEP, default=None)
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--sweep-pool", action="store_true",
-                    help="also time the expert-pool workloads (32 experts, k = 1, 2; skewed, balanced)")
+    ap.add_argument("--no-pool", action="store_true",
+                    help="skip the expert-pool workloads (32 experts, k = 1, 2; skewed, balanced)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -21,7 +21,8 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().double().numpy()
 
 
-def assert_close(got: torch.Tensor, want: np.ndarray, what: str, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
+def assert_close(got: torch.Tensor, want: np.ndarray, what: str, max_abs=MAX_ABS, mean_abs=MEAN_ABS,
+                 allow_scale: bool = False):
     """Max-abs / mean-abs check against the oracle.
 
     The bounds hold as stated for outputs of rms <= 1/2, which covers every
@@ -29,10 +30,13 @@ def assert_close(got: torch.Tensor, want: np.ndarray, what: str, max_abs=MAX_ABS
     Each bf16 rounding on the path (Q, K, V, P, slots, y) is relative to the
     value rounded (unit roundoff 2^-8 ~ 3.9e-3), so for larger outputs -- a
     sequence of a few tokens, where o is a single V row and |y| ~ 1 -- both
-    bounds scale with 2 * rms(want).
+    bounds scale with 2 * rms(want). Only sequences shorter than one 128-row
+    tile may use that scaling (allow_scale); everywhere else the bounds are
+    the stated ones and the check fails if the outputs are larger.
     """
     g = to_f64(got).reshape(want.shape)
     scale = max(1.0, 2.0 * float(np.sqrt(np.mean(np.square(want)))) if want.size else 1.0)
+    assert allow_scale or scale == 1.0, f"{what}: rms(want) above 1/2 outside the short-sequence cases"
     max_abs, mean_abs = max_abs * scale, mean_abs * scale
     err = np.abs(g - want)
     assert np.isfinite(g).all(), f"{what}: non-finite values"
@@ -53,9 +57,17 @@ def device_inputs(inp: synth.LayerInputs) -> dict:
     return d
 
 
-def run_steps(rsq, shape: synth.LayerShape, d: dict) -> dict:
+def n_slots(shape: synth.LayerShape, flags: int = 0) -> int:
+    """Slots per token of the output construction chosen by `flags`."""
+    import routed_sparse_query_b200 as rsq
+    no_shared = flags & (rsq.GQE_FLAG_OUT_HARD | rsq.GQE_FLAG_OUT_WEIGHTED_CONCAT)
+    return shape.k * shape.G + (0 if no_shared else 2)
+
+
+def run_steps(rsq, shape: synth.LayerShape, d: dict, flags: int = 0) -> dict:
     """GQE layer through the five step entry points; returns every output."""
-    cfg = rsq.GQEConfig.of(shape)
+    cfg = rsq.GQEConfig.of(shape, flags)
+    S = n_slots(shape, flags)
     B, T, G, M, k, dh = shape.B, shape.T, shape.G, shape.M, shape.k, shape.d_head
     R, N = B * T, G * M
     dev = torch.device("cuda")
@@ -69,7 +81,7 @@ def run_steps(rsq, shape: synth.LayerShape, d: dict) -> dict:
     o["tok"] = torch.empty(k * G * R, dtype=torch.int32, device=dev)
     o["slot_pos"] = torch.empty(R, G, k, dtype=torch.int32, device=dev)
     o["Qv"] = torch.empty(B, G, k, T, dh, dtype=torch.bfloat16, device=dev)
-    o["Qs"] = torch.empty(B, T, dh, dtype=torch.bfloat16, device=dev)
+    o["Qs"] = torch.empty(B, T, dh, dtype=torch.bfloat16, device=dev) if S == k * G + 2 else None
     ws = torch.empty(max(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_DISPATCH), 16), dtype=torch.uint8,
                      device=dev)
     rsq.gqe_dispatch(cfg, o["idx"], d["x"], d["W_q"], d["W_qs"], o["counts"], o["offsets"],
@@ -77,7 +89,7 @@ def run_steps(rsq, shape: synth.LayerShape, d: dict) -> dict:
     o["K"] = torch.empty(B, G, T, dh, dtype=torch.bfloat16, device=dev)
     o["V"] = torch.empty(B, G, T, dh, dtype=torch.bfloat16, device=dev)
     rsq.gqe_kv_proj(cfg, d["x"], d["W_k"], d["W_v"], o["K"], o["V"])
-    o["slots"] = torch.zeros(R, (k * G + 2) * dh, dtype=torch.bfloat16, device=dev)
+    o["slots"] = torch.zeros(R, S * dh, dtype=torch.bfloat16, device=dev)
     wsa = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_ATTENTION), dtype=torch.uint8, device=dev)
     rsq.gqe_attention_fwd(cfg, o["Qv"], o["Qs"], o["K"], o["V"], o["slots"], wsa)
     o["y"] = torch.empty(R, shape.d_model, dtype=torch.bfloat16, device=dev)
@@ -87,8 +99,8 @@ def run_steps(rsq, shape: synth.LayerShape, d: dict) -> dict:
     return o
 
 
-def run_layer(rsq, shape, d: dict):
-    cfg = rsq.GQEConfig.of(shape)
+def run_layer(rsq, shape, d: dict, flags: int = 0):
+    cfg = rsq.GQEConfig.of(shape, flags)
     ws = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_LAYER), dtype=torch.uint8, device="cuda")
     y = torch.empty(shape.R, shape.d_model, dtype=torch.bfloat16, device="cuda")
     rsq.gqe_layer_fwd(cfg, d["x"], d["W_r"], d["b_r"], d["W_q"], d["W_qs"], d["W_k"], d["W_v"],

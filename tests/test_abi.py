@@ -119,3 +119,31 @@ def test_attention_split_kv_plan(rsq):
     assert large == 256
     rows = 9 * 16 * 2 * 128  # streams x items (chunk of 5 KV tiles: 16 per stream) x 2 tiles x 128 rows
     assert small >= rows * 64 * 4 + rows * 8  # fp32 partial O rows and (m, l) pairs
+
+
+def test_output_construction_flags(rsq):
+    # At most one output construction; the ablation ones (no weighted slot, no
+    # shared head) have kG slots, the others kG+2; the decode step takes the
+    # layer's construction only.
+    c = _cfg(rsq)
+    R, G, k, dh = 2048, 8, 1, 64
+    for flags, S in ((0, k * G + 2), (rsq.GQE_FLAG_SLOT_GROUP_MEAN, k * G + 2),
+                     (rsq.GQE_FLAG_OUT_HARD, k * G), (rsq.GQE_FLAG_OUT_WEIGHTED_CONCAT, k * G)):
+        c.flags = flags
+        total = rsq.gqe_workspace_bytes(c, rsq.GQE_WS_LAYER)
+        slots = rsq.gqe_workspace_offset(c, rsq.GQE_WS_LAYER, "slots")
+        assert total > 0 and slots + R * S * dh * 2 <= total
+        assert rsq.gqe_workspace_bytes(c, rsq.GQE_WS_DECODE) == (0 if flags else
+                                                                 rsq.gqe_workspace_bytes(c, rsq.GQE_WS_DECODE))
+    c.flags = rsq.GQE_FLAG_OUT_HARD | rsq.GQE_FLAG_SLOT_GROUP_MEAN
+    assert rsq.gqe_workspace_bytes(c, rsq.GQE_WS_LAYER) == 0
+    lib = rsq.lib()
+    assert lib.gqe_router_topk(ctypes.byref(c), None, None, None, None, None, None,
+                               None) == rsq.GQE_ERR_INVALID
+    c.flags = 1 << 7  # unknown bit
+    assert rsq.gqe_workspace_bytes(c, rsq.GQE_WS_LAYER) == 0
+    # The ablation constructions take no shared head: Qs / W_qs may be NULL.
+    c.flags = rsq.GQE_FLAG_OUT_HARD
+    p = ctypes.c_void_p(0x1000_0000)  # aligned; never dereferenced (workspace too small)
+    st = lib.gqe_dispatch(ctypes.byref(c), p, p, p, None, p, p, p, p, p, None, p, 16, None)
+    assert st == rsq.GQE_ERR_WORKSPACE

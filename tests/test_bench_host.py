@@ -1,6 +1,7 @@
 """Host-side logic of bench.py (CPU only): the FLOP model against the values
 the active-FLOP formula gives for the measured workloads, the launch counts,
-and the configuration of the opt-in expert-pool sweep."""
+the per-call roofline fractions, the short summary table and the
+configuration of the expert-pool sweep."""
 import math
 
 import bench
@@ -46,3 +47,31 @@ def test_pool_sweep_configuration():
         assert (s.G, s.M, s.T, s.d_model) == (8, 4, 32768, 1024)
         if skew:
             assert (s.M, s.k) in synth.SKEW_BETA
+
+
+def test_call_fractions():
+    # 1 ms per call over 2 steps: each fraction is work / 0.5 ms / peak.
+    s = synth.SEQ2K
+    pk = {"bf16": 1000.0, "hbm": 5000.0}
+    per = {c: 1.0 for c in ("router", "dispatch", "kv", "attention", "output")}
+    fr = bench.call_fractions(s, per, 2, pk)
+    rb = 2048 * 1024 * 2 + 1024 * 16 * 4 + 2048 * 8 * 12
+    assert math.isclose(fr["router_hbm_frac"], round(rb / 0.5e-3 / 1e9 / 5000.0, 4))
+    f = bench.flops(s)
+    assert math.isclose(fr["kv_tensor_frac"], round(f["kv"] / 0.5e-3 / 1e12 / 1000.0, 4))
+    assert math.isclose(fr["dispatch_tensor_frac"], round(f["q"] / 0.5e-3 / 1e12 / 1000.0, 4))
+    assert math.isclose(fr["attention_tensor_frac"], round(f["attention"] / 0.5e-3 / 1e12 / 1000.0, 4))
+
+
+def test_summary_table():
+    out = {"config": {"workload": "seq2k: x"}, "ms_per_step": 0.07, "roofline": {"frac": 0.1},
+           "dense_gqa": {"ms_per_step": 0.06, "speedup_gqe_over_dense": 0.857},
+           "fractions": {"router_hbm_frac": 0.05},
+           "sweep": [{"workload": "seq32k: y", "gqe_ms": 2.0, "dense_ms": 3.0, "speedup": 1.5,
+                      "attn_frac_of_bf16_peak": 0.5}],
+           "pool_sweep": [{"workload": "pool4_k1 (skewed): z", "gqe_ms": 1.0, "dense_ms": 3.0,
+                           "speedup": 3.0, "attn_frac_of_bf16_peak": 0.4, "hot_expert_share": 0.8}]}
+    rows = bench.summary_of(out)["per_workload"]
+    assert [r["workload"] for r in rows] == ["seq2k", "seq32k", "pool4_k1 (skewed)"]
+    assert rows[0]["speedup"] == 0.857 and rows[0]["router_hbm_frac"] == 0.05
+    assert rows[2]["hot_expert_share"] == 0.8

@@ -81,9 +81,17 @@ def test_decode_step_matches_oracle(rsq, name):
     assert rsq.gqe_read_status() == 0
     ref = oracle.gqe_decode_step(xn, Kf, Vf, f["W_r"], f["b_r"], f["W_q"], f["W_qs"], f["W_k"],
                                  f["W_v"], f["W_o"], G, shape.M, shape.k, dh)
-    assert_close(y, ref["y"], "y")
-    assert_close(Kc[:, :, T - 1], ref["k_new"], "new K")
-    assert_close(Vc[:, :, T - 1], ref["v_new"], "new V")
+    # The step's routing: bit-exact indices, weights within 2e-6.
+    sel = (B, G, shape.k)
+    idx = rsq.workspace_view(ws, cfg, rsq.GQE_WS_DECODE, "idx", torch.int32, sel)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"]), "decode router indices differ"
+    for item in ("r", "omega"):
+        got = rsq.workspace_view(ws, cfg, rsq.GQE_WS_DECODE, item, torch.float32, sel)
+        np.testing.assert_allclose(got.cpu().numpy(), ref[item], rtol=0, atol=2e-6)
+    short = T < 128  # a few cached keys: o is close to single V rows
+    assert_close(y, ref["y"], "y", allow_scale=short)
+    assert_close(Kc[:, :, T - 1], ref["k_new"], "new K", allow_scale=short)
+    assert_close(Vc[:, :, T - 1], ref["v_new"], "new V", allow_scale=short)
     # Only position T-1 of the cache changed.
     keep = torch.ones(Kc.shape[2], dtype=torch.bool, device="cuda")
     keep[T - 1] = False
@@ -106,7 +114,7 @@ def test_dense_decode_step_matches_oracle(rsq, name):
     assert rsq.gqe_read_status() == 0
     ref = oracle.gqa_dense_decode_step(xn, Kf, Vf, f["W_q"], f["W_k"], f["W_v"], f["W_o_dense"], G,
                                        shape.M, dh)
-    assert_close(y, ref["y"], "y (dense decode)")
+    assert_close(y, ref["y"], "y (dense decode)", allow_scale=T < 128)
 
 
 def test_decode_step_agrees_with_prefill_layer(rsq):

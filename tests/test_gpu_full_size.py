@@ -6,7 +6,10 @@ attention, slots and y at sampled rows: the first and last rows of each
 sequence, rows on both sides of 128-row tile boundaries (the first tile, the
 middle, the last full and the ragged last tile) and a few seeded random rows.
 Integer outputs must be bit-exact; floating-point outputs within the layer
-tolerance (max-abs 2e-2, mean-abs 2e-3).
+tolerance (max-abs 2e-2, mean-abs 2e-3). The two long-context workloads
+(262144 and 1048576 tokens) are checked the same way, with the oracle's K/V
+built only up to each sequence's last sampled row and K/V compared at the
+sampled rows.
 """
 import numpy as np
 import pytest
@@ -68,6 +71,53 @@ def test_full_size_sampled_rows(rsq, name):
     # The fused entry point gives the same y.
     y, _ = run_layer(rsq, shape, device_inputs(inp))
     assert torch.equal(y, o["y"]), "gqe_layer_fwd differs from the step calls"
+
+
+LONG = {"seq256k": synth.SEQ256K, "seq1m": synth.SEQ1M}
+
+
+def sample_rows_long(shape: synth.LayerShape, strata: int = 24, seed: int = 11) -> np.ndarray:
+    """Tile edges at the start, middle and end of the sequence, plus one
+    seeded row in each of `strata` equal stretches of positions."""
+    T = shape.T
+    pos = {0, 1, 127, 128, 129, T // 2 - 1, T // 2, T - 129, T - 128, T - 2, T - 1}
+    rng = np.random.default_rng(seed)
+    edges = np.linspace(0, T, strata + 1).astype(np.int64)
+    pos |= {int(rng.integers(lo, hi)) for lo, hi in zip(edges[:-1], edges[1:])}
+    pos = sorted(p for p in pos if 0 <= p < T)
+    return np.array([b * T + p for b in range(shape.B) for p in pos], dtype=np.int64)
+
+
+@pytest.mark.parametrize("name", list(LONG))
+def test_long_context_sampled_rows(rsq, name):
+    # The long-context workloads (262144 and 1048576 tokens) against the
+    # oracle: router output and token lists bit-exact in full; K, V, slots
+    # and y at stratified sampled rows, each evaluated from the definition
+    # against the full causal prefix of its sequence.
+    shape = LONG[name]
+    inp = synth.make_layer_inputs(shape, seed=2026, with_dense=False)
+    rows = sample_rows_long(shape)
+    ref = oracle.gqe_layer(inp, rows=rows, full_kv=False)
+    o = run_steps(rsq, shape, device_inputs(inp))
+    assert np.array_equal(o["idx"].cpu().numpy(), ref["idx"]), "router indices differ"
+    assert np.array_equal(o["counts"].cpu().numpy().reshape(shape.N, shape.B), ref["counts"])
+    assert np.array_equal(o["offsets"].cpu().numpy(), ref["offsets"])
+    assert np.array_equal(o["tok"].cpu().numpy(), ref["tok"]), "token lists differ"
+    assert np.array_equal(o["slot_pos"].cpu().numpy(), ref["slot_pos"])
+    np.testing.assert_allclose(o["r"].cpu().numpy(), ref["r"], rtol=0, atol=2e-6)
+    np.testing.assert_allclose(o["omega"].cpu().numpy(), ref["omega"], rtol=0, atol=2e-6)
+    b = torch.from_numpy(rows // shape.T).cuda()
+    t = torch.from_numpy(rows % shape.T).cuda()
+    assert_close(o["K"][b, :, t], ref["K_rows"], "K")
+    assert_close(o["V"][b, :, t], ref["V_rows"], "V")
+    sel = torch.from_numpy(rows).cuda()
+    assert_close(o["slots"].index_select(0, sel), ref["slots"], "slots")
+    assert_close(o["y"].index_select(0, sel), ref["y"], "y")
+    y_steps = o["y"]
+    del o
+    torch.cuda.empty_cache()
+    y, _ = run_layer(rsq, shape, device_inputs(inp))
+    assert torch.equal(y, y_steps), "gqe_layer_fwd differs from the step calls"
 
 
 def test_long_sequence_layouts_agree_bitwise(rsq):

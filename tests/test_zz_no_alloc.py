@@ -14,7 +14,7 @@ import torch
 
 import synth
 from synth import LayerShape
-from gpu_common import assert_close, device_inputs, to_f64
+from gpu_common import device_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -62,10 +62,11 @@ def test_noalloc_dispatch_matches_workspace_dispatch(rsq, shape):
                                  got["offsets"], got["tok"], got["slot_pos"], got["Qv"], got["Qs"])
         torch.cuda.synchronize()
         assert rsq.gqe_read_status() == 0
-        for name in ("counts", "offsets", "tok", "slot_pos"):
+        # Same kernels, tiles and inputs; only the scratch's place differs, so
+        # every output is bitwise equal (a stale tile-table entry would change
+        # which rows a tile covers).
+        for name in ("counts", "offsets", "tok", "slot_pos", "Qv", "Qs"):
             assert torch.equal(got[name], ref[name]), name
-        for name in ("Qv", "Qs"):
-            assert_close(got[name], to_f64(ref[name]), name)
         results.append(got["tok"].cpu().numpy())
     assert not np.array_equal(results[0], results[1])  # the second call really re-dispatched
 
