@@ -256,12 +256,38 @@ def device_inputs_seeded(shape: synth.LayerShape, seed: int) -> dict:
     return d
 
 
+def _graph(f):
+    """f captured once as a CUDA graph (on a side stream; warm calls made before),
+    or None where capture is not possible: replays then time device work only,
+    with no host issue time between the kernels of a step."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            f()
+        torch.cuda.current_stream().wait_stream(s)
+        return g
+    except Exception:  # noqa: BLE001 - capture unavailable: eager calls
+        torch.cuda.synchronize()
+        return None
+
+
 def time_steps(layer: Layer, steps: int, warmup: int, flush, sync_ranks) -> dict:
-    """Times `steps` layer passes; returns total ms and per-call ms sums."""
+    """Times `steps` layer passes call by call (each entry point captured as its
+    own CUDA graph and replayed, events between them); returns total ms and
+    per-call ms sums."""
     import torch
     for _ in range(warmup):
         for c in Layer.CALLS:
             getattr(layer, c)()
+    torch.cuda.synchronize()
+    graphs = {c: _graph(getattr(layer, c)) for c in Layer.CALLS}
+    run = {c: (graphs[c].replay if graphs[c] is not None else getattr(layer, c)) for c in Layer.CALLS}
+    for _ in range(2):
+        for c in Layer.CALLS:
+            run[c]()
     torch.cuda.synchronize()
     n = len(Layer.CALLS)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
@@ -272,7 +298,7 @@ def time_steps(layer: Layer, steps: int, warmup: int, flush, sync_ranks) -> dict
             flush()
         ev[i][0].record()
         for j, c in enumerate(Layer.CALLS):
-            getattr(layer, c)()
+            run[c]()
             ev[i][j + 1].record()
     torch.cuda.synchronize()
     sync_ranks()
@@ -282,12 +308,13 @@ def time_steps(layer: Layer, steps: int, warmup: int, flush, sync_ranks) -> dict
         total += ev[i][0].elapsed_time(ev[i][n])
         for j, c in enumerate(Layer.CALLS):
             per[c] += ev[i][j].elapsed_time(ev[i][j + 1])
-    return {"total_ms": total, "per_call_ms": per}
+    return {"total_ms": total, "per_call_ms": per, "graphs": all(g is not None for g in graphs.values())}
 
 
-def time_layer(rsq, shape, d, steps, warmup, flush, sync_ranks=lambda: None) -> float:
+def time_layer(rsq, shape, d, steps, warmup, flush, sync_ranks=lambda: None, eager: bool = False) -> float:
     """Total ms of `steps` passes of the whole layer through its one entry
-    point, gqe_layer_fwd (device time per step; L2 flushed before each)."""
+    point, gqe_layer_fwd (device time per step; L2 flushed before each when
+    `flush` is given), replayed from a CUDA graph unless `eager`."""
     import torch
     cfg = rsq.GQEConfig.of(shape, rsq.GQE_FLAG_WS_CLEAN)
     ws = torch.zeros(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_LAYER), dtype=torch.uint8, device="cuda")
@@ -297,14 +324,21 @@ def time_layer(rsq, shape, d, steps, warmup, flush, sync_ranks=lambda: None) -> 
         rsq.gqe_layer_fwd(cfg, d["x"], d["W_r"], d["b_r"], d["W_q"], d["W_qs"], d["W_k"], d["W_v"],
                           d["W_o"], y, ws)
 
-    return _time_calls(f, steps, warmup, flush, sync_ranks)
+    return _time_calls(f, steps, warmup, flush, sync_ranks, eager)
 
 
-def _time_calls(f, steps, warmup, flush, sync_ranks=lambda: None) -> float:
+def _time_calls(f, steps, warmup, flush, sync_ranks=lambda: None, eager: bool = False) -> float:
     import torch
     for _ in range(warmup):
         f()
     torch.cuda.synchronize()
+    if not eager:
+        g = _graph(f)
+        if g is not None:
+            f = g.replay
+            for _ in range(2):
+                f()
+            torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
     sync_ranks()
@@ -320,7 +354,7 @@ def _time_calls(f, steps, warmup, flush, sync_ranks=lambda: None) -> float:
     return sum(a.elapsed_time(b) for a, b in ev)
 
 
-def time_dense(rsq, shape, d, steps, warmup, flush) -> float:
+def time_dense(rsq, shape, d, steps, warmup, flush, eager: bool = False) -> float:
     import torch
     cfg = rsq.GQEConfig.of(shape, rsq.GQE_FLAG_WS_CLEAN)
     ws = torch.zeros(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_DENSE), dtype=torch.uint8, device="cuda")
@@ -329,7 +363,7 @@ def time_dense(rsq, shape, d, steps, warmup, flush) -> float:
     def f():
         rsq.gqa_dense_fwd(cfg, d["x"], d["W_q"], d["W_k"], d["W_v"], d["W_o_dense"], y, ws)
 
-    return _time_calls(f, steps, warmup, flush)
+    return _time_calls(f, steps, warmup, flush, eager=eager)
 
 
 def time_e2e(rsq, shape, d, steps, warmup) -> dict:
@@ -520,6 +554,8 @@ def run_ours(args, rank: int, world: int, dist):
     with ClockSampler(torch.cuda.current_device()) as clk:
         # The step: one pass of the whole layer through gqe_layer_fwd.
         layer_ms = time_layer(rsq, shape, d, args.steps, warmup, flush, sync_ranks)
+        # The same call issued from Python every step (host issue time included).
+        eager_ms = time_layer(rsq, shape, d, args.steps, warmup, flush, sync_ranks, eager=True)
         # The same steps call by call, for the per-call times (roofline).
         res = time_steps(layer, args.steps, warmup, flush, sync_ranks)
     if rsq.gqe_read_status() != 0:
@@ -533,6 +569,9 @@ def run_ours(args, rank: int, world: int, dist):
 
     dense_ms = max_over_ranks(time_dense(rsq, shape, d, args.steps, warmup, flush) / args.steps,
                               dist, "cuda")
+    dense_eager_ms = max_over_ranks(time_dense(rsq, shape, d, args.steps, warmup, flush, eager=True) /
+                                    args.steps, dist, "cuda")
+    eager_ms = max_over_ranks(eager_ms, dist, "cuda") / args.steps
     if dist is not None:
         dist.barrier()
     if rank != 0:
@@ -555,6 +594,8 @@ def run_ours(args, rank: int, world: int, dist):
         "config": {"workload": f"{args.workload}: {describe(shape)}", "global_batch": shape.B * world,
                    "seq_len": shape.T, "parallelism": f"replicas{world}",
                    "l2": "flushed (256 MiB write) before every timed step",
+                   "timing": "one gqe_layer_fwd call per step, captured once as a CUDA graph and replayed "
+                             "(device time; eager_ms_per_step: the call issued from Python every step)",
                    "inputs": "seeded synth recipe: x ~ N(0,1) bf16, weights ~ N(0,1/d_model) bf16, "
                              "router fp32"},
         "gpu_launches": layer_launches(shape) * args.steps,
@@ -566,10 +607,14 @@ def run_ours(args, rank: int, world: int, dist):
         "roofline": roof,
         "breakdown_ms_per_step": {c: v / args.steps for c, v in res["per_call_ms"].items()},
         "fractions": call_fractions(shape, res["per_call_ms"], args.steps, pk),
-        "breakdown_note": "per entry point, timed call by call in a second loop of the same steps",
+        "breakdown_note": "per entry point, each captured as its own CUDA graph, replayed call by call "
+                          "in a second loop of the same steps",
+        "eager_ms_per_step": eager_ms,
         "dense_gqa": {"ms_per_step": dense_ms,
                       "tokens_per_s": shape.R * world / (dense_ms / 1e3),
-                      "speedup_gqe_over_dense": dense_ms / ms_per_step},
+                      "speedup_gqe_over_dense": dense_ms / ms_per_step,
+                      "eager_ms_per_step": dense_eager_ms,
+                      "eager_speedup": dense_eager_ms / eager_ms},
         "pages_speedup_context": PAGES_SPEEDUP,
     }
     if world == 1 and not args.no_sweep:

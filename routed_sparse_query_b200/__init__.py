@@ -29,6 +29,7 @@ GQE_WS_DECODE, GQE_WS_DENSE_DECODE = 5, 6
 GQE_FLAG_WS_CLEAN, GQE_FLAG_EXPERT_MAJOR = 1, 2
 # Output constructions (at most one): see include/gqe.h.
 GQE_FLAG_SLOT_GROUP_MEAN, GQE_FLAG_OUT_HARD, GQE_FLAG_OUT_WEIGHTED_CONCAT = 4, 8, 16
+GQE_FLAG_NO_SHARED_HEAD = 32  # a shard of the layer split over KV groups (no shared head)
 OUTPUT_MODE_FLAGS = {"gqe": 0, "group_mean": GQE_FLAG_SLOT_GROUP_MEAN, "hard": GQE_FLAG_OUT_HARD,
                      "weighted_concat": GQE_FLAG_OUT_WEIGHTED_CONCAT}
 ITEMS = {"idx": 1, "r": 2, "omega": 3, "counts": 4, "offsets": 5, "tok": 6, "slot_pos": 7,

@@ -31,12 +31,15 @@ def assert_close(got: torch.Tensor, want: np.ndarray, what: str, max_abs=MAX_ABS
     value rounded (unit roundoff 2^-8 ~ 3.9e-3), so for larger outputs -- a
     sequence of a few tokens, where o is a single V row and |y| ~ 1 -- both
     bounds scale with 2 * rms(want). Only sequences shorter than one 128-row
-    tile may use that scaling (allow_scale); everywhere else the bounds are
-    the stated ones and the check fails if the outputs are larger.
+    tile use that scaling (allow_scale); everywhere else the bounds are the
+    stated ones, unscaled. (K, V and the queries are projections of rms ~1 at
+    every length; their one bf16 rounding, below 2^-9 of the value, keeps them
+    inside the stated bounds.)
     """
     g = to_f64(got).reshape(want.shape)
-    scale = max(1.0, 2.0 * float(np.sqrt(np.mean(np.square(want)))) if want.size else 1.0)
-    assert allow_scale or scale == 1.0, f"{what}: rms(want) above 1/2 outside the short-sequence cases"
+    scale = 1.0
+    if allow_scale and want.size:
+        scale = max(1.0, 2.0 * float(np.sqrt(np.mean(np.square(want)))))
     max_abs, mean_abs = max_abs * scale, mean_abs * scale
     err = np.abs(g - want)
     assert np.isfinite(g).all(), f"{what}: non-finite values"
