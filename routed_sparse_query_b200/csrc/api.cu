@@ -194,7 +194,7 @@ gqe_status dispatch_and_project(const gqe_config& c, const int32_t* idx, const g
   int e = launch_dispatch_lists(c, idx, counts, offsets, tok, slot_pos, ws, L, stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
   char* w = static_cast<char*>(ws);
-  return cuda_status(gemm_q_routed(c, x, W_q, W_qs, idx, offsets, tok, w + L.qtiles,
+  return cuda_status(gemm_q_routed(c, x, W_q, W_qs, idx, tok, w + L.qtiles,
                                    reinterpret_cast<const int32_t*>(w + L.n_qtiles), L.max_qtiles,
                                    Qv, Qs, (c.flags & GQE_FLAG_EXPERT_MAJOR) != 0u, stream));
 }

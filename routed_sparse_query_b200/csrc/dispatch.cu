@@ -11,8 +11,8 @@
 //              the tile's tokens of the same expert (ascending t), so the
 //              lists are stable and bit-exact.
 // When the tile counts are few (kFusedScanMax), every scatter CTA computes
-// the prefix sum it needs itself and CTA 0 also writes the shared outputs, so
-// steps 2 and 3 are one launch.
+// the prefix sum it needs itself and one more CTA writes the shared outputs,
+// so steps 2 and 3 are one launch.
 // Only the selected experts receive rows ("a router selects a sparse subset
 // of k query-head experts from each GQA group": gist.science Technical
 // Summary, Methodology), and every group gets exactly k entries per token.
@@ -190,9 +190,11 @@ __device__ void write_list_meta(const ListArgs& a, int total) {
   int qbase = block_exclusive_scan(nq, &nq_total);
   for (int i = lo; i < hi; ++i) {
     const int e = i / a.B, b = i % a.B;
-    const int c = a.counts[i];
+    const int c = a.counts[i], start = a.offsets[i];
     for (int s = 0; s < c; s += kQTileRows) {
-      if (qbase < a.max_qtiles) a.qtiles[qbase] = make_int4(e, b, s, min(kQTileRows, c - s));
+      // (expert, sequence, first list entry, rows): the GEMM reads its rows'
+      // positions straight from tok.
+      if (qbase < a.max_qtiles) a.qtiles[qbase] = make_int4(e, b, start + s, min(kQTileRows, c - s));
       ++qbase;
     }
   }

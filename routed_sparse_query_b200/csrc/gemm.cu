@@ -70,7 +70,6 @@ struct Epi {
 struct Gather {
   const uint16_t* x;
   const int32_t* tok;
-  const int32_t* offsets;
   const int4* qtiles;
   const int32_t* n_qtiles;
   const int32_t* idx;
@@ -160,7 +159,7 @@ __global__ void __launch_bounds__(192, 2)
         const int4 qt = ga.qtiles[q];
         e = qt.x;
         b = qt.y;
-        list0 = ga.offsets[e * ga.B + b] + qt.z;
+        list0 = qt.z;
         rows = qt.w;
         n0 = e * ga.dh;
       }
@@ -500,7 +499,7 @@ int gemm_output(const gqe_config& c, uint16_t* slots, const float* omega, const 
 }
 
 int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const uint16_t* W_qs,
-                  const int32_t* idx, const int32_t* offsets, const int32_t* tok, const void* qtiles,
+                  const int32_t* idx, const int32_t* tok, const void* qtiles,
                   const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, uint16_t* Qs,
                   bool expert_major, void* stream) {
   const int N = c.G * c.M;
@@ -513,7 +512,6 @@ int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, c
   Gather g;
   g.x = x;
   g.tok = tok;
-  g.offsets = offsets;
   g.qtiles = static_cast<const int4*>(qtiles);
   g.n_qtiles = n_qtiles;
   g.idx = idx;

@@ -54,7 +54,7 @@ struct DispatchWs {
   size_t masks;        // uint64 [R]: selection bitmask per token
   size_t tile_counts;  // int32 [N][num_tiles]
   size_t tile_base;    // int32 [N][num_tiles]
-  size_t qtiles;       // int4  [max_qtiles]: (e, b, start, rows)
+  size_t qtiles;       // int4  [max_qtiles]: (e, b, first list entry, rows)
   size_t n_qtiles;     // int32 [1]
   size_t total;
   int num_tiles;
@@ -117,7 +117,7 @@ int gemm_kv(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const u
 // expert_major: Qv is written in token-list order ([k*G*B*T, dh], row = list
 // entry) instead of slot-major [B, G, k, T, dh].
 int gemm_q_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const uint16_t* W_qs,
-                  const int32_t* idx, const int32_t* offsets, const int32_t* tok, const void* qtiles,
+                  const int32_t* idx, const int32_t* tok, const void* qtiles,
                   const int32_t* n_qtiles, int max_qtiles, uint16_t* Qv, uint16_t* Qs,
                   bool expert_major, void* stream);
 // The shared-head query projection alone (Qs [B, T, dh]); the same tiles and

@@ -33,10 +33,14 @@ def test_projection_flops():
 
 
 def test_launch_counts():
-    # seq2k: 8 dispatch tiles x 16 experts fit the fused scan + scatter.
+    # seq2k and 4 x 8k: the tile counts (8 or 128 tiles x 16 experts) fit the
+    # fused scan + scatter after the count kernel; 1M tokens: 4096 x 16 tile
+    # counts take the separate scan.
     assert bench.launches(synth.SEQ2K) == {"router": 1, "dispatch": 3, "kv": 1, "attention": 1,
                                            "output": 1}
     assert bench.layer_launches(synth.SEQ2K) == 8
+    assert bench.launches(synth.BATCH4_8K)["dispatch"] == 3
+    assert bench.launches(synth.SEQ1M)["dispatch"] == 4
     # d_head = 32: the weighted slot is its own kernel before W_O.
     assert bench.launches(synth.TINY)["output"] == 2
 

@@ -89,8 +89,22 @@ def test_seq2k_layer_matches_oracle(rsq):
     _check_float_parts(o, ref, shape)
     y, ws = run_layer(rsq, shape, d)
     assert torch.equal(y, o["y"]), "gqe_layer_fwd differs from the step calls"
-    # T = 2048 runs the split-KV attention; a second call on the same scratch
-    # (merge counters reset by the previous call) gives the same slots.
+
+
+def test_split_kv_attention_repeated_calls(rsq):
+    # T = 3072 (9 streams): the split-KV attention with pairs of unequal chunk
+    # counts; the layer matches the oracle, and further calls on the same
+    # scratch (merge counters reset by the previous call) give the same slots,
+    # with and without GQE_FLAG_WS_CLEAN.
+    shape = LayerShape(B=1, T=3072, d_model=1024, G=8, M=2, k=1, d_head=64)
+    inp = synth.make_layer_inputs(shape, seed=12)
+    ref = oracle.gqe_layer(inp)
+    d = device_inputs(inp)
+    o = run_steps(rsq, shape, d)
+    _check_integer_parts(o, ref, shape)
+    _check_float_parts(o, ref, shape)
+    y, ws = run_layer(rsq, shape, d)
+    assert torch.equal(y, o["y"]), "gqe_layer_fwd differs from the step calls"
     cfg = rsq.GQEConfig.of(shape)
     wsa = torch.empty(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_ATTENTION), dtype=torch.uint8,
                       device="cuda")

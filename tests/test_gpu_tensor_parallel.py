@@ -2,8 +2,9 @@
 part (routing of the whole layer, its groups' dispatch, K/V, attention and
 W_O rows, the shared head on the rank of group 0) runs one after another on
 the same GPU, with no collective; the partial outputs summed on the device
-must match the oracle's layer, and each shard's token lists must be the
-oracle's lists of its groups."""
+must match the oracle's layer (within the layer tolerance plus the bf16
+rounding of each shard's partial output), and each shard's token lists must be
+the oracle's lists of its groups."""
 import numpy as np
 import pytest
 import torch
@@ -35,6 +36,7 @@ def test_group_shards_sum_to_the_layer(rsq, world, shape):
     ref = oracle.gqe_layer(inp)
     d = device_inputs(inp)
     y_sum = torch.zeros(shape.R, shape.d_model, dtype=torch.float32, device="cuda")
+    rounding = 0.0  # each shard's y is rounded to bf16 (unit roundoff 2^-9) before the sum
     for rank in range(world):
         shard = GroupShard(world, rank, shape.G, shape.M, shape.k, shape.d_head)
         Wq, Wk, Wv, Wo = shard_weights(shard, d["W_q"], d["W_k"], d["W_v"], d["W_o"])
@@ -44,7 +46,9 @@ def test_group_shards_sum_to_the_layer(rsq, world, shape):
         torch.cuda.synchronize()
         assert rsq.gqe_read_status() == 0
         y_sum += y.float()
+        rounding += float(y.float().abs().max()) * 2.0 ** -9
         lists = oracle.dispatch(ref["idx"][:, shard.g0:shard.g1], shape.B, shape.T, shard.G_local, shape.M)
         assert np.array_equal(layer.tok.cpu().numpy(), lists["tok"])
         assert np.array_equal(layer.offsets.cpu().numpy(), lists["offsets"])
-    assert_close(y_sum, ref["y"], f"sum of {world} shards")
+    # The layer's bounds, plus the bf16 rounding of each shard's partial output.
+    assert_close(y_sum, ref["y"], f"sum of {world} shards", max_abs=2e-2 + rounding)
