@@ -545,14 +545,14 @@ def run_ours(args, rank: int, world: int, dist):
     d = device_inputs_from_synth(inp)
     layer = Layer(rsq, shape, d)
     flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    read_buf = torch.zeros(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+    read_buf = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
     def flush():
         # Write 256 MiB (evicts every input of the step from the 126 MB L2),
         # then read another 256 MiB, so that the dirty lines of the write are
         # written back before the step and L2 holds clean, unrelated lines.
         flush_buf.zero_()
-        read_buf.sum()
+        read_buf.sum()  # float32: one reduction, no widened temporary
 
     def sync_ranks():
         if dist is not None:
