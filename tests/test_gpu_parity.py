@@ -51,6 +51,14 @@ CASES = {
     "k_equals_m": (LayerShape(B=1, T=260, d_model=256, G=4, M=2, k=2, d_head=32), {}),
     "t1": (LayerShape(B=3, T=1, d_model=128, G=2, M=2, k=1, d_head=64), {}),
     "t5_dh32": (LayerShape(B=2, T=5, d_model=64, G=2, M=3, k=2, d_head=32), {}),
+    # Query-projection weights of one expert larger than the resident limit
+    # (d_model x d_head bf16 > 128 KB): the per-tile routed Q GEMM.
+    "wide_d1536": (LayerShape(B=1, T=300, d_model=1536, G=4, M=2, k=1, d_head=64), {}),
+    # The same width with d_head = 32: 24 K blocks resident.
+    "d1536_dh32": (LayerShape(B=2, T=200, d_model=1536, G=2, M=3, k=2, d_head=32), {}),
+    # At least two query tiles per SM: the routed Q GEMM with the expert's
+    # weights resident in shared memory (routed tiles, then shared-head tiles).
+    "resident_w": (LayerShape(B=2, T=2400, d_model=256, G=8, M=2, k=1, d_head=64), {}),
 }
 
 
