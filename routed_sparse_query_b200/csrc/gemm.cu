@@ -15,9 +15,10 @@
 //    tile per CTA.
 //  - W_O projection (step a11): plain row-major output. With d_head = 64 the
 //    weighted slot (step a10) is exactly one K block of A: the epilogue warps,
-//    idle during the main loop, compute it from the routed slots and omega,
-//    write it into that K block's stage in the swizzled layout (and, in the
-//    CTAs of the first column tile, back to the slot buffer), and the TMA warp
+//    idle during the main loop, sum it from the routed slots' stages as they
+//    land (weighted by omega), write it into that K block's stage in the
+//    swizzled layout (and, in the CTAs of the first column tile, back to the
+//    slot buffer), and the TMA warp
 //    loads only B for that block.
 //
 // Warp roles (192 threads): warp 0 issues TMA loads, warp 1 issues the UMMAs
@@ -126,7 +127,9 @@ __global__ void __launch_bounds__(192, 2)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], GATHER ? 129u : 1u);
-      mbar_init(&empty[s], 1u);
+      // With the weighted slot fused, the 128 epilogue threads read every
+      // stage too and release it along with the UMMAs.
+      mbar_init(&empty[s], (!GATHER && epi.kb_w >= 0) ? 129u : 1u);
     }
     mbar_init(accb, 1u);
     mbar_init(drain, 1u);
@@ -270,51 +273,76 @@ __global__ void __launch_bounds__(192, 2)
     }
     if (!GATHER && epi.kb_w >= 0) {
       // Weighted slot: the same fp32 sum, in the same order, as the
-      // stand-alone weighted-slot kernel, rounded to bf16. Thread i takes
-      // 16-byte chunk i % 8 of rows i / 8, i / 8 + 16, ... (8 threads read one
-      // slot row segment together), writes it into the block's stage once the
-      // stage is free, and (first column tile) into the slot buffer.
+      // stand-alone weighted-slot kernel, rounded to bf16. The kG routed
+      // slots are the first K blocks of A, so the sum is taken from their
+      // stages as they land: thread i takes 16-byte chunk i % 8 of rows
+      // i / 8, i / 8 + 16, ... (8 threads read one slot row segment
+      // together), and these threads release every stage along with the
+      // UMMAs. The sum goes into the weighted block's stage once that stage
+      // is free, and (first column tile) into the slot buffer. Rows past the
+      // end are zero in the stages and get omega 0.
       const int i = threadIdx.x - 64;
       const int c = i & 7;
-      uint4 o[8];
-#pragma unroll 2
-      for (int pass = 0; pass < 8; ++pass) {
-        const int row = m0 + pass * 16 + (i >> 3);
-        if (row < epi.rows) {
-          const uint16_t* base = epi.wslots + static_cast<size_t>(row) * epi.lda + c * 8;
-          const float* w = epi.omega + static_cast<size_t>(row) * epi.gk;
-          float acc[8];
+      float acc[8][8];
 #pragma unroll
-          for (int x = 0; x < 8; ++x) acc[x] = 0.0f;
-#pragma unroll 4
-          for (int gs = 0; gs < epi.gk; ++gs) {
-            const float wi = __ldg(w + gs);
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + gs * BK));
+      for (int pass = 0; pass < 8; ++pass)
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc[pass][x] = 0.0f;
+      // omega of this thread's rows for slot gs (read one block ahead).
+      auto omega_of = [&](int gs, float (&w)[8]) {
+#pragma unroll
+        for (int pass = 0; pass < 8; ++pass) {
+          const int row = m0 + pass * 16 + (i >> 3);
+          w[pass] = (gs < epi.gk && row < epi.rows) ? __ldg(epi.omega + static_cast<size_t>(row) * epi.gk + gs)
+                                                    : 0.0f;
+        }
+      };
+      float wn[8];
+      omega_of(0, wn);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % C::STAGES;
+        const uint32_t ph = (kb / C::STAGES) & 1;
+        if (kb == epi.kb_w) {
+          uint4 o[8];
+#pragma unroll
+          for (int pass = 0; pass < 8; ++pass) {
+            o[pass] = make_uint4(pack_bf16x2(acc[pass][0], acc[pass][1]), pack_bf16x2(acc[pass][2], acc[pass][3]),
+                                 pack_bf16x2(acc[pass][4], acc[pass][5]), pack_bf16x2(acc[pass][6], acc[pass][7]));
+            const int row = m0 + pass * 16 + (i >> 3);
+            if (blockIdx.y == 0 && row < epi.rows)
+              *reinterpret_cast<uint4*>(epi.wslots + static_cast<size_t>(row) * epi.lda + epi.kb_w * BK +
+                                        c * 8) = o[pass];
+          }
+          if (!mbar_wait(wfree, 0, abort_flag)) break;
+          uint8_t* stage = sA + s * C::A_BYTES;
+#pragma unroll
+          for (int pass = 0; pass < 8; ++pass) {
+            const int r = pass * 16 + (i >> 3);
+            *reinterpret_cast<uint4*>(stage + r * 128 + ((c ^ (r & 7)) << 4)) = o[pass];
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(wready);
+        }
+        if (!mbar_wait(&full[s], ph, abort_flag)) break;
+        if (kb < epi.gk) {
+          float w[8];
+#pragma unroll
+          for (int pass = 0; pass < 8; ++pass) w[pass] = wn[pass];
+          omega_of(kb + 1, wn);
+          const uint8_t* stage = sA + s * C::A_BYTES;
+#pragma unroll
+          for (int pass = 0; pass < 8; ++pass) {
+            const int r = pass * 16 + (i >> 3);
+            const uint4 v = *reinterpret_cast<const uint4*>(stage + r * 128 + ((c ^ (r & 7)) << 4));
             const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int i2 = 0; i2 < 4; ++i2) {
-              acc[2 * i2] = fmaf(wi, __uint_as_float(u[i2] << 16), acc[2 * i2]);
-              acc[2 * i2 + 1] = fmaf(wi, __uint_as_float(u[i2] & 0xffff0000u), acc[2 * i2 + 1]);
+              acc[pass][2 * i2] = fmaf(w[pass], __uint_as_float(u[i2] << 16), acc[pass][2 * i2]);
+              acc[pass][2 * i2 + 1] = fmaf(w[pass], __uint_as_float(u[i2] & 0xffff0000u), acc[pass][2 * i2 + 1]);
             }
           }
-          o[pass] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                               pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
-          if (blockIdx.y == 0)
-            *reinterpret_cast<uint4*>(epi.wslots + static_cast<size_t>(row) * epi.lda + epi.kb_w * BK +
-                                      c * 8) = o[pass];
-        } else {
-          o[pass] = make_uint4(0u, 0u, 0u, 0u);
         }
-      }
-      if (mbar_wait(wfree, 0, abort_flag)) {
-        uint8_t* stage = sA + (epi.kb_w % C::STAGES) * C::A_BYTES;
-#pragma unroll
-        for (int pass = 0; pass < 8; ++pass) {
-          const int r = pass * 16 + (i >> 3);
-          *reinterpret_cast<uint4*>(stage + r * 128 + ((c ^ (r & 7)) << 4)) = o[pass];
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(wready);
+        mbar_arrive(&empty[s]);
       }
     }
     const bool have = mbar_wait(accb, 0, abort_flag);
