@@ -33,6 +33,9 @@ CASES = {
     "chunk_edge_257": LayerShape(B=2, T=257, d_model=256, G=4, M=2, k=1, d_head=64),
     "pool4_k2": LayerShape(B=2, T=700, d_model=256, G=8, M=4, k=2, d_head=64),
     "long_2k": LayerShape(B=2, T=2048, d_model=1024, G=8, M=2, k=1, d_head=64),
+    # 128 (sequence, group) pairs: spans of 2 chunks of 256 keys (the streaming
+    # form's online softmax across chunks), the last span one partial chunk.
+    "spans_4097": LayerShape(B=16, T=4097, d_model=256, G=8, M=2, k=1, d_head=64),
 }
 
 
@@ -99,7 +102,7 @@ def test_decode_step_matches_oracle(rsq, name):
     assert torch.equal(Vc[:, :, keep], V_before[:, :, keep])
 
 
-@pytest.mark.parametrize("name", ["t5_k2", "chunk_edge_257", "pool4_k2"])
+@pytest.mark.parametrize("name", ["t5_k2", "chunk_edge_257", "pool4_k2", "spans_4097"])
 def test_dense_decode_step_matches_oracle(rsq, name):
     shape = CASES[name]
     inp, d, Kc, Vc, x_new = _setup(rsq, shape, seed=78)
