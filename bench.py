@@ -367,6 +367,25 @@ def time_dense(rsq, shape, d, steps, warmup, flush, eager: bool = False) -> floa
     return _time_calls(f, steps, warmup, flush, eager=eager)
 
 
+def gpu_local_cpus() -> set | None:
+    """The host CPUs that NVML reports as local to the current GPU (its NUMA
+    node), intersected with the ones this process may run on; None if NVML
+    or the query is unavailable. A read-only query."""
+    import torch
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(torch.cuda.current_device())
+        uuid = str(getattr(props, "uuid", ""))
+        h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid if not uuid.startswith("GPU-") else uuid).encode())
+        words = pynvml.nvmlDeviceGetCpuAffinity(h, (os.cpu_count() + 63) // 64)
+        local = {64 * i + bit for i, w in enumerate(words) for bit in range(64) if (int(w) >> bit) & 1}
+        cpus = local & os.sched_getaffinity(0)
+        return cpus or None
+    except Exception:  # noqa: BLE001 - no NVML, no binding
+        return None
+
+
 def time_e2e(rsq, shape, d, steps, warmup) -> dict:
     """gqe_layer_fwd with x copied in from pinned host memory and y copied
     back, every step, inside the timed region, pipelined: stage i copies in
@@ -375,6 +394,21 @@ def time_e2e(rsq, shape, d, steps, warmup) -> dict:
     Each stage is captured once as a CUDA graph (one per buffer parity) and
     replayed, so the host issues one launch per step; if capture is not
     possible the same stages run eagerly."""
+    import torch
+    # The pinned host buffers are placed on the GPU's own NUMA node: this
+    # thread runs on the CPUs local to the GPU while it allocates and drives
+    # the copies (the previous affinity is restored afterwards).
+    saved = os.sched_getaffinity(0)
+    local = gpu_local_cpus()
+    if local is not None:
+        os.sched_setaffinity(0, local)
+    try:
+        return _time_e2e(rsq, shape, d, steps, warmup, local)
+    finally:
+        os.sched_setaffinity(0, saved)
+
+
+def _time_e2e(rsq, shape, d, steps, warmup, local) -> dict:
     import torch
     cfg = rsq.GQEConfig.of(shape, rsq.GQE_FLAG_WS_CLEAN)
     ws = torch.zeros(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_LAYER), dtype=torch.uint8, device="cuda")
@@ -430,7 +464,7 @@ def time_e2e(rsq, shape, d, steps, warmup) -> dict:
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     return {"ms": ms, "h2d": x_h.numel() * 2, "d2h": y_h.numel() * 2,
-            "graph": graphs is not None}
+            "graph": graphs is not None, "host_cpus": len(local) if local is not None else None}
 
 
 def roofline_of(shape, per_call_ms: dict, steps: int, pk: dict, traffic=None):
@@ -610,6 +644,8 @@ def run_ours(args, rank: int, world: int, dist):
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"], "api": "gqe_layer_fwd",
+                "host_buffers": (f"pinned, allocated from the {e2e['host_cpus']} CPUs local to the GPU"
+                                 if e2e["host_cpus"] else "pinned (GPU-local CPUs unknown)"),
                 "pipelining": "copies of steps i+1 (in) and i-1 (out) overlap the layer of step i",
                 "cuda_graph_stages": e2e["graph"]},
         "roofline": roof,
