@@ -664,6 +664,8 @@ def run_ours(args, rank: int, world: int, dist):
     if world == 1 and not args.no_sweep:
         out["sweep"] = sweep(rsq, pk, args)
         out["decode"] = decode_bench(rsq, pk, args.steps)
+        if shape.T <= 8192:
+            out["backward"] = backward_bench(rsq, shape, d)
     if world == 1 and not args.no_pool:
         out["pool_sweep"] = sweep_pool(rsq, pk, args)
     if world == 1 and not args.no_cpu:
@@ -673,6 +675,37 @@ def run_ours(args, rank: int, world: int, dist):
         out["cpu_baseline"]["host_cores"] = os.cpu_count()
     out["summary"] = summary_of(out)
     return out
+
+
+def backward_bench(rsq, shape, d, steps: int = 5) -> dict:
+    """One gqe_layer_bwd call (forward recomputation included) on the bench
+    workload, CUDA-event timed after two warm-up calls; dy ~ N(0, 1)."""
+    import torch
+    cfg = rsq.GQEConfig.of(shape, rsq.GQE_FLAG_WS_CLEAN)
+    ws = torch.zeros(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_BACKWARD), dtype=torch.uint8, device="cuda")
+    R, dm, dh, N, G = shape.R, shape.d_model, shape.d_head, shape.N, shape.G
+    f32 = lambda *sh: torch.empty(*sh, dtype=torch.float32, device="cuda")  # noqa: E731
+    g = torch.Generator(device="cuda").manual_seed(7)
+    dy = torch.randn(R, dm, device="cuda", generator=g)
+    outs = (f32(R, dm), f32(dm, N), f32(N), f32(dm, N * dh), f32(dm, dh), f32(dm, G * dh), f32(dm, G * dh),
+            f32((shape.k * G + 2) * dh, dm))
+
+    def f():
+        rsq.gqe_layer_bwd(cfg, d["x"], d["W_r"], d["b_r"], d["W_q"], d["W_qs"], d["W_k"], d["W_v"], d["W_o"], dy,
+                          *outs, ws)
+    for _ in range(2):
+        f()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        f()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return {"workload": describe(shape), "ms_per_call": ms, "tokens_per_s": R / (ms / 1e3), "steps": steps,
+            "path": "first CUDA-core path (forward recomputed first; fp32 GEMMs, attention backward, router "
+                    "backward through the weighted slot); no tensor cores yet"}
 
 
 DECODE = {"batch": 64, "cache": 32768}  # decode measurement: 64 sequences, 32k cached tokens

@@ -118,7 +118,8 @@ enum {
   GQE_WS_DENSE = 3,    /* everything gqa_dense_fwd keeps between its steps */
   GQE_WS_ATTENTION = 4, /* scratch of gqe_attention_fwd (split-KV partials) */
   GQE_WS_DECODE = 5,    /* scratch of gqe_decode_step */
-  GQE_WS_DENSE_DECODE = 6 /* scratch of gqa_dense_decode_step */
+  GQE_WS_DENSE_DECODE = 6, /* scratch of gqa_dense_decode_step */
+  GQE_WS_BACKWARD = 7      /* scratch of gqe_layer_bwd */
 };
 
 /* Items inside the GQE_WS_LAYER / GQE_WS_DENSE workspaces (for inspection). */
@@ -364,6 +365,31 @@ gqe_status gqa_dense_decode_step(const gqe_config* cfg, const gqe_bf16* x, const
                                  const gqe_bf16* W_o_dense, gqe_bf16* K_cache, gqe_bf16* V_cache,
                                  int32_t cache_capacity, gqe_bf16* y, void* ws, size_t ws_bytes,
                                  gqe_stream_t stream);
+
+/*
+ * Backward of the layer (the default output construction; cfg->flags may
+ * hold GQE_FLAG_WS_CLEAN only, else GQE_ERR_UNSUPPORTED): given
+ * dy = dL/dy [B*T, d_model] (fp32), the gradients of L with the router's
+ * top-k selection held fixed -- the selection is a discrete choice, and the
+ * weighted slot is the layer's differentiable path from the loss to the
+ * router ("a differentiable path for the language-modelling loss to reach the
+ * router": gist.science Technical Summary, Output Construction). Through the
+ * weighted slot the router gets d(omega) = <o, dS_w>, the quotient rule of
+ * omega = p_sel / sum(p_sel) and each group's softmax Jacobian. The forward
+ * is recomputed first (as gqe_layer_fwd, into the scratch) and the gradients
+ * use its bf16 intermediates (routing, Q, K, V, slots), accumulated in fp32.
+ * Outputs (fp32, overwritten): dx [B*T, d_model], dW_r [d_model, N],
+ * db_r [N] (NULL: not computed), dW_q [d_model, N*d_head],
+ * dW_qs [d_model, d_head], dW_k, dW_v [d_model, G*d_head],
+ * dW_o [(kG+2)*d_head, d_model]. Inputs as in gqe_layer_fwd.
+ * Scratch: >= gqe_workspace_bytes(cfg, GQE_WS_BACKWARD). A first path on the
+ * CUDA cores (no tensor cores yet).
+ */
+gqe_status gqe_layer_bwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r, const float* b_r,
+                         const gqe_bf16* W_q, const gqe_bf16* W_qs, const gqe_bf16* W_k, const gqe_bf16* W_v,
+                         const gqe_bf16* W_o, const float* dy, float* dx, float* dW_r, float* db_r,
+                         float* dW_q, float* dW_qs, float* dW_k, float* dW_v, float* dW_o, void* ws,
+                         size_t ws_bytes, gqe_stream_t stream);
 
 #ifdef __cplusplus
 }

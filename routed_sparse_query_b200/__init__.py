@@ -25,7 +25,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 GQE_OK, GQE_ERR_INVALID, GQE_ERR_UNSUPPORTED, GQE_ERR_WORKSPACE = 0, 1, 2, 3
 GQE_ERR_CUDA, GQE_ERR_TIMEOUT, GQE_ERR_DEVICE_CHECK = 4, 5, 6
 GQE_WS_DISPATCH, GQE_WS_LAYER, GQE_WS_DENSE, GQE_WS_ATTENTION = 1, 2, 3, 4
-GQE_WS_DECODE, GQE_WS_DENSE_DECODE = 5, 6
+GQE_WS_DECODE, GQE_WS_DENSE_DECODE, GQE_WS_BACKWARD = 5, 6, 7
 GQE_FLAG_WS_CLEAN, GQE_FLAG_EXPERT_MAJOR = 1, 2
 # Output constructions (at most one): see include/gqe.h.
 GQE_FLAG_SLOT_GROUP_MEAN, GQE_FLAG_OUT_HARD, GQE_FLAG_OUT_WEIGHTED_CONCAT = 4, 8, 16
@@ -40,7 +40,7 @@ EXPORTED = ("gqe_workspace_bytes", "gqe_workspace_offset", "gqe_router_topk", "g
             "gqe_kv_proj", "gqe_attention_fwd", "gqe_output_proj", "gqe_layer_fwd",
             "gqa_dense_fwd", "gqe_read_status", "gqe_selftest_wait_timeout",
             "gqe_status_string", "gqe_version", "gqe_dispatch_noalloc", "gqe_attention_fwd_compact",
-            "gqe_decode_step", "gqa_dense_decode_step")
+            "gqe_decode_step", "gqa_dense_decode_step", "gqe_layer_bwd")
 
 
 class GQEConfig(ctypes.Structure):
@@ -80,6 +80,7 @@ _sig = {
                                        _P, _P, ctypes.c_size_t, _P]),
     "gqa_dense_decode_step": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P,
                                              _P, ctypes.c_size_t, _P]),
+    "gqe_layer_bwd": (ctypes.c_int, [_CFG] + [_P] * 18 + [ctypes.c_size_t, _P]),
     "gqe_read_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32)]),
     "gqe_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
     "gqe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -174,6 +175,14 @@ def gqe_layer_fwd(cfg, x, W_r, b_r, W_q, W_qs, W_k, W_v, W_o, y, ws, stream=None
     _check(_lib.gqe_layer_fwd(_cfg(cfg), _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(W_q), _ptr(W_qs),
                               _ptr(W_k), _ptr(W_v), _ptr(W_o), _ptr(y), _ptr(ws),
                               ws.numel() * ws.element_size(), _stream(stream)), "gqe_layer_fwd")
+
+
+def gqe_layer_bwd(cfg, x, W_r, b_r, W_q, W_qs, W_k, W_v, W_o, dy, dx, dW_r, db_r, dW_q, dW_qs, dW_k, dW_v,
+                  dW_o, ws, stream=None):
+    _check(_lib.gqe_layer_bwd(_cfg(cfg), _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(W_q), _ptr(W_qs), _ptr(W_k),
+                              _ptr(W_v), _ptr(W_o), _ptr(dy), _ptr(dx), _ptr(dW_r), _ptr(db_r), _ptr(dW_q),
+                              _ptr(dW_qs), _ptr(dW_k), _ptr(dW_v), _ptr(dW_o), _ptr(ws),
+                              ws.numel() * ws.element_size(), _stream(stream)), "gqe_layer_bwd")
 
 
 def gqa_dense_fwd(cfg, x, W_q, W_k, W_v, W_o_dense, y, ws, stream=None):

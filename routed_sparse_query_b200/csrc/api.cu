@@ -82,6 +82,38 @@ LayerWs layer_ws(const gqe_config& c) {
   return L;
 }
 
+// Backward: the layer's workspace (the recomputed forward), y of the
+// recomputation, then the fp32 gradients in flight.
+struct BwdWs {
+  LayerWs L;
+  size_t y, dS, dOr, dOs, dz, stats, dQr, dQs, dQfull, dKf, dVf, total;
+};
+
+BwdWs bwd_ws(const gqe_config& c) {
+  BwdWs W{};
+  W.L = layer_ws(c);
+  const size_t R = static_cast<size_t>(c.B) * c.T, dh = c.d_head;
+  const size_t gk = static_cast<size_t>(c.G) * c.k, N = static_cast<size_t>(c.G) * c.M;
+  size_t o = W.L.total;
+  auto put = [&](size_t& field, size_t bytes) {
+    field = o;
+    o = round256(o + bytes);
+  };
+  put(W.y, R * c.d_model * 2);
+  put(W.dS, R * (gk + 2) * dh * 4);
+  put(W.dOr, R * gk * dh * 4);
+  put(W.dOs, R * dh * 4);
+  put(W.dz, R * N * 4);
+  put(W.stats, static_cast<size_t>(c.B) * (gk + 1) * c.T * 3 * 4);
+  put(W.dQr, R * gk * dh * 4);
+  put(W.dQs, R * dh * 4);
+  put(W.dQfull, R * N * dh * 4);
+  put(W.dKf, R * c.G * dh * 4);
+  put(W.dVf, R * c.G * dh * 4);
+  W.total = o;
+  return W;
+}
+
 // Decode step: the layer's per-token buffers for B rows (one new token per
 // sequence; K/V go to the caller's cache), then the decode attention scratch.
 gqe_config decode_rows_cfg(const gqe_config& c) {
@@ -224,6 +256,8 @@ size_t gqe_workspace_bytes(const gqe_config* cfg, int which) {
   switch (which) {
     case GQE_WS_DISPATCH: return dispatch_ws_layout(*cfg).total;
     case GQE_WS_LAYER: return layer_ws(*cfg).total;
+    case GQE_WS_BACKWARD:
+      return (cfg->flags & ~GQE_FLAG_WS_CLEAN) != 0u ? 0 : bwd_ws(*cfg).total;
     case GQE_WS_DENSE: return dense_ws(*cfg).total;
     case GQE_WS_ATTENTION: {
       const size_t t = attention_plan(*cfg, n_streams(*cfg)).total;
@@ -400,6 +434,70 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
                                      L.total - L.aws, true, stream);
   if (ea != cudaSuccess) return GQE_ERR_CUDA;
   return gqe_output_proj(cfg, H(L.slots), F(L.omega), W_o, y, stream);
+}
+
+gqe_status gqe_layer_bwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r, const float* b_r,
+                         const gqe_bf16* W_q, const gqe_bf16* W_qs, const gqe_bf16* W_k, const gqe_bf16* W_v,
+                         const gqe_bf16* W_o, const float* dy, float* dx, float* dW_r, float* db_r,
+                         float* dW_q, float* dW_qs, float* dW_k, float* dW_v, float* dW_o, void* ws,
+                         size_t ws_bytes, gqe_stream_t stream) {
+  const gqe_status s = check_cfg(cfg);
+  if (s != GQE_OK) return s;
+  if ((cfg->flags & ~GQE_FLAG_WS_CLEAN) != 0u) return GQE_ERR_UNSUPPORTED;  // the default construction only
+  if (!all_aligned(x, W_r, W_q, W_qs, W_k, W_v, W_o, dy, dx, dW_r, dW_q, dW_qs, dW_k, dW_v, dW_o) ||
+      ws == nullptr || !aligned16(ws) || (b_r != nullptr && (reinterpret_cast<uintptr_t>(b_r) & 3u)) ||
+      (db_r != nullptr && (reinterpret_cast<uintptr_t>(db_r) & 3u)))
+    return GQE_ERR_INVALID;
+  const gqe_config& c = *cfg;
+  const BwdWs W = bwd_ws(c);
+  if (ws_bytes < W.total) return GQE_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  auto Fp = [&](size_t o) { return reinterpret_cast<float*>(w + o); };
+  auto Hp = [&](size_t o) { return reinterpret_cast<uint16_t*>(w + o); };
+  // The forward, into the layer part of the workspace (routing, Q, K, V, slots).
+  gqe_status st = gqe_layer_fwd(cfg, x, W_r, b_r, W_q, W_qs, W_k, W_v, W_o, reinterpret_cast<gqe_bf16*>(w + W.y),
+                                ws, W.L.total, stream);
+  if (st != GQE_OK) return st;
+  const LayerWs& L = W.L;
+  const long long R = static_cast<long long>(c.B) * c.T;
+  const int d = c.d_model, dh = c.d_head, gk = c.G * c.k, N = c.G * c.M, Sdh = (gk + 2) * dh;
+  const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
+  const uint16_t* slots = Hp(L.slots);
+  const int Ri = static_cast<int>(R);
+  int e = cudaSuccess;
+  auto ok = [&](int r) { e = r; return r == cudaSuccess; };
+  // a11: dS = dy W_O^T; dW_O = S^T dy.
+  ok(bwd_gemm(dy, d, 1, reinterpret_cast<const uint16_t*>(W_o), 1, d, Fp(W.dS), Sdh, Ri, Sdh, d, false, stream)) &&
+      ok(bwd_gemm(slots, 1, Sdh, dy, d, 1, dW_o, d, Sdh, d, Ri, false, stream)) &&
+      // a10, a4, a2: slots and router -> dO, dz.
+      ok(bwd_slots_router(c, xb, W_r, b_r, reinterpret_cast<const int32_t*>(w + L.idx), Fp(L.omega), slots,
+                          Fp(W.dS), Fp(W.dOr), Fp(W.dOs), Fp(W.dz), stream)) &&
+      // a1: dW_r = x^T dz, db = sum dz, dx = dz W_r^T.
+      ok(bwd_gemm(xb, 1, d, Fp(W.dz), N, 1, dW_r, N, d, N, Ri, false, stream)) &&
+      (db_r == nullptr || ok(bwd_colsum(Fp(W.dz), db_r, R, N, stream))) &&
+      ok(bwd_gemm(Fp(W.dz), N, 1, W_r, 1, N, dx, d, Ri, d, N, false, stream)) &&
+      // a8: attention -> dq, dK, dV.
+      ok(bwd_attention(c, Hp(L.Qv), Hp(L.Qs), Hp(L.K), Hp(L.V), Fp(W.dOr), Fp(W.dOs), Fp(W.stats), Fp(W.dQr),
+                       Fp(W.dQs), Fp(W.dKf), Fp(W.dVf), stream)) &&
+      // a7: routed queries (scattered to their experts' columns) and the shared head.
+      ok(bwd_scatter_dq(c, Fp(W.dQr), reinterpret_cast<const int32_t*>(w + L.idx), Fp(W.dQfull), stream)) &&
+      ok(bwd_gemm(xb, 1, d, Fp(W.dQfull), static_cast<long long>(N) * dh, 1, dW_q, static_cast<long long>(N) * dh, d,
+                  N * dh, Ri, false, stream)) &&
+      ok(bwd_gemm(Fp(W.dQfull), static_cast<long long>(N) * dh, 1, reinterpret_cast<const uint16_t*>(W_q), 1,
+                  static_cast<long long>(N) * dh, dx, d, Ri, d, N * dh, true, stream)) &&
+      ok(bwd_gemm(xb, 1, d, Fp(W.dQs), dh, 1, dW_qs, dh, d, dh, Ri, false, stream)) &&
+      ok(bwd_gemm(Fp(W.dQs), dh, 1, reinterpret_cast<const uint16_t*>(W_qs), 1, dh, dx, d, Ri, d, dh, true,
+                  stream)) &&
+      // a6: K and V.
+      ok(bwd_gemm(xb, 1, d, Fp(W.dKf), static_cast<long long>(c.G) * dh, 1, dW_k, static_cast<long long>(c.G) * dh,
+                  d, c.G * dh, Ri, false, stream)) &&
+      ok(bwd_gemm(Fp(W.dKf), static_cast<long long>(c.G) * dh, 1, reinterpret_cast<const uint16_t*>(W_k), 1,
+                  static_cast<long long>(c.G) * dh, dx, d, Ri, d, c.G * dh, true, stream)) &&
+      ok(bwd_gemm(xb, 1, d, Fp(W.dVf), static_cast<long long>(c.G) * dh, 1, dW_v, static_cast<long long>(c.G) * dh,
+                  d, c.G * dh, Ri, false, stream)) &&
+      ok(bwd_gemm(Fp(W.dVf), static_cast<long long>(c.G) * dh, 1, reinterpret_cast<const uint16_t*>(W_v), 1,
+                  static_cast<long long>(c.G) * dh, dx, d, Ri, d, c.G * dh, true, stream));
+  return cuda_status(e);
 }
 
 gqe_status gqa_dense_fwd(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf16* W_q,

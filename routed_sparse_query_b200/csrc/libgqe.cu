@@ -7,3 +7,4 @@
 #include "decode.cu"
 #include "api.cu"
 #include "noalloc.cu"
+#include "backward.cu"
