@@ -86,30 +86,43 @@ LayerWs layer_ws(const gqe_config& c) {
 // recomputation, then the fp32 gradients in flight.
 struct BwdWs {
   LayerWs L;
-  size_t y, dS, dOr, dOs, dz, stats, dQr, dQs, dQfull, dKf, dVf, total;
+  size_t y, dS, dOr, dOs, dz, stats, dQr, dQs, dKf, dVf;  // fp32
+  size_t dy16, WoT, sT, xT, WcT, Y;                       // bf16 operands of the tensor-core GEMMs
+  long long ldR, ldS, Kcat, zoff;
+  size_t total;
 };
 
 BwdWs bwd_ws(const gqe_config& c) {
   BwdWs W{};
   W.L = layer_ws(c);
-  const size_t R = static_cast<size_t>(c.B) * c.T, dh = c.d_head;
+  const size_t R = static_cast<size_t>(c.B) * c.T, dh = c.d_head, d = c.d_model;
   const size_t gk = static_cast<size_t>(c.G) * c.k, N = static_cast<size_t>(c.G) * c.M;
+  const size_t Sdh = (gk + 2) * dh;
+  W.ldR = static_cast<long long>((R + 7) / 8 * 8);
+  W.ldS = static_cast<long long>((Sdh + 63) / 64 * 64);
+  W.zoff = static_cast<long long>(N * dh + dh + 2 * c.G * dh);
+  W.Kcat = W.zoff + static_cast<long long>((N + 63) / 64 * 64);
   size_t o = W.L.total;
   auto put = [&](size_t& field, size_t bytes) {
     field = o;
     o = round256(o + bytes);
   };
-  put(W.y, R * c.d_model * 2);
-  put(W.dS, R * (gk + 2) * dh * 4);
+  put(W.y, R * d * 2);
+  put(W.dS, R * Sdh * 4);
   put(W.dOr, R * gk * dh * 4);
   put(W.dOs, R * dh * 4);
   put(W.dz, R * N * 4);
   put(W.stats, static_cast<size_t>(c.B) * (gk + 1) * c.T * 3 * 4);
   put(W.dQr, R * gk * dh * 4);
   put(W.dQs, R * dh * 4);
-  put(W.dQfull, R * N * dh * 4);
   put(W.dKf, R * c.G * dh * 4);
   put(W.dVf, R * c.G * dh * 4);
+  put(W.dy16, R * d * 2);
+  put(W.WoT, d * W.ldS * 2);
+  put(W.sT, Sdh * W.ldR * 2);
+  put(W.xT, d * W.ldR * 2);
+  put(W.WcT, static_cast<size_t>(W.Kcat) * d * 2);
+  put(W.Y, R * W.Kcat * 2);
   W.total = o;
   return W;
 }
@@ -464,39 +477,43 @@ gqe_status gqe_layer_bwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
   const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
   const uint16_t* slots = Hp(L.slots);
   const int Ri = static_cast<int>(R);
+  const long long c1 = static_cast<long long>(N) * dh, c2 = c1 + dh, c3 = c2 + static_cast<long long>(c.G) * dh,
+                  c4 = W.zoff, Kc = W.Kcat;
+  const int Gdh = c.G * dh;
+  uint16_t* dy16 = Hp(W.dy16);
+  uint16_t* WcT = Hp(W.WcT);
+  uint16_t* Y = Hp(W.Y);
+  auto U = [](const gqe_bf16* p) { return reinterpret_cast<const uint16_t*>(p); };
   int e = cudaSuccess;
   auto ok = [&](int r) { e = r; return r == cudaSuccess; };
-  // a11: dS = dy W_O^T; dW_O = S^T dy.
-  ok(bwd_gemm(dy, d, 1, reinterpret_cast<const uint16_t*>(W_o), 1, d, Fp(W.dS), Sdh, Ri, Sdh, d, false, stream)) &&
-      ok(bwd_gemm(slots, 1, Sdh, dy, d, 1, dW_o, d, Sdh, d, Ri, false, stream)) &&
-      // a10, a4, a2: slots and router -> dO, dz.
+  // a11: dS = dy W_O^T; dW_O = S^T dy (tensor cores, bf16 operands).
+  ok(bwd_cast(dy, d, R, d, dy16, d, stream)) && ok(bwd_transpose(U(W_o), d, Sdh, d, Hp(W.WoT), W.ldS, stream)) &&
+      ok(gemm_f32out(dy16, d, Ri, d, Hp(W.WoT), W.ldS, Sdh, Fp(W.dS), Sdh, stream)) &&
+      ok(bwd_transpose(slots, Sdh, Ri, Sdh, Hp(W.sT), W.ldR, stream)) &&
+      ok(gemm_f32out(Hp(W.sT), W.ldR, Sdh, Ri, dy16, d, d, dW_o, d, stream)) &&
+      // a10, a4, a2: slots and router -> dO, dz; db = sum dz.
       ok(bwd_slots_router(c, xb, W_r, b_r, reinterpret_cast<const int32_t*>(w + L.idx), Fp(L.omega), slots,
                           Fp(W.dS), Fp(W.dOr), Fp(W.dOs), Fp(W.dz), stream)) &&
-      // a1: dW_r = x^T dz, db = sum dz, dx = dz W_r^T.
-      ok(bwd_gemm(xb, 1, d, Fp(W.dz), N, 1, dW_r, N, d, N, Ri, false, stream)) &&
       (db_r == nullptr || ok(bwd_colsum(Fp(W.dz), db_r, R, N, stream))) &&
-      ok(bwd_gemm(Fp(W.dz), N, 1, W_r, 1, N, dx, d, Ri, d, N, false, stream)) &&
       // a8: attention -> dq, dK, dV.
       ok(bwd_attention(c, Hp(L.Qv), Hp(L.Qs), Hp(L.K), Hp(L.V), Fp(W.dOr), Fp(W.dOs), Fp(W.stats), Fp(W.dQr),
                        Fp(W.dQs), Fp(W.dKf), Fp(W.dVf), stream)) &&
-      // a7: routed queries (scattered to their experts' columns) and the shared head.
-      ok(bwd_scatter_dq(c, Fp(W.dQr), reinterpret_cast<const int32_t*>(w + L.idx), Fp(W.dQfull), stream)) &&
-      ok(bwd_gemm(xb, 1, d, Fp(W.dQfull), static_cast<long long>(N) * dh, 1, dW_q, static_cast<long long>(N) * dh, d,
-                  N * dh, Ri, false, stream)) &&
-      ok(bwd_gemm(Fp(W.dQfull), static_cast<long long>(N) * dh, 1, reinterpret_cast<const uint16_t*>(W_q), 1,
-                  static_cast<long long>(N) * dh, dx, d, Ri, d, N * dh, true, stream)) &&
-      ok(bwd_gemm(xb, 1, d, Fp(W.dQs), dh, 1, dW_qs, dh, d, dh, Ri, false, stream)) &&
-      ok(bwd_gemm(Fp(W.dQs), dh, 1, reinterpret_cast<const uint16_t*>(W_qs), 1, dh, dx, d, Ri, d, dh, true,
-                  stream)) &&
-      // a6: K and V.
-      ok(bwd_gemm(xb, 1, d, Fp(W.dKf), static_cast<long long>(c.G) * dh, 1, dW_k, static_cast<long long>(c.G) * dh,
-                  d, c.G * dh, Ri, false, stream)) &&
-      ok(bwd_gemm(Fp(W.dKf), static_cast<long long>(c.G) * dh, 1, reinterpret_cast<const uint16_t*>(W_k), 1,
-                  static_cast<long long>(c.G) * dh, dx, d, Ri, d, c.G * dh, true, stream)) &&
-      ok(bwd_gemm(xb, 1, d, Fp(W.dVf), static_cast<long long>(c.G) * dh, 1, dW_v, static_cast<long long>(c.G) * dh,
-                  d, c.G * dh, Ri, false, stream)) &&
-      ok(bwd_gemm(Fp(W.dVf), static_cast<long long>(c.G) * dh, 1, reinterpret_cast<const uint16_t*>(W_v), 1,
-                  static_cast<long long>(c.G) * dh, dx, d, Ri, d, c.G * dh, true, stream));
+      // a7, a6, a1: Y = [dQ (routed, scattered to their experts) | dQs | dK | dV | dz];
+      // dx = Y [W_q | W_qs | W_k | W_v | W_r]^T; each weight gradient = x^T (its columns of Y).
+      ok(bwd_pack(c, Fp(W.dQr), Fp(W.dQs), Fp(W.dKf), Fp(W.dVf), Fp(W.dz), reinterpret_cast<const int32_t*>(w + L.idx),
+                  Y, static_cast<int>(Kc), stream)) &&
+      ok(bwd_transpose(U(W_q), c1, d, static_cast<int>(c1), WcT, d, stream)) &&
+      ok(bwd_transpose(U(W_qs), dh, d, dh, WcT + c1 * d, d, stream)) &&
+      ok(bwd_transpose(U(W_k), Gdh, d, Gdh, WcT + c2 * d, d, stream)) &&
+      ok(bwd_transpose(U(W_v), Gdh, d, Gdh, WcT + c3 * d, d, stream)) &&
+      ok(bwd_transpose(W_r, N, d, N, WcT + c4 * d, d, stream)) &&
+      ok(gemm_f32out(Y, Kc, Ri, static_cast<int>(c4 + N), WcT, d, d, dx, d, stream)) &&
+      ok(bwd_transpose(xb, d, Ri, d, Hp(W.xT), W.ldR, stream)) &&
+      ok(gemm_f32out(Hp(W.xT), W.ldR, d, Ri, Y, Kc, static_cast<int>(c1), dW_q, c1, stream)) &&
+      ok(gemm_f32out(Hp(W.xT), W.ldR, d, Ri, Y + c1, Kc, dh, dW_qs, dh, stream)) &&
+      ok(gemm_f32out(Hp(W.xT), W.ldR, d, Ri, Y + c2, Kc, Gdh, dW_k, Gdh, stream)) &&
+      ok(gemm_f32out(Hp(W.xT), W.ldR, d, Ri, Y + c3, Kc, Gdh, dW_v, Gdh, stream)) &&
+      ok(gemm_f32out(Hp(W.xT), W.ldR, d, Ri, Y + c4, Kc, N, dW_r, N, stream));
   return cuda_status(e);
 }
 

@@ -6,12 +6,16 @@
 // router": gist.science Technical Summary, "Output Construction"; pptc.cn
 // blog section 4.3).
 //
-// A first, plain path on the CUDA cores, in fp32 throughout, on the forward's
-// own intermediates (recomputed by the forward kernels: routing, Q, K, V,
-// slots):
-//   - gemm_f32_kernel: C (+)= A B for any strides of A and B (bf16 or fp32),
-//     64 x 64 tiles through shared memory. It carries dS = dy W_O^T,
-//     dW_O = S^T dy and every weight and input gradient of the projections;
+// On the forward's own intermediates (recomputed by the forward kernels:
+// routing, Q, K, V, slots). The contractions of the projections (dS = dy W_O^T,
+// dW_O = S^T dy, dx and every weight gradient) run on the tensor cores
+// through the projection GEMM (fp32 output) on bf16 copies of their
+// operands, made here:
+//   - transpose_kernel / cast_kernel: bf16 copies (x^T, S^T, W_O^T, the
+//     projection weights transposed, dy);
+//   - pack_grads_kernel: the rows of [dQ of every expert | dQ of the shared
+//     head | dK | dV | dz] in bf16, the A operand of dx and the B operand of
+//     every weight gradient;
 //   - slot_router_bwd_kernel, one CTA per token: the slots' backward (routed
 //     outputs, shared head, weighted slot) and the router's (the renormalised
 //     weights' quotient rule, then each group's softmax Jacobian) -> dz;
@@ -35,59 +39,6 @@ namespace bwd_impl {
 
 __device__ __forceinline__ float to_f(uint16_t v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
 __device__ __forceinline__ float to_f(float v) { return v; }
-
-template <typename TA, typename TB>
-__global__ void __launch_bounds__(256) gemm_f32_kernel(const TA* A, long long sam, long long sak, const TB* B,
-                                                       long long sbk, long long sbn, float* C, long long ldc,
-                                                       int M, int N, int K, int beta) {
-  __shared__ float As[16][65];  // [k][m]
-  __shared__ float Bs[16][65];  // [k][n]
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const long long m0 = static_cast<long long>(blockIdx.y) * 64, n0 = static_cast<long long>(blockIdx.x) * 64;
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    for (int q = threadIdx.x; q < 1024; q += 256) {
-      const int mm = q >> 4, ka = q & 15;
-      const long long gm = m0 + mm;
-      const int gk = k0 + ka;
-      As[ka][mm] = (gm < M && gk < K) ? to_f(A[gm * sam + gk * sak]) : 0.0f;
-      const int kb = q >> 6, nn = q & 63;
-      const long long gn = n0 + nn;
-      const int gk2 = k0 + kb;
-      Bs[kb][nn] = (gk2 < K && gn < N) ? to_f(B[gk2 * sbk + gn * sbn]) : 0.0f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a[i] = As[kk][ty * 4 + i];
-        b[i] = Bs[kk][tx * 4 + i];
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const long long gm = m0 + ty * 4 + i, gn = n0 + tx * 4 + j;
-      if (gm < M && gn < N) {
-        float v = acc[i][j];
-        if (beta) v += C[gm * ldc + gn];
-        C[gm * ldc + gn] = v;
-      }
-    }
-}
 
 struct SlotArgs {
   const uint16_t* x;      // [R, d]
@@ -475,22 +426,71 @@ __global__ void __launch_bounds__(256) attn_keys_bwd_kernel(AttnBwdArgs a) {
   }
 }
 
-// dQfull[r, e*dh + c] = dq of the slot of row r that selected expert e, 0 for
-// the experts the row did not select.
-__global__ void scatter_dq_kernel(const float* dQr, const int32_t* idx, float* dQfull, long long R, int G,
-                                  int M, int k, int dh) {
-  const long long n = R * G * M * dh;
+__device__ __forceinline__ uint16_t bf16_rn(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+
+// out[c, r] = bf16(in[r, c]) for r < rows, c < cols: 32 x 32 tiles through
+// shared memory (block 32 x 8), both sides coalesced.
+template <typename TI>
+__global__ void __launch_bounds__(256) transpose_kernel(const TI* in, long long ldi, int rows, int cols,
+                                                        uint16_t* out, long long ldo) {
+  __shared__ float tile[32][33];
+  const long long r0 = static_cast<long long>(blockIdx.y) * 32, c0 = static_cast<long long>(blockIdx.x) * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const long long r = r0 + i, c = c0 + threadIdx.x;
+    tile[i][threadIdx.x] = (r < rows && c < cols) ? to_f(in[r * ldi + c]) : 0.0f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const long long c = c0 + i, r = r0 + threadIdx.x;
+    if (c < cols && r < rows) out[c * ldo + r] = bf16_rn(tile[threadIdx.x][i]);
+  }
+}
+
+// out[r, c] = bf16(in[r, c]) (row strides ldi, ldo).
+__global__ void cast_kernel(const float* in, long long ldi, long long rows, int cols, uint16_t* out, long long ldo) {
+  const long long n = rows * cols;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(i % dh);
-    const long long re = i / dh;
-    const int e = static_cast<int>(re % (G * M));
-    const long long r = re / (G * M);
-    const int g = e / M, j = e - g * M;
-    float v = 0.0f;
-    for (int s = 0; s < k; ++s)
-      if (idx[(r * G + g) * k + s] == j) v = dQr[((r * G + g) * k + s) * dh + c];
-    dQfull[i] = v;
+    const long long r = i / cols;
+    const int c = static_cast<int>(i - r * cols);
+    out[r * ldo + c] = bf16_rn(in[r * ldi + c]);
+  }
+}
+
+// Row r of Y (bf16, ld columns): [dQ of every expert (the slot of row r that
+// selected expert e, 0 where none did) | dQ of the shared head | dK | dV |
+// dz | 0 padding]. Each thread writes two adjacent columns.
+__global__ void pack_grads_kernel(const float* dQr, const float* dQs, const float* dKf, const float* dVf,
+                                  const float* dz, const int32_t* idx, uint16_t* Y, long long R, int G, int M,
+                                  int k, int dh, int ld) {
+  const int N = G * M, c1 = N * dh, c2 = c1 + dh, c3 = c2 + G * dh, c4 = c3 + G * dh, c5 = c4 + N;
+  const int half = ld / 2;
+  const long long n = R * half;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / half;
+    const int c = 2 * static_cast<int>(i - r * half);
+    float v[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int cc = c + q;
+      if (cc < c1) {
+        const int e = cc / dh, col = cc - e * dh, g = e / M, j = e - g * M;
+        const int32_t* ip = idx + (r * G + g) * k;
+        for (int s = 0; s < k; ++s)
+          if (ip[s] == j) v[q] = dQr[((r * G + g) * k + s) * dh + col];
+      } else if (cc < c2) {
+        v[q] = dQs[r * dh + (cc - c1)];
+      } else if (cc < c3) {
+        v[q] = dKf[r * G * dh + (cc - c2)];
+      } else if (cc < c4) {
+        v[q] = dVf[r * G * dh + (cc - c3)];
+      } else if (cc < c5) {
+        v[q] = dz[r * N + (cc - c4)];
+      }
+    }
+    *reinterpret_cast<uint32_t*>(Y + r * ld + c) = static_cast<uint32_t>(bf16_rn(v[0])) |
+                                                  (static_cast<uint32_t>(bf16_rn(v[1])) << 16);
   }
 }
 
@@ -512,22 +512,29 @@ __global__ void colsum_kernel(const float* dz, float* db, long long R, int N) {
 }  // namespace bwd_impl
 using namespace bwd_impl;
 
-template <typename TA, typename TB>
-int bwd_gemm(const TA* A, long long sam, long long sak, const TB* B, long long sbk, long long sbn, float* C,
-             long long ldc, int M, int N, int K, bool accumulate, void* stream) {
-  if (M <= 0 || N <= 0) return cudaSuccess;
-  const dim3 grid(static_cast<unsigned>((N + 63) / 64), static_cast<unsigned>((M + 63) / 64));
+template <typename TI>
+int bwd_transpose(const TI* in, long long ldi, int rows, int cols, uint16_t* out, long long ldo, void* stream) {
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
+  const dim3 grid(static_cast<unsigned>((cols + 31) / 32), static_cast<unsigned>((rows + 31) / 32));
   if (grid.y > 65535u) return cudaErrorInvalidConfiguration;
-  gemm_f32_kernel<TA, TB><<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(A, sam, sak, B, sbk, sbn, C, ldc,
-                                                                              M, N, K, accumulate ? 1 : 0);
+  transpose_kernel<TI><<<grid, dim3(32, 8), 0, static_cast<cudaStream_t>(stream)>>>(in, ldi, rows, cols, out, ldo);
   return cudaGetLastError();
 }
-template int bwd_gemm<uint16_t, float>(const uint16_t*, long long, long long, const float*, long long, long long,
-                                       float*, long long, int, int, int, bool, void*);
-template int bwd_gemm<float, uint16_t>(const float*, long long, long long, const uint16_t*, long long, long long,
-                                       float*, long long, int, int, int, bool, void*);
-template int bwd_gemm<float, float>(const float*, long long, long long, const float*, long long, long long,
-                                    float*, long long, int, int, int, bool, void*);
+template int bwd_transpose<uint16_t>(const uint16_t*, long long, int, int, uint16_t*, long long, void*);
+template int bwd_transpose<float>(const float*, long long, int, int, uint16_t*, long long, void*);
+
+int bwd_cast(const float* in, long long ldi, long long rows, int cols, uint16_t* out, long long ldo, void* stream) {
+  cast_kernel<<<1024, 256, 0, static_cast<cudaStream_t>(stream)>>>(in, ldi, rows, cols, out, ldo);
+  return cudaGetLastError();
+}
+
+int bwd_pack(const gqe_config& c, const float* dQr, const float* dQs, const float* dKf, const float* dVf,
+             const float* dz, const int32_t* idx, uint16_t* Y, int ld, void* stream) {
+  const long long R = static_cast<long long>(c.B) * c.T;
+  pack_grads_kernel<<<1184, 256, 0, static_cast<cudaStream_t>(stream)>>>(dQr, dQs, dKf, dVf, dz, idx, Y, R, c.G,
+                                                                         c.M, c.k, c.d_head, ld);
+  return cudaGetLastError();
+}
 
 int bwd_slots_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r,
                      const int32_t* idx, const float* omega, const uint16_t* slots, const float* dS, float* dOr,
@@ -556,13 +563,6 @@ int bwd_attention(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, c
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   attn_keys_bwd_kernel<<<static_cast<unsigned>(key_ctas), 256, smem_keys, st>>>(a);
-  return cudaGetLastError();
-}
-
-int bwd_scatter_dq(const gqe_config& c, const float* dQr, const int32_t* idx, float* dQfull, void* stream) {
-  const long long R = static_cast<long long>(c.B) * c.T;
-  scatter_dq_kernel<<<1024, 256, 0, static_cast<cudaStream_t>(stream)>>>(dQr, idx, dQfull, R, c.G, c.M, c.k,
-                                                                         c.d_head);
   return cudaGetLastError();
 }
 

@@ -69,6 +69,11 @@ struct Epi {
   const float* omega = nullptr;
   uint16_t* wslots = nullptr;  // A itself, written back by the blockIdx.y == 0 CTAs
   int lda = 0;                 // A row length (elements)
+  // fp32 output instead (row-major, row stride ldf): C[row, col] for
+  // row < rows, col < cols. fvec: ldf and outf allow 16-byte stores.
+  float* outf = nullptr;
+  long long ldf = 0;
+  int fvec = 0;
 };
 
 struct Gather {
@@ -370,6 +375,28 @@ __global__ void __launch_bounds__(192, 2)
         uint32_t v[32];
         tmem_ld32(trow + cc * 32, v);
         if (valid) store32_bf16((shared_tile ? ga.Qs : ga.Qv) + obase + cc * 32, v);
+      }
+    } else if (epi.outf != nullptr) {
+      const int row = m0 + r;
+      const bool valid = have && row < epi.rows;
+      float* orow = epi.outf + static_cast<long long>(row) * epi.ldf;
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(trow + cc * 32, v);
+        const int col0 = n0 + cc * 32;
+        if (!valid || col0 >= epi.cols) continue;
+        if (epi.fvec && col0 + 32 <= epi.cols) {
+          float4* d4 = reinterpret_cast<float4*>(orow + col0);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            d4[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                 __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col0 + j < epi.cols) orow[col0 + j] = __uint_as_float(v[j]);
+        }
       }
     } else {
       const int row = m0 + r;
@@ -753,6 +780,47 @@ Epi head_split(uint16_t* out, int T, int H, int dh, int R) {
 
 }  // namespace gemm_impl
 using namespace gemm_impl;
+
+// C[M, N] (fp32, row stride ldc) = A[M, K] B[K, N]: A bf16 with K contiguous
+// (row stride lda), B bf16 with N contiguous (row stride ldb). Rows, columns
+// and K blocks past the ends read as zero (TMA fill) and are not stored.
+int gemm_f32out(const uint16_t* A, long long lda, int M, int K, const uint16_t* B, long long ldb, int N,
+                float* C, long long ldc, void* stream) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  if (K <= 0 || ((lda | ldb) & 7) != 0 || ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B)) & 15u))
+    return cudaErrorInvalidValue;
+  const long long mt = (M + BM - 1) / BM;
+  int BN = 128;
+  if (N <= 32) BN = 32;
+  else if (N <= 64 || mt * ((N + 127) / 128) < 148) BN = 64;
+  const long long nt = (N + BN - 1) / BN;
+  if (mt > 0x7fffffffll || nt > 65535) return cudaErrorInvalidConfiguration;
+  // B's inner extent is rounded up to whole boxes: the caller's rows are at
+  // least that long (columns past N only reach C columns that are not stored).
+  const int batom = BN >= 64 ? 64 : BN;
+  const long long nb = (N + batom - 1) / batom * batom;
+  if (nb > ldb) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16_2d(&ta, A, K, M, lda, 64, BM)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tb, B, nb, K, ldb, batom, BK)) return cudaErrorInvalidValue;
+  Epi e;
+  e.out = nullptr;
+  e.T = M;
+  e.hd = N;
+  e.sb = e.sh = e.st = 0;
+  e.rows = M;
+  e.cols = N;
+  e.outf = C;
+  e.ldf = ldc;
+  e.fvec = ((ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(C) & 15u) == 0) ? 1 : 0;
+  const dim3 grid(static_cast<unsigned>(mt), static_cast<unsigned>(nt), 1);
+  Gather g{};
+  switch (BN) {
+    case 128: return launch<128, false>(ta, tb, tb, e, e, g, K, grid, stream);
+    case 64: return launch<64, false>(ta, tb, tb, e, e, g, K, grid, stream);
+    default: return launch<32, false>(ta, tb, tb, e, e, g, K, grid, stream);
+  }
+}
 
 int gemm_kv(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
             uint16_t* K, uint16_t* V, void* stream) {

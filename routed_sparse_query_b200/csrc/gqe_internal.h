@@ -156,18 +156,24 @@ int attention_dense(const gqe_config& c, const uint16_t* Q, const uint16_t* K, c
                     uint16_t* O, void* ws, size_t ws_bytes, bool counters_zeroed, void* stream);
 int zero_attention_counters(const gqe_config& c, int H, void* ws, void* stream);
 
-// Backward of the layer (backward.cu): plain CUDA-core kernels, fp32.
-// C[m, n] (+)= sum_k A[m*sam + k*sak] B[k*sbk + n*sbn] (A, B bf16 or fp32).
-template <typename TA, typename TB>
-int bwd_gemm(const TA* A, long long sam, long long sak, const TB* B, long long sbk, long long sbn, float* C,
-             long long ldc, int M, int N, int K, bool accumulate, void* stream);
+// fp32-output tensor-core GEMM (gemm.cu): C[M, N] = A[M, K] B[K, N], A bf16
+// K-contiguous (row stride lda), B bf16 N-contiguous (row stride ldb, rows at
+// least N rounded up to 64 long); lda, ldb multiples of 8.
+int gemm_f32out(const uint16_t* A, long long lda, int M, int K, const uint16_t* B, long long ldb, int N,
+                float* C, long long ldc, void* stream);
+
+// Backward of the layer (backward.cu).
+template <typename TI>
+int bwd_transpose(const TI* in, long long ldi, int rows, int cols, uint16_t* out, long long ldo, void* stream);
+int bwd_cast(const float* in, long long ldi, long long rows, int cols, uint16_t* out, long long ldo, void* stream);
+int bwd_pack(const gqe_config& c, const float* dQr, const float* dQs, const float* dKf, const float* dVf,
+             const float* dz, const int32_t* idx, uint16_t* Y, int ld, void* stream);
 int bwd_slots_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r,
                      const int32_t* idx, const float* omega, const uint16_t* slots, const float* dS, float* dOr,
                      float* dOs, float* dz, void* stream);
 int bwd_attention(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
                   const uint16_t* V, const float* dOr, const float* dOs, float* stats, float* dQr, float* dQs,
                   float* dKf, float* dVf, void* stream);
-int bwd_scatter_dq(const gqe_config& c, const float* dQr, const int32_t* idx, float* dQfull, void* stream);
 int bwd_colsum(const float* dz, float* db, long long R, int N, void* stream);
 
 // Decode step. cfg.T = keys after the step (the new token sits at T - 1),
