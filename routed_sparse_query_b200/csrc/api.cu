@@ -87,7 +87,7 @@ LayerWs layer_ws(const gqe_config& c) {
 struct BwdWs {
   LayerWs L;
   size_t y, dS, dOr, dOs, dz, stats, dQr, dQs, dKf, dVf;  // fp32
-  size_t dy16, WoT, sT, xT, WcT, Y;                       // bf16 operands of the tensor-core GEMMs
+  size_t dy16, WoT, sT, xT, WcT, Y, dO16;                 // bf16 operands of the tensor-core GEMMs
   long long ldR, ldS, Kcat, zoff;
   size_t total;
 };
@@ -112,7 +112,7 @@ BwdWs bwd_ws(const gqe_config& c) {
   put(W.dOr, R * gk * dh * 4);
   put(W.dOs, R * dh * 4);
   put(W.dz, R * N * 4);
-  put(W.stats, static_cast<size_t>(c.B) * (gk + 1) * c.T * 3 * 4);
+  put(W.stats, static_cast<size_t>(c.B) * (gk + 1) * c.T * 8);
   put(W.dQr, R * gk * dh * 4);
   put(W.dQs, R * dh * 4);
   put(W.dKf, R * c.G * dh * 4);
@@ -123,6 +123,7 @@ BwdWs bwd_ws(const gqe_config& c) {
   put(W.xT, d * W.ldR * 2);
   put(W.WcT, static_cast<size_t>(W.Kcat) * d * 2);
   put(W.Y, R * W.Kcat * 2);
+  put(W.dO16, R * (gk + 1) * dh * 2);
   W.total = o;
   return W;
 }
@@ -493,11 +494,11 @@ gqe_status gqe_layer_bwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
       ok(gemm_f32out(Hp(W.sT), W.ldR, Sdh, Ri, dy16, d, d, dW_o, d, stream)) &&
       // a10, a4, a2: slots and router -> dO, dz; db = sum dz.
       ok(bwd_slots_router(c, xb, W_r, b_r, reinterpret_cast<const int32_t*>(w + L.idx), Fp(L.omega), slots,
-                          Fp(W.dS), Fp(W.dOr), Fp(W.dOs), Fp(W.dz), stream)) &&
+                          Fp(W.dS), Fp(W.dOr), Fp(W.dOs), Fp(W.dz), Hp(W.dO16), stream)) &&
       (db_r == nullptr || ok(bwd_colsum(Fp(W.dz), db_r, R, N, stream))) &&
       // a8: attention -> dq, dK, dV.
-      ok(bwd_attention(c, Hp(L.Qv), Hp(L.Qs), Hp(L.K), Hp(L.V), Fp(W.dOr), Fp(W.dOs), Fp(W.stats), Fp(W.dQr),
-                       Fp(W.dQs), Fp(W.dKf), Fp(W.dVf), stream)) &&
+      ok(bwd_attention_tc(c, Hp(L.Qv), Hp(L.Qs), Hp(L.K), Hp(L.V), Hp(W.dO16), Fp(W.dOr), Fp(W.dOs), slots,
+                          Fp(W.stats), Fp(W.dQr), Fp(W.dQs), Fp(W.dKf), Fp(W.dVf), stream)) &&
       // a7, a6, a1: Y = [dQ (routed, scattered to their experts) | dQs | dK | dV | dz];
       // dx = Y [W_q | W_qs | W_k | W_v | W_r]^T; each weight gradient = x^T (its columns of Y).
       ok(bwd_pack(c, Fp(W.dQr), Fp(W.dQs), Fp(W.dKf), Fp(W.dVf), Fp(W.dz), reinterpret_cast<const int32_t*>(w + L.idx),

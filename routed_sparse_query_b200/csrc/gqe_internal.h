@@ -170,10 +170,13 @@ int bwd_pack(const gqe_config& c, const float* dQr, const float* dQs, const floa
              const float* dz, const int32_t* idx, uint16_t* Y, int ld, void* stream);
 int bwd_slots_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r,
                      const int32_t* idx, const float* omega, const uint16_t* slots, const float* dS, float* dOr,
-                     float* dOs, float* dz, void* stream);
-int bwd_attention(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
-                  const uint16_t* V, const float* dOr, const float* dOs, float* stats, float* dQr, float* dQs,
-                  float* dKf, float* dVf, void* stream);
+                     float* dOs, float* dz, uint16_t* dO16, void* stream);
+// Attention backward on tcgen05 (attn_bwd.cu): dq of every stream, dK and dV
+// of every group; stats [B, G*k+1, T] float2 scratch.
+int bwd_attention_tc(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
+                     const uint16_t* V, const uint16_t* dO16, const float* dOr, const float* dOs,
+                     const uint16_t* slots, float* stats, float* dQr, float* dQs, float* dKf, float* dVf,
+                     void* stream);
 int bwd_colsum(const float* dz, float* db, long long R, int N, void* stream);
 
 // Decode step. cfg.T = keys after the step (the new token sits at T - 1),

@@ -8,3 +8,4 @@
 #include "api.cu"
 #include "noalloc.cu"
 #include "backward.cu"
+#include "attn_bwd.cu"
