@@ -677,6 +677,22 @@ def run_ours(args, rank: int, world: int, dist):
     return out
 
 
+def backward_flops(shape) -> float:
+    """Algorithmic FLOPs of one layer backward (selection fixed; the forward
+    recomputation not counted). Attention, per stream and causal (query, key)
+    pair: S recomputed, dP = dO V^T, dQ, dK, dV -- five products of 2 dh
+    FLOPs. Projections: dS = dy W_O^T and dW_O = S^T dy (2 R d S dh each),
+    dx and the weight gradients over the concatenated columns
+    [Q of every expert | shared Q | K | V | router] (2 R d C each)."""
+    B, T, d, G, M, k, dh = shape.B, shape.T, shape.d_model, shape.G, shape.M, shape.k, shape.d_head
+    R, N = B * T, G * M
+    streams = B * (G * k + 1)
+    attn = 5 * 2 * dh * (T * (T + 1) // 2) * streams
+    sdh = (G * k + 2) * dh
+    cols = N * dh + dh + 2 * G * dh + N
+    return float(attn + 2 * (2 * R * d * sdh) + 2 * (2 * R * d * cols))
+
+
 def backward_bench(rsq, shape, d, steps: int = 5) -> dict:
     """One gqe_layer_bwd call (forward recomputation included) on the bench
     workload, CUDA-event timed after two warm-up calls; dy ~ N(0, 1)."""
@@ -703,9 +719,12 @@ def backward_bench(rsq, shape, d, steps: int = 5) -> dict:
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
+    fl = backward_flops(shape)
     return {"workload": describe(shape), "ms_per_call": ms, "tokens_per_s": R / (ms / 1e3), "steps": steps,
-            "path": "first CUDA-core path (forward recomputed first; fp32 GEMMs, attention backward, router "
-                    "backward through the weighted slot); no tensor cores yet"}
+            "flops": fl, "tflops_excl_forward": fl / (ms / 1e3) / 1e12,
+            "path": "forward recomputed (attention keeps each row's log-sum-exp); tcgen05 attention backward "
+                    "(dQ per query tile, dK/dV per key tile); projection gradients on the tcgen05 GEMM with an "
+                    "fp32 epilogue; router backward through the weighted slot on the CUDA cores"}
 
 
 DECODE = {"batch": 64, "cache": 32768}  # decode measurement: 64 sequences, 32k cached tokens
@@ -871,7 +890,15 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-pool", action="store_true",
                     help="skip the expert-pool workloads (32 experts, k = 1, 2; skewed, balanced)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time only the layer backward (gqe_layer_bwd) on --workload, --steps calls")
     args = ap.parse_args()
+    if args.backward:
+        import routed_sparse_query_b200 as rsq
+        shape = WORKLOADS[args.workload]
+        d = device_inputs_from_synth(synth.make_layer_inputs(shape))
+        print(json.dumps(backward_bench(rsq, shape, d, steps=args.steps)), flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -376,14 +376,16 @@ gqe_status gqa_dense_decode_step(const gqe_config* cfg, const gqe_bf16* x, const
  * router": gist.science Technical Summary, Output Construction). Through the
  * weighted slot the router gets d(omega) = <o, dS_w>, the quotient rule of
  * omega = p_sel / sum(p_sel) and each group's softmax Jacobian. The forward
- * is recomputed first (as gqe_layer_fwd, into the scratch) and the gradients
- * use its bf16 intermediates (routing, Q, K, V, slots), accumulated in fp32.
+ * is recomputed first (as gqe_layer_fwd, into the scratch; the attention also
+ * keeps each row's log-sum-exp) and the gradients use its bf16 intermediates
+ * (routing, Q, K, V, slots). The products run on the tensor cores with bf16
+ * operands (dy, dO, P, dS and the gradients of Q, K, V and the router logits
+ * each rounded once) and fp32 accumulation; the result is deterministic.
  * Outputs (fp32, overwritten): dx [B*T, d_model], dW_r [d_model, N],
  * db_r [N] (NULL: not computed), dW_q [d_model, N*d_head],
  * dW_qs [d_model, d_head], dW_k, dW_v [d_model, G*d_head],
  * dW_o [(kG+2)*d_head, d_model]. Inputs as in gqe_layer_fwd.
- * Scratch: >= gqe_workspace_bytes(cfg, GQE_WS_BACKWARD). A first path on the
- * CUDA cores (no tensor cores yet).
+ * Scratch: >= gqe_workspace_bytes(cfg, GQE_WS_BACKWARD).
  */
 gqe_status gqe_layer_bwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r, const float* b_r,
                          const gqe_bf16* W_q, const gqe_bf16* W_qs, const gqe_bf16* W_k, const gqe_bf16* W_v,

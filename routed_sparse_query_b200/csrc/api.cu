@@ -86,8 +86,9 @@ LayerWs layer_ws(const gqe_config& c) {
 // recomputation, then the fp32 gradients in flight.
 struct BwdWs {
   LayerWs L;
-  size_t y, dS, dOr, dOs, dz, stats, dQr, dQs, dKf, dVf;  // fp32
+  size_t y, dS, dOr, dOs, dz, stats, dQr, dQs, dKp, dVp;  // fp32
   size_t dy16, WoT, sT, xT, WcT, Y, dO16;                 // bf16 operands of the tensor-core GEMMs
+  size_t lse, zl;                                         // the forward attention's row statistics; logits
   long long ldR, ldS, Kcat, zoff;
   size_t total;
 };
@@ -112,11 +113,11 @@ BwdWs bwd_ws(const gqe_config& c) {
   put(W.dOr, R * gk * dh * 4);
   put(W.dOs, R * dh * 4);
   put(W.dz, R * N * 4);
-  put(W.stats, static_cast<size_t>(c.B) * (gk + 1) * c.T * 8);
+  put(W.stats, static_cast<size_t>(c.B) * (gk + 1) * ((c.T + 63) / 64 * 64) * 8);
   put(W.dQr, R * gk * dh * 4);
   put(W.dQs, R * dh * 4);
-  put(W.dKf, R * c.G * dh * 4);
-  put(W.dVf, R * c.G * dh * 4);
+  put(W.dKp, R * (gk + 1) * dh * 4);
+  put(W.dVp, R * (gk + 1) * dh * 4);
   put(W.dy16, R * d * 2);
   put(W.WoT, d * W.ldS * 2);
   put(W.sT, Sdh * W.ldR * 2);
@@ -124,6 +125,8 @@ BwdWs bwd_ws(const gqe_config& c) {
   put(W.WcT, static_cast<size_t>(W.Kcat) * d * 2);
   put(W.Y, R * W.Kcat * 2);
   put(W.dO16, R * (gk + 1) * dh * 2);
+  put(W.lse, static_cast<size_t>(c.B) * (gk + 1) * ((c.T + 63) / 64 * 64) * 4);
+  put(W.zl, R * N * 4);
   W.total = o;
   return W;
 }
@@ -393,10 +396,12 @@ gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* 
   return cuda_status(gemm_output(*cfg, slots, omega, W_o, y, stream));
 }
 
-gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
-                         const float* b_r, const gqe_bf16* W_q, const gqe_bf16* W_qs,
-                         const gqe_bf16* W_k, const gqe_bf16* W_v, const gqe_bf16* W_o,
-                         gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream_t stream) {
+// The layer forward; lse (optional, slot-major attention only) receives the
+// attention rows' log-sum-exp for the backward.
+static gqe_status layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r, const float* b_r,
+                            const gqe_bf16* W_q, const gqe_bf16* W_qs, const gqe_bf16* W_k, const gqe_bf16* W_v,
+                            const gqe_bf16* W_o, gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream_t stream,
+                            float* lse) {
   const gqe_status s = check_cfg(cfg);
   if (s != GQE_OK) return s;
   const bool shared = has_shared_head(*cfg);
@@ -445,9 +450,16 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
                      ? attention_gqe_em(*cfg, H(L.Qv), H(L.Qs), H(L.K), H(L.V), I(L.idx), I(L.offsets),
                                         I(L.tok), H(L.slots), stream)
                      : attention_gqe(*cfg, H(L.Qv), H(L.Qs), H(L.K), H(L.V), H(L.slots), w + L.aws,
-                                     L.total - L.aws, true, stream);
+                                     L.total - L.aws, true, stream, lse);
   if (ea != cudaSuccess) return GQE_ERR_CUDA;
   return gqe_output_proj(cfg, H(L.slots), F(L.omega), W_o, y, stream);
+}
+
+gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
+                         const float* b_r, const gqe_bf16* W_q, const gqe_bf16* W_qs,
+                         const gqe_bf16* W_k, const gqe_bf16* W_v, const gqe_bf16* W_o,
+                         gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream_t stream) {
+  return layer_fwd(cfg, x, W_r, b_r, W_q, W_qs, W_k, W_v, W_o, y, ws, ws_bytes, stream, nullptr);
 }
 
 gqe_status gqe_layer_bwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r, const float* b_r,
@@ -469,8 +481,8 @@ gqe_status gqe_layer_bwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
   auto Fp = [&](size_t o) { return reinterpret_cast<float*>(w + o); };
   auto Hp = [&](size_t o) { return reinterpret_cast<uint16_t*>(w + o); };
   // The forward, into the layer part of the workspace (routing, Q, K, V, slots).
-  gqe_status st = gqe_layer_fwd(cfg, x, W_r, b_r, W_q, W_qs, W_k, W_v, W_o, reinterpret_cast<gqe_bf16*>(w + W.y),
-                                ws, W.L.total, stream);
+  gqe_status st = layer_fwd(cfg, x, W_r, b_r, W_q, W_qs, W_k, W_v, W_o, reinterpret_cast<gqe_bf16*>(w + W.y), ws,
+                            W.L.total, stream, Fp(W.lse));
   if (st != GQE_OK) return st;
   const LayerWs& L = W.L;
   const long long R = static_cast<long long>(c.B) * c.T;
@@ -493,15 +505,15 @@ gqe_status gqe_layer_bwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
       ok(bwd_transpose(slots, Sdh, Ri, Sdh, Hp(W.sT), W.ldR, stream)) &&
       ok(gemm_f32out(Hp(W.sT), W.ldR, Sdh, Ri, dy16, d, d, dW_o, d, stream)) &&
       // a10, a4, a2: slots and router -> dO, dz; db = sum dz.
-      ok(bwd_slots_router(c, xb, W_r, b_r, reinterpret_cast<const int32_t*>(w + L.idx), Fp(L.omega), slots,
+      ok(bwd_slots_router(c, xb, W_r, b_r, Fp(W.zl), reinterpret_cast<const int32_t*>(w + L.idx), Fp(L.omega), slots,
                           Fp(W.dS), Fp(W.dOr), Fp(W.dOs), Fp(W.dz), Hp(W.dO16), stream)) &&
       (db_r == nullptr || ok(bwd_colsum(Fp(W.dz), db_r, R, N, stream))) &&
       // a8: attention -> dq, dK, dV.
       ok(bwd_attention_tc(c, Hp(L.Qv), Hp(L.Qs), Hp(L.K), Hp(L.V), Hp(W.dO16), Fp(W.dOr), Fp(W.dOs), slots,
-                          Fp(W.stats), Fp(W.dQr), Fp(W.dQs), Fp(W.dKf), Fp(W.dVf), stream)) &&
+                          Fp(W.lse), Fp(W.stats), Fp(W.dQr), Fp(W.dQs), Fp(W.dKp), Fp(W.dVp), stream)) &&
       // a7, a6, a1: Y = [dQ (routed, scattered to their experts) | dQs | dK | dV | dz];
       // dx = Y [W_q | W_qs | W_k | W_v | W_r]^T; each weight gradient = x^T (its columns of Y).
-      ok(bwd_pack(c, Fp(W.dQr), Fp(W.dQs), Fp(W.dKf), Fp(W.dVf), Fp(W.dz), reinterpret_cast<const int32_t*>(w + L.idx),
+      ok(bwd_pack(c, Fp(W.dQr), Fp(W.dQs), Fp(W.dKp), Fp(W.dVp), Fp(W.dz), reinterpret_cast<const int32_t*>(w + L.idx),
                   Y, static_cast<int>(Kc), stream)) &&
       ok(bwd_transpose(U(W_q), c1, d, static_cast<int>(c1), WcT, d, stream)) &&
       ok(bwd_transpose(U(W_qs), dh, d, dh, WcT + c1 * d, d, stream)) &&

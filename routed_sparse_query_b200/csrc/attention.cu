@@ -81,6 +81,10 @@ struct AttnParams {
   const int32_t* offsets;  // [N*B + 1]: list starts in (expert, sequence) order
   const int32_t* tok;      // list entries: positions t
   const int32_t* idx;      // [B*T, G, k]: selections (the output slot of a row)
+  // Optional (slot-major streams only): each row's log-sum-exp in base 2 of
+  // s log2(e)/sqrt(dh), lse[stream][lse_ld] (the backward's softmax statistics).
+  float* lse;
+  int lse_ld;
 };
 
 // Expert-major decode: routed unit u -> (list l = e*B + b, pair q of its
@@ -656,6 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tO + c * 32, v);
           if (row_ok) store_row32(dst + c * 32, v, inv);
         }
+        if (p.lse != nullptr && row_ok) p.lse[static_cast<size_t>(bh) * p.lse_ld + qi] = m + log2f(l);
       }
     } else {
       // Split-KV: publish this chunk's unnormalised rows (O relative to the
@@ -713,6 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint16_t* dst = p.out + (static_cast<size_t>(b) * p.T + qi) * p.ldo + slot * DH;
           const float inv = 1.0f / lt;
+          if (p.lse != nullptr) p.lse[static_cast<size_t>(bh) * p.lse_ld + qi] = ms + log2f(lt);
 #pragma unroll
           for (int c = 0; c < DH / 32; ++c) {
             uint32_t v[32];
@@ -749,7 +755,7 @@ int launch_attn(const CUtensorMap& q, const CUtensorMap& qs, const CUtensorMap& 
 
 int run(const gqe_config& c, const uint16_t* Q, uint64_t nq_streams, const uint16_t* Qs,
         const uint16_t* K, const uint16_t* V, uint16_t* out, int ldo, int H, int dense, void* ws,
-        size_t ws_bytes, bool counters_zeroed, void* stream) {
+        size_t ws_bytes, bool counters_zeroed, void* stream, float* lse = nullptr) {
   const int dh = c.d_head;
   const AttnPlan plan = attention_plan(c, H);
   if (plan.total > 0 && (ws == nullptr || ws_bytes < plan.total)) return cudaErrorInvalidValue;
@@ -776,6 +782,8 @@ int run(const gqe_config& c, const uint16_t* Q, uint64_t nq_streams, const uint1
   p.out = out;
   p.ldo = ldo;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(dh)));
+  p.lse = lse;
+  p.lse_ld = (c.T + 63) / 64 * 64;
   char* w = static_cast<char*>(ws);
   p.part = plan.total ? reinterpret_cast<float*>(w + plan.part) : nullptr;
   p.part_ml = plan.total ? reinterpret_cast<float2*>(w + plan.ml) : nullptr;
@@ -874,9 +882,9 @@ AttnPlan attention_plan(const gqe_config& c, int H) {
 
 int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
                   const uint16_t* V, uint16_t* slots, void* ws, size_t ws_bytes,
-                  bool counters_zeroed, void* stream) {
+                  bool counters_zeroed, void* stream, float* lse) {
   return run(c, Qv, static_cast<uint64_t>(c.B) * c.G * c.k, Qs, K, V, slots, n_slots(c) * c.d_head,
-             n_streams(c), 0, ws, ws_bytes, counters_zeroed, stream);
+             n_streams(c), 0, ws, ws_bytes, counters_zeroed, stream, lse);
 }
 
 int attention_gqe_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const uint16_t* K,

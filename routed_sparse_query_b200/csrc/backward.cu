@@ -36,10 +36,51 @@ namespace bwd_impl {
 __device__ __forceinline__ float to_f(uint16_t v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
 __device__ __forceinline__ float to_f(float v) { return v; }
 
+// Router logits z[r, e] = x[r] . W_r[:, e] + b[e] in fp32 (as the forward's
+// router forms them), 16 rows per CTA; W_r and the 16 rows of x are staged
+// in shared memory, then thread (row i, expert e) of a pass takes one dot
+// product over d.
+constexpr int kLogitRows = 16;
+__global__ void __launch_bounds__(256) logits_kernel(const uint16_t* x, const float* W_r, const float* b_r,
+                                                     float* z, long long R, int d, int N) {
+  extern __shared__ float4 Ws4[];  // W_r [d][N] (d N is a multiple of 4: d is one of 64), then x rows [16][d] bf16
+  const float* Ws = reinterpret_cast<const float*>(Ws4);
+  const int nw = d * N / 4;
+  uint4* xs4 = reinterpret_cast<uint4*>(Ws4 + nw);
+  const float4* W4 = reinterpret_cast<const float4*>(W_r);
+  const long long r0 = static_cast<long long>(blockIdx.x) * kLogitRows;
+  const int rows = static_cast<int>(R - r0 < kLogitRows ? R - r0 : kLogitRows);
+  const int xw = d / 8;  // 16-byte words per x row
+#pragma unroll 8
+  for (int i = threadIdx.x; i < nw; i += blockDim.x) Ws4[i] = __ldg(W4 + i);
+#pragma unroll 4
+  for (int i = threadIdx.x; i < rows * xw; i += blockDim.x)
+    xs4[i] = __ldg(reinterpret_cast<const uint4*>(x + r0 * d) + i);
+  __syncthreads();
+  const int per = blockDim.x / N;  // rows per pass
+  const int e = threadIdx.x % N, i0 = threadIdx.x / N;
+  if (i0 >= per) return;
+  for (int i = i0; i < rows; i += per) {
+    const uint4* xr = xs4 + i * xw;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four partial sums, added in a fixed order
+    for (int c8 = 0; c8 < xw; ++c8) {
+      const uint4 v = xr[c8];
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[q] = fmaf(__uint_as_float(u[q] << 16), Ws[(c8 * 8 + 2 * q) * N + e], acc[q]);
+        acc[q] = fmaf(__uint_as_float(u[q] & 0xffff0000u), Ws[(c8 * 8 + 2 * q + 1) * N + e], acc[q]);
+      }
+    }
+    z[(r0 + i) * N + e] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + (b_r != nullptr ? b_r[e] : 0.0f);
+  }
+}
+
 struct SlotArgs {
   const uint16_t* x;      // [R, d]
   const float* W_r;       // [d, N]
   const float* b_r;       // [N] or null
+  const float* zl;        // [R, N]: the router logits (logits_kernel)
   const int32_t* idx;     // [R, G, k]
   const float* omega;     // [R, G, k] (the forward's weights)
   const uint16_t* slots;  // [R, S*dh] (S = kG+2)
@@ -58,19 +99,12 @@ __global__ void __launch_bounds__(256) slot_router_bwd_kernel(SlotArgs a) {
   const int r = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = a.G * a.M, gk = a.G * a.k, dh = a.dh, Sdh = (gk + 2) * dh;
-  const uint16_t* xr = a.x + static_cast<size_t>(r) * a.d;
   const float* dSr = a.dS + static_cast<size_t>(r) * Sdh;
   const float* dSw = dSr + (gk + 1) * dh;
   const uint16_t* orow = a.slots + static_cast<size_t>(r) * Sdh;
   const float* om = a.omega + static_cast<size_t>(r) * gk;
   // Logits (fp32) and each group's softmax.
-  for (int e = warp; e < N; e += 8) {
-    float s = 0.0f;
-    for (int i = lane; i < a.d; i += 32) s = fmaf(to_f(xr[i]), a.W_r[static_cast<size_t>(i) * N + e], s);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) z[e] = s + (a.b_r != nullptr ? a.b_r[e] : 0.0f);
-  }
+  for (int e = tid; e < N; e += blockDim.x) z[e] = a.zl[static_cast<size_t>(r) * N + e];
   // dw[g, s] = <o[g, s], dS_w>.
   for (int q = warp; q < gk; q += 8) {
     float s = 0.0f;
@@ -164,38 +198,54 @@ __global__ void cast_kernel(const float* in, long long ldi, long long rows, int 
 
 // Row r of Y (bf16, ld columns): [dQ of every expert (the slot of row r that
 // selected expert e, 0 where none did) | dQ of the shared head | dK | dV |
-// dz | 0 padding]. Each thread writes two adjacent columns.
-__global__ void pack_grads_kernel(const float* dQr, const float* dQs, const float* dKf, const float* dVf,
-                                  const float* dz, const int32_t* idx, uint16_t* Y, long long R, int G, int M,
-                                  int k, int dh, int ld) {
-  const int N = G * M, c1 = N * dh, c2 = c1 + dh, c3 = c2 + G * dh, c4 = c3 + G * dh, c5 = c4 + N;
-  const int half = ld / 2;
-  const long long n = R * half;
+// dz | 0 padding]. dK and dV of group g are the sums, in stream order, of the
+// per-stream parts dKp, dVp [B, G k + 1, T, dh] of its k routed streams (and
+// of the shared head for group 0). Each thread writes 8 adjacent columns;
+// the segment bounds before dz are multiples of 32, so 8 columns never
+// straddle two of them.
+__global__ void pack_grads_kernel(const float* dQr, const float* dQs, const float* dKp, const float* dVp,
+                                  const float* dz, const int32_t* idx, uint16_t* Y, long long R, int T, int G,
+                                  int M, int k, int dh, int ld) {
+  const int N = G * M, gk = G * k, c1 = N * dh, c2 = c1 + dh, c3 = c2 + G * dh, c4 = c3 + G * dh, c5 = c4 + N;
+  const int per_row = ld / 8;
+  const long long n = R * per_row;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long r = i / half;
-    const int c = 2 * static_cast<int>(i - r * half);
-    float v[2] = {0.0f, 0.0f};
+    const long long r = i / per_row;
+    const int c = 8 * static_cast<int>(i - r * per_row);
+    const long long bb = r / T, t = r - bb * T;
+    float v[8];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int cc = c + q;
-      if (cc < c1) {
-        const int e = cc / dh, col = cc - e * dh, g = e / M, j = e - g * M;
-        const int32_t* ip = idx + (r * G + g) * k;
-        for (int s = 0; s < k; ++s)
-          if (ip[s] == j) v[q] = dQr[((r * G + g) * k + s) * dh + col];
-      } else if (cc < c2) {
-        v[q] = dQs[r * dh + (cc - c1)];
-      } else if (cc < c3) {
-        v[q] = dKf[r * G * dh + (cc - c2)];
-      } else if (cc < c4) {
-        v[q] = dVf[r * G * dh + (cc - c3)];
-      } else if (cc < c5) {
-        v[q] = dz[r * N + (cc - c4)];
-      }
+    for (int q = 0; q < 8; ++q) v[q] = 0.0f;
+    auto add8 = [&](const float* src) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(src)), b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+      v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    };
+    if (c < c1) {
+      const int e = c / dh, col = c - e * dh, g = e / M, j = e - g * M;
+      const int32_t* ip = idx + (r * G + g) * k;
+      for (int s = 0; s < k; ++s)
+        if (ip[s] == j) add8(dQr + ((r * G + g) * k + s) * dh + col);
+    } else if (c < c2) {
+      add8(dQs + r * dh + (c - c1));
+    } else if (c < c4) {
+      const bool is_k = c < c3;
+      const int x = c - (is_k ? c2 : c3), g = x / dh, col = x - g * dh;
+      const float* part = is_k ? dKp : dVp;
+      for (int s = 0; s < k; ++s) add8(part + ((bb * (gk + 1) + g * k + s) * T + t) * dh + col);
+      if (g == 0) add8(part + ((bb * (gk + 1) + gk) * T + t) * dh + col);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (c + q < c5) v[q] = dz[r * N + (c + q - c4)];
     }
-    *reinterpret_cast<uint32_t*>(Y + r * ld + c) = static_cast<uint32_t>(bf16_rn(v[0])) |
-                                                  (static_cast<uint32_t>(bf16_rn(v[1])) << 16);
+    uint4 o;
+    o.x = pack_bf16x2(v[0], v[1]);
+    o.y = pack_bf16x2(v[2], v[3]);
+    o.z = pack_bf16x2(v[4], v[5]);
+    o.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(Y + r * ld + c) = o;
   }
 }
 
@@ -233,19 +283,29 @@ int bwd_cast(const float* in, long long ldi, long long rows, int cols, uint16_t*
   return cudaGetLastError();
 }
 
-int bwd_pack(const gqe_config& c, const float* dQr, const float* dQs, const float* dKf, const float* dVf,
+int bwd_pack(const gqe_config& c, const float* dQr, const float* dQs, const float* dKp, const float* dVp,
              const float* dz, const int32_t* idx, uint16_t* Y, int ld, void* stream) {
   const long long R = static_cast<long long>(c.B) * c.T;
-  pack_grads_kernel<<<1184, 256, 0, static_cast<cudaStream_t>(stream)>>>(dQr, dQs, dKf, dVf, dz, idx, Y, R, c.G,
-                                                                         c.M, c.k, c.d_head, ld);
+  pack_grads_kernel<<<1184, 256, 0, static_cast<cudaStream_t>(stream)>>>(dQr, dQs, dKp, dVp, dz, idx, Y, R, c.T,
+                                                                         c.G, c.M, c.k, c.d_head, ld);
   return cudaGetLastError();
 }
 
-int bwd_slots_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r,
+int bwd_slots_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r, float* zl,
                      const int32_t* idx, const float* omega, const uint16_t* slots, const float* dS, float* dOr,
                      float* dOs, float* dz, uint16_t* dO16, void* stream) {
-  SlotArgs a{x, W_r, b_r, idx, omega, slots, dS, dOr, dOs, dz, dO16, c.d_model, c.G, c.M, c.k, c.d_head, c.T};
-  slot_router_bwd_kernel<<<c.B * c.T, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  const long long R = static_cast<long long>(c.B) * c.T;
+  const int N = c.G * c.M;
+  const int smem = c.d_model * N * static_cast<int>(sizeof(float)) + kLogitRows * c.d_model * 2;
+  cudaError_t e = static_cast<cudaError_t>(ensure_smem<logits_kernel>(smem));
+  if (e != cudaSuccess) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  logits_kernel<<<static_cast<unsigned>((R + kLogitRows - 1) / kLogitRows), 256, smem, st>>>(x, W_r, b_r, zl, R,
+                                                                                           c.d_model, N);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  SlotArgs a{x, W_r, b_r, zl, idx, omega, slots, dS, dOr, dOs, dz, dO16, c.d_model, c.G, c.M, c.k, c.d_head, c.T};
+  slot_router_bwd_kernel<<<static_cast<unsigned>(R), 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -144,9 +144,11 @@ struct AttnPlan {
 AttnPlan attention_plan(const gqe_config& c, int H);
 // counters_zeroed: the caller has zeroed the split-KV arrival counters of ws
 // earlier on the stream (zero_attention_counters); otherwise the call does.
+// lse (optional): each stream's rows' log-sum-exp, base 2 of s log2(e)/sqrt(dh),
+// [B*(G*k+1)][T rounded up to 64].
 int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
                   const uint16_t* V, uint16_t* slots, void* ws, size_t ws_bytes,
-                  bool counters_zeroed, void* stream);
+                  bool counters_zeroed, void* stream, float* lse = nullptr);
 // Expert-major routed attention (Qe in token-list order, rows masked by
 // their positions tok[]) plus the shared head, one launch, no scratch.
 int attention_gqe_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const uint16_t* K,
@@ -166,17 +168,20 @@ int gemm_f32out(const uint16_t* A, long long lda, int M, int K, const uint16_t* 
 template <typename TI>
 int bwd_transpose(const TI* in, long long ldi, int rows, int cols, uint16_t* out, long long ldo, void* stream);
 int bwd_cast(const float* in, long long ldi, long long rows, int cols, uint16_t* out, long long ldo, void* stream);
-int bwd_pack(const gqe_config& c, const float* dQr, const float* dQs, const float* dKf, const float* dVf,
+int bwd_pack(const gqe_config& c, const float* dQr, const float* dQs, const float* dKp, const float* dVp,
              const float* dz, const int32_t* idx, uint16_t* Y, int ld, void* stream);
-int bwd_slots_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r,
+// zl: [B*T, G*M] fp32 scratch for the router logits.
+int bwd_slots_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r, float* zl,
                      const int32_t* idx, const float* omega, const uint16_t* slots, const float* dS, float* dOr,
                      float* dOs, float* dz, uint16_t* dO16, void* stream);
 // Attention backward on tcgen05 (attn_bwd.cu): dq of every stream, dK and dV
-// of every group; stats [B, G*k+1, T] float2 scratch.
+// of every stream (dKp, dVp [B, G*k+1, T, dh]; summed per group by bwd_pack);
+// lse: the forward attention's row statistics; stats: [B, G*k+1, T rounded
+// up to 64] float2 scratch.
 int bwd_attention_tc(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
                      const uint16_t* V, const uint16_t* dO16, const float* dOr, const float* dOs,
-                     const uint16_t* slots, float* stats, float* dQr, float* dQs, float* dKf, float* dVf,
-                     void* stream);
+                     const uint16_t* slots, const float* lse, float* stats, float* dQr, float* dQs, float* dKp,
+                     float* dVp, void* stream);
 int bwd_colsum(const float* dz, float* db, long long R, int N, void* stream);
 
 // Decode step. cfg.T = keys after the step (the new token sits at T - 1),

@@ -32,6 +32,17 @@ def test_projection_flops():
     assert f["router"] == 2 * R * d * 16
 
 
+def test_backward_flops():
+    # seq2k (B=1, T=2048, d=1024, G=8, M=2, k=1, dh=64): attention 5 products
+    # x 2*64 FLOPs x 2048*2049/2 pairs x 9 streams; dS and dW_O 2*2048*1024*640
+    # each; dx and the weight gradients 2*2048*1024*(1024 + 64 + 1024 + 16) each.
+    s = synth.SEQ2K
+    attn = 5 * 128 * (2048 * 2049 // 2) * 9
+    proj = 2 * (2 * 2048 * 1024 * 640) + 2 * (2 * 2048 * 1024 * 2128)
+    assert bench.backward_flops(s) == attn + proj
+    assert round(bench.backward_flops(s) / 1e9, 1) == 35.3
+
+
 def test_launch_counts():
     # seq2k and 4 x 8k: the tile counts (8 or 128 tiles x 16 experts) fit the
     # fused scan + scatter after the count kernel; 1M tokens: 4096 x 16 tile
