@@ -88,7 +88,7 @@ struct BwdWs {
   LayerWs L;
   size_t y, dS, dOr, dOs, dz, stats, dQr, dQs, dKp, dVp;  // fp32
   size_t dy16, WoT, sT, xT, WcT, Y, dO16;                 // bf16 operands of the tensor-core GEMMs
-  size_t lse, zl;                                         // the forward attention's row statistics; logits
+  size_t lse, zl, Drow;                                   // the forward attention's row statistics; logits; dO . O
   long long ldR, ldS, Kcat, zoff;
   size_t total;
 };
@@ -114,10 +114,10 @@ BwdWs bwd_ws(const gqe_config& c) {
   put(W.dOs, R * dh * 4);
   put(W.dz, R * N * 4);
   put(W.stats, static_cast<size_t>(c.B) * (gk + 1) * ((c.T + 63) / 64 * 64) * 8);
-  put(W.dQr, R * gk * dh * 4);
-  put(W.dQs, R * dh * 4);
-  put(W.dKp, R * (gk + 1) * dh * 4);
-  put(W.dVp, R * (gk + 1) * dh * 4);
+  put(W.dQr, 2 * R * gk * dh * 4);
+  put(W.dQs, 2 * R * dh * 4);
+  put(W.dKp, 2 * R * (gk + 1) * dh * 4);
+  put(W.dVp, 2 * R * (gk + 1) * dh * 4);
   put(W.dy16, R * d * 2);
   put(W.WoT, d * W.ldS * 2);
   put(W.sT, Sdh * W.ldR * 2);
@@ -127,6 +127,7 @@ BwdWs bwd_ws(const gqe_config& c) {
   put(W.dO16, R * (gk + 1) * dh * 2);
   put(W.lse, static_cast<size_t>(c.B) * (gk + 1) * ((c.T + 63) / 64 * 64) * 4);
   put(W.zl, R * N * 4);
+  put(W.Drow, static_cast<size_t>(c.B) * (gk + 1) * ((c.T + 63) / 64 * 64) * 4);
   W.total = o;
   return W;
 }
@@ -506,11 +507,11 @@ gqe_status gqe_layer_bwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
       ok(gemm_f32out(Hp(W.sT), W.ldR, Sdh, Ri, dy16, d, d, dW_o, d, stream)) &&
       // a10, a4, a2: slots and router -> dO, dz; db = sum dz.
       ok(bwd_slots_router(c, xb, W_r, b_r, Fp(W.zl), reinterpret_cast<const int32_t*>(w + L.idx), Fp(L.omega), slots,
-                          Fp(W.dS), Fp(W.dOr), Fp(W.dOs), Fp(W.dz), Hp(W.dO16), stream)) &&
+                          Fp(W.dS), Fp(W.dOr), Fp(W.dOs), Fp(W.dz), Hp(W.dO16), Fp(W.Drow), stream)) &&
       (db_r == nullptr || ok(bwd_colsum(Fp(W.dz), db_r, R, N, stream))) &&
       // a8: attention -> dq, dK, dV.
-      ok(bwd_attention_tc(c, Hp(L.Qv), Hp(L.Qs), Hp(L.K), Hp(L.V), Hp(W.dO16), Fp(W.dOr), Fp(W.dOs), slots,
-                          Fp(W.lse), Fp(W.stats), Fp(W.dQr), Fp(W.dQs), Fp(W.dKp), Fp(W.dVp), stream)) &&
+      ok(bwd_attention_tc(c, Hp(L.Qv), Hp(L.Qs), Hp(L.K), Hp(L.V), Hp(W.dO16), Fp(W.Drow), Fp(W.lse), Fp(W.stats),
+                          Fp(W.dQr), Fp(W.dQs), Fp(W.dKp), Fp(W.dVp), stream)) &&
       // a7, a6, a1: Y = [dQ (routed, scattered to their experts) | dQs | dK | dV | dz];
       // dx = Y [W_q | W_qs | W_k | W_v | W_r]^T; each weight gradient = x^T (its columns of Y).
       ok(bwd_pack(c, Fp(W.dQr), Fp(W.dQs), Fp(W.dKp), Fp(W.dVp), Fp(W.dz), reinterpret_cast<const int32_t*>(w + L.idx),

@@ -15,16 +15,17 @@
 // thread of warp 0 issues the TMA loads and the UMMAs. The S / dP products of
 // item n + 1 go into the other of two TMEM buffers while the threads work on
 // item n.
-//   attn_bwd_q_kernel, one CTA per 128 query rows of a stream: over the
-//     64-key tiles up to the diagonal, S = Q K^T and dP = dO V^T, P from the
-//     row's log-sum-exp (kept by the forward), dS in bf16 over S, and
-//     dQ += dS K (A from TMEM). The rows' (lse, D) go to a stats buffer for
-//     the second kernel.
-//   attn_bwd_kv_kernel, one CTA per 128 keys of one stream: for every
-//     64-query tile from the diagonal on, S^T = K Q^T and dP^T = V dO^T, P^T
-//     and dS^T written back in bf16, then dV += P^T dO and dK += dS^T Q. The
-//     per-stream dK, dV are summed over a group's streams later, in a fixed
-//     order, so the result is deterministic.
+//   attn_bwd_q_kernel, two CTAs per 128 query rows of a stream (each half
+//     of the 64-key tiles up to the diagonal): S = Q K^T and dP = dO V^T, P
+//     from the row's log-sum-exp (kept by the forward), dS in bf16 over S,
+//     and dQ += dS K (A from TMEM). The rows' (lse, D) go to a stats buffer
+//     for the second kernel.
+//   attn_bwd_kv_kernel, two CTAs per 128 keys of one stream (each half of the
+//     64-query tiles from the diagonal on): S^T = K Q^T and dP^T = V dO^T,
+//     P^T and dS^T written back in bf16, then dV += P^T dO and dK += dS^T Q.
+// Each CTA writes its own part of dQ, dK, dV; the parts, and dK, dV over a
+// group's streams, are summed later in a fixed order, so the result is
+// deterministic.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -60,15 +61,13 @@ struct Params {
   int B, T, Tp, G, k, H;  // Tp: T rounded up to 64 (row stride of stats); H = G k + 1 streams
   float scale;            // 1 / sqrt(dh)
   float scale_log2;       // log2(e) / sqrt(dh)
-  const float* dOr;       // [B*T, G*k, dh] fp32
-  const float* dOs;       // [B*T, dh]
-  const uint16_t* slots;  // [B*T, Sdh]: the forward's attention outputs (stream h = slot h)
-  int Sdh;
+  const float* Drow;      // [B, H, Tp]: D = dO . O of each row
   const float* lse;       // [B, H, Tp]: each row's log-sum-exp (base 2 of s log2(e)/sqrt(dh)), from the forward
   float2* stats;          // [B, H, Tp]: (lse, D) for the key kernel
-  float* dQr;             // [B*T, G*k, dh]
-  float* dQs;             // [B*T, dh]
-  float* dKp;             // [B, H, T, dh]: dK of each stream
+  // Outputs in two parts [2][...], one per half of a CTA pair's tiles.
+  float* dQr;             // [2][B*T, G*k, dh]
+  float* dQs;             // [2][B*T, dh]
+  float* dKp;             // [2][B, H, T, dh]: dK of each stream
   float* dVp;
 };
 
@@ -122,15 +121,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_q_kernel(const __grid_co
 
   const int gk = p.G * p.k, H = p.H;
   const int nq = (p.T + 127) / 128;
-  const int qt = nq - 1 - static_cast<int>(blockIdx.x % nq);  // longest rows first
-  const int h = static_cast<int>((blockIdx.x / nq) % H);
-  const int b = static_cast<int>(blockIdx.x / (nq * H));
+  // Two CTAs per (stream, query tile), each taking half of its key tiles.
+  const int part = static_cast<int>(blockIdx.x & 1);
+  const int rest = static_cast<int>(blockIdx.x >> 1);
+  const int qt = nq - 1 - rest % nq;  // longest rows first
+  const int h = (rest / nq) % H;
+  const int b = rest / (nq * H);
   const int g = h < gk ? h / p.k : 0;
   const int t0 = qt * 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hc = warp >> 2;                    // column half
   const int row = (warp & 3) * 32 + lane;      // TMEM lane = query row in the tile
-  const int total = min(2 * qt + 2, (p.T + 63) / 64);  // 64-key tiles up to the diagonal
+  const int ntiles = min(2 * qt + 2, (p.T + 63) / 64);  // 64-key tiles up to the diagonal
+  const int mid = (ntiles + 1) / 2;
+  const int j0 = part ? mid : 0;
+  const int total = part ? ntiles - mid : mid;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1u);
@@ -157,8 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_q_kernel(const __grid_co
     const int s = n % kStages;
     if (!mbar_wait(&kv_empty[s], ((n / kStages) & 1) ^ 1u, abort_flag)) return false;
     mbar_arrive_expect_tx(&kv_full[s], 2u * C::ROWS64);
-    tma_load_3d(sK + s * C::ROWS64, &tmK, &kv_full[s], 0, 64 * n, b * p.G + g);
-    tma_load_3d(sV + s * C::ROWS64, &tmV, &kv_full[s], 0, 64 * n, b * p.G + g);
+    tma_load_3d(sK + s * C::ROWS64, &tmK, &kv_full[s], 0, 64 * (j0 + n), b * p.G + g);
+    tma_load_3d(sV + s * C::ROWS64, &tmV, &kv_full[s], 0, 64 * (j0 + n), b * p.G + g);
     issued = n + 1;
     return true;
   };
@@ -190,29 +195,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_q_kernel(const __grid_co
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
     prefetch_tmap(&tmdO);
-    mbar_arrive_expect_tx(q_full, 2u * C::ROWS128);
-    if (h < gk) tma_load_3d(sQ, &tmQv, q_full, 0, t0, b * gk + h);
-    else tma_load_3d(sQ, &tmQs, q_full, 0, t0, b);
-    tma_load_3d(sdO, &tmdO, q_full, 0, t0, b * H + h);
+    if (total > 0) {  // an empty half loads nothing (no copy may outlive the CTA)
+      mbar_arrive_expect_tx(q_full, 2u * C::ROWS128);
+      if (h < gk) tma_load_3d(sQ, &tmQv, q_full, 0, t0, b * gk + h);
+      else tma_load_3d(sQ, &tmQs, q_full, 0, t0, b);
+      tma_load_3d(sdO, &tmdO, q_full, 0, t0, b * H + h);
+    }
     for (int n = 0; n < kAhead && n < total; ++n)
       if (!load(n)) break;
   }
   __syncwarp();
-  if (warp == 0) issue(0);
+  if (warp == 0 && total > 0) issue(0);
 
-  // Row of this thread; D = dO . O from the fp32 gradient and the forward's output.
+  // Row of this thread, its log-sum-exp and D.
   const int t = t0 + row;
   const bool row_ok = t < p.T;
   const size_t r = static_cast<size_t>(b) * p.T + t;
-  float D = 0.0f;
-  if (row_ok) {
-    const float* dO = h < gk ? p.dOr + (r * gk + h) * DH : p.dOs + r * DH;
-    const uint16_t* O = p.slots + r * p.Sdh + static_cast<size_t>(h) * DH;
-#pragma unroll 8
-    for (int c = 0; c < DH; ++c) D = fmaf(dO[c], bf16f(O[c]), D);
-  }
+  const size_t srow = (static_cast<size_t>(b) * H + h) * p.Tp + t;
   const float sl = p.scale_log2;
-  const float lse = row_ok ? p.lse[(static_cast<size_t>(b) * H + h) * p.Tp + t] : 0.0f;
+  const float lse = row_ok ? p.lse[srow] : 0.0f;
+  const float D = row_ok ? p.Drow[srow] : 0.0f;
 
   bool ok = true;
   int n = 0;
@@ -230,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_q_kernel(const __grid_co
     tc_fence_after();
     if (threadIdx.x == 0 && n + kAhead < total) load(n + kAhead);
     __syncwarp();
-    const int ub = 64 * n + 32 * hc;  // first key of this thread's columns
+    const int ub = 64 * (j0 + n) + 32 * hc;  // first key of this thread's columns
     uint32_t va[32], pa[32], w[16];
     tmem_ld32_nowait(tS + lane_base + 32 * hc, va);
     tmem_ld32_nowait(tS + 64 + lane_base + 32 * hc, pa);
@@ -265,16 +267,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_q_kernel(const __grid_co
   const bool have = __syncthreads_and(ok && mbar_wait(done, 0, abort_flag));
   tc_fence_after();
   if (have && hc * 32 < DH) {
+    const size_t R = static_cast<size_t>(p.B) * p.T;
+    float* dq = h < gk ? p.dQr + part * R * gk * DH + (r * gk + h) * DH : p.dQs + part * R * DH + r * DH;
     uint32_t v[32];
-    tmem_ld32(tA + lane_base + 32 * hc, v);
-    if (row_ok) store_rows32<DH>((h < gk ? p.dQr + (r * gk + h) * DH : p.dQs + r * DH) + 32 * hc, v, p.scale);
+    if (total > 0) {
+      tmem_ld32(tA + lane_base + 32 * hc, v);
+    } else {  // no key tiles in this half: its part is zero
+#pragma unroll
+      for (int c = 0; c < 32; ++c) v[c] = 0u;
+    }
+    if (row_ok) store_rows32<DH>(dq + 32 * hc, v, p.scale);
   }
-  if (have && hc == 0 && row_ok) p.stats[(static_cast<size_t>(b) * H + h) * p.Tp + t] = make_float2(lse, D);
+  if (have && part == 0 && hc == 0 && row_ok) p.stats[srow] = make_float2(lse, D);
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && !have) {
     volatile int none = 0;
-    mbar_wait(q_full, 0, &none, 500000000ull);
+    if (total > 0) mbar_wait(q_full, 0, &none, 500000000ull);
     drain_loads(kv_full, issued);
   }
   if (warp == 0) {
@@ -310,15 +319,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kv_kernel(const __grid_c
 
   const int gk = p.G * p.k, H = p.H;
   const int nk = (p.T + 127) / 128;
-  const int kb = static_cast<int>(blockIdx.x % nk);  // longest query ranges first
-  const int h = static_cast<int>((blockIdx.x / nk) % H);
-  const int b = static_cast<int>(blockIdx.x / (nk * H));
+  // Two CTAs per (stream, key tile), each taking half of its query tiles.
+  const int part = static_cast<int>(blockIdx.x & 1);
+  const int rest = static_cast<int>(blockIdx.x >> 1);
+  const int kb = rest % nk;  // longest query ranges first
+  const int h = (rest / nk) % H;
+  const int b = rest / (nk * H);
   const int g = h < gk ? h / p.k : 0;
   const int u0 = kb * 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hc = warp >> 2;
   const int row = (warp & 3) * 32 + lane;  // TMEM lane = key row in the tile
-  const int total = (p.T + 63) / 64 - 2 * kb;  // 64-query tiles from the diagonal on
+  const int ntiles = (p.T + 63) / 64 - 2 * kb;  // 64-query tiles from the diagonal on
+  const int mid = (ntiles + 1) / 2;
+  const int jq0 = 2 * kb + (part ? mid : 0);  // first query tile of this CTA
+  const int total = part ? ntiles - mid : mid;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1u);
@@ -345,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kv_kernel(const __grid_c
   auto load = [&](int n) -> bool {
     const int s = n % kStages;
     if (!mbar_wait(&q_empty[s], ((n / kStages) & 1) ^ 1u, abort_flag)) return false;
-    const int j = 2 * kb + n;
+    const int j = jq0 + n;
     uint8_t* st = ring + s * C::KV_STAGE;
     mbar_arrive_expect_tx(&q_full[s], 2u * C::ROWS64 + 512u);
     if (h < gk) tma_load_3d(st, &tmQv, &q_full[s], 0, 64 * j, b * gk + h);
@@ -383,14 +398,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kv_kernel(const __grid_c
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
     prefetch_tmap(&tmdO);
-    mbar_arrive_expect_tx(kv_full, 2u * C::ROWS128);
-    tma_load_3d(sK, &tmK, kv_full, 0, u0, b * p.G + g);
-    tma_load_3d(sV, &tmV, kv_full, 0, u0, b * p.G + g);
+    if (total > 0) {  // an empty half loads nothing (no copy may outlive the CTA)
+      mbar_arrive_expect_tx(kv_full, 2u * C::ROWS128);
+      tma_load_3d(sK, &tmK, kv_full, 0, u0, b * p.G + g);
+      tma_load_3d(sV, &tmV, kv_full, 0, u0, b * p.G + g);
+    }
     for (int n = 0; n < kAhead && n < total; ++n)
       if (!load(n)) break;
   }
   __syncwarp();
-  if (warp == 0) issue(0);
+  if (warp == 0 && total > 0) issue(0);
 
   const int u = u0 + row;  // key of this thread
   const float sl = p.scale_log2;
@@ -411,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kv_kernel(const __grid_c
     if (threadIdx.x == 0 && n + kAhead < total) load(n + kAhead);
     __syncwarp();
     const float2* sst = reinterpret_cast<const float2*>(ring + s * C::KV_STAGE + 2 * C::ROWS64) + 32 * hc;
-    const int tq0 = 64 * (2 * kb + n) + 32 * hc;  // first query of this thread's columns
+    const int tq0 = 64 * (jq0 + n) + 32 * hc;  // first query of this thread's columns
     uint32_t va[32], pa[32], pw[16], dw[16];
     tmem_ld32_nowait(tS + lane_base + 32 * hc, va);
     tmem_ld32_nowait(tS + 64 + lane_base + 32 * hc, pa);
@@ -455,15 +472,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kv_kernel(const __grid_c
     }
   }
   if (warp == 0) umma_commit_elect(done);
-  const bool have = __syncthreads_and(ok && total > 0 && mbar_wait(done, 0, abort_flag));
+  const bool have = __syncthreads_and(ok && mbar_wait(done, 0, abort_flag));
   tc_fence_after();
   if (have) {
     // Column half 0 drains dK, half 1 dV.
-    const size_t o = ((static_cast<size_t>(b) * H + h) * p.T + u) * DH;
+    const size_t o = static_cast<size_t>(part) * p.B * H * p.T * DH + ((static_cast<size_t>(b) * H + h) * p.T + u) * DH;
 #pragma unroll
     for (int cc = 0; cc < DH / 32; ++cc) {
       uint32_t v[32];
-      tmem_ld32((hc == 0 ? tK : tV) + lane_base + 32 * cc, v);
+      if (total > 0) {
+        tmem_ld32((hc == 0 ? tK : tV) + lane_base + 32 * cc, v);
+      } else {  // no query tiles in this half: its part is zero
+#pragma unroll
+        for (int c = 0; c < 32; ++c) v[c] = 0u;
+      }
       if (u < p.T) store_rows32<DH>((hc == 0 ? p.dKp : p.dVp) + o + 32 * cc, v, hc == 0 ? p.scale : 1.0f);
     }
   }
@@ -471,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kv_kernel(const __grid_c
   __syncthreads();
   if (threadIdx.x == 0 && !have) {
     volatile int none = 0;
-    mbar_wait(kv_full, 0, &none, 500000000ull);
+    if (total > 0) mbar_wait(kv_full, 0, &none, 500000000ull);
     drain_loads(q_full, issued);
   }
   if (warp == 0) {
@@ -508,7 +530,7 @@ int launch_bwd(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, cons
   constexpr int kOneCtaSmem = 120 * 1024;
   const int smem_q = static_cast<int>(Cf::SMEM_Q) > kOneCtaSmem ? static_cast<int>(Cf::SMEM_Q) : kOneCtaSmem;
   const int smem_kv = static_cast<int>(Cf::SMEM_KV) > kOneCtaSmem ? static_cast<int>(Cf::SMEM_KV) : kOneCtaSmem;
-  const long long ctas = static_cast<long long>(c.B) * H * ((c.T + 127) / 128);
+  const long long ctas = 2ll * c.B * H * ((c.T + 127) / 128);
   if (ctas > 0x7fffffffll) return cudaErrorInvalidConfiguration;
   int e = ensure_smem<attn_bwd_q_kernel<DH>>(smem_q);
   if (e == cudaSuccess) e = ensure_smem<attn_bwd_kv_kernel<DH>>(smem_kv);
@@ -524,15 +546,14 @@ int launch_bwd(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, cons
 }  // namespace attn_bwd_impl
 
 int bwd_attention_tc(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
-                     const uint16_t* V, const uint16_t* dO16, const float* dOr, const float* dOs,
-                     const uint16_t* slots, const float* lse, float* stats, float* dQr, float* dQs, float* dKp,
-                     float* dVp, void* stream) {
+                     const uint16_t* V, const uint16_t* dO16, const float* Drow, const float* lse, float* stats,
+                     float* dQr, float* dQs, float* dKp, float* dVp, void* stream) {
   using namespace attn_bwd_impl;
   const int gk = c.G * c.k;
   Params p{c.B, c.T, (c.T + 63) / 64 * 64, c.G, c.k, gk + 1,
            static_cast<float>(1.0 / std::sqrt(static_cast<double>(c.d_head))),
            static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.d_head))),
-           dOr, dOs, slots, (gk + 2) * c.d_head, lse, reinterpret_cast<float2*>(stats), dQr, dQs, dKp, dVp};
+           Drow, lse, reinterpret_cast<float2*>(stats), dQr, dQs, dKp, dVp};
   switch (c.d_head) {
     case 64: return launch_bwd<64>(c, Qv, Qs, K, V, dO16, p, stream);
     case 32: return launch_bwd<32>(c, Qv, Qs, K, V, dO16, p, stream);

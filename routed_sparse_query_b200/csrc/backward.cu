@@ -89,7 +89,8 @@ struct SlotArgs {
   float* dOs;             // [R, dh]
   float* dz;              // [R, N]
   uint16_t* dO16;         // [B, G*k + 1, T, dh]: dO per stream in bf16 (the attention backward's operand)
-  int d, G, M, k, dh, T;
+  float* Drow;            // [B, G*k + 1, Tp]: D = dO . O per stream and row (the attention backward's)
+  int d, G, M, k, dh, T, Tp;
 };
 
 // One CTA (256 threads) per token row.
@@ -163,6 +164,17 @@ __global__ void __launch_bounds__(256) slot_router_bwd_kernel(SlotArgs a) {
     a.dOs[static_cast<size_t>(r) * dh + c] = v;
     o16[gk * hs + c] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
   }
+  // D = dO . O of every stream (O = the forward's slot, bf16), one warp per stream.
+  for (int h = warp; h <= gk; h += 8) {
+    float sd = 0.0f;
+    for (int c = lane; c < dh; c += 32) {
+      const float v = h < gk ? dSr[h * dh + c] + om[h] * dSw[c] : dSr[gk * dh + c];
+      sd = fmaf(v, to_f(orow[h * dh + c]), sd);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sd += __shfl_xor_sync(0xffffffffu, sd, o);
+    if (lane == 0) a.Drow[(static_cast<size_t>(bb) * (gk + 1) + h) * a.Tp + t] = sd;
+  }
 }
 
 __device__ __forceinline__ uint16_t bf16_rn(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
@@ -200,7 +212,8 @@ __global__ void cast_kernel(const float* in, long long ldi, long long rows, int 
 // selected expert e, 0 where none did) | dQ of the shared head | dK | dV |
 // dz | 0 padding]. dK and dV of group g are the sums, in stream order, of the
 // per-stream parts dKp, dVp [B, G k + 1, T, dh] of its k routed streams (and
-// of the shared head for group 0). Each thread writes 8 adjacent columns;
+// of the shared head for group 0); each of dQ, dK, dV arrives in two parts
+// [2][...] that are added here. Each thread writes 8 adjacent columns;
 // the segment bounds before dz are multiples of 32, so 8 columns never
 // straddle two of them.
 __global__ void pack_grads_kernel(const float* dQr, const float* dQs, const float* dKp, const float* dVp,
@@ -222,19 +235,25 @@ __global__ void pack_grads_kernel(const float* dQr, const float* dQs, const floa
       v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
       v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
     };
+    // Every attention gradient comes in two parts (the two halves of the
+    // tiles an attention-backward CTA pair covers), added in a fixed order.
     if (c < c1) {
       const int e = c / dh, col = c - e * dh, g = e / M, j = e - g * M;
       const int32_t* ip = idx + (r * G + g) * k;
       for (int s = 0; s < k; ++s)
-        if (ip[s] == j) add8(dQr + ((r * G + g) * k + s) * dh + col);
+        if (ip[s] == j)
+          for (int hf = 0; hf < 2; ++hf) add8(dQr + hf * R * gk * dh + ((r * G + g) * k + s) * dh + col);
     } else if (c < c2) {
-      add8(dQs + r * dh + (c - c1));
+      for (int hf = 0; hf < 2; ++hf) add8(dQs + hf * R * dh + r * dh + (c - c1));
     } else if (c < c4) {
       const bool is_k = c < c3;
       const int x = c - (is_k ? c2 : c3), g = x / dh, col = x - g * dh;
       const float* part = is_k ? dKp : dVp;
-      for (int s = 0; s < k; ++s) add8(part + ((bb * (gk + 1) + g * k + s) * T + t) * dh + col);
-      if (g == 0) add8(part + ((bb * (gk + 1) + gk) * T + t) * dh + col);
+      const long long half_sz = R * (gk + 1) * dh;
+      for (int hf = 0; hf < 2; ++hf) {
+        for (int s = 0; s < k; ++s) add8(part + hf * half_sz + ((bb * (gk + 1) + g * k + s) * T + t) * dh + col);
+        if (g == 0) add8(part + hf * half_sz + ((bb * (gk + 1) + gk) * T + t) * dh + col);
+      }
     } else {
 #pragma unroll
       for (int q = 0; q < 8; ++q)
@@ -293,7 +312,7 @@ int bwd_pack(const gqe_config& c, const float* dQr, const float* dQs, const floa
 
 int bwd_slots_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r, float* zl,
                      const int32_t* idx, const float* omega, const uint16_t* slots, const float* dS, float* dOr,
-                     float* dOs, float* dz, uint16_t* dO16, void* stream) {
+                     float* dOs, float* dz, uint16_t* dO16, float* Drow, void* stream) {
   const long long R = static_cast<long long>(c.B) * c.T;
   const int N = c.G * c.M;
   const int smem = c.d_model * N * static_cast<int>(sizeof(float)) + kLogitRows * c.d_model * 2;
@@ -304,7 +323,8 @@ int bwd_slots_router(const gqe_config& c, const uint16_t* x, const float* W_r, c
                                                                                            c.d_model, N);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  SlotArgs a{x, W_r, b_r, zl, idx, omega, slots, dS, dOr, dOs, dz, dO16, c.d_model, c.G, c.M, c.k, c.d_head, c.T};
+  SlotArgs a{x,  W_r, b_r,       zl,  idx,    omega,  slots,    dS,      dOr, dOs, dz,
+             dO16, Drow, c.d_model, c.G, c.M, c.k, c.d_head, c.T, (c.T + 63) / 64 * 64};
   slot_router_bwd_kernel<<<static_cast<unsigned>(R), 256, 0, st>>>(a);
   return cudaGetLastError();
 }

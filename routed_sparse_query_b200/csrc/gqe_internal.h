@@ -173,15 +173,15 @@ int bwd_pack(const gqe_config& c, const float* dQr, const float* dQs, const floa
 // zl: [B*T, G*M] fp32 scratch for the router logits.
 int bwd_slots_router(const gqe_config& c, const uint16_t* x, const float* W_r, const float* b_r, float* zl,
                      const int32_t* idx, const float* omega, const uint16_t* slots, const float* dS, float* dOr,
-                     float* dOs, float* dz, uint16_t* dO16, void* stream);
+                     float* dOs, float* dz, uint16_t* dO16, float* Drow, void* stream);
 // Attention backward on tcgen05 (attn_bwd.cu): dq of every stream, dK and dV
-// of every stream (dKp, dVp [B, G*k+1, T, dh]; summed per group by bwd_pack);
+// of every stream (dKp, dVp [B, G*k+1, T, dh]; summed per group by bwd_pack),
+// each output in two parts [2][...] (summed by bwd_pack); Drow: D = dO . O;
 // lse: the forward attention's row statistics; stats: [B, G*k+1, T rounded
 // up to 64] float2 scratch.
 int bwd_attention_tc(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
-                     const uint16_t* V, const uint16_t* dO16, const float* dOr, const float* dOs,
-                     const uint16_t* slots, const float* lse, float* stats, float* dQr, float* dQs, float* dKp,
-                     float* dVp, void* stream);
+                     const uint16_t* V, const uint16_t* dO16, const float* Drow, const float* lse, float* stats,
+                     float* dQr, float* dQs, float* dKp, float* dVp, void* stream);
 int bwd_colsum(const float* dz, float* db, long long R, int N, void* stream);
 
 // Decode step. cfg.T = keys after the step (the new token sits at T - 1),
