@@ -28,8 +28,6 @@
 //    GQE_ERR_WORKSPACE before anything is launched.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "gqe_internal.h"
 
 namespace gqe {
@@ -38,27 +36,13 @@ namespace noalloc_impl {
 constexpr size_t kScratchBytes = size_t(4) << 20;  // 4 MiB per device
 static __device__ __align__(256) unsigned char scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex mu;
-void* dev_ptr[kMaxDevices] = {nullptr};
-
-// Device address of `scratch` on the current device (looked up once per device).
+// Device address of `scratch` in the current context, looked up on every
+// call: a cached address would dangle after a device reset or a context
+// re-creation in the same process.
 void* scratch_address(cudaError_t* err) {
-  int dev = 0;
-  *err = cudaGetDevice(&dev);
-  if (*err != cudaSuccess) return nullptr;
-  if (dev < 0 || dev >= kMaxDevices) {
-    *err = cudaErrorInvalidDevice;
-    return nullptr;
-  }
-  std::lock_guard<std::mutex> lock(mu);
-  if (dev_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    *err = cudaGetSymbolAddress(&p, scratch);
-    if (*err != cudaSuccess) return nullptr;
-    dev_ptr[dev] = p;
-  }
-  return dev_ptr[dev];
+  void* p = nullptr;
+  *err = cudaGetSymbolAddress(&p, scratch);
+  return *err == cudaSuccess ? p : nullptr;
 }
 
 }  // namespace noalloc_impl

@@ -45,7 +45,18 @@ def _close(got, want, what):
 
 @pytest.mark.parametrize("name", list(CASES))
 def test_layer_backward_matches_oracle(rsq, name):
-    s = CASES[name]
+    _check(rsq, CASES[name], 0)
+
+
+def test_layer_backward_at_the_bench_workload(rsq):
+    # seq2k (B=1, T=2048, d_model=1024, G=8, M=2, k=1, d_head=64), the call
+    # `bench.py --backward` times, with its flags (a zeroed workspace declared
+    # clean): the full attention-backward grid (two CTAs per 128-row tile,
+    # 16 x 16 tiles per stream), every gradient against the fp64 oracle.
+    _check(rsq, synth.SEQ2K, rsq.GQE_FLAG_WS_CLEAN)
+
+
+def _check(rsq, s, flags):
     inp = synth.make_layer_inputs(s, seed=31)
     f = oracle._f64_inputs(inp)
     rt = oracle.router(f["x"], f["W_r"], f["b_r"], s.G, s.M, s.k)
@@ -54,7 +65,7 @@ def test_layer_backward_matches_oracle(rsq, name):
     ref = bw.backward(f["x"], f["W_r"], f["b_r"], f["W_q"], f["W_qs"], f["W_k"], f["W_v"], f["W_o"],
                       B=s.B, T=s.T, G=s.G, M=s.M, dh=s.d_head, idx=rt["idx"], dy=dy.astype(np.float64))
     d = device_inputs(inp)
-    cfg = rsq.GQEConfig.of(s)
+    cfg = rsq.GQEConfig.of(s, flags)
     ws = torch.zeros(rsq.gqe_workspace_bytes(cfg, rsq.GQE_WS_BACKWARD), dtype=torch.uint8, device="cuda")
     dev = lambda *shape: torch.empty(*shape, dtype=torch.float32, device="cuda")  # noqa: E731
     N, dh, R, dm = s.N, s.d_head, s.R, s.d_model
