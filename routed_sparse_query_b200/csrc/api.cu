@@ -50,8 +50,20 @@ gqe_status check_cfg(const gqe_config* c) {
 gqe_status cuda_status(int e) { return e == cudaSuccess ? GQE_OK : GQE_ERR_CUDA; }
 
 struct LayerWs {
-  size_t idx, r, omega, counts, offsets, tok, slot_pos, Qv, Qs, K, V, slots, dws, aws, total;
+  size_t idx, r, omega, counts, offsets, tok, slot_pos, Qv, Qs, K, V, slots, Qd, dws, aws, total;
 };
+
+// Short batches (at most this many rows, d_head 64, slot-major attention):
+// the queries of every expert come from one dense GEMM and the routed rows
+// are copied into the slot-major streams, so the dispatch lists and the
+// gathered routed Q GEMM leave the critical path (at the price of the
+// unselected experts' projection FLOPs). The routed Q rows are the same
+// values either way.
+constexpr long long kGatherRows = 4096;
+bool gather_path(const gqe_config& c) {
+  return c.d_head == 64 && (c.flags & GQE_FLAG_EXPERT_MAJOR) == 0u &&
+         static_cast<long long>(c.B) * c.T <= kGatherRows;
+}
 
 LayerWs layer_ws(const gqe_config& c) {
   const size_t R = static_cast<size_t>(c.B) * c.T;
@@ -76,6 +88,7 @@ LayerWs layer_ws(const gqe_config& c) {
   put(L.K, R * c.G * dh * 2);
   put(L.V, R * c.G * dh * 2);
   put(L.slots, R * n_slots(c) * dh * 2);
+  put(L.Qd, gather_path(c) ? R * N * dh * 2 : 0);  // every expert's queries [B][N][T][dh]
   put(L.dws, dispatch_ws_layout(c).total);
   put(L.aws, attention_plan(c, n_streams(c)).total);
   L.total = o;
@@ -402,7 +415,7 @@ gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* 
 static gqe_status layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r, const float* b_r,
                             const gqe_bf16* W_q, const gqe_bf16* W_qs, const gqe_bf16* W_k, const gqe_bf16* W_v,
                             const gqe_bf16* W_o, gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream_t stream,
-                            float* lse) {
+                            float* lse, bool allow_gather) {
   const gqe_status s = check_cfg(cfg);
   if (s != GQE_OK) return s;
   const bool shared = has_shared_head(*cfg);
@@ -423,6 +436,7 @@ static gqe_status layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const floa
     return GQE_ERR_CUDA;
   // K/V projection on the side stream (falls back to the caller's stream).
   cudaStream_t main_st = static_cast<cudaStream_t>(stream);
+  const bool gather = allow_gather && gather_path(*cfg);
   {
     std::lock_guard<std::mutex> guard(g_side_mu);
     // The router goes first (it heads the critical path); the K/V projection
@@ -441,9 +455,17 @@ static gqe_status layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const floa
     if (shared && gemm_q_shared(*cfg, x, W_qs, H(L.Qs), side ? side->s : stream) != cudaSuccess)
       return GQE_ERR_CUDA;
     if (side != nullptr && cudaEventRecord(side->join, side->s) != cudaSuccess) return GQE_ERR_CUDA;
-    st = dispatch_and_project(*cfg, I(L.idx), x, W_q, W_qs, I(L.counts), I(L.offsets), I(L.tok),
-                              I(L.slot_pos), H(L.Qv), nullptr, w + L.dws, L.total - L.dws, stream);
-    if (st != GQE_OK) return st;
+    if (gather) {
+      // Short batch: every expert's queries in one dense GEMM, then the
+      // routed rows copied into the slot-major streams (no token lists).
+      if (gemm_q_dense(*cfg, x, W_q, H(L.Qd), stream) != cudaSuccess ||
+          gather_routed_q(*cfg, H(L.Qd), I(L.idx), H(L.Qv), stream) != cudaSuccess)
+        return GQE_ERR_CUDA;
+    } else {
+      st = dispatch_and_project(*cfg, I(L.idx), x, W_q, W_qs, I(L.counts), I(L.offsets), I(L.tok),
+                                I(L.slot_pos), H(L.Qv), nullptr, w + L.dws, L.total - L.dws, stream);
+      if (st != GQE_OK) return st;
+    }
     if (side != nullptr && cudaStreamWaitEvent(main_st, side->join, 0) != cudaSuccess)
       return GQE_ERR_CUDA;
   }
@@ -460,7 +482,7 @@ gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
                          const float* b_r, const gqe_bf16* W_q, const gqe_bf16* W_qs,
                          const gqe_bf16* W_k, const gqe_bf16* W_v, const gqe_bf16* W_o,
                          gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream_t stream) {
-  return layer_fwd(cfg, x, W_r, b_r, W_q, W_qs, W_k, W_v, W_o, y, ws, ws_bytes, stream, nullptr);
+  return layer_fwd(cfg, x, W_r, b_r, W_q, W_qs, W_k, W_v, W_o, y, ws, ws_bytes, stream, nullptr, true);
 }
 
 gqe_status gqe_layer_bwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r, const float* b_r,
@@ -483,7 +505,7 @@ gqe_status gqe_layer_bwd(const gqe_config* cfg, const gqe_bf16* x, const float* 
   auto Hp = [&](size_t o) { return reinterpret_cast<uint16_t*>(w + o); };
   // The forward, into the layer part of the workspace (routing, Q, K, V, slots).
   gqe_status st = layer_fwd(cfg, x, W_r, b_r, W_q, W_qs, W_k, W_v, W_o, reinterpret_cast<gqe_bf16*>(w + W.y), ws,
-                            W.L.total, stream, Fp(W.lse));
+                            W.L.total, stream, Fp(W.lse), true);
   if (st != GQE_OK) return st;
   const LayerWs& L = W.L;
   const long long R = static_cast<long long>(c.B) * c.T;
