@@ -293,8 +293,11 @@ gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* 
  * side stream owned by the library (one per device) that forks from `stream`
  * after the router and joins it before the attention, so the call is still
  * stream-ordered as a whole (and captures into a CUDA graph as a fork/join).
- * The results are bitwise those of the step calls. Arguments as in the calls
- * above.
+ * The results are bitwise those of the step calls. Batches of at most 4096
+ * rows with d_head 64 (slot-major) take every expert's queries from one dense
+ * GEMM that stores only the routed rows: the token lists (COUNTS, OFFSETS,
+ * TOK, SLOT_POS) of the workspace are then not written. Arguments as in the
+ * calls above.
  */
 gqe_status gqe_layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r,
                          const float* b_r, const gqe_bf16* W_q, const gqe_bf16* W_qs,

@@ -50,15 +50,15 @@ gqe_status check_cfg(const gqe_config* c) {
 gqe_status cuda_status(int e) { return e == cudaSuccess ? GQE_OK : GQE_ERR_CUDA; }
 
 struct LayerWs {
-  size_t idx, r, omega, counts, offsets, tok, slot_pos, Qv, Qs, K, V, slots, Qd, dws, aws, total;
+  size_t idx, r, omega, counts, offsets, tok, slot_pos, Qv, Qs, K, V, slots, dws, aws, total;
 };
 
 // Short batches (at most this many rows, d_head 64, slot-major attention):
-// the queries of every expert come from one dense GEMM and the routed rows
-// are copied into the slot-major streams, so the dispatch lists and the
-// gathered routed Q GEMM leave the critical path (at the price of the
-// unselected experts' projection FLOPs). The routed Q rows are the same
-// values either way.
+// the queries of every expert come from one dense GEMM whose epilogue stores
+// only the routed rows, straight into the slot-major streams, so the dispatch
+// lists and the gathered routed Q GEMM leave the critical path (at the price
+// of the unselected experts' projection FLOPs). The routed Q rows are the
+// same values either way.
 constexpr long long kGatherRows = 4096;
 bool gather_path(const gqe_config& c) {
   return c.d_head == 64 && (c.flags & GQE_FLAG_EXPERT_MAJOR) == 0u &&
@@ -88,7 +88,6 @@ LayerWs layer_ws(const gqe_config& c) {
   put(L.K, R * c.G * dh * 2);
   put(L.V, R * c.G * dh * 2);
   put(L.slots, R * n_slots(c) * dh * 2);
-  put(L.Qd, gather_path(c) ? R * N * dh * 2 : 0);  // every expert's queries [B][N][T][dh]
   put(L.dws, dispatch_ws_layout(c).total);
   put(L.aws, attention_plan(c, n_streams(c)).total);
   L.total = o;
@@ -450,18 +449,23 @@ static gqe_status layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const floa
     // The side stream also takes the shared-head query projection (it reads
     // only x), so the routed Q projection on the critical path has only the
     // routed tiles.
-    const gqe_status kv = gqe_kv_proj(cfg, x, W_k, W_v, H(L.K), H(L.V), side ? side->s : stream);
-    if (kv != GQE_OK) return kv;
-    if (shared && gemm_q_shared(*cfg, x, W_qs, H(L.Qs), side ? side->s : stream) != cudaSuccess)
-      return GQE_ERR_CUDA;
-    if (side != nullptr && cudaEventRecord(side->join, side->s) != cudaSuccess) return GQE_ERR_CUDA;
     if (gather) {
-      // Short batch: every expert's queries in one dense GEMM, then the
-      // routed rows copied into the slot-major streams (no token lists).
-      if (gemm_q_dense(*cfg, x, W_q, H(L.Qd), stream) != cudaSuccess ||
-          gather_routed_q(*cfg, H(L.Qd), I(L.idx), H(L.Qv), stream) != cudaSuccess)
+      // Short batch: the shared head's queries first (they join before the
+      // attention), then K/V on the side stream; every expert's queries in
+      // one dense GEMM on this stream, the routed rows stored straight into
+      // the slot-major streams (no token lists).
+      if (shared && gemm_q_shared(*cfg, x, W_qs, H(L.Qs), side ? side->s : stream) != cudaSuccess)
         return GQE_ERR_CUDA;
+      const gqe_status kv = gqe_kv_proj(cfg, x, W_k, W_v, H(L.K), H(L.V), side ? side->s : stream);
+      if (kv != GQE_OK) return kv;
+      if (side != nullptr && cudaEventRecord(side->join, side->s) != cudaSuccess) return GQE_ERR_CUDA;
+      if (gemm_q_all_routed(*cfg, x, W_q, I(L.idx), H(L.Qv), stream) != cudaSuccess) return GQE_ERR_CUDA;
     } else {
+      const gqe_status kv = gqe_kv_proj(cfg, x, W_k, W_v, H(L.K), H(L.V), side ? side->s : stream);
+      if (kv != GQE_OK) return kv;
+      if (shared && gemm_q_shared(*cfg, x, W_qs, H(L.Qs), side ? side->s : stream) != cudaSuccess)
+        return GQE_ERR_CUDA;
+      if (side != nullptr && cudaEventRecord(side->join, side->s) != cudaSuccess) return GQE_ERR_CUDA;
       st = dispatch_and_project(*cfg, I(L.idx), x, W_q, W_qs, I(L.counts), I(L.offsets), I(L.tok),
                                 I(L.slot_pos), H(L.Qv), nullptr, w + L.dws, L.total - L.dws, stream);
       if (st != GQE_OK) return st;

@@ -451,33 +451,4 @@ int launch_scale_slots(const gqe_config& c, uint16_t* slots, const float* omega,
                     static_cast<int>(R), gk, c.d_head, n_slots(c) * c.d_head);
 }
 
-// Routed queries of a short batch: every expert's queries were projected
-// (Qd [B][N][T][dh]); the slot-major streams take each token's row of the
-// expert its slot selected. One thread per 16 bytes of an output row.
-__global__ void gather_routed_q_kernel(const uint16_t* Qd, const int32_t* idx, uint16_t* Qv, int B, int T, int G,
-                                       int M, int k, int dh) {
-  const int per_row = dh / 8;
-  const long long rows = static_cast<long long>(B) * G * k * T;
-  const long long n = rows * per_row;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long row = i / per_row;  // ((b G + g) k + s) T + t
-    const int c = static_cast<int>(i - row * per_row);
-    const int t = static_cast<int>(row % T);
-    const long long bgs = row / T;
-    const int s = static_cast<int>(bgs % k);
-    const int g = static_cast<int>((bgs / k) % G);
-    const int b = static_cast<int>(bgs / (static_cast<long long>(k) * G));
-    const int e = g * M + __ldg(idx + ((static_cast<long long>(b) * T + t) * G + g) * k + s);
-    const uint4* src = reinterpret_cast<const uint4*>(Qd + ((static_cast<long long>(b) * G * M + e) * T + t) * dh);
-    reinterpret_cast<uint4*>(Qv + row * dh)[c] = __ldg(src + c);
-  }
-}
-
-int gather_routed_q(const gqe_config& c, const uint16_t* Qd, const int32_t* idx, uint16_t* Qv, void* stream) {
-  gather_routed_q_kernel<<<2 * device_sms(), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      Qd, idx, Qv, c.B, c.T, c.G, c.M, c.k, c.d_head);
-  return cudaGetLastError();
-}
-
 }  // namespace gqe

@@ -74,6 +74,12 @@ struct Epi {
   float* outf = nullptr;
   long long ldf = 0;
   int fvec = 0;
+  // Routed head-split output (every expert's queries computed, only the
+  // routed ones stored): column block h is expert h of the row's token; it
+  // goes to slot s of its group, out + ((b G + g) k + s) sh + t st + c, where
+  // sel[row][g][s] == h % M; rows that did not select h store nothing.
+  const int32_t* sel = nullptr;
+  int G = 0, M = 0, k = 0;
 };
 
 struct Gather {
@@ -409,7 +415,16 @@ __global__ void __launch_bounds__(192, 2)
         const int col0 = n0 + cc * 32;
         if (valid && col0 < epi.cols) {
           const int h = col0 / epi.hd, c = col0 % epi.hd;
-          store32_bf16(epi.out + bb * epi.sb + h * epi.sh + t * epi.st + c, v);
+          if (epi.sel != nullptr) {
+            const int g = h / epi.M, j = h - g * epi.M;
+            const int32_t* ip = epi.sel + (static_cast<size_t>(row) * epi.G + g) * epi.k;
+            for (int s2 = 0; s2 < epi.k; ++s2)
+              if (__ldg(ip + s2) == j)
+                store32_bf16(epi.out + ((static_cast<long long>(bb) * epi.G + g) * epi.k + s2) * epi.sh +
+                                 t * epi.st + c, v);
+          } else {
+            store32_bf16(epi.out + bb * epi.sb + h * epi.sh + t * epi.st + c, v);
+          }
         }
       }
     }
@@ -854,6 +869,18 @@ int gemm_q_dense(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, ui
   const int R = c.B * c.T;
   const int N = c.G * c.M;
   const Epi e = head_split(Q, c.T, N, c.d_head, R);
+  return dense_gemm(x, R, c.d_model, W_q, nullptr, N * c.d_head, e, e, 1, stream);
+}
+
+int gemm_q_all_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const int32_t* idx,
+                      uint16_t* Qv, void* stream) {
+  const int R = c.B * c.T;
+  const int N = c.G * c.M;
+  Epi e = head_split(Qv, c.T, N, c.d_head, R);
+  e.sel = idx;
+  e.G = c.G;
+  e.M = c.M;
+  e.k = c.k;
   return dense_gemm(x, R, c.d_model, W_q, nullptr, N * c.d_head, e, e, 1, stream);
 }
 

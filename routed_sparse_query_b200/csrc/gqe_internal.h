@@ -149,9 +149,10 @@ AttnPlan attention_plan(const gqe_config& c, int H);
 int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, const uint16_t* K,
                   const uint16_t* V, uint16_t* slots, void* ws, size_t ws_bytes,
                   bool counters_zeroed, void* stream, float* lse = nullptr);
-// Routed queries copied out of every expert's queries: Qv[b][g][s][t] =
-// Qd[b][g M + idx[b T + t][g][s]][t] (Qd [B][G*M][T][dh], as gemm_q_dense).
-int gather_routed_q(const gqe_config& c, const uint16_t* Qd, const int32_t* idx, uint16_t* Qv, void* stream);
+// Every expert's queries in one dense GEMM, only the routed rows stored:
+// Qv[b][g][s][t] = x[b T + t] W_q[:, e], e = g M + idx[b T + t][g][s].
+int gemm_q_all_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const int32_t* idx,
+                      uint16_t* Qv, void* stream);
 // Expert-major routed attention (Qe in token-list order, rows masked by
 // their positions tok[]) plus the shared head, one launch, no scratch.
 int attention_gqe_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const uint16_t* K,
