@@ -449,7 +449,16 @@ static gqe_status layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const floa
     // The side stream also takes the shared-head query projection (it reads
     // only x), so the routed Q projection on the critical path has only the
     // routed tiles.
-    if (gather) {
+    if (gather && cfg->M == 2) {
+      // Short batch, two experts per group: K, V and every expert's queries
+      // (the routed rows stored straight into the slot-major streams) in one
+      // launch of four outputs; the shared head's queries on the side stream.
+      if (shared && gemm_q_shared(*cfg, x, W_qs, H(L.Qs), side ? side->s : stream) != cudaSuccess)
+        return GQE_ERR_CUDA;
+      if (side != nullptr && cudaEventRecord(side->join, side->s) != cudaSuccess) return GQE_ERR_CUDA;
+      if (gemm_kvq_routed(*cfg, x, W_k, W_v, W_q, I(L.idx), H(L.K), H(L.V), H(L.Qv), stream) != cudaSuccess)
+        return GQE_ERR_CUDA;
+    } else if (gather) {
       // Short batch: the shared head's queries first (they join before the
       // attention), then K/V on the side stream; every expert's queries in
       // one dense GEMM on this stream, the routed rows stored straight into

@@ -80,6 +80,7 @@ struct Epi {
   // sel[row][g][s] == h % M; rows that did not select h store nothing.
   const int32_t* sel = nullptr;
   int G = 0, M = 0, k = 0;
+  int h0 = 0;  // expert of column block 0 (a launch over a slice of the experts)
 };
 
 struct Gather {
@@ -111,7 +112,10 @@ __device__ __forceinline__ void store32_bf16(uint16_t* dst, const uint32_t (&v)[
 template <int BN, bool GATHER>
 __global__ void __launch_bounds__(192, 2)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                const __grid_constant__ CUtensorMap tmB1, const Epi epi0, const Epi epi1,
+                const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
+                const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ Epi epi0,
+                const __grid_constant__ Epi epi1, const __grid_constant__ Epi epi2,
+                const __grid_constant__ Epi epi3,
                 const Gather ga, const int K) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -130,8 +134,10 @@ __global__ void __launch_bounds__(192, 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool z1 = blockIdx.z == 1 || (GATHER && blockIdx.x >= static_cast<unsigned>(ga.max_qtiles));
-  const CUtensorMap* tmB = z1 ? &tmB1 : &tmB0;
-  const Epi& epi = z1 ? epi1 : epi0;
+  // Output z of up to four (B operand, epilogue) pairs of one launch.
+  const int zi = GATHER ? (z1 ? 1 : 0) : static_cast<int>(blockIdx.z);
+  const CUtensorMap* tmB = zi == 0 ? &tmB0 : zi == 1 ? &tmB1 : zi == 2 ? &tmB2 : &tmB3;
+  const Epi& epi = zi == 0 ? epi0 : zi == 1 ? epi1 : zi == 2 ? epi2 : epi3;
 
   const int nk = (K + BK - 1) / BK;
 
@@ -416,7 +422,7 @@ __global__ void __launch_bounds__(192, 2)
         if (valid && col0 < epi.cols) {
           const int h = col0 / epi.hd, c = col0 % epi.hd;
           if (epi.sel != nullptr) {
-            const int g = h / epi.M, j = h - g * epi.M;
+            const int g = (epi.h0 + h) / epi.M, j = epi.h0 + h - g * epi.M;
             const int32_t* ip = epi.sel + (static_cast<size_t>(row) * epi.G + g) * epi.k;
             for (int s2 = 0; s2 < epi.k; ++s2)
               if (__ldg(ip + s2) == j)
@@ -737,13 +743,20 @@ __global__ void __launch_bounds__(q_threads(GW), 1)
 }
 
 template <int BN, bool GATHER>
-int launch(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const Epi& e0,
-           const Epi& e1, const Gather& g, int K, dim3 grid, void* stream) {
+int launch(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const CUtensorMap& B2,
+           const CUtensorMap& B3, const Epi& e0, const Epi& e1, const Epi& e2, const Epi& e3, const Gather& g,
+           int K, dim3 grid, void* stream) {
   using C = GemmCfg<BN>;
   const int e = ensure_smem<gemm_kernel<BN, GATHER>>(static_cast<int>(C::SMEM));
   if (e != cudaSuccess) return e;
-  return launch_pdl(gemm_kernel<BN, GATHER>, grid, dim3(192), C::SMEM, stream, A, B0, B1, e0, e1,
+  return launch_pdl(gemm_kernel<BN, GATHER>, grid, dim3(192), C::SMEM, stream, A, B0, B1, B2, B3, e0, e1, e2, e3,
                     g, K);
+}
+
+template <int BN, bool GATHER>
+int launch(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const Epi& e0,
+           const Epi& e1, const Gather& g, int K, dim3 grid, void* stream) {
+  return launch<BN, GATHER>(A, B0, B1, B1, B1, e0, e1, e1, e1, g, K, grid, stream);
 }
 
 template <int DH>
@@ -882,6 +895,36 @@ int gemm_q_all_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_
   e.M = c.M;
   e.k = c.k;
   return dense_gemm(x, R, c.d_model, W_q, nullptr, N * c.d_head, e, e, 1, stream);
+}
+
+int gemm_kvq_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
+                    const uint16_t* W_q, const int32_t* idx, uint16_t* K, uint16_t* V, uint16_t* Qv, void* stream) {
+  const int R = c.B * c.T, dh = c.d_head;
+  const int Nkv = c.G * dh, Nq = c.G * c.M * dh;
+  if (Nq != 2 * Nkv || Nkv % 64 != 0) return cudaErrorInvalidValue;
+  const int BN = Nkv % 128 == 0 ? 128 : 64;
+  const long long mt = (R + BM - 1) / BM;
+  CUtensorMap ta, tk, tv, tq0, tq1;
+  if (!make_tmap_bf16_2d(&ta, x, c.d_model, R, c.d_model, 64, BM) ||
+      !make_tmap_bf16_2d(&tk, W_k, Nkv, c.d_model, Nkv, 64, BK) ||
+      !make_tmap_bf16_2d(&tv, W_v, Nkv, c.d_model, Nkv, 64, BK) ||
+      !make_tmap_bf16_2d(&tq0, W_q, Nkv, c.d_model, Nq, 64, BK) ||
+      !make_tmap_bf16_2d(&tq1, W_q + Nkv, Nkv, c.d_model, Nq, 64, BK))
+    return cudaErrorInvalidValue;
+  const Epi ek = head_split(K, c.T, c.G, dh, R);
+  const Epi ev = head_split(V, c.T, c.G, dh, R);
+  Epi eq0 = head_split(Qv, c.T, c.G * c.M, dh, R);
+  eq0.cols = Nkv;
+  eq0.sel = idx;
+  eq0.G = c.G;
+  eq0.M = c.M;
+  eq0.k = c.k;
+  Epi eq1 = eq0;
+  eq1.h0 = c.G;  // the second half of the experts' columns
+  const dim3 grid(static_cast<unsigned>(mt), static_cast<unsigned>(Nkv / BN), 4);
+  Gather g{};
+  if (BN == 128) return launch<128, false>(ta, tk, tv, tq0, tq1, ek, ev, eq0, eq1, g, c.d_model, grid, stream);
+  return launch<64, false>(ta, tk, tv, tq0, tq1, ek, ev, eq0, eq1, g, c.d_model, grid, stream);
 }
 
 int gemm_rowmajor(const uint16_t* A, int rows, int K, const uint16_t* W, int N, uint16_t* out,
