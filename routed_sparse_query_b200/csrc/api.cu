@@ -456,7 +456,7 @@ static gqe_status layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const floa
       if (shared && gemm_q_shared(*cfg, x, W_qs, H(L.Qs), side ? side->s : stream) != cudaSuccess)
         return GQE_ERR_CUDA;
       if (side != nullptr && cudaEventRecord(side->join, side->s) != cudaSuccess) return GQE_ERR_CUDA;
-      if (gemm_kvq_routed(*cfg, x, W_k, W_v, W_q, I(L.idx), H(L.K), H(L.V), H(L.Qv), stream) != cudaSuccess)
+      if (gemm_kvq(*cfg, x, W_k, W_v, W_q, I(L.idx), H(L.K), H(L.V), H(L.Qv), stream) != cudaSuccess)
         return GQE_ERR_CUDA;
     } else if (gather) {
       // Short batch: the shared head's queries first (they join before the
@@ -583,7 +583,12 @@ gqe_status gqa_dense_fwd(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf1
   int e = (c.flags & GQE_FLAG_WS_CLEAN) != 0u ? cudaSuccess
                                                 : zero_attention_counters(c, c.G * c.M, w + L.aws, stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
-  {
+  if (gather_path(c) && c.M == 2) {
+    // Short batches, two heads per group: K, V and Q in one launch of four
+    // outputs (the same fusion as the GQE layer's short path).
+    e = gemm_kvq(c, x, W_k, W_v, W_q, nullptr, H(L.K), H(L.V), H(L.Q), stream);
+    if (e != cudaSuccess) return GQE_ERR_CUDA;
+  } else {
     // K/V projection beside the Q projection (side stream, as in gqe_layer_fwd).
     std::lock_guard<std::mutex> guard(g_side_mu);
     cudaStream_t main_st = static_cast<cudaStream_t>(stream);

@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(192, 2)
                 store32_bf16(epi.out + ((static_cast<long long>(bb) * epi.G + g) * epi.k + s2) * epi.sh +
                                  t * epi.st + c, v);
           } else {
-            store32_bf16(epi.out + bb * epi.sb + h * epi.sh + t * epi.st + c, v);
+            store32_bf16(epi.out + bb * epi.sb + (epi.h0 + h) * epi.sh + t * epi.st + c, v);
           }
         }
       }
@@ -897,8 +897,8 @@ int gemm_q_all_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_
   return dense_gemm(x, R, c.d_model, W_q, nullptr, N * c.d_head, e, e, 1, stream);
 }
 
-int gemm_kvq_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
-                    const uint16_t* W_q, const int32_t* idx, uint16_t* K, uint16_t* V, uint16_t* Qv, void* stream) {
+int gemm_kvq(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
+             const uint16_t* W_q, const int32_t* idx, uint16_t* K, uint16_t* V, uint16_t* Q, void* stream) {
   const int R = c.B * c.T, dh = c.d_head;
   const int Nkv = c.G * dh, Nq = c.G * c.M * dh;
   if (Nq != 2 * Nkv || Nkv % 64 != 0) return cudaErrorInvalidValue;
@@ -913,14 +913,14 @@ int gemm_kvq_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_k,
     return cudaErrorInvalidValue;
   const Epi ek = head_split(K, c.T, c.G, dh, R);
   const Epi ev = head_split(V, c.T, c.G, dh, R);
-  Epi eq0 = head_split(Qv, c.T, c.G * c.M, dh, R);
+  Epi eq0 = head_split(Q, c.T, c.G * c.M, dh, R);
   eq0.cols = Nkv;
-  eq0.sel = idx;
+  eq0.sel = idx;  // null: every expert's queries stored ([B][G*M][T][dh])
   eq0.G = c.G;
   eq0.M = c.M;
   eq0.k = c.k;
   Epi eq1 = eq0;
-  eq1.h0 = c.G;  // the second half of the experts' columns
+  eq1.h0 = c.G;  // the second half of the heads' columns
   const dim3 grid(static_cast<unsigned>(mt), static_cast<unsigned>(Nkv / BN), 4);
   Gather g{};
   if (BN == 128) return launch<128, false>(ta, tk, tv, tq0, tq1, ek, ev, eq0, eq1, g, c.d_model, grid, stream);

@@ -153,10 +153,12 @@ int attention_gqe(const gqe_config& c, const uint16_t* Qv, const uint16_t* Qs, c
 // Qv[b][g][s][t] = x[b T + t] W_q[:, e], e = g M + idx[b T + t][g][s].
 int gemm_q_all_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_q, const int32_t* idx,
                       uint16_t* Qv, void* stream);
-// K, V and every expert's queries (routed rows stored, as gemm_q_all_routed)
-// in one launch of four outputs; needs G*M*dh = 2*G*dh (M = 2).
-int gemm_kvq_routed(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
-                    const uint16_t* W_q, const int32_t* idx, uint16_t* K, uint16_t* V, uint16_t* Qv, void* stream);
+// K, V and every head's queries in one launch of four outputs (needs
+// G*M*dh = 2*G*dh, M = 2). idx non-null: only the routed rows are stored, into
+// the slot-major streams Q = Qv (as gemm_q_all_routed); null: every head's
+// queries, Q [B][G*M][T][dh] (as gemm_q_dense).
+int gemm_kvq(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const uint16_t* W_v,
+             const uint16_t* W_q, const int32_t* idx, uint16_t* K, uint16_t* V, uint16_t* Q, void* stream);
 // Expert-major routed attention (Qe in token-list order, rows masked by
 // their positions tok[]) plus the shared head, one launch, no scratch.
 int attention_gqe_em(const gqe_config& c, const uint16_t* Qe, const uint16_t* Qs, const uint16_t* K,
