@@ -81,6 +81,12 @@ struct Epi {
   const int32_t* sel = nullptr;
   int G = 0, M = 0, k = 0;
   int h0 = 0;  // expert of column block 0 (a launch over a slice of the experts)
+  // The main loop reads only the layer's inputs (x, W), complete before the
+  // previous kernel started, since every kernel of the chain lets its
+  // dependents start only after its own wait. So it runs while the previous
+  // kernel (the router) finishes, and the epilogue threads wait for that kernel
+  // before they read its selections or store anything.
+  int late_wait = 0;
 };
 
 struct Gather {
@@ -164,7 +170,8 @@ __global__ void __launch_bounds__(192, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  pdl_wait();
+  const bool late = !GATHER && epi.late_wait != 0;
+  if (!late) pdl_wait();
   pdl_launch_dependents();
 
   // Tile of this CTA (read after pdl_wait: the routed tile table is produced
@@ -362,6 +369,7 @@ __global__ void __launch_bounds__(192, 2)
         mbar_arrive(&empty[s]);
       }
     }
+    if (late) pdl_wait();
     const bool have = mbar_wait(accb, 0, abort_flag);
     tc_fence_after();
     const int r = q * 32 + lane;
@@ -911,8 +919,8 @@ int gemm_kvq(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const 
       !make_tmap_bf16_2d(&tq0, W_q, Nkv, c.d_model, Nq, 64, BK) ||
       !make_tmap_bf16_2d(&tq1, W_q + Nkv, Nkv, c.d_model, Nq, 64, BK))
     return cudaErrorInvalidValue;
-  const Epi ek = head_split(K, c.T, c.G, dh, R);
-  const Epi ev = head_split(V, c.T, c.G, dh, R);
+  Epi ek = head_split(K, c.T, c.G, dh, R);
+  Epi ev = head_split(V, c.T, c.G, dh, R);
   Epi eq0 = head_split(Q, c.T, c.G * c.M, dh, R);
   eq0.cols = Nkv;
   eq0.sel = idx;  // null: every expert's queries stored ([B][G*M][T][dh])
@@ -921,6 +929,9 @@ int gemm_kvq(const gqe_config& c, const uint16_t* x, const uint16_t* W_k, const 
   eq0.k = c.k;
   Epi eq1 = eq0;
   eq1.h0 = c.G;  // the second half of the heads' columns
+  if (idx != nullptr) {  // the main loop overlaps the router; the epilogues wait for it
+    ek.late_wait = ev.late_wait = eq0.late_wait = eq1.late_wait = 1;
+  }
   const dim3 grid(static_cast<unsigned>(mt), static_cast<unsigned>(Nkv / BN), 4);
   Gather g{};
   if (BN == 128) return launch<128, false>(ta, tk, tv, tq0, tq1, ek, ev, eq0, eq1, g, c.d_model, grid, stream);
