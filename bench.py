@@ -60,10 +60,18 @@ def launches(s: synth.LayerShape) -> dict:
             "output": 1 if s.d_head == 64 else 2}
 
 
+SHORT_BATCH_ROWS = 4096  # the library's short-batch path: B*T rows at most, d_head 64
+
+
 def layer_launches(s: synth.LayerShape) -> int:
-    """Kernels of this library per gqe_layer_fwd call: the step calls' kernels,
-    with the shared-head query projection as its own GEMM on the side stream
-    (after the K/V GEMM) instead of tiles of the routed Q GEMM."""
+    """Kernels of this library per gqe_layer_fwd call. Long batches: the step
+    calls' kernels, with the shared-head query projection as its own GEMM on
+    the side stream instead of tiles of the routed Q GEMM. Short batches
+    (B*T <= 4096, d_head 64): router, shared-head Q GEMM, the projections
+    (one fused K/V/Q GEMM when M = 2, else a K/V GEMM and an every-expert Q
+    GEMM), attention and W_O -- no token-list kernels."""
+    if s.B * s.T <= SHORT_BATCH_ROWS and s.d_head == 64:
+        return 1 + 1 + (1 if s.M == 2 else 2) + 1 + launches(s)["output"]
     return sum(launches(s).values()) + 1
 
 

@@ -49,7 +49,11 @@ def test_launch_counts():
     # counts take the separate scan.
     assert bench.launches(synth.SEQ2K) == {"router": 1, "dispatch": 3, "kv": 1, "attention": 1,
                                            "output": 1}
-    assert bench.layer_launches(synth.SEQ2K) == 8
+    # gqe_layer_fwd at seq2k takes the short-batch path: router, shared-head Q
+    # GEMM, fused K/V/Q GEMM, attention, W_O.
+    assert bench.layer_launches(synth.SEQ2K) == 5
+    # 4 x 8k: the step kernels (router, 3 dispatch, K/V, attention, W_O) + shared Q.
+    assert bench.layer_launches(synth.BATCH4_8K) == 8
     assert bench.launches(synth.BATCH4_8K)["dispatch"] == 3
     assert bench.launches(synth.SEQ1M)["dispatch"] == 4
     # d_head = 32: the weighted slot is its own kernel before W_O.
