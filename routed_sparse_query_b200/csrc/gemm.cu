@@ -783,7 +783,8 @@ int dense_gemm(const uint16_t* A, int rows, int K, const uint16_t* W0, const uin
   int BN = 256;
   const long long mt = (rows + BM - 1) / BM;
   if (N % 256 != 0 || mt * (N / 256) * nz < 148) BN = 128;
-  if (N % 128 != 0) BN = 64;
+  // Fewer 128-wide tiles than SMs: 64-wide ones (two CTAs per SM fit).
+  if (N % 128 != 0 || mt * (N / 128) * nz < 148) BN = 64;
   if (N % 64 != 0) BN = 32;
   if (N % 32 != 0) return cudaErrorInvalidValue;
   CUtensorMap ta, tb0, tb1;
