@@ -59,10 +59,10 @@ struct LayerWs {
 // lists and the gathered routed Q GEMM leave the critical path (at the price
 // of the unselected experts' projection FLOPs). The routed Q rows are the
 // same values either way.
-constexpr long long kGatherRows = 4096;
-bool gather_path(const gqe_config& c) {
+constexpr long long kShortBatchRows = 4096;
+bool short_batch_path(const gqe_config& c) {
   return c.d_head == 64 && (c.flags & GQE_FLAG_EXPERT_MAJOR) == 0u &&
-         static_cast<long long>(c.B) * c.T <= kGatherRows;
+         static_cast<long long>(c.B) * c.T <= kShortBatchRows;
 }
 
 LayerWs layer_ws(const gqe_config& c) {
@@ -414,7 +414,7 @@ gqe_status gqe_output_proj(const gqe_config* cfg, gqe_bf16* slots, const float* 
 static gqe_status layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const float* W_r, const float* b_r,
                             const gqe_bf16* W_q, const gqe_bf16* W_qs, const gqe_bf16* W_k, const gqe_bf16* W_v,
                             const gqe_bf16* W_o, gqe_bf16* y, void* ws, size_t ws_bytes, gqe_stream_t stream,
-                            float* lse, bool allow_gather) {
+                            float* lse, bool allow_short) {
   const gqe_status s = check_cfg(cfg);
   if (s != GQE_OK) return s;
   const bool shared = has_shared_head(*cfg);
@@ -435,7 +435,7 @@ static gqe_status layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const floa
     return GQE_ERR_CUDA;
   // K/V projection on the side stream (falls back to the caller's stream).
   cudaStream_t main_st = static_cast<cudaStream_t>(stream);
-  const bool gather = allow_gather && gather_path(*cfg);
+  const bool short_batch = allow_short && short_batch_path(*cfg);
   {
     std::lock_guard<std::mutex> guard(g_side_mu);
     // The router goes first (it heads the critical path); the K/V projection
@@ -449,7 +449,7 @@ static gqe_status layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const floa
     // The side stream also takes the shared-head query projection (it reads
     // only x), so the routed Q projection on the critical path has only the
     // routed tiles.
-    if (gather && cfg->M == 2) {
+    if (short_batch && cfg->M == 2) {
       // Short batch, two experts per group: K, V and every expert's queries
       // (the routed rows stored straight into the slot-major streams) in one
       // launch of four outputs; the shared head's queries on the side stream.
@@ -458,7 +458,7 @@ static gqe_status layer_fwd(const gqe_config* cfg, const gqe_bf16* x, const floa
       if (side != nullptr && cudaEventRecord(side->join, side->s) != cudaSuccess) return GQE_ERR_CUDA;
       if (gemm_kvq(*cfg, x, W_k, W_v, W_q, I(L.idx), H(L.K), H(L.V), H(L.Qv), stream) != cudaSuccess)
         return GQE_ERR_CUDA;
-    } else if (gather) {
+    } else if (short_batch) {
       // Short batch: the shared head's queries first (they join before the
       // attention), then K/V on the side stream; every expert's queries in
       // one dense GEMM on this stream, the routed rows stored straight into
@@ -583,7 +583,7 @@ gqe_status gqa_dense_fwd(const gqe_config* cfg, const gqe_bf16* x, const gqe_bf1
   int e = (c.flags & GQE_FLAG_WS_CLEAN) != 0u ? cudaSuccess
                                                 : zero_attention_counters(c, c.G * c.M, w + L.aws, stream);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
-  if (gather_path(c) && c.M == 2) {
+  if (short_batch_path(c) && c.M == 2) {
     // Short batches, two heads per group: K, V and Q in one launch of four
     // outputs (the same fusion as the GQE layer's short path).
     e = gemm_kvq(c, x, W_k, W_v, W_q, nullptr, H(L.K), H(L.V), H(L.Q), stream);
