@@ -197,6 +197,50 @@ __global__ void __launch_bounds__(256) transpose_kernel(const TI* in, long long 
   }
 }
 
+// The bf16 transpose on 64 x 64 tiles (block 32 x 8): each thread moves
+// pairs of elements, so a warp reads and writes 128 contiguous bytes of a
+// row. Needs even row strides and 4-byte aligned bases.
+__global__ void __launch_bounds__(256) transpose_pairs_kernel(const uint16_t* in, long long ldi, int rows, int cols,
+                                                              uint16_t* out, long long ldo) {
+  __shared__ uint16_t tile[64][66];
+  const long long r0 = static_cast<long long>(blockIdx.y) * 64, c0 = static_cast<long long>(blockIdx.x) * 64;
+  const int tx = threadIdx.x;
+  for (int i = threadIdx.y; i < 64; i += 8) {
+    const long long r = r0 + i, c = c0 + 2 * tx;
+    uint32_t v = 0u;
+    if (r < rows && c + 1 < cols) v = __ldg(reinterpret_cast<const uint32_t*>(in + r * ldi + c));
+    else if (r < rows && c < cols) v = in[r * ldi + c];
+    tile[i][2 * tx] = static_cast<uint16_t>(v & 0xffffu);
+    tile[i][2 * tx + 1] = static_cast<uint16_t>(v >> 16);
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 64; i += 8) {
+    const long long c = c0 + i, r = r0 + 2 * tx;
+    if (c >= cols) continue;
+    const uint32_t lo = tile[2 * tx][i], hi = tile[2 * tx + 1][i];
+    if (r + 1 < rows) *reinterpret_cast<uint32_t*>(out + c * ldo + r) = lo | (hi << 16);
+    else if (r < rows) out[c * ldo + r] = static_cast<uint16_t>(lo);
+  }
+}
+
+// out[r, c] = bf16(in[r, c]) (row strides ldi, ldo), four columns per thread
+// where the row strides and cols allow 16-byte loads.
+__global__ void cast4_kernel(const float* in, long long ldi, long long rows, int cols, uint16_t* out,
+                             long long ldo) {
+  const int q = cols / 4;
+  const long long n = rows * q;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / q;
+    const int c = 4 * static_cast<int>(i - r * q);
+    const float4 v = __ldg(reinterpret_cast<const float4*>(in + r * ldi + c));
+    uint2 o;
+    o.x = pack_bf16x2(v.x, v.y);
+    o.y = pack_bf16x2(v.z, v.w);
+    *reinterpret_cast<uint2*>(out + r * ldo + c) = o;
+  }
+}
+
 // out[r, c] = bf16(in[r, c]) (row strides ldi, ldo).
 __global__ void cast_kernel(const float* in, long long ldi, long long rows, int cols, uint16_t* out, long long ldo) {
   const long long n = rows * cols;
@@ -289,6 +333,14 @@ using namespace bwd_impl;
 template <typename TI>
 int bwd_transpose(const TI* in, long long ldi, int rows, int cols, uint16_t* out, long long ldo, void* stream) {
   if (rows <= 0 || cols <= 0) return cudaSuccess;
+  if (sizeof(TI) == 2 && ((ldi | ldo) & 1) == 0 &&
+      ((reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(out)) & 3u) == 0) {
+    const dim3 grid(static_cast<unsigned>((cols + 63) / 64), static_cast<unsigned>((rows + 63) / 64));
+    if (grid.y > 65535u) return cudaErrorInvalidConfiguration;
+    transpose_pairs_kernel<<<grid, dim3(32, 8), 0, static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const uint16_t*>(in), ldi, rows, cols, out, ldo);
+    return cudaGetLastError();
+  }
   const dim3 grid(static_cast<unsigned>((cols + 31) / 32), static_cast<unsigned>((rows + 31) / 32));
   if (grid.y > 65535u) return cudaErrorInvalidConfiguration;
   transpose_kernel<TI><<<grid, dim3(32, 8), 0, static_cast<cudaStream_t>(stream)>>>(in, ldi, rows, cols, out, ldo);
@@ -298,7 +350,11 @@ template int bwd_transpose<uint16_t>(const uint16_t*, long long, int, int, uint1
 template int bwd_transpose<float>(const float*, long long, int, int, uint16_t*, long long, void*);
 
 int bwd_cast(const float* in, long long ldi, long long rows, int cols, uint16_t* out, long long ldo, void* stream) {
-  cast_kernel<<<1024, 256, 0, static_cast<cudaStream_t>(stream)>>>(in, ldi, rows, cols, out, ldo);
+  if (((ldi | ldo | cols) & 3) == 0 &&
+      ((reinterpret_cast<uintptr_t>(in) & 15u) | (reinterpret_cast<uintptr_t>(out) & 7u)) == 0)
+    cast4_kernel<<<1184, 256, 0, static_cast<cudaStream_t>(stream)>>>(in, ldi, rows, cols, out, ldo);
+  else
+    cast_kernel<<<1024, 256, 0, static_cast<cudaStream_t>(stream)>>>(in, ldi, rows, cols, out, ldo);
   return cudaGetLastError();
 }
 
